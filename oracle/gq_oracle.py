@@ -1,0 +1,471 @@
+"""Plain CPU oracle for layer-wise GPTQ / RTN 4-bit weight quantization.
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring.  Float work is fp64
+except where the method takes an integer decision (a quantisation code, a
+stored 16-bit scale): those decisions are taken in IEEE float32 with the same
+operation order as the kernels, so both sides decide in the same precision.
+
+Sources (page title -- section):
+
+* [RTN]  "GPT-2 Quantization Reconstruction Error" -- "What this project
+  does": 4-bit symmetric per-channel quantisation, one scale per output row,
+  15 discrete levels, dequantised back to float; per-layer output MSE.
+* [AFF]  "Model Quantization Mechanics: Precision Reduction and Weight
+  Formatting" -- section 1: affine quantisation W_q = round(W/S) + Z,
+  W_deq = S (W_q - Z); group-wise quantisation with g = 128.  Section 2.1:
+  objective ||WX - W^X||^2; Cholesky decomposition of the inverse Hessian.
+* [OBQ]  "GPTQ: Post-Training INT4" -- "OBQ Foundation" (objective),
+  "Hessian-Based Weight Update" (H = 2 X X^T, OBS update), "The GPTQ
+  Algorithm" (fixed left-to-right order, lazy blocks of B = 128 columns, the
+  scaled error and the in-block / trailing updates), "Group Quantization"
+  (groups of consecutive weights; 4.25 / 4.125 bits per weight), "Running
+  GPTQ with AutoGPTQ" (damp_percent, desc_act, sym).
+* [LES]  "GPTQ and AWQ" (Inference and Serving, lesson 17) -- "Your turn"
+  (the 0.26 / 0.26 pair) and "Example 1.1" (rounding with the error carried
+  forward).
+
+Readings taken where the pages are silent, ambiguous or garbled:
+
+1. H = 2 X^T X with X stored tokens x d_in (the listing's orientation); no
+   1/N normalisation.  Codes are invariant to a positive scale of H.
+2. Damping: H_jj += damp * mean(diag H) with damp = 0.01 (the AutoGPTQ
+   config's damp_percent), not the listing's fixed 1e-6 * I.
+3. Dead columns (H_jj == 0): H_jj := 1 and W[:, j] := 0, before damping.
+4. The listing's "H_inv" is read as the upper Cholesky factor U of H^-1
+   (H^-1 = U^T U): h_inv_jj -> U_jj, H_inv[j, j+1:] -> U[j, j+1:].  This is
+   what section 2.1 of the quantisation-mechanics page describes, and only
+   this form equals the OBS update (checked against ``obs_quantize``).
+5. The OBS update prints H where H_F^-1 is meant: delta_F =
+   -(w_q - q^) [H_F^-1]_{F,q} / [H_F^-1]_qq.
+6. quantize_to_int on one column: a group's scale (and zero) is computed
+   from that group's *current* (already updated) weights when the group's
+   first column is reached; for per-channel (group_size = -1) once from the
+   initial row.  group_size must divide block_size.
+7. Symmetric grid: 15 levels -7..7, s = absmax / 7.  Affine grid: 0..15,
+   s = (max' - min') / 15 with min' = min(min, 0), max' = max(max, 0),
+   z = rint(-min' / s).  The 16-bit scale is used for quantising and
+   dequantising.  A scale that is 0 in fp16 (all-zero group, or underflow)
+   becomes 1 with z = 0; a scale above the fp16 range saturates to 65504.
+8. Rounding is round-half-to-even.
+9. Act-order: perm = stable argsort(-diag H) after damping; groups are
+   consecutive columns in permuted order; g_idx[c] is the group of original
+   column c; codes are returned in original column order.
+"""
+from __future__ import annotations
+
+import itertools
+from dataclasses import dataclass
+
+import numpy as np
+
+F32 = np.float32
+F16_MAX = F32(65504.0)
+
+__all__ = [
+    "hessian", "hessian_entries", "damp_hessian", "act_order_perm",
+    "upper_factor_of_inverse", "sym_params", "affine_params", "quantize_codes",
+    "dequantize_codes", "pack_nibbles", "unpack_nibbles", "rtn_quantize",
+    "GptqResult", "gptq_quantize", "dequantize_packed", "recon_sse",
+    "recon_sse_trace", "bits_per_weight", "obs_quantize", "bruteforce_row",
+    "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
+    "gptq_layer",
+]
+
+
+# --------------------------------------------------------------------------
+# Hessian, damping, act-order, inverse factor
+# --------------------------------------------------------------------------
+
+def hessian(X) -> np.ndarray:
+    """H = 2 X^T X in fp64 ("GPTQ: Post-Training INT4", "Hessian-Based Weight
+    Update"; X is tokens x d_in as in the listing of "The GPTQ Algorithm").
+
+    X holds bf16 values (any float dtype that represents them exactly)."""
+    X64 = np.asarray(X, dtype=np.float64)
+    return 2.0 * (X64.T @ X64)
+
+
+def hessian_entries(X, rows, cols) -> np.ndarray:
+    """The sub-block H[rows][:, cols] of H = 2 X^T X, each entry computed
+    straight from its definition (for sampled checks at large sizes)."""
+    X64 = np.asarray(X, dtype=np.float64)
+    return 2.0 * (X64[:, rows].T @ X64[:, cols])
+
+
+def damp_hessian(H, damp_percent=0.01):
+    """Dead-column fix, then H_jj += damp * mean(diag H).
+
+    Damping follows the damp_percent knob of "GPTQ: Post-Training INT4" --
+    "Running GPTQ with AutoGPTQ" (reading 2); dead columns are reading 3.
+    Returns (H_damped, dead_mask)."""
+    H = np.array(H, dtype=np.float64, copy=True)
+    d = H.shape[0]
+    diag = np.diag(H).copy()
+    dead = diag == 0.0
+    idx = np.arange(d)
+    H[idx[dead], idx[dead]] = 1.0
+    lam = damp_percent * np.mean(np.diag(H))
+    H[idx, idx] += lam
+    return H, dead
+
+
+def act_order_perm(H_damped) -> np.ndarray:
+    """Columns in order of descending diag H, ties by lower index first
+    (desc_act of "Running GPTQ with AutoGPTQ"; reading 9)."""
+    return np.argsort(-np.diag(H_damped), kind="stable").astype(np.int64)
+
+
+def upper_factor_of_inverse(H) -> np.ndarray:
+    """U upper triangular with H^-1 = U^T U.
+
+    The route the pages describe: Cholesky of H, its inverse (the listing's
+    cholesky_inverse), then the Cholesky factor of H^-1 ("Model Quantization
+    Mechanics", section 2.1: "a Cholesky decomposition of the inverse
+    Hessian").  Raises numpy.linalg.LinAlgError if H is not positive
+    definite."""
+    L = np.linalg.cholesky(H)                    # H = L L^T
+    Linv = np.linalg.inv(L)
+    Hinv = Linv.T @ Linv                         # H^-1
+    Hinv = 0.5 * (Hinv + Hinv.T)
+    Lh = np.linalg.cholesky(Hinv)                # H^-1 = Lh Lh^T
+    return np.ascontiguousarray(Lh.T)            # U = Lh^T
+
+
+# --------------------------------------------------------------------------
+# Quantisation grid (float32 decisions, see module docstring)
+# --------------------------------------------------------------------------
+
+def _to_fp16_scale(s32):
+    s32 = np.minimum(np.asarray(s32, dtype=F32), F16_MAX)
+    s16 = s32.astype(np.float16)
+    degenerate = s16 == np.float16(0)
+    s16 = np.where(degenerate, np.float16(1.0), s16)
+    return s16, degenerate
+
+
+def sym_params(vals, bits=4):
+    """Symmetric scale per row of ``vals`` (rows x group): s = absmax / qmax,
+    qmax = 2^(bits-1) - 1 (7 -> 15 levels, "GPT-2 Quantization
+    Reconstruction Error").  Returns (scale fp16, zero fp16 = 0)."""
+    v = np.asarray(vals, dtype=F32)
+    qmax = F32(2 ** (bits - 1) - 1)
+    amax = np.max(np.abs(v), axis=-1)
+    s16, _ = _to_fp16_scale(amax / qmax)
+    return s16, np.zeros_like(s16)
+
+
+def affine_params(vals, bits=4):
+    """Affine scale and zero per row ("Model Quantization Mechanics",
+    section 1): the range [min', max'] always contains 0, s = range / maxq,
+    z = rint(-min' / s) clamped to the code range (reading 7)."""
+    v = np.asarray(vals, dtype=F32)
+    maxq = F32(2 ** bits - 1)
+    mn = np.minimum(np.min(v, axis=-1), F32(0))
+    mx = np.maximum(np.max(v, axis=-1), F32(0))
+    s16, degenerate = _to_fp16_scale((mx - mn) / maxq)
+    z = np.rint(-mn / s16.astype(F32)).astype(F32)
+    z = np.clip(z, F32(0), maxq)
+    z = np.where(degenerate, F32(0), z)
+    return s16, z.astype(np.float16)
+
+
+def quantize_codes(w, s16, z16, sym, bits=4):
+    """Integer codes c = clamp(rint(w / s) + z) in float32 (RNE)."""
+    w32 = np.asarray(w, dtype=F32)
+    s = np.asarray(s16).astype(F32)
+    z = np.asarray(z16).astype(F32)
+    if sym:
+        lo, hi = F32(-(2 ** (bits - 1) - 1)), F32(2 ** (bits - 1) - 1)
+    else:
+        lo, hi = F32(0), F32(2 ** bits - 1)
+    c = np.rint(w32 / s) + z
+    c = np.clip(c, lo, hi)
+    return c.astype(np.int64)
+
+
+def dequantize_codes(c, s16, z16):
+    """W_deq = S (W_q - Z) ("Model Quantization Mechanics", section 1)."""
+    return np.asarray(s16).astype(np.float64) * (
+        np.asarray(c, dtype=np.float64) - np.asarray(z16).astype(np.float64))
+
+
+def pack_nibbles(codes, sym, bits=4):
+    """Pack [rows, d_in] codes into uint32 words of 8 nibbles along d_in;
+    nibble k of word j is column 8j + k (low nibble first).  Symmetric codes
+    are stored with an offset of 2^(bits-1) (so 8 is the zero level)."""
+    assert bits == 4
+    c = np.asarray(codes, dtype=np.int64)
+    nib = (c + 8) if sym else c
+    assert nib.min(initial=0) >= 0 and nib.max(initial=0) <= 15
+    rows, d_in = nib.shape
+    nib = nib.reshape(rows, d_in // 8, 8).astype(np.uint64)
+    words = np.zeros((rows, d_in // 8), dtype=np.uint64)
+    for k in range(8):
+        words |= nib[:, :, k] << np.uint64(4 * k)
+    return words.astype(np.uint32)
+
+
+def unpack_nibbles(words, d_in, sym, bits=4):
+    """Inverse of ``pack_nibbles``."""
+    assert bits == 4
+    w = np.asarray(words, dtype=np.uint32).astype(np.uint64)
+    rows = w.shape[0]
+    out = np.zeros((rows, w.shape[1], 8), dtype=np.int64)
+    for k in range(8):
+        out[:, :, k] = ((w >> np.uint64(4 * k)) & np.uint64(0xF)).astype(np.int64)
+    out = out.reshape(rows, -1)[:, :d_in]
+    return out - 8 if sym else out
+
+
+def bits_per_weight(d_out, d_in, group_size, sym, act_order=False):
+    """Storage cost of the packed output in bits per weight: 4 bits per code
+    plus one 16-bit scale (and one 16-bit zero unless symmetric) per group
+    ("GPTQ: Post-Training INT4", "Group Quantization"), plus a 32-bit group
+    index per input column when the columns are act-ordered."""
+    n_groups = 1 if group_size == -1 else d_in // group_size
+    bits = 4 * d_out * d_in + 16 * d_out * n_groups
+    if not sym:
+        bits += 16 * d_out * n_groups
+    if act_order:
+        bits += 32 * d_in
+    return bits / (d_out * d_in)
+
+
+# --------------------------------------------------------------------------
+# RTN baseline
+# --------------------------------------------------------------------------
+
+def rtn_quantize(W, group_size=-1, sym=True, bits=4):
+    """Round-to-nearest on the raw weights, per channel (group_size = -1) or
+    per group of consecutive weights in a row.
+
+    Returns dict(codes [d_out, d_in] int, scales fp16 [d_out, n_groups],
+    zeros fp16 [d_out, n_groups], qpacked uint32 [d_out, d_in / 8])."""
+    W32 = np.asarray(W, dtype=F32)
+    d_out, d_in = W32.shape
+    g = d_in if group_size == -1 else group_size
+    n_groups = d_in // g
+    codes = np.zeros((d_out, d_in), dtype=np.int64)
+    scales = np.zeros((d_out, n_groups), dtype=np.float16)
+    zeros = np.zeros((d_out, n_groups), dtype=np.float16)
+    for gi in range(n_groups):
+        blk = W32[:, gi * g:(gi + 1) * g]
+        s, z = sym_params(blk, bits) if sym else affine_params(blk, bits)
+        scales[:, gi] = s
+        zeros[:, gi] = z
+        codes[:, gi * g:(gi + 1) * g] = quantize_codes(blk, s[:, None], z[:, None], sym, bits)
+    return dict(codes=codes, scales=scales, zeros=zeros,
+                qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None)
+
+
+# --------------------------------------------------------------------------
+# GPTQ
+# --------------------------------------------------------------------------
+
+@dataclass
+class GptqResult:
+    codes: np.ndarray      # [d_out, d_in] int, original column order
+    scales: np.ndarray     # [d_out, n_groups] fp16, group order of the (permuted) columns
+    zeros: np.ndarray      # [d_out, n_groups] fp16
+    g_idx: np.ndarray      # [d_in] int32, group of each original column
+    qpacked: np.ndarray    # [d_out, d_in / 8] uint32 (None unless d_in % 8 == 0)
+    W_hat: np.ndarray      # [d_out, d_in] fp64 dequantised, original column order
+
+
+def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
+                  perm=None, dead=None) -> GptqResult:
+    """GPTQ on one layer given U (upper, H^-1 = U^T U, in the column order
+    the layer is processed in).
+
+    Follows "GPTQ: Post-Training INT4", "The GPTQ Algorithm": columns left
+    to right in blocks of ``block_size``; for each column the code from the
+    current weights, the scaled error delta = (w - q) / U_jj, the in-block
+    update w[j+1:end] -= delta * U[j, j+1:end]; after the block the lazy
+    trailing update W[:, end:] -= Err @ U[blk, end:].  Group parameters per
+    reading 6.  ``perm`` (act-order) gives the processing order of the
+    original columns; ``dead`` columns are zeroed first."""
+    W = np.array(W, dtype=np.float64, copy=True)
+    d_out, d_in = W.shape
+    if dead is not None:
+        W[:, np.asarray(dead, dtype=bool)] = 0.0
+    if perm is not None:
+        perm = np.asarray(perm, dtype=np.int64)
+        W = W[:, perm]
+    g = d_in if group_size == -1 else group_size
+    if group_size != -1:
+        assert d_in % g == 0 and block_size % g == 0
+    n_groups = d_in // g
+    lo = -(2 ** (bits - 1) - 1) if sym else 0
+    params = sym_params if sym else affine_params
+
+    codes = np.zeros((d_out, d_in), dtype=np.int64)
+    Q = np.zeros((d_out, d_in), dtype=np.float64)
+    scales = np.zeros((d_out, n_groups), dtype=np.float16)
+    zeros = np.zeros((d_out, n_groups), dtype=np.float16)
+    if group_size == -1:
+        s, z = params(W.astype(F32), bits)
+        scales[:, 0], zeros[:, 0] = s, z
+    for b0 in range(0, d_in, block_size):
+        b1 = min(b0 + block_size, d_in)
+        Wb = W[:, b0:b1].copy()
+        Err = np.zeros_like(Wb)
+        for j in range(b1 - b0):
+            col = b0 + j
+            if group_size != -1 and col % g == 0:
+                s, z = params(Wb[:, j:j + g].astype(F32), bits)
+                scales[:, col // g], zeros[:, col // g] = s, z
+            gi = 0 if group_size == -1 else col // g
+            s, z = scales[:, gi], zeros[:, gi]
+            w = Wb[:, j]
+            c = quantize_codes(w, s, z, sym, bits)
+            q = dequantize_codes(c, s, z)
+            codes[:, col] = c
+            Q[:, col] = q
+            delta = (w - q) / U[col, col]
+            Err[:, j] = delta
+            Wb[:, j + 1:] -= np.outer(delta, U[col, col + 1:b1])
+        W[:, b0:b1] = Wb
+        W[:, b1:] -= Err @ U[b0:b1, b1:]
+
+    g_perm = np.arange(d_in) // g
+    if perm is not None:
+        inv = np.empty_like(perm)
+        inv[perm] = np.arange(d_in)
+        codes = codes[:, inv]
+        Q = Q[:, inv]
+        g_idx = g_perm[inv]
+    else:
+        g_idx = g_perm
+    assert codes.min() >= lo
+    return GptqResult(codes=codes, scales=scales, zeros=zeros,
+                      g_idx=g_idx.astype(np.int32),
+                      qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None,
+                      W_hat=Q)
+
+
+def gptq_layer(W, X, bits=4, group_size=-1, block_size=128, sym=True,
+               damp_percent=0.01, act_order=False):
+    """The whole per-layer path: H = 2 X^T X, dead columns and damping,
+    optional act-order, U, then GPTQ.  Returns (GptqResult, H_undamped,
+    U, perm, dead)."""
+    H0 = hessian(X)
+    Hd, dead = damp_hessian(H0, damp_percent)
+    perm = act_order_perm(Hd) if act_order else None
+    Hp = Hd[np.ix_(perm, perm)] if perm is not None else Hd
+    U = upper_factor_of_inverse(Hp)
+    res = gptq_quantize(W, U, bits=bits, group_size=group_size,
+                        block_size=block_size, sym=sym, perm=perm, dead=dead)
+    return res, H0, U, perm, dead
+
+
+def dequantize_packed(qpacked, scales, zeros, d_in, group_size, sym,
+                      g_idx=None, bits=4):
+    """W^ from packed codes and the stored 16-bit scales / zeros."""
+    c = unpack_nibbles(qpacked, d_in, sym, bits)
+    if g_idx is None:
+        g = d_in if group_size == -1 else group_size
+        g_idx = np.arange(d_in) // g
+    g_idx = np.asarray(g_idx, dtype=np.int64)
+    s = np.asarray(scales)[:, g_idx]
+    z = np.asarray(zeros)[:, g_idx] if not sym else np.zeros_like(s)
+    return dequantize_codes(c, s, z)
+
+
+# --------------------------------------------------------------------------
+# Reconstruction error
+# --------------------------------------------------------------------------
+
+def recon_sse(W, W_hat, X) -> float:
+    """||W X^T - W^ X^T||_F^2 in fp64 -- the layer-wise objective of "GPTQ:
+    Post-Training INT4", "OBQ Foundation", with X tokens x d_in.  The MSE is
+    this divided by n_tok * d_out."""
+    dW = np.asarray(W, dtype=np.float64) - np.asarray(W_hat, dtype=np.float64)
+    Y = dW @ np.asarray(X, dtype=np.float64).T
+    return float(np.sum(Y * Y))
+
+
+def recon_sse_trace(W, W_hat, H_undamped) -> float:
+    """Second route to the same number: trace(dW H dW^T) / 2 with the
+    undamped H = 2 X^T X (pin only)."""
+    dW = np.asarray(W, dtype=np.float64) - np.asarray(W_hat, dtype=np.float64)
+    return float(np.sum((dW @ H_undamped) * dW) / 2.0)
+
+
+# --------------------------------------------------------------------------
+# References used by the pins
+# --------------------------------------------------------------------------
+
+def obs_quantize(w, H, quantize):
+    """Per-step OBS on one row with the Hessian re-inverted on the remaining
+    set F at every step ("GPTQ: Post-Training INT4", "Hessian-Based Weight
+    Update", read with H_F^-1 as in reading 5), columns taken left to right.
+    ``quantize(col, value) -> dequantised value``.  Returns the dequantised
+    row."""
+    w = np.array(w, dtype=np.float64, copy=True)
+    d = w.shape[0]
+    out = np.zeros(d)
+    for q in range(d):
+        F = np.arange(q, d)
+        HinvF = np.linalg.inv(H[np.ix_(F, F)])
+        qhat = quantize(q, w[q])
+        out[q] = qhat
+        err = w[q] - qhat
+        w[F] -= err * HinvF[:, 0] / HinvF[0, 0]
+    return out
+
+
+def bruteforce_row(w, H_undamped, levels_per_col):
+    """Exhaustive minimum of (w - q) H (w - q)^T / 2 over every code vector,
+    ``levels_per_col[k]`` listing the dequantised values allowed at column
+    k.  Returns (best q, best error)."""
+    w = np.asarray(w, dtype=np.float64)
+    best, best_q = np.inf, None
+    for q in itertools.product(*levels_per_col):
+        r = w - np.asarray(q)
+        e = float(r @ H_undamped @ r) / 2.0
+        if e < best:
+            best, best_q = e, np.asarray(q)
+    return best_q, best
+
+
+def round_to_grid(w, step):
+    """Round each weight alone to the nearest multiple of ``step`` ("GPTQ and
+    AWQ", "Part 1. Rounding each weight alone")."""
+    return [np.rint(v / step) * step for v in w]
+
+
+def round_error_carried_forward(w, step):
+    """Round left to right, removing the previous rounding error from the
+    next weight before rounding it ("GPTQ and AWQ", "Example 1.1")."""
+    out, carry = [], 0.0
+    for v in w:
+        t = v + carry
+        q = np.rint(t / step) * step
+        carry = t - q
+        out.append(q)
+    return out
+
+
+def gptq_fixed_grid(w_row, X, step, damp_percent=0.01, block_size=128):
+    """GPTQ on a single row with a fixed unbounded grid of spacing ``step``
+    (the lesson's setting), same loop as ``gptq_quantize``.  Returns the
+    dequantised row."""
+    w = np.array(w_row, dtype=np.float64, copy=True)[None, :]
+    H, _ = damp_hessian(hessian(X), damp_percent)
+    U = upper_factor_of_inverse(H)
+    d = w.shape[1]
+    Q = np.zeros_like(w)
+    for b0 in range(0, d, block_size):
+        b1 = min(b0 + block_size, d)
+        Wb = w[:, b0:b1].copy()
+        Err = np.zeros_like(Wb)
+        for j in range(b1 - b0):
+            col = b0 + j
+            q = np.rint(Wb[:, j] / step) * step
+            Q[:, col] = q
+            delta = (Wb[:, j] - q) / U[col, col]
+            Err[:, j] = delta
+            Wb[:, j + 1:] -= np.outer(delta, U[col, col + 1:b1])
+        w[:, b0:b1] = Wb
+        w[:, b1:] -= Err @ U[b0:b1, b1:]
+    return Q[0]

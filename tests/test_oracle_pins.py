@@ -1,0 +1,379 @@
+"""Pins of the CPU oracle to what the pages and the mathematics fix.
+
+Each test ties one oracle function to something other than itself: values
+printed on the pages (fixtures under tests/golden/), brute force on tiny
+inputs, closed forms, or an independent derivation (per-step OBS with a
+re-inverted Hessian, the reversed Cholesky route to U, the trace form of the
+reconstruction error).  Chosen so that a dropped term, a wrong sign or index,
+or a transposed operand in the oracle fails at least one of them.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+F32 = np.float32
+
+
+# -------------------------------------------------------------- the lesson
+
+def test_lesson_nearest_and_carried_forward(golden):
+    g = golden("lesson_example_1_1.txt")
+    w, x, step = g["weights"], g["inputs"], g["step"]
+    true = sum(a * b for a, b in zip(w, x))
+    near = O.round_to_grid(w, step)
+    comp = O.round_error_carried_forward(w, step)
+    assert [round(v, 1) for v in near] == g["nearest"]
+    assert [round(v, 1) for v in comp] == g["compensated"]
+    assert round(abs(sum(a * b for a, b in zip(near, x)) - true), 2) == g["nearest_abs_error"]
+    assert round(abs(sum(a * b for a, b in zip(comp, x)) - true), 2) == g["compensated_abs_error"]
+
+
+def test_lesson_gptq_reaches_bruteforce_optimum(golden):
+    """GPTQ on the lesson's row (one token, inputs 1.0, grid step 0.1) makes
+    the output error 0.04, the same as the best of all code vectors and far
+    below round-to-nearest's 0.14."""
+    g = golden("lesson_example_1_1.txt")
+    w = np.array(g["weights"])
+    X = np.array(g["inputs"])[None, :]
+    q = O.gptq_fixed_grid(w, X, g["step"], damp_percent=0.01)
+    err_gptq = abs(float((q - w) @ X[0]))
+    cands = [[np.floor(v / 0.1) * 0.1, np.ceil(v / 0.1) * 0.1] for v in w]
+    best = min(abs(float((np.array(c) - w) @ X[0])) for c in itertools.product(*cands))
+    assert round(err_gptq, 2) == g["compensated_abs_error"]
+    assert round(best, 2) == g["compensated_abs_error"]
+    assert err_gptq < g["nearest_abs_error"]
+
+
+def test_pair_case(golden):
+    g = golden("pair_case.txt")
+    w, x = np.array(g["weights"]), np.array(g["inputs"])
+    outs = {c: float(np.array(c) @ x) for c in itertools.product(g["grid"], repeat=2)}
+    best = min(outs.items(), key=lambda kv: abs(kv[1] - w @ x))
+    assert round(best[1], 2) == g["best_output"]
+    assert round(abs(best[1] - w @ x), 2) == g["best_abs_error"]
+    near = O.round_to_grid(w, 0.1)
+    assert round(float(np.dot(near, x)), 2) == g["nearest_output"]
+    assert round(abs(float(np.dot(near, x)) - w @ x), 2) == g["nearest_abs_error"]
+    assert round(abs(0.4 - w @ x), 2) == g["both_down_abs_error"]
+    # GPTQ with two equal unit inputs reduces to carrying the error forward
+    q = O.gptq_fixed_grid(w, x[None, :], 0.1, damp_percent=0.01)
+    assert [round(v, 1) for v in q] == g["carried_forward"]
+    assert [round(v, 1) for v in O.round_error_carried_forward(w, 0.1)] == g["carried_forward"]
+
+
+# -------------------------------------------------------------- Hessian
+
+def test_hessian_bruteforce_definition():
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((7, 5))
+    H = O.hessian(X)
+    for i in range(5):
+        for j in range(5):
+            ref = 0.0
+            for t in range(7):
+                ref += 2.0 * X[t, i] * X[t, j]
+            assert abs(H[i, j] - ref) < 1e-12
+    sub = O.hessian_entries(X, [1, 3], [0, 4])
+    assert np.allclose(sub, H[np.ix_([1, 3], [0, 4])], rtol=0, atol=1e-13)
+
+
+def test_damp_and_dead_columns_closed_form():
+    H = np.diag([4.0, 0.0, 2.0])
+    H[0, 2] = H[2, 0] = 1.0
+    Hd, dead = O.damp_hessian(H, 0.01)
+    assert dead.tolist() == [False, True, False]
+    lam = 0.01 * (4.0 + 1.0 + 2.0) / 3.0
+    assert np.allclose(np.diag(Hd), [4.0 + lam, 1.0 + lam, 2.0 + lam], rtol=0, atol=1e-15)
+    assert Hd[0, 2] == 1.0 and Hd[2, 0] == 1.0
+
+
+def test_act_order_perm_stable_descending():
+    H = np.diag([1.0, 5.0, 3.0, 5.0, 0.5])
+    assert O.act_order_perm(H).tolist() == [1, 3, 2, 0, 4]
+
+
+def test_upper_factor_against_reversed_cholesky():
+    """U from the pages' route (Cholesky, inverse, Cholesky of the inverse)
+    equals the independent reversal identity U = J chol(J H J)^-1 J, and
+    U^T U H = I."""
+    rng = np.random.default_rng(2)
+    for d in (1, 3, 8, 33):
+        A = rng.standard_normal((2 * d + 3, d))
+        H, _ = O.damp_hessian(O.hessian(A), 0.01)
+        U = O.upper_factor_of_inverse(H)
+        J = np.eye(d)[::-1]
+        Lr = np.linalg.cholesky(J @ H @ J)
+        U2 = J @ np.linalg.inv(Lr) @ J
+        assert np.allclose(U, np.triu(U), atol=0)
+        assert np.max(np.abs(U - U2)) <= 1e-10 * np.max(np.abs(U))
+        assert np.max(np.abs(U.T @ U @ H - np.eye(d))) < 1e-9
+        assert np.all(np.diag(U) > 0)
+
+
+def test_not_positive_definite_raises():
+    with pytest.raises(np.linalg.LinAlgError):
+        O.upper_factor_of_inverse(-np.eye(3))
+
+
+# -------------------------------------------------------------- grid
+
+def test_sym_grid_has_15_levels(golden):
+    g = golden("sym_grid.txt")
+    rng = np.random.default_rng(3)
+    v = np.concatenate([np.linspace(-1.0, 1.0, 97), rng.uniform(-0.9, 0.9, 4000)])
+    v = v[None, :].astype(F32)
+    s, z = O.sym_params(v, int(g["bits"]))
+    c = O.quantize_codes(v, s[:, None], z[:, None], True, int(g["bits"]))
+    assert len(np.unique(c)) == int(g["levels"])
+    assert c.min() == -7 and c.max() == 7
+    amax_i = np.argmax(np.abs(v[0]))
+    assert abs(c[0, amax_i]) == 7
+    # negation symmetry of the grid
+    c_neg = O.quantize_codes(-v, s[:, None], z[:, None], True)
+    assert np.array_equal(c_neg, -c)
+    # points on the grid map to themselves
+    grid = (np.arange(-7, 8) * s.astype(np.float64)[0])[None, :]
+    cg = O.quantize_codes(grid, s[:, None], z[:, None], True)
+    assert np.array_equal(cg[0], np.arange(-7, 8))
+    assert np.array_equal(O.dequantize_codes(cg, s[:, None], z[:, None]), grid)
+
+
+def test_affine_grid_formula():
+    """W_q = round(W/S) + Z in 0..15, W_deq = S (W_q - Z): zero is exact, the
+    range ends map to the end codes, the rounding error is at most half a
+    step (plus the fp16 rounding of S at the far end)."""
+    rng = np.random.default_rng(4)
+    for shift in (0.0, 0.05, -0.05, 0.5):
+        v = (rng.standard_normal((16, 128)) * 0.02 + shift).astype(F32)
+        s, z = O.affine_params(v)
+        c = O.quantize_codes(v, s[:, None], z[:, None], False)
+        assert c.min() >= 0 and c.max() <= 15
+        deq = O.dequantize_codes(c, s[:, None], z[:, None])
+        zero_c = O.quantize_codes(np.zeros((16, 1), F32), s[:, None], z[:, None], False)
+        assert np.all(O.dequantize_codes(zero_c, s[:, None], z[:, None]) == 0.0)
+        step = s.astype(np.float64)[:, None]
+        assert np.all(np.abs(deq - v) <= 0.5 * step * 1.02 + 1e-12)
+        mn = np.minimum(v.min(1), 0)
+        mx = np.maximum(v.max(1), 0)
+        c_mn = O.quantize_codes(mn[:, None], s[:, None], z[:, None], False)[:, 0]
+        c_mx = O.quantize_codes(mx[:, None], s[:, None], z[:, None], False)[:, 0]
+        assert np.all(c_mn <= 1) and np.all(c_mx >= 14)
+
+
+def test_degenerate_group():
+    v = np.zeros((2, 8), F32)
+    for sym in (True, False):
+        s, z = O.sym_params(v) if sym else O.affine_params(v)
+        assert np.all(s == np.float16(1.0)) and np.all(z == 0)
+        c = O.quantize_codes(v, s[:, None], z[:, None], sym)
+        assert np.all(c == 0)
+
+
+def test_pack_layout_and_roundtrip():
+    codes = np.arange(16, dtype=np.int64)[None, :]
+    words = O.pack_nibbles(codes, sym=False)
+    assert words.tolist() == [[0x76543210, 0xFEDCBA98]]
+    sym_codes = np.arange(-7, 9, dtype=np.int64)[None, :].clip(-7, 7)
+    assert np.array_equal(O.unpack_nibbles(O.pack_nibbles(sym_codes, True), 16, True), sym_codes)
+    rng = np.random.default_rng(5)
+    c = rng.integers(0, 16, size=(5, 64))
+    assert np.array_equal(O.unpack_nibbles(O.pack_nibbles(c, False), 64, False), c)
+
+
+def test_storage_bits_per_weight(golden):
+    g = golden("storage_bits.txt")
+    gs = int(g["group_size"])
+    assert O.bits_per_weight(8, 1024, gs, sym=True) == g["bits_symmetric"]
+    assert O.bits_per_weight(8, 1024, gs, sym=False) == g["bits_affine"]
+    W = np.random.default_rng(6).standard_normal((8, 1024)).astype(F32) * 0.02
+    for sym, key in ((True, "bits_symmetric"), (False, "bits_affine")):
+        r = O.rtn_quantize(W, gs, sym)
+        nbytes = r["qpacked"].nbytes + r["scales"].nbytes + (0 if sym else r["zeros"].nbytes)
+        assert nbytes * 8 / W.size == g[key]
+    assert O.bits_per_weight(8, 768, -1, True) == 4 + 16 / 768
+
+
+# -------------------------------------------------------------- GPTQ
+
+def _row_quantizer(w_row, sym):
+    s, z = O.sym_params(w_row[None].astype(F32)) if sym else O.affine_params(w_row[None].astype(F32))
+
+    def q(col, v):
+        c = O.quantize_codes(np.array([[v]]), s[:, None], z[:, None], sym)
+        return float(O.dequantize_codes(c, s[:, None], z[:, None])[0, 0])
+    return q
+
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_cholesky_form_equals_per_step_obs(sym):
+    """GPTQ's Cholesky form equals OBS with H_F re-inverted at every step,
+    for tiny d_in <= 8, with any lazy block size."""
+    rng = np.random.default_rng(7 if sym else 8)
+    for t in range(40):
+        d = int(rng.integers(2, 9))
+        n = int(rng.integers(1, 3 * d))
+        X = rng.standard_normal((n, d)) * rng.lognormal(0, 0.5, d)
+        W = rng.standard_normal((4, d)) * 0.1
+        H, _ = O.damp_hessian(O.hessian(X), 0.01)
+        U = O.upper_factor_of_inverse(H)
+        r = O.gptq_quantize(W, U, group_size=-1, block_size=128, sym=sym)
+        for bs in (1, 2, 3):
+            rb = O.gptq_quantize(W, U, group_size=-1, block_size=bs, sym=sym)
+            assert np.array_equal(rb.codes, r.codes)
+        for i in range(4):
+            ref = O.obs_quantize(W[i], H, _row_quantizer(W[i], sym))
+            assert np.array_equal(ref, r.W_hat[i]), (t, i)
+
+
+def _fixed_scale_levels(s, z, sym, d):
+    codes = range(-7, 8) if sym else range(0, 16)
+    lv = [float(s) * (c - float(z)) for c in codes]
+    return [lv] * d
+
+
+def test_bruteforce_bounds_gptq():
+    """On tiny layers with the scale GPTQ picked: the exhaustive optimum is
+    never worse than GPTQ; on correlated inputs (duplicated / near-collinear
+    columns) GPTQ beats round-to-nearest."""
+    rng = np.random.default_rng(9)
+    wins = 0
+    for t in range(12):
+        d = 4
+        base = rng.standard_normal((24, 2))
+        X = np.concatenate([base, base + 0.05 * rng.standard_normal((24, 2))], 1)
+        W = rng.standard_normal((1, d)) * 0.1
+        H0 = O.hessian(X)
+        Hd, _ = O.damp_hessian(H0, 0.01)
+        U = O.upper_factor_of_inverse(Hd)
+        r = O.gptq_quantize(W, U, group_size=-1, sym=True)
+        rtn = O.rtn_quantize(W.astype(F32), -1, True)
+        assert r.scales[0, 0] == rtn["scales"][0, 0]
+        w_rtn = O.dequantize_codes(rtn["codes"], rtn["scales"], rtn["zeros"])
+        e_gptq = O.recon_sse(W, r.W_hat, X)
+        e_rtn = O.recon_sse(W, w_rtn, X)
+        _, e_best = O.bruteforce_row(W[0], H0, _fixed_scale_levels(r.scales[0, 0], 0, True, d))
+        assert e_best <= e_gptq * (1 + 1e-12) + 1e-15
+        assert e_best <= e_rtn * (1 + 1e-12) + 1e-15
+        assert e_gptq <= e_rtn * (1 + 1e-12)
+        wins += e_gptq < e_rtn * (1 - 1e-9)
+    assert wins >= 3
+
+
+def test_diagonal_hessian_reduces_to_rtn():
+    """Orthogonal inputs give a diagonal H and a diagonal U, so GPTQ has
+    nothing to feed forward and equals RTN exactly (codes and scales)."""
+    rng = np.random.default_rng(10)
+    d = 256
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    X = np.diag(rng.lognormal(0, 0.5, d)) @ np.eye(d)
+    W = (rng.standard_normal((16, d)) * 0.02).astype(F32)
+    for gs in (-1, 128, 32):
+        for sym in (True, False):
+            res, H0, U, _, _ = O.gptq_layer(W, X, group_size=gs, sym=sym)
+            assert np.count_nonzero(np.triu(U, 1)) == 0
+            rtn = O.rtn_quantize(W, gs, sym)
+            assert np.array_equal(res.codes, rtn["codes"])
+            assert np.array_equal(res.scales, rtn["scales"])
+            assert np.array_equal(res.qpacked, rtn["qpacked"])
+    del Q
+
+
+def test_hessian_scale_invariance_and_identity_perm():
+    rng = np.random.default_rng(11)
+    d = 64
+    X = rng.standard_normal((200, d)) * rng.lognormal(0, 0.5, d)
+    W = rng.standard_normal((8, d)) * 0.02
+    Hd, _ = O.damp_hessian(O.hessian(X), 0.01)
+    for gs in (-1, 32):
+        a = O.gptq_quantize(W, O.upper_factor_of_inverse(Hd), group_size=gs, block_size=32)
+        b = O.gptq_quantize(W, O.upper_factor_of_inverse(7.3 * Hd), group_size=gs, block_size=32)
+        c = O.gptq_quantize(W, O.upper_factor_of_inverse(Hd), group_size=gs, block_size=32,
+                            perm=np.arange(d))
+        assert np.array_equal(a.codes, b.codes)
+        assert np.array_equal(a.codes, c.codes) and np.array_equal(a.scales, c.scales)
+
+
+def test_act_order_groups_and_g_idx():
+    rng = np.random.default_rng(12)
+    d = 64
+    X = rng.standard_normal((300, d)) * rng.lognormal(0, 0.7, d)
+    W = rng.standard_normal((8, d)) * 0.02
+    res, H0, U, perm, dead = O.gptq_layer(W, X, group_size=16, sym=False, act_order=True)
+    assert sorted(perm.tolist()) == list(range(d))
+    inv = np.empty(d, int)
+    inv[perm] = np.arange(d)
+    assert np.array_equal(res.g_idx, inv // 16)
+    # dequantising with g_idx reproduces the oracle's W_hat
+    Wh = O.dequantize_packed(res.qpacked, res.scales, res.zeros, d, 16, False, g_idx=res.g_idx)
+    assert np.array_equal(Wh, res.W_hat)
+    # the permuted problem is the plain problem on permuted columns
+    plain = O.gptq_quantize(W[:, perm], U, group_size=16, sym=False)
+    assert np.array_equal(plain.codes, res.codes[:, perm])
+
+
+def test_gptq_not_worse_than_rtn_on_correlated_layer():
+    rng = np.random.default_rng(13)
+    d, n = 128, 400
+    base = rng.standard_normal((n, 16))
+    X = base @ rng.standard_normal((16, d)) + 0.1 * rng.standard_normal((n, d))
+    W = rng.standard_normal((32, d)) * 0.02
+    for gs, sym in ((-1, True), (32, True), (32, False)):
+        res, *_ = O.gptq_layer(W, X, group_size=gs, sym=sym, block_size=64)
+        rtn = O.rtn_quantize(W.astype(F32), gs, sym)
+        w_rtn = O.dequantize_packed(rtn["qpacked"], rtn["scales"], rtn["zeros"], d, gs, sym)
+        assert O.recon_sse(W, res.W_hat, X) < 0.8 * O.recon_sse(W, w_rtn, X)
+
+
+def test_mse_two_routes():
+    rng = np.random.default_rng(14)
+    X = rng.standard_normal((90, 40))
+    W = rng.standard_normal((7, 40))
+    Wh = W + 0.01 * rng.standard_normal((7, 40))
+    a = O.recon_sse(W, Wh, X)
+    b = O.recon_sse_trace(W, Wh, O.hessian(X))
+    assert abs(a - b) <= 1e-12 * a
+    Y = (W - Wh) @ X.T
+    assert abs(a - sum(float(v) ** 2 for v in Y.ravel())) <= 1e-12 * a
+
+
+def test_dead_columns_zeroed():
+    rng = np.random.default_rng(15)
+    X = rng.standard_normal((50, 16))
+    X[:, 3] = 0.0
+    W = rng.standard_normal((4, 16)) * 0.02
+    res, H0, U, perm, dead = O.gptq_layer(W, X, group_size=-1)
+    assert dead.tolist() == [j == 3 for j in range(16)]
+    assert np.all(res.W_hat[:, 3] == 0.0)
+
+
+# -------------------------------------------------------------- planted mistakes
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Plant plausible mistakes in a copy of the GPTQ loop and check that the
+    OBS-equivalence pin rejects each one."""
+    rng = np.random.default_rng(16)
+    d, rows = 6, 64
+    X = rng.standard_normal((10, d)) * rng.lognormal(0, 0.5, d)
+    W = rng.standard_normal((rows, d)) * 0.1
+    H, _ = O.damp_hessian(O.hessian(X), 0.01)
+    U = O.upper_factor_of_inverse(H)
+    Hinv = np.linalg.inv(H)
+    refs = [O.obs_quantize(W[i], H, _row_quantizer(W[i], True)) for i in range(rows)]
+
+    def matches(Uuse, bs=128):
+        r = O.gptq_quantize(W, Uuse, group_size=-1, block_size=bs)
+        return all(np.array_equal(refs[i], r.W_hat[i]) for i in range(rows))
+
+    assert matches(U) and matches(U, 2)
+    # full inverse instead of its Cholesky factor (the listing read literally)
+    assert not matches(np.triu(Hinv))
+    # transposed factor (lower instead of upper)
+    assert not matches(np.ascontiguousarray(U.T))
+    # a wrong sign of the update
+    assert not matches(np.diag(np.diag(U)) - np.triu(U, 1))
+    # the lazy trailing update dropped (only the 2-column in-block updates kept)
+    blockdiag = np.kron(np.eye(d // 2), np.ones((2, 2))) * U
+    assert not matches(blockdiag, 2)
