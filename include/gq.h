@@ -1,0 +1,228 @@
+/*
+ * gq.h -- C ABI of libgq.so: layer-wise 4-bit post-training weight
+ * quantization (GPTQ and round-to-nearest) on NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title -- section):
+ *   "GPTQ: Post-Training INT4" -- "OBQ Foundation", "Hessian-Based Weight
+ *       Update", "The GPTQ Algorithm", "Group Quantization", "Running GPTQ
+ *       with AutoGPTQ".
+ *   "Model Quantization Mechanics: Precision Reduction and Weight
+ *       Formatting" -- section 1 (affine and group-wise quantization),
+ *       section 2.1 (GPTQ objective; Cholesky factor of the inverse Hessian).
+ *   "GPT-2 Quantization Reconstruction Error" -- "What this project does"
+ *       (4-bit symmetric per-channel RTN with 15 levels; per-layer MSE).
+ *
+ * Conventions shared by every entry point:
+ *   - Every array pointer is a DEVICE pointer owned by the caller, except
+ *     the ones whose name ends in _host.  Arrays are dense and row-major.
+ *   - The library allocates no device memory.  Entry points that need
+ *     scratch take a caller-owned workspace (ws, ws_bytes) whose minimum
+ *     size the matching gq_*_workspace_size() returns; ws must be 256-byte
+ *     aligned.  Workspace contents need not be initialised.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  An entry point returns before the GPU
+ *     work finishes unless it documents a synchronisation.
+ *   - Argument errors are detected on the host and returned before any
+ *     launch; nothing is written then.  GQ_ERR_CUDA reports a launch or
+ *     runtime error (gq_last_error() gives the text).
+ *   - Shapes: W is d_out x d_in; X (calibration activations) is
+ *     n_tok x d_in in bf16.  d_in must be a positive multiple of 8;
+ *     d_out, n_tok >= 1.  Only bits == 4 is implemented.
+ *   - Packed codes: uint32 words of 8 nibbles along d_in, qpacked is
+ *     [d_out][d_in/8]; nibble k (bits 4k..4k+3) of word j is column 8j+k.
+ *     Symmetric codes c in -7..7 are stored as c+8; affine codes 0..15 as is.
+ *   - Scales and zeros are IEEE fp16 bit patterns (uint16), [d_out][n_groups]
+ *     with n_groups = d_in / group_size, or 1 for group_size == -1.  Zeros
+ *     hold the integer zero-point 0..15 (0 for symmetric).
+ *   - group_size is -1 (one group per output row) or a multiple of 8 that
+ *     divides d_in; for GPTQ it must also divide block_size.
+ *   - Inputs must be finite; non-finite values give unspecified codes.
+ */
+#ifndef GQ_H
+#define GQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t gq_status;
+enum {
+  GQ_OK = 0,
+  GQ_ERR_ARG = 1,         /* null pointer, bad flag or unsupported option   */
+  GQ_ERR_SHAPE = 2,       /* sizes violate the rules above                  */
+  GQ_ERR_DTYPE = 3,       /* unknown gq_dtype                               */
+  GQ_ERR_WORKSPACE = 4,   /* ws too small or misaligned                     */
+  GQ_ERR_NOT_PD = 5,      /* damped Hessian not positive definite           */
+  GQ_ERR_NONFINITE = 6,   /* a non-finite value where one is not allowed    */
+  GQ_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up             */
+  GQ_ERR_CUDA = 8         /* CUDA runtime / launch error                    */
+};
+
+typedef int32_t gq_dtype;
+enum { GQ_F32 = 0, GQ_F16 = 1, GQ_BF16 = 2 };
+
+/* Human-readable name of a status code (static string). */
+const char *gq_status_string(gq_status s);
+
+/* Detail of the last error returned on the calling host thread (static,
+ * thread-local; empty string if none). */
+const char *gq_last_error(void);
+
+/* Number of kernels this library has launched in the process so far. */
+uint64_t gq_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * Hessian accumulation.
+ * "GPTQ: Post-Training INT4", "Hessian-Based Weight Update": the Hessian
+ * of the layer-wise objective is H = 2 X X^T, the same for every output
+ * row; with X stored tokens x d_in (the orientation of the listing in "The
+ * GPTQ Algorithm") this is H = 2 X^T X.  The call is additive, so a
+ * calibration set larger than memory is fed in several calls.
+ *
+ *   X   [n_tok][d_in] bf16 (device, read only, 16-byte aligned)
+ *   H   [d_in][d_in] fp32 (device, in/out): on return
+ *       H := sym(H) + 2 X^T X, where sym(H) takes the upper triangle
+ *       (i <= j) of the incoming H and mirrors it; the result is exactly
+ *       symmetric.
+ *   ws  >= gq_hessian_workspace_size(n_tok, d_in) bytes.
+ * Accumulates in fp32 on the tensor cores (bf16 x bf16 products are exact
+ * in fp32), in fixed token chunks whose partial sums are added in a fixed
+ * order: results are deterministic run to run.
+ * ---------------------------------------------------------------------- */
+size_t gq_hessian_workspace_size(int64_t n_tok, int64_t d_in);
+gq_status gq_hessian_accumulate(const void *X_bf16, int64_t n_tok, int64_t d_in,
+                                float *H, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Damping, act-order and the upper Cholesky factor of the inverse Hessian.
+ * "GPTQ: Post-Training INT4", "Running GPTQ with AutoGPTQ" (damp_percent,
+ * desc_act) and "The GPTQ Algorithm" (Cholesky of H, then its inverse);
+ * "Model Quantization Mechanics", section 2.1 (GPTQ uses a Cholesky
+ * decomposition of the inverse Hessian).
+ *
+ * Steps, in order:
+ *   1. dead columns: where H_jj == 0, set H_jj := 1 and mark the column
+ *      (dead_out[j] = 1, else 0); GPTQ zeroes those weight columns;
+ *   2. H_jj += damp_percent * mean_j(H_jj);
+ *   3. act_order != 0: perm = the columns by descending H_jj, ties by lower
+ *      index first (written to perm_out), and H := H[perm][:, perm];
+ *   4. U := the upper-triangular matrix with positive diagonal such that
+ *      H^-1 = U^T U (written to U; the strictly lower part is zero).
+ *
+ *   H          [d_in][d_in] fp32, exactly symmetric (device, in; used as
+ *              scratch: contents unspecified on return)
+ *   perm_out   [d_in] int32 (device, out) -- required iff act_order != 0
+ *   dead_out   [d_in] uint8 (device, out) or NULL
+ *   U          [d_in][d_in] fp32 (device, out)
+ *   info_dev   int32 (device, out) or NULL: -1 on success, else the index
+ *              (in processing order) of the first non-positive or
+ *              non-finite pivot.
+ *   info_host  int32 (host, out) or NULL.  If non-NULL the call
+ *              synchronises the stream once at its end, stores the info
+ *              value there and returns GQ_ERR_NOT_PD on failure.
+ *   ws         >= gq_damp_cholesky_workspace_size(d_in) bytes.
+ * Computed in fp32: a blocked Cholesky of the index-reversed matrix, whose
+ * reversed inverse is U (no separate inverse of H is formed).
+ * ---------------------------------------------------------------------- */
+size_t gq_damp_cholesky_workspace_size(int64_t d_in);
+gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent,
+                                   int act_order, int32_t *perm_out, uint8_t *dead_out,
+                                   float *U, int32_t *info_dev, int32_t *info_host,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * GPTQ on one layer.
+ * "GPTQ: Post-Training INT4", "The GPTQ Algorithm": columns in a fixed
+ * left-to-right order (the act-order permutation if given) in blocks of
+ * block_size columns; for column j of a block the code q of the current
+ * weight w, the scaled error delta = (w - q) / U_jj, the in-block update
+ * w[j+1:end] -= delta * U[j, j+1:end]; after the block the lazy trailing
+ * update W[:, end:] -= Err * U[blk, end:].  A group's scale (and zero) is
+ * taken from that group's current (already updated) weights when its first
+ * column is reached ("Group Quantization"); per-channel (group_size == -1)
+ * scales come from the initial row.  Symmetric grid: s = absmax / 7, codes
+ * -7..7; affine ("Model Quantization Mechanics", section 1): s = (max' -
+ * min') / 15 with the range widened to contain 0, z = rint(-min'/s),
+ * codes 0..15.  The fp16-rounded scale is the one used; a scale that is 0
+ * in fp16 becomes 1 (and z = 0); codes are rint(w / s) + z clamped, with
+ * IEEE division and round-half-to-even, in fp32.
+ *
+ *   W          [d_out][d_in] in w_dtype (device, read only; not modified)
+ *   U          [d_in][d_in] fp32 upper factor from gq_damp_cholesky_inverse
+ *              (in processing order)
+ *   bits       4
+ *   group_size -1 or a multiple of 8 dividing d_in and block_size
+ *   block_size a multiple of 32 (the pages' value is 128)
+ *   sym        1 symmetric, 0 affine
+ *   perm       [d_in] int32 processing order (act-order) or NULL
+ *   dead       [d_in] uint8 dead-column mask or NULL
+ *   qpacked    [d_out][d_in/8] uint32 (out), original column order
+ *   scales     [d_out][n_groups] fp16 bits (out); with perm, group k holds
+ *              processing positions k*g .. k*g+g-1
+ *   zeros      [d_out][n_groups] fp16 bits (out) or NULL (sym)
+ *   g_idx      [d_in] int32 (out) or NULL: the group of each original
+ *              column (position in perm / group_size)
+ *   ws         >= gq_gptq_workspace_size(d_out, d_in, block_size) bytes;
+ *              holds the fp32 working copy of W.
+ * ---------------------------------------------------------------------- */
+size_t gq_gptq_workspace_size(int64_t d_out, int64_t d_in, int block_size);
+gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
+                                 const float *U, int bits, int group_size, int block_size,
+                                 int sym, const int32_t *perm, const uint8_t *dead,
+                                 uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
+                                 int32_t *g_idx, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Round-to-nearest baseline with int4 packing.
+ * "GPT-2 Quantization Reconstruction Error", "What this project does"
+ * (per output row scale, 15 levels), "Model Quantization Mechanics",
+ * section 1 (affine; groups of g consecutive weights), "GPTQ: Post-Training
+ * INT4", "Group Quantization" (4 + 16/g (+16/g) bits per weight).  Same
+ * grid, rounding and storage as gq_gptq_quantize_layer, on the raw weights
+ * with no feedback.  Bit-exact and deterministic.
+ *
+ *   W        [d_out][d_in] in w_dtype (device, read only, 16-byte aligned)
+ *   qpacked  [d_out][d_in/8] uint32 (out)
+ *   scales   [d_out][n_groups] fp16 bits (out)
+ *   zeros    [d_out][n_groups] fp16 bits (out) or NULL (written with 0
+ *            when sym and non-NULL)
+ * ---------------------------------------------------------------------- */
+gq_status gq_rtn_quantize_pack(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
+                               int bits, int group_size, int sym, uint32_t *qpacked,
+                               uint16_t *scales, uint16_t *zeros, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Layer reconstruction error.
+ * "Model Quantization Mechanics", section 2.1 and "GPTQ: Post-Training
+ * INT4", "OBQ Foundation": the objective ||W X - W^ X||^2 (here with X
+ * tokens x d_in: ||(W - W^) X^T||_F^2); "GPT-2 Quantization Reconstruction
+ * Error" reports it per layer as an MSE over the layer's outputs.
+ *
+ *   W, w_dtype         original weights [d_out][d_in] (device)
+ *   qpacked, scales,   the quantised layer (device), as produced above;
+ *   zeros, g_idx       zeros NULL when sym; g_idx NULL unless act-order
+ *   X                  [n_tok][d_in] bf16 (device, 16-byte aligned)
+ *   sse_dev            double (device, out): SSE = ||(W - W^) X^T||_F^2
+ *   sse_host, mse_host double (host, out) or NULL; if either is non-NULL
+ *                      the call synchronises the stream once at its end.
+ *                      MSE = SSE / (n_tok * d_out).
+ *   ws                 >= gq_recon_workspace_size(d_out, d_in, n_tok) bytes
+ * W - W^ is formed in fp32 and fed to the tensor cores as a bf16 hi + lo
+ * pair (X is exactly bf16); squares are summed in fp32 per tile and in
+ * fp64 across tiles in a fixed order (deterministic).
+ * ---------------------------------------------------------------------- */
+size_t gq_recon_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok);
+gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
+                         const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
+                         int64_t d_out, int64_t d_in, int group_size, int sym,
+                         const void *X_bf16, int64_t n_tok, double *sse_dev,
+                         double *sse_host, double *mse_host, void *ws, size_t ws_bytes,
+                         void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GQ_H */

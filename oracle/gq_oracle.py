@@ -165,7 +165,7 @@ def affine_params(vals, bits=4):
     s16, degenerate = _to_fp16_scale((mx - mn) / maxq)
     z = np.rint(-mn / s16.astype(F32)).astype(F32)
     z = np.clip(z, F32(0), maxq)
-    z = np.where(degenerate, F32(0), z)
+    z = np.where(degenerate, F32(0), z) + F32(0.0)      # -0 -> +0
     return s16, z.astype(np.float16)
 
 

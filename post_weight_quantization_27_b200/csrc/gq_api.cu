@@ -1,0 +1,275 @@
+// extern "C" entry points of libgq.so: argument validation, workspace
+// sizing, and dispatch to the kernels.  See include/gq.h for the contract.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "gq_device.cuh"
+#include "gq_internal.h"
+
+namespace gq {
+
+std::atomic<uint64_t> g_launches{0};
+static thread_local std::string t_last_error;
+
+gq_status fail(gq_status s, const std::string &msg) {
+  t_last_error = msg;
+  return s;
+}
+
+gq_status check_launch(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return GQ_OK;
+  return fail(GQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+gq_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt,
+                       size_t elem_bytes, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+                       uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(GQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_elems * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  return GQ_OK;
+}
+
+}  // namespace gq
+
+using namespace gq;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+gq_status check_dtype(gq_dtype dt) {
+  if (dt != GQ_F32 && dt != GQ_F16 && dt != GQ_BF16) return fail(GQ_ERR_DTYPE, "unknown w_dtype");
+  return GQ_OK;
+}
+
+gq_status check_layer(int64_t d_out, int64_t d_in) {
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0)
+    return fail(GQ_ERR_SHAPE, "need d_out >= 1 and d_in a positive multiple of 8");
+  if (d_in > (int64_t(1) << 30) || d_out > (int64_t(1) << 31))
+    return fail(GQ_ERR_SHAPE, "layer too large");
+  return GQ_OK;
+}
+
+gq_status check_group(int group_size, int64_t d_in) {
+  if (group_size == -1) return GQ_OK;
+  if (group_size < 8 || group_size % 8 != 0 || d_in % group_size != 0)
+    return fail(GQ_ERR_SHAPE, "group_size must be -1 or a multiple of 8 dividing d_in");
+  return GQ_OK;
+}
+
+gq_status check_ws(const void *ws, size_t have, size_t need) {
+  if (need == 0) return GQ_OK;
+  if (!ws || have < need)
+    return fail(GQ_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) +
+                                      " bytes, have " + std::to_string(have));
+  if (!aligned(ws, 256)) return fail(GQ_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  return GQ_OK;
+}
+
+#define GQ_TRY(x)                         \
+  do {                                    \
+    const gq_status _s = (x);             \
+    if (_s != GQ_OK) return _s;           \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *gq_status_string(gq_status s) {
+  switch (s) {
+    case GQ_OK: return "GQ_OK";
+    case GQ_ERR_ARG: return "GQ_ERR_ARG";
+    case GQ_ERR_SHAPE: return "GQ_ERR_SHAPE";
+    case GQ_ERR_DTYPE: return "GQ_ERR_DTYPE";
+    case GQ_ERR_WORKSPACE: return "GQ_ERR_WORKSPACE";
+    case GQ_ERR_NOT_PD: return "GQ_ERR_NOT_PD";
+    case GQ_ERR_NONFINITE: return "GQ_ERR_NONFINITE";
+    case GQ_ERR_TIMEOUT: return "GQ_ERR_TIMEOUT";
+    case GQ_ERR_CUDA: return "GQ_ERR_CUDA";
+  }
+  return "GQ_UNKNOWN_STATUS";
+}
+
+const char *gq_last_error(void) { return t_last_error.c_str(); }
+
+uint64_t gq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t gq_hessian_workspace_size(int64_t n_tok, int64_t d_in) {
+  if (n_tok < 0 || d_in < 8 || d_in % 8 != 0) return 0;
+  return hessian_plan(n_tok, d_in).ws_bytes;
+}
+
+gq_status gq_hessian_accumulate(const void *X_bf16, int64_t n_tok, int64_t d_in, float *H,
+                                void *ws, size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  if (!H || (n_tok > 0 && !X_bf16)) return fail(GQ_ERR_ARG, "null pointer");
+  if (n_tok < 0 || d_in < 8 || d_in % 8 != 0)
+    return fail(GQ_ERR_SHAPE, "need n_tok >= 0 and d_in a positive multiple of 8");
+  if (d_in > 65536 || n_tok > (int64_t(1) << 31) - 64)
+    return fail(GQ_ERR_SHAPE, "d_in or n_tok too large");
+  if (n_tok > 0 && !aligned(X_bf16, 16)) return fail(GQ_ERR_ARG, "X must be 16-byte aligned");
+  const HessPlan p = hessian_plan(n_tok, d_in);
+  GQ_TRY(check_ws(ws, ws_bytes, p.ws_bytes));
+  return launch_hessian(X_bf16, n_tok, d_in, H, ws, p, static_cast<cudaStream_t>(stream));
+}
+
+size_t gq_damp_cholesky_workspace_size(int64_t d_in) {
+  if (d_in < 8 || d_in % 8 != 0) return 0;
+  return chol_ws_bytes(d_in);
+}
+
+gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent, int act_order,
+                                   int32_t *perm_out, uint8_t *dead_out, float *U,
+                                   int32_t *info_dev, int32_t *info_host, void *ws,
+                                   size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  if (!H || !U) return fail(GQ_ERR_ARG, "null pointer");
+  if (act_order != 0 && !perm_out) return fail(GQ_ERR_ARG, "act_order needs perm_out");
+  if (!(damp_percent >= 0.0f) || !(damp_percent < 1e30f))
+    return fail(GQ_ERR_ARG, "damp_percent must be finite and >= 0");
+  if (d_in < 8 || d_in % 8 != 0 || d_in > 65536)
+    return fail(GQ_ERR_SHAPE, "d_in must be a multiple of 8 in [8, 65536]");
+  GQ_TRY(check_ws(ws, ws_bytes, chol_ws_bytes(d_in)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GQ_TRY(launch_damp_chol(H, d_in, damp_percent, act_order, perm_out, dead_out, U, info_dev, ws,
+                          st));
+  if (info_host) {
+    int32_t info = -1;
+    const int32_t *src = info_dev ? info_dev : reinterpret_cast<const int32_t *>(ws) + 1;
+    if (cudaMemcpyAsync(&info, src, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return check_launch("damp_cholesky sync");
+    *info_host = info;
+    if (info >= 0)
+      return fail(GQ_ERR_NOT_PD, "damped Hessian not positive definite at column " +
+                                     std::to_string(info));
+  }
+  return GQ_OK;
+}
+
+size_t gq_gptq_workspace_size(int64_t d_out, int64_t d_in, int block_size) {
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || block_size < 32 || block_size % 32 != 0) return 0;
+  return gptq_ws_bytes(d_out, d_in, block_size);
+}
+
+gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
+                                 const float *U, int bits, int group_size, int block_size,
+                                 int sym, const int32_t *perm, const uint8_t *dead,
+                                 uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
+                                 int32_t *g_idx, void *ws, size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  GQ_TRY(check_dtype(w_dtype));
+  if (!W || !U || !qpacked || !scales) return fail(GQ_ERR_ARG, "null pointer");
+  if (bits != 4) return fail(GQ_ERR_ARG, "only bits == 4 is implemented");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
+  GQ_TRY(check_layer(d_out, d_in));
+  GQ_TRY(check_group(group_size, d_in));
+  if (block_size < 32 || block_size % 32 != 0 || block_size > 256)
+    return fail(GQ_ERR_ARG, "block_size must be a multiple of 32 in [32, 256]");
+  if (group_size != -1 && block_size % group_size != 0)
+    return fail(GQ_ERR_ARG, "group_size must divide block_size");
+  if (!aligned(W, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
+  GQ_TRY(check_ws(ws, ws_bytes, gptq_ws_bytes(d_out, d_in, block_size)));
+  return launch_gptq(W, w_dtype, d_out, d_in, U, group_size, block_size, sym, perm, dead,
+                     qpacked, scales, zeros, g_idx, ws, static_cast<cudaStream_t>(stream));
+}
+
+gq_status gq_rtn_quantize_pack(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
+                               int bits, int group_size, int sym, uint32_t *qpacked,
+                               uint16_t *scales, uint16_t *zeros, void *stream) {
+  t_last_error.clear();
+  GQ_TRY(check_dtype(w_dtype));
+  if (!W || !qpacked || !scales) return fail(GQ_ERR_ARG, "null pointer");
+  if (bits != 4) return fail(GQ_ERR_ARG, "only bits == 4 is implemented");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
+  GQ_TRY(check_layer(d_out, d_in));
+  GQ_TRY(check_group(group_size, d_in));
+  if (!aligned(W, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
+  return launch_rtn(W, w_dtype, d_out, d_in, group_size, sym, qpacked, scales, zeros,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t gq_recon_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok) {
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || n_tok < 0) return 0;
+  return recon_ws_bytes(d_out, d_in, n_tok);
+}
+
+gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
+                         const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
+                         int64_t d_out, int64_t d_in, int group_size, int sym,
+                         const void *X_bf16, int64_t n_tok, double *sse_dev, double *sse_host,
+                         double *mse_host, void *ws, size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  GQ_TRY(check_dtype(w_dtype));
+  if (!W || !qpacked || !scales || !sse_dev || (n_tok > 0 && !X_bf16))
+    return fail(GQ_ERR_ARG, "null pointer");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
+  GQ_TRY(check_layer(d_out, d_in));
+  GQ_TRY(check_group(group_size, d_in));
+  if (n_tok < 0 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
+  if (!aligned(W, 16) || (n_tok > 0 && !aligned(X_bf16, 16)))
+    return fail(GQ_ERR_ARG, "W and X must be 16-byte aligned");
+  GQ_TRY(check_ws(ws, ws_bytes, recon_ws_bytes(d_out, d_in, n_tok)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GQ_TRY(launch_recon(W, w_dtype, qpacked, scales, zeros, g_idx, d_out, d_in, group_size, sym,
+                      X_bf16, n_tok, sse_dev, ws, st));
+  if (sse_host || mse_host) {
+    double sse = 0.0;
+    if (cudaMemcpyAsync(&sse, sse_dev, sizeof(double), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return check_launch("recon_error sync");
+    if (sse_host) *sse_host = sse;
+    if (mse_host) *mse_host = n_tok > 0 ? sse / (static_cast<double>(n_tok) * d_out) : 0.0;
+  }
+  return GQ_OK;
+}
+
+}  // extern "C"

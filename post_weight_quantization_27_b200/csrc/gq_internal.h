@@ -1,0 +1,65 @@
+// Host-side declarations shared by the libgq translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <string>
+
+#include "../../include/gq.h"
+
+namespace gq {
+
+extern std::atomic<uint64_t> g_launches;
+inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Sets the thread-local error text and returns `s`.
+gq_status fail(gq_status s, const std::string &msg);
+// GQ_ERR_CUDA with the text of the pending CUDA error, or GQ_OK.
+gq_status check_launch(const char *what);
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// 2-D bf16 / fp32 tensor map with 128-byte swizzle: inner extent `inner`
+// elements (contiguous), outer extent `outer` rows with a row pitch of
+// `pitch_elems` elements; box of box_inner x box_outer.
+gq_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt,
+                       size_t elem_bytes, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+                       uint32_t box_inner, uint32_t box_outer);
+
+int num_sms();
+
+// ---- kernels (each returns GQ_OK or GQ_ERR_CUDA after launching) ----
+gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, int group_size,
+                     int sym, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
+                     cudaStream_t st);
+
+struct HessPlan {
+  int n_bi, n_bj, n_tiles, n_split, nkb_total, kb_per_split;
+  size_t ws_bytes;
+};
+HessPlan hessian_plan(int64_t n_tok, int64_t d_in);
+gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, void *ws,
+                         const HessPlan &plan, cudaStream_t st);
+
+size_t chol_ws_bytes(int64_t d);
+gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32_t *perm_out,
+                           uint8_t *dead_out, float *U, int32_t *info_dev, void *ws,
+                           cudaStream_t st);
+
+size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size);
+gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,
+                      int group_size, int block_size, int sym, const int32_t *perm,
+                      const uint8_t *dead, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
+                      int32_t *g_idx, void *ws, cudaStream_t st);
+
+size_t recon_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok);
+gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
+                       const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
+                       int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
+                       int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st);
+
+}  // namespace gq

@@ -1,0 +1,309 @@
+// H += 2 X^T X on the 5th-generation tensor cores.
+//
+// "GPTQ: Post-Training INT4" -- "Hessian-Based Weight Update": the layer
+// Hessian is H = 2 X X^T (X as d_in x tokens), the same for every output
+// row; with X stored tokens x d_in it is 2 X^T X.
+//
+// Design (sm_100a, one CTA per SM, persistent):
+//   * H is symmetric, so only 128 x 256 output tiles that touch the upper
+//     triangle are computed (about half the dense work).
+//   * warp 0 issues TMA loads of X boxes (64 columns x 64 tokens, 128-byte
+//     swizzle, no multicast) into a 4-stage shared-memory ring; A = X^T and
+//     B = X^T are both "MN-major" operands of tcgen05.mma (columns of X
+//     are contiguous), so no transpose is ever materialised.
+//   * warp 1 (one elected thread) issues tcgen05.mma kind::f16 bf16 x bf16
+//     -> fp32 into one of two 256-column TMEM accumulators.  Every 1024
+//     tokens the accumulator is handed to the epilogue and the other one
+//     is used, so the tensor pipe never waits for the drain.
+//   * warps 2..9 add each 1024-token partial into fp32 registers (one TMEM
+//     lane = one tile row per thread).  Short accumulation chains inside
+//     the tensor core keep the fp32 error small at 262144 tokens.
+//   * tiles are split over token ranges when there are too few tiles for
+//     the SMs; each (split, tile) writes its raw partial tile to the
+//     workspace and a second kernel adds the splits in a fixed order,
+//     scales by 2, adds the incoming H and mirrors the upper triangle:
+//     the result is deterministic and exactly symmetric.
+#include "gq_device.cuh"
+#include "gq_internal.h"
+
+namespace gq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, CHUNK_KB = 16;
+constexpr int A_BYTES = BM * BK * 2;  // two 64x64 boxes
+constexpr int B_BYTES = BN * BK * 2;  // four 64x64 boxes
+constexpr int BOX_BYTES = 64 * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 320;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+struct HessArgs {
+  int n_bj, n_tiles, n_split, kb_per_split, nkb_total;
+  float *P;
+  int *status;
+};
+
+// Tiles of row-block b are the column blocks b/2 .. n_bj-1 (a 128-row block
+// starting at 128b meets the diagonal in column block floor(128b/256)).
+__host__ __device__ __forceinline__ int64_t tile_row_start(int64_t b, int64_t n_bj) {
+  const int64_t k = b >> 1;
+  return b * n_bj - (k * (k - 1) + (b & 1) * k);
+}
+__device__ __forceinline__ void tile_coords(int t, int n_bj, int &bi, int &bj) {
+  int lo = 0, hi = 2 * n_bj;  // row_start is increasing in b
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_row_start(mid, n_bj) <= t) lo = mid; else hi = mid;
+  }
+  bi = lo;
+  bj = (lo >> 1) + (t - static_cast<int>(tile_row_start(lo, n_bj)));
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    hessian_mma_kernel(const __grid_constant__ CUtensorMap tmX, HessArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + STAGES;
+  uint64_t *acc_full = bars + 2 * STAGES;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) tma_prefetch_desc(&tmX);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = a.n_tiles * a.n_split;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int split = item / a.n_tiles, t = item % a.n_tiles;
+        int bi, bj;
+        tile_coords(t, a.n_bj, bi, bj);
+        const int kb0 = split * a.kb_per_split;
+        const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          uint8_t *sa = smem + s * STAGE_BYTES;
+          uint8_t *sb = sa + A_BYTES;
+          const int tok = kb * BK;
+          tma_load_2d(sa, &tmX, &full[s], bi * BM, tok);
+          tma_load_2d(sa + BOX_BYTES, &tmX, &full[s], bi * BM + 64, tok);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tma_load_2d(sb + q * BOX_BYTES, &tmX, &full[s], bj * BN + 64 * q, tok);
+        }
+      }
+      // every load issued must have landed before the CTA may exit
+      const uint32_t n_wait = it < STAGES ? it : STAGES;
+      for (uint32_t k = 0; k < n_wait; ++k) {
+        const uint32_t j = it - 1 - k;
+        if (!mbar_wait(&full[j % STAGES], (j / STAGES) & 1)) ok = false;
+      }
+      if (!ok) set_status(a.status, kDevTimeout);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0, ch = 0;
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, true, true);
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int split = item / a.n_tiles;
+        const int kb0 = split * a.kb_per_split;
+        const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
+        for (int c0 = kb0; c0 < kb1 && ok; c0 += CHUNK_KB, ++ch) {
+          const int c1 = min(c0 + CHUNK_KB, kb1);
+          const uint32_t buf = ch & 1, use = ch >> 1;
+          if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + buf * BN;
+          for (int kb = c0; kb < c1; ++kb, ++it) {
+            const uint32_t s = it % STAGES, r = it / STAGES;
+            if (!mbar_wait(&full[s], r & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              // 16 tokens = two 8-row swizzle atoms of 1024 bytes
+              const uint64_t ad = smem_desc_sw128(sa + kk * 2048, BOX_BYTES, 1024);
+              const uint64_t bd = smem_desc_sw128(sb + kk * 2048, BOX_BYTES, 1024);
+              mma_bf16(d_tmem, ad, bd, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
+          }
+          if (!ok) break;
+          mma_commit(&acc_full[buf]);
+        }
+      }
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) ok = false;
+      if (!ok) set_status(a.status, kDevTimeout);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..9
+    const int quarter = warp & 3;        // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;    // which 128 of the 256 columns
+    const int row = quarter * 32 + lane;
+    uint32_t ch = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int split = item / a.n_tiles;
+      const int kb0 = split * a.kb_per_split;
+      const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
+      float m[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) m[i] = 0.0f;
+      for (int c0 = kb0; c0 < kb1; c0 += CHUNK_KB, ++ch) {
+        const uint32_t buf = ch & 1, use = ch >> 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN + half * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) m[c * 32 + i] += v[i];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
+      if (!ok) break;
+      float *dst = a.P + (static_cast<size_t>(item) * BM + row) * BN + half * 128;
+#pragma unroll
+      for (int c = 0; c < 128; c += 4)
+        *reinterpret_cast<float4 *>(dst + c) = make_float4(m[c], m[c + 1], m[c + 2], m[c + 3]);
+    }
+    if (!ok && lane == 0) set_status(a.status, kDevTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// H[i][j] (i <= j) := H[i][j] + 2 * sum_s P_s(i, j); H[j][i] := H[i][j].
+__global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__ H, int d,
+                                                             const float *__restrict__ P,
+                                                             int n_tiles, int n_bj, int n_split,
+                                                             const int *status) {
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  if (bi > bj) return;
+  __shared__ float tile[32][33];
+  const bool bad = status != nullptr && *status != 0;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = bi * 32 + r, j = bj * 32 + tx;
+    float val = 0.0f;
+    if (i < d && j < d && i <= j) {
+      const int tb = i / BM, tj = j / BN;
+      const int t = static_cast<int>(tile_row_start(tb, n_bj)) + (tj - (tb >> 1));
+      float sum = 0.0f;
+      for (int s = 0; s < n_split; ++s)
+        sum += P[(static_cast<size_t>(s * n_tiles + t) * BM + (i - tb * BM)) * BN + (j - tj * BN)];
+      val = H[static_cast<size_t>(i) * d + j] + 2.0f * sum;
+      if (bad) val = __int_as_float(0x7fc00000);
+      H[static_cast<size_t>(i) * d + j] = val;
+    }
+    tile[r][tx] = val;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int j = bj * 32 + r, i = bi * 32 + tx;
+    if (i < d && j < d && i < j) H[static_cast<size_t>(j) * d + i] = tile[tx][r];
+  }
+}
+
+}  // namespace
+
+HessPlan hessian_plan(int64_t n_tok, int64_t d_in) {
+  HessPlan p{};
+  p.n_bi = static_cast<int>((d_in + BM - 1) / BM);
+  p.n_bj = static_cast<int>((d_in + BN - 1) / BN);
+  p.n_tiles = static_cast<int>(tile_row_start(p.n_bi, p.n_bj));
+  p.nkb_total = static_cast<int>((n_tok + BK - 1) / BK);
+  int split = 1;
+  const int target = 2 * num_sms();
+  if (p.nkb_total > 0 && p.n_tiles < target) {
+    const int want = (target + p.n_tiles - 1) / p.n_tiles;
+    const int most = p.nkb_total / 4 > 1 ? p.nkb_total / 4 : 1;
+    split = want < most ? want : most;
+  }
+  if (p.nkb_total == 0) {
+    p.n_split = 0;
+    p.kb_per_split = 0;
+  } else {
+    p.kb_per_split = (p.nkb_total + split - 1) / split;
+    p.n_split = (p.nkb_total + p.kb_per_split - 1) / p.kb_per_split;
+  }
+  p.ws_bytes = kWsHeader + static_cast<size_t>(p.n_split) * p.n_tiles * BM * BN * sizeof(float);
+  return p;
+}
+
+gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, void *ws,
+                         const HessPlan &p, cudaStream_t st) {
+  int *status = static_cast<int *>(ws);
+  float *P = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kWsHeader);
+  if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
+  const int n_items = p.n_tiles * p.n_split;
+  if (n_items > 0) {
+    CUtensorMap tm;
+    gq_status s = make_tmap_2d(&tm, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d_in, n_tok, d_in,
+                               64, BK);
+    if (s != GQ_OK) return s;
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaFuncSetAttribute(hessian_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(SMEM_BYTES));
+      attr_set = true;
+    }
+    HessArgs a{p.n_bj, p.n_tiles, p.n_split, p.kb_per_split, p.nkb_total, P, status};
+    const int grid = n_items < num_sms() ? n_items : num_sms();
+    hessian_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, a);
+    count_launch();
+    s = check_launch("hessian_mma_kernel");
+    if (s != GQ_OK) return s;
+  }
+  const int nb = static_cast<int>((d_in + 31) / 32);
+  hessian_finish_kernel<<<dim3(nb, nb), 256, 0, st>>>(H, static_cast<int>(d_in), P, p.n_tiles,
+                                                      p.n_bj, p.n_split, status);
+  count_launch();
+  return check_launch("hessian_finish_kernel");
+}
+
+}  // namespace gq

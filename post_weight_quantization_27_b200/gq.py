@@ -1,0 +1,260 @@
+"""ctypes binding of libgq.so (declared in include/gq.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current CUDA stream.  Loading fails
+loudly if libgq.so has not been built; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgq.so")
+
+GQ_F32, GQ_F16, GQ_BF16 = 0, 1, 2
+_DTYPES = {torch.float32: GQ_F32, torch.float16: GQ_F16, torch.bfloat16: GQ_BF16}
+
+_c_i64, _c_int, _c_f32, _c_vp, _c_sz = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class GQError(RuntimeError):
+    def __init__(self, status: int, name: str, detail: str, where: str):
+        super().__init__(f"{where}: {name} ({detail})")
+        self.status = status
+        self.name = name
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgq.so (loaded once)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m post_weight_quantization_27_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.gq_status_string.restype = ctypes.c_char_p
+    L.gq_status_string.argtypes = [_c_int]
+    L.gq_last_error.restype = ctypes.c_char_p
+    L.gq_last_error.argtypes = []
+    L.gq_launch_count.restype = ctypes.c_uint64
+    L.gq_launch_count.argtypes = []
+    L.gq_hessian_workspace_size.restype = _c_sz
+    L.gq_hessian_workspace_size.argtypes = [_c_i64, _c_i64]
+    L.gq_hessian_accumulate.restype = _c_int
+    L.gq_hessian_accumulate.argtypes = [_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_damp_cholesky_workspace_size.restype = _c_sz
+    L.gq_damp_cholesky_workspace_size.argtypes = [_c_i64]
+    L.gq_damp_cholesky_inverse.restype = _c_int
+    L.gq_damp_cholesky_inverse.argtypes = [_c_vp, _c_i64, _c_f32, _c_int, _c_vp, _c_vp, _c_vp,
+                                           _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_gptq_workspace_size.restype = _c_sz
+    L.gq_gptq_workspace_size.argtypes = [_c_i64, _c_i64, _c_int]
+    L.gq_gptq_quantize_layer.restype = _c_int
+    L.gq_gptq_quantize_layer.argtypes = [_c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_int, _c_int,
+                                         _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
+                                         _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_rtn_quantize_pack.restype = _c_int
+    L.gq_rtn_quantize_pack.argtypes = [_c_vp, _c_int, _c_i64, _c_i64, _c_int, _c_int, _c_int,
+                                       _c_vp, _c_vp, _c_vp, _c_vp]
+    L.gq_recon_workspace_size.restype = _c_sz
+    L.gq_recon_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64]
+    L.gq_recon_error.restype = _c_int
+    L.gq_recon_error.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
+                                 _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp,
+                                 _c_sz, _c_vp]
+    _lib = L
+    return L
+
+
+EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_workspace_size",
+           "gq_hessian_accumulate", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
+           "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
+           "gq_recon_workspace_size", "gq_recon_error")
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        L = lib()
+        raise GQError(status, L.gq_status_string(status).decode(),
+                      L.gq_last_error().decode(), where)
+
+
+def _p(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A caller-owned workspace buffer (256-byte aligned by the allocator)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def launch_count() -> int:
+    return int(lib().gq_launch_count())
+
+
+# ------------------------------------------------------------------ Hessian
+
+def hessian_workspace_size(n_tok: int, d_in: int) -> int:
+    return int(lib().gq_hessian_workspace_size(n_tok, d_in))
+
+
+def hessian_accumulate(X: torch.Tensor, H: torch.Tensor, ws: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """H := sym(H) + 2 X^T X (in place); X [n_tok, d_in] bf16, H fp32."""
+    _dev(X, "X", torch.bfloat16)
+    n_tok, d_in = X.shape
+    _dev(H, "H", torch.float32, (d_in, d_in))
+    need = hessian_workspace_size(n_tok, d_in)
+    ws = workspace(need, X.device) if ws is None else ws
+    _check(lib().gq_hessian_accumulate(_p(X), n_tok, d_in, _p(H), _p(ws), ws.numel(),
+                                       _stream(stream)), "gq_hessian_accumulate")
+    return H
+
+
+def hessian(X: torch.Tensor, stream=None) -> torch.Tensor:
+    H = torch.zeros((X.shape[1], X.shape[1]), dtype=torch.float32, device=X.device)
+    return hessian_accumulate(X, H, stream=stream)
+
+
+# ------------------------------------------------------------------ damp + Cholesky
+
+def damp_cholesky_workspace_size(d_in: int) -> int:
+    return int(lib().gq_damp_cholesky_workspace_size(d_in))
+
+
+def damp_cholesky_inverse(H: torch.Tensor, damp_percent: float = 0.01, act_order: bool = False,
+                          U: torch.Tensor | None = None, check: bool = True,
+                          ws: torch.Tensor | None = None, stream=None):
+    """Dead columns, damping, optional act-order and U (H^-1 = U^T U).
+
+    H is used as scratch.  Returns (U, perm or None, dead uint8, info int32
+    device tensor).  With check=True the call synchronises and raises
+    GQError(GQ_ERR_NOT_PD) if the damped H is not positive definite."""
+    _dev(H, "H", torch.float32)
+    d = H.shape[0]
+    dev = H.device
+    U = torch.empty((d, d), dtype=torch.float32, device=dev) if U is None else _dev(U, "U", torch.float32, (d, d))
+    perm = torch.empty(d, dtype=torch.int32, device=dev) if act_order else None
+    dead = torch.empty(d, dtype=torch.uint8, device=dev)
+    info = torch.empty(1, dtype=torch.int32, device=dev)
+    info_host = ctypes.c_int32(-1)
+    ws = workspace(damp_cholesky_workspace_size(d), dev) if ws is None else ws
+    st = lib().gq_damp_cholesky_inverse(_p(H), d, float(damp_percent), int(bool(act_order)),
+                                        _p(perm), _p(dead), _p(U), _p(info),
+                                        ctypes.byref(info_host) if check else None,
+                                        _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_damp_cholesky_inverse")
+    return U, perm, dead, info
+
+
+# ------------------------------------------------------------------ GPTQ
+
+def gptq_workspace_size(d_out: int, d_in: int, block_size: int = 128) -> int:
+    return int(lib().gq_gptq_workspace_size(d_out, d_in, block_size))
+
+
+def _n_groups(d_in: int, group_size: int) -> int:
+    return 1 if group_size == -1 else d_in // group_size
+
+
+def _outputs(d_out, d_in, group_size, sym, dev, with_g_idx):
+    ng = _n_groups(d_in, group_size)
+    return dict(qpacked=torch.empty((d_out, d_in // 8), dtype=torch.int32, device=dev),
+                scales=torch.empty((d_out, ng), dtype=torch.float16, device=dev),
+                zeros=None if sym else torch.empty((d_out, ng), dtype=torch.float16, device=dev),
+                g_idx=torch.empty(d_in, dtype=torch.int32, device=dev) if with_g_idx else None)
+
+
+def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, bits: int = 4, group_size: int = -1,
+                        block_size: int = 128, sym: bool = True, perm: torch.Tensor | None = None,
+                        dead: torch.Tensor | None = None, out: dict | None = None,
+                        ws: torch.Tensor | None = None, stream=None) -> dict:
+    """GPTQ on one layer.  Returns dict(qpacked int32 [d_out, d_in/8] (uint32
+    bit patterns), scales fp16, zeros fp16 or None, g_idx int32 or None)."""
+    _dev(W, "W")
+    if W.dtype not in _DTYPES:
+        raise ValueError(f"unsupported W dtype {W.dtype}")
+    d_out, d_in = W.shape
+    _dev(U, "U", torch.float32, (d_in, d_in))
+    if perm is not None:
+        _dev(perm, "perm", torch.int32, (d_in,))
+    if dead is not None:
+        _dev(dead, "dead", torch.uint8, (d_in,))
+    o = _outputs(d_out, d_in, group_size, sym, W.device, perm is not None) if out is None else out
+    ws = workspace(gptq_workspace_size(d_out, d_in, block_size), W.device) if ws is None else ws
+    st = lib().gq_gptq_quantize_layer(_p(W), _DTYPES[W.dtype], d_out, d_in, _p(U), bits,
+                                      group_size, block_size, int(bool(sym)), _p(perm), _p(dead),
+                                      _p(o["qpacked"]), _p(o["scales"]), _p(o["zeros"]),
+                                      _p(o["g_idx"]), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_gptq_quantize_layer")
+    return o
+
+
+# ------------------------------------------------------------------ RTN
+
+def rtn_quantize_pack(W: torch.Tensor, bits: int = 4, group_size: int = -1, sym: bool = True,
+                      out: dict | None = None, stream=None) -> dict:
+    """Round-to-nearest with int4 packing.  Same output layout as GPTQ."""
+    _dev(W, "W")
+    if W.dtype not in _DTYPES:
+        raise ValueError(f"unsupported W dtype {W.dtype}")
+    d_out, d_in = W.shape
+    o = _outputs(d_out, d_in, group_size, sym, W.device, False) if out is None else out
+    st = lib().gq_rtn_quantize_pack(_p(W), _DTYPES[W.dtype], d_out, d_in, bits, group_size,
+                                    int(bool(sym)), _p(o["qpacked"]), _p(o["scales"]),
+                                    _p(o["zeros"]), _stream(stream))
+    _check(st, "gq_rtn_quantize_pack")
+    return o
+
+
+# ------------------------------------------------------------------ reconstruction error
+
+def recon_workspace_size(d_out: int, d_in: int, n_tok: int) -> int:
+    return int(lib().gq_recon_workspace_size(d_out, d_in, n_tok))
+
+
+def recon_error(W: torch.Tensor, q: dict, X: torch.Tensor, group_size: int = -1,
+                sym: bool = True, sync: bool = True, sse: torch.Tensor | None = None,
+                ws: torch.Tensor | None = None, stream=None):
+    """SSE = ||(W - W^) X^T||_F^2 of a quantised layer ``q`` (dict as
+    returned above).  With sync=True returns (sse, mse) as Python floats;
+    otherwise the device fp64 tensor holding the SSE."""
+    _dev(W, "W")
+    _dev(X, "X", torch.bfloat16)
+    d_out, d_in = W.shape
+    n_tok = X.shape[0]
+    sse = torch.empty(1, dtype=torch.float64, device=W.device) if sse is None else sse
+    ws = workspace(recon_workspace_size(d_out, d_in, n_tok), W.device) if ws is None else ws
+    sse_h, mse_h = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    st = lib().gq_recon_error(_p(W), _DTYPES[W.dtype], _p(q["qpacked"]), _p(q["scales"]),
+                              _p(q.get("zeros")), _p(q.get("g_idx")), d_out, d_in, group_size,
+                              int(bool(sym)), _p(X), n_tok, _p(sse),
+                              ctypes.byref(sse_h) if sync else None,
+                              ctypes.byref(mse_h) if sync else None,
+                              _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_recon_error")
+    return (sse_h.value, mse_h.value) if sync else sse

@@ -1,0 +1,89 @@
+"""The C-ABI library loads without a GPU, exports every symbol the header
+declares, sizes workspaces, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_27_b200 import gq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    txt = open(os.path.join(ROOT, "include", "gq.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(gq_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = gq.lib()
+    names = _header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(gq.EXPORTS) <= set(names)
+
+
+def test_status_strings_and_counter():
+    L = gq.lib()
+    assert L.gq_status_string(0) == b"GQ_OK"
+    assert L.gq_status_string(5) == b"GQ_ERR_NOT_PD"
+    assert gq.launch_count() >= 0
+
+
+def test_workspace_sizes():
+    assert gq.hessian_workspace_size(2048, 768) > 256
+    assert gq.hessian_workspace_size(0, 768) >= 256
+    assert gq.hessian_workspace_size(10, 7) == 0
+    assert gq.damp_cholesky_workspace_size(768) > 0
+    assert gq.gptq_workspace_size(768, 768, 128) > 0
+    assert gq.recon_workspace_size(768, 768, 2048) > 0
+
+
+FAKE = ctypes.c_void_p(4096)   # never dereferenced: every call below fails validation
+
+
+@pytest.mark.parametrize("args,code", [
+    # bad dtype
+    (dict(dt=7, d_out=8, d_in=8, bits=4, g=-1, sym=1), 3),
+    # d_in not a multiple of 8
+    (dict(dt=0, d_out=8, d_in=12, bits=4, g=-1, sym=1), 2),
+    # group does not divide d_in
+    (dict(dt=0, d_out=8, d_in=64, bits=4, g=48, sym=1), 2),
+    # bits != 4
+    (dict(dt=0, d_out=8, d_in=64, bits=3, g=-1, sym=1), 1),
+    # affine without zeros
+    (dict(dt=0, d_out=8, d_in=64, bits=4, g=-1, sym=0), 1),
+])
+def test_rtn_argument_errors(args, code):
+    L = gq.lib()
+    st = L.gq_rtn_quantize_pack(FAKE, args["dt"], args["d_out"], args["d_in"], args["bits"],
+                                args["g"], args["sym"], FAKE, FAKE, None, None)
+    assert st == code
+    assert L.gq_last_error() != b""
+
+
+def test_other_argument_errors():
+    L = gq.lib()
+    # null H
+    assert L.gq_hessian_accumulate(FAKE, 64, 64, None, FAKE, 1 << 20, None) == 1
+    # workspace too small
+    assert L.gq_hessian_accumulate(FAKE, 64, 64, FAKE, FAKE, 8, None) == 4
+    # act_order without perm_out
+    assert L.gq_damp_cholesky_inverse(FAKE, 64, 0.01, 1, None, None, FAKE, None, None,
+                                      FAKE, 1 << 30, None) == 1
+    # negative damping
+    assert L.gq_damp_cholesky_inverse(FAKE, 64, -1.0, 0, None, None, FAKE, None, None,
+                                      FAKE, 1 << 30, None) == 1
+    # group_size must divide block_size
+    assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 192, FAKE, 4, 96, 128, 1, None, None,
+                                    FAKE, FAKE, None, None, FAKE, 1 << 40, None) == 1
+    # misaligned workspace
+    assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 128, FAKE, 4, 128, 128, 1, None, None, FAKE,
+                                    FAKE, None, None, ctypes.c_void_p(4096 + 8), 1 << 40,
+                                    None) == 4
+    # recon: null sse_dev
+    assert L.gq_recon_error(FAKE, 0, FAKE, FAKE, None, None, 8, 64, -1, 1, FAKE, 16, None,
+                            None, None, FAKE, 1 << 30, None) == 1

@@ -1,0 +1,81 @@
+"""RTN quantize + pack on the GPU against the oracle: codes, scales, zeros
+and packed bytes bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from post_weight_quantization_27_b200 import gq, inputs as I
+from tests.gpu_util import f16, u32
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def _check(W: torch.Tensor, group_size: int, sym: bool, rows=None):
+    Wd = W.cuda()
+    out = gq.rtn_quantize_pack(Wd, 4, group_size, sym)
+    torch.cuda.synchronize()
+    Wn = W.float().numpy()
+    if rows is not None:
+        Wn = Wn[rows]
+    ref = O.rtn_quantize(Wn, group_size, sym)
+    q = u32(out["qpacked"])
+    s = f16(out["scales"])
+    if rows is not None:
+        q, s = q[rows], s[rows]
+    assert np.array_equal(q, ref["qpacked"])
+    assert np.array_equal(s.view(np.uint16), ref["scales"].view(np.uint16))
+    if not sym:
+        z = f16(out["zeros"])
+        if rows is not None:
+            z = z[rows]
+        assert np.array_equal(z.view(np.uint16), ref["zeros"].view(np.uint16))
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("group_size,sym", [(-1, True), (-1, False), (128, True), (128, False),
+                                            (32, True), (8, False), (64, True), (256, False)])
+@pytest.mark.parametrize("shape", [(7, 256), (33, 768), (130, 1024)])
+def test_rtn_bit_exact(dt, group_size, sym, shape):
+    d_out, d_in = shape
+    if group_size != -1 and d_in % group_size:
+        pytest.skip("group does not divide d_in")
+    g = torch.Generator().manual_seed(d_out * 1000 + d_in + (group_size % 97))
+    W = (torch.randn(shape, generator=g) * 0.02).to(DT[dt])
+    W[0, :8] = 0                                        # zero words
+    if d_out > 2:
+        W[2] = 0                                        # an all-zero row
+    _check(W, group_size, sym)
+
+
+@pytest.mark.parametrize("d_in", [8, 2048, 2056, 4096, 28672])
+def test_rtn_per_channel_long_rows(d_in):
+    g = torch.Generator().manual_seed(d_in)
+    W = (torch.randn((5, d_in), generator=g) * 0.01).to(torch.float16)
+    _check(W, -1, True)
+    _check(W, -1, False)
+
+
+def test_rtn_rounding_ties():
+    """Values exactly half-way between two levels round to even."""
+    s = 0.25
+    row = np.array([7 * s, -1.5 * s, 2.5 * s, 0.5 * s, -0.5 * s, 3.5 * s, -2.5 * s, 6.5 * s],
+                   dtype=np.float32)
+    W = torch.from_numpy(np.tile(row, (3, 2)))
+    _check(W, -1, True)
+    _check(W, 8, True)
+    _check(W, 16, False)
+
+
+@pytest.mark.parametrize("workload,idx", [(2, 48), (3, 3), (4, 6), (5, 1)])
+def test_rtn_full_size_layers(workload, idx):
+    """Full-size layers of the workloads; the oracle checks every row of the
+    GPT-2 lm_head and 96 sampled rows of the larger layers."""
+    spec = I.workload_layers(workload)[idx]
+    W = I.make_weights(spec)
+    rows = None
+    if spec.d_out * spec.d_in > 50_000_000:
+        rows = np.sort(np.random.default_rng(idx).choice(spec.d_out, 96, replace=False))
+    _check(W, spec.group_size, spec.sym, rows)
