@@ -27,7 +27,8 @@
  *     runtime error (gq_last_error() gives the text).
  *   - Shapes: W is d_out x d_in; X (calibration activations) is
  *     n_tok x d_in in bf16.  d_in must be a positive multiple of 8;
- *     d_out, n_tok >= 1.  Only bits == 4 is implemented.
+ *     d_out >= 1; n_tok >= 0 (an empty calibration batch adds nothing).
+ *     Only bits == 4 is implemented.
  *   - Packed codes: uint32 words of 8 nibbles along d_in, qpacked is
  *     [d_out][d_in/8]; nibble k (bits 4k..4k+3) of word j is column 8j+k.
  *     Symmetric codes c in -7..7 are stored as c+8; affine codes 0..15 as is.
@@ -35,7 +36,7 @@
  *     with n_groups = d_in / group_size, or 1 for group_size == -1.  Zeros
  *     hold the integer zero-point 0..15 (0 for symmetric).
  *   - group_size is -1 (one group per output row) or a multiple of 8 that
- *     divides d_in; for GPTQ it must also divide block_size.
+ *     divides d_in; for GPTQ it is -1, 32, 64 or 128 and divides block_size.
  *   - Inputs must be finite; non-finite values give unspecified codes.
  */
 #ifndef GQ_H
@@ -117,9 +118,9 @@ gq_status gq_hessian_accumulate(const void *X_bf16, int64_t n_tok, int64_t d_in,
  *   perm_out   [d_in] int32 (device, out) -- required iff act_order != 0
  *   dead_out   [d_in] uint8 (device, out) or NULL
  *   U          [d_in][d_in] fp32 (device, out)
- *   info_dev   int32 (device, out) or NULL: -1 on success, else the index
- *              (in processing order) of the first non-positive or
- *              non-finite pivot.
+ *   info_dev   int32 (device, out) or NULL: -1 on success, else a column
+ *              (in processing order) at which the factorisation met a
+ *              non-positive or non-finite pivot.
  *   info_host  int32 (host, out) or NULL.  If non-NULL the call
  *              synchronises the stream once at its end, stores the info
  *              value there and returns GQ_ERR_NOT_PD on failure.
@@ -154,8 +155,8 @@ gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent,
  *   U          [d_in][d_in] fp32 upper factor from gq_damp_cholesky_inverse
  *              (in processing order)
  *   bits       4
- *   group_size -1 or a multiple of 8 dividing d_in and block_size
- *   block_size a multiple of 32 (the pages' value is 128)
+ *   group_size -1, 32, 64 or 128, dividing d_in and block_size
+ *   block_size 32, 64 or 128 (the pages' value is 128)
  *   sym        1 symmetric, 0 affine
  *   perm       [d_in] int32 processing order (act-order) or NULL
  *   dead       [d_in] uint8 dead-column mask or NULL

@@ -270,10 +270,29 @@ class GptqResult:
     g_idx: np.ndarray      # [d_in] int32, group of each original column
     qpacked: np.ndarray    # [d_out, d_in / 8] uint32 (None unless d_in % 8 == 0)
     W_hat: np.ndarray      # [d_out, d_in] fp64 dequantised, original column order
+    n_followed: int = 0    # tie decisions adopted from ``follow``
+
+
+def _tie_dist(x):
+    """Distance of x from the nearest rounding boundary k + 1/2."""
+    f = np.asarray(x, dtype=np.float64)
+    return np.abs(f - np.floor(f) - 0.5)
+
+
+def _fp16_tie_dist(s32):
+    """Distance (in fp16 ulps) of an fp32 scale from the nearest fp16
+    rounding boundary."""
+    s = np.asarray(s32, dtype=np.float64)
+    lo = s.astype(np.float16).astype(np.float64)
+    up = np.nextafter(lo.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+    dn = np.nextafter(lo.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
+    ulp = np.where(s >= lo, up - lo, lo - dn)
+    mid = np.where(s >= lo, (lo + up) / 2, (lo + dn) / 2)
+    return np.abs(s - mid) / np.where(ulp > 0, ulp, 1.0)
 
 
 def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
-                  perm=None, dead=None) -> GptqResult:
+                  perm=None, dead=None, follow=None, tie_tol=1e-3) -> GptqResult:
     """GPTQ on one layer given U (upper, H^-1 = U^T U, in the column order
     the layer is processed in).
 
@@ -283,7 +302,17 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     update w[j+1:end] -= delta * U[j, j+1:end]; after the block the lazy
     trailing update W[:, end:] -= Err @ U[blk, end:].  Group parameters per
     reading 6.  ``perm`` (act-order) gives the processing order of the
-    original columns; ``dead`` columns are zeroed first."""
+    original columns; ``dead`` columns are zeroed first.
+
+    ``follow`` (optional, dict with "codes" [d_out, d_in] in original column
+    order and "scales"/"zeros" [d_out, n_groups]) is the output of another
+    implementation.  Where the oracle's own decision is a rounding tie --
+    the value w/s lies within ``tie_tol`` steps of k + 1/2, or the fp32
+    scale within ``tie_tol`` fp16 ulps of an fp16 rounding boundary -- both
+    roundings are correct, and the oracle takes the other implementation's
+    choice so that the rest of the row can be checked along it.  Nowhere
+    else does ``follow`` change anything; ``n_followed`` counts the
+    adopted decisions."""
     W = np.array(W, dtype=np.float64, copy=True)
     d_out, d_in = W.shape
     if dead is not None:
@@ -302,8 +331,37 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     Q = np.zeros((d_out, d_in), dtype=np.float64)
     scales = np.zeros((d_out, n_groups), dtype=np.float16)
     zeros = np.zeros((d_out, n_groups), dtype=np.float16)
+    n_followed = 0
+    if follow is not None:
+        f_codes = np.asarray(follow["codes"], dtype=np.int64)
+        if perm is not None:
+            f_codes = f_codes[:, perm]
+        f_scales = np.asarray(follow["scales"], dtype=np.float16)
+        f_zeros = (np.asarray(follow["zeros"], dtype=np.float16)
+                   if not sym else np.zeros_like(f_scales))
+
+    def group(vals, gi):
+        nonlocal n_followed
+        s, z = params(vals, bits)
+        if follow is not None:
+            v = np.asarray(vals, dtype=F32)
+            if sym:
+                s32 = np.max(np.abs(v), axis=-1) / F32(2 ** (bits - 1) - 1)
+                ztie = np.zeros(len(s), dtype=bool)
+            else:
+                mn = np.minimum(np.min(v, axis=-1), F32(0))
+                mx = np.maximum(np.max(v, axis=-1), F32(0))
+                s32 = (mx - mn) / F32(2 ** bits - 1)
+                ztie = _tie_dist(-mn.astype(np.float64) / s.astype(np.float64)) < tie_tol
+            tie = (_fp16_tie_dist(s32) < tie_tol) | ztie
+            take = tie & ((f_scales[:, gi] != s) | (f_zeros[:, gi] != z))
+            s = np.where(take, f_scales[:, gi], s)
+            z = np.where(take, f_zeros[:, gi], z)
+            n_followed += int(take.sum())
+        return s, z
+
     if group_size == -1:
-        s, z = params(W.astype(F32), bits)
+        s, z = group(W.astype(F32), 0)
         scales[:, 0], zeros[:, 0] = s, z
     for b0 in range(0, d_in, block_size):
         b1 = min(b0 + block_size, d_in)
@@ -312,12 +370,18 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
         for j in range(b1 - b0):
             col = b0 + j
             if group_size != -1 and col % g == 0:
-                s, z = params(Wb[:, j:j + g].astype(F32), bits)
+                s, z = group(Wb[:, j:j + g].astype(F32), col // g)
                 scales[:, col // g], zeros[:, col // g] = s, z
             gi = 0 if group_size == -1 else col // g
             s, z = scales[:, gi], zeros[:, gi]
             w = Wb[:, j]
             c = quantize_codes(w, s, z, sym, bits)
+            if follow is not None:
+                r = w.astype(F32).astype(np.float64) / s.astype(np.float64)
+                take = ((_tie_dist(r) < tie_tol) & (f_codes[:, col] != c)
+                        & (np.abs(f_codes[:, col] - c) == 1))
+                c = np.where(take, f_codes[:, col], c)
+                n_followed += int(take.sum())
             q = dequantize_codes(c, s, z)
             codes[:, col] = c
             Q[:, col] = q
@@ -338,13 +402,13 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
         g_idx = g_perm
     assert codes.min() >= lo
     return GptqResult(codes=codes, scales=scales, zeros=zeros,
-                      g_idx=g_idx.astype(np.int32),
+                      g_idx=g_idx.astype(np.int32), n_followed=n_followed,
                       qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None,
                       W_hat=Q)
 
 
 def gptq_layer(W, X, bits=4, group_size=-1, block_size=128, sym=True,
-               damp_percent=0.01, act_order=False):
+               damp_percent=0.01, act_order=False, follow=None, tie_tol=1e-3):
     """The whole per-layer path: H = 2 X^T X, dead columns and damping,
     optional act-order, U, then GPTQ.  Returns (GptqResult, H_undamped,
     U, perm, dead)."""
@@ -354,7 +418,8 @@ def gptq_layer(W, X, bits=4, group_size=-1, block_size=128, sym=True,
     Hp = Hd[np.ix_(perm, perm)] if perm is not None else Hd
     U = upper_factor_of_inverse(Hp)
     res = gptq_quantize(W, U, bits=bits, group_size=group_size,
-                        block_size=block_size, sym=sym, perm=perm, dead=dead)
+                        block_size=block_size, sym=sym, perm=perm, dead=dead,
+                        follow=follow, tie_tol=tie_tol)
     return res, H0, U, perm, dead
 
 

@@ -1,0 +1,454 @@
+// Damping, dead columns, act-order, and U with H^-1 = U^T U, all in fp32.
+//
+// "GPTQ: Post-Training INT4" -- "Running GPTQ with AutoGPTQ": damp_percent
+// (H += damp * mean diag H) and desc_act (columns by descending diag H);
+// "The GPTQ Algorithm": Cholesky of H, then its inverse; "Model
+// Quantization Mechanics", section 2.1: GPTQ uses a Cholesky factor of the
+// inverse Hessian.
+//
+// Instead of inverting H and factoring the inverse, this file uses the
+// identity U = J L^-1 J, where J reverses the index order and L is the
+// lower Cholesky factor of A = J H J: U is upper triangular with positive
+// diagonal and U^T U = J L^-T L^-1 J = J A^-1 J = H^-1, so by uniqueness it
+// is the upper Cholesky factor of H^-1.  Two d^3/3 steps instead of three.
+//
+// Memory: A is gathered (reversed, act-order permuted) into the U buffer
+// and factored in place; X = L^-1 is built in the H buffer (the caller's H
+// is scratch); the last kernel writes U = J X J back into the U buffer.
+// Blocked right-looking algorithms with 128-wide panels; one CTA factors a
+// diagonal block in shared memory, the panel solve and the trailing
+// updates run as tiled fp32 GEMMs over the whole GPU.
+#include <cfloat>
+#include <climits>
+
+#include "gq_device.cuh"
+#include "gq_internal.h"
+
+namespace gq {
+namespace {
+
+constexpr int NB = 128;  // panel width
+
+struct CholWs {
+  int *status;    // [0] device status, [1] info (first bad pivot, INT_MAX if none)
+  double *mean;   // scratch for the damping mean
+  float *key;     // [d] diag after damping (act-order keys)
+  float *linv;    // [n_panels][NB][NB] inverse of each diagonal block of L
+};
+
+CholWs carve(void *ws, int64_t d) {
+  uint8_t *p = static_cast<uint8_t *>(ws);
+  CholWs w;
+  w.status = reinterpret_cast<int *>(p);
+  w.mean = reinterpret_cast<double *>(p + 64);
+  size_t off = kWsHeader;
+  w.key = reinterpret_cast<float *>(p + off);
+  off += round_up(static_cast<size_t>(d) * sizeof(float), 256);
+  w.linv = reinterpret_cast<float *>(p + off);
+  return w;
+}
+
+// ---------------------------------------------------------------- damping
+// One block: dead columns (H_jj == 0 -> 1), the mean of the diagonal in
+// fp64 (fixed reduction order), then H_jj += damp * mean.
+__global__ void __launch_bounds__(1024) damp_kernel(float *__restrict__ H, int64_t d, float damp,
+                                                    uint8_t *__restrict__ dead_out,
+                                                    float *__restrict__ key, int *status) {
+  __shared__ double red[1024];
+  double s = 0.0;
+  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
+    float hjj = H[j * d + j];
+    const bool dead = hjj == 0.0f;
+    if (dead) hjj = 1.0f;
+    if (dead_out) dead_out[j] = dead ? 1 : 0;
+    s += static_cast<double>(hjj);
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 512; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const double lam = static_cast<double>(damp) * (red[0] / static_cast<double>(d));
+  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
+    float hjj = H[j * d + j];
+    if (hjj == 0.0f) hjj = 1.0f;
+    const float v = static_cast<float>(static_cast<double>(hjj) + lam);
+    H[j * d + j] = v;
+    key[j] = v;
+  }
+  if (threadIdx.x == 0) {
+    status[0] = 0;
+    status[1] = INT_MAX;
+  }
+}
+
+// ---------------------------------------------------------------- act-order
+// perm[rank(i)] = i with rank(i) = #{j : key_j > key_i} + #{j < i : key_j == key_i},
+// i.e. a stable sort by descending key.
+__global__ void __launch_bounds__(256) rank_kernel(const float *__restrict__ key, int64_t d,
+                                                   int32_t *__restrict__ perm) {
+  __shared__ float tile[256];
+  // NaN keys count as -FLT_MAX so that the ranks always form a permutation
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  float ki = i < d ? key[i] : 0.0f;
+  if (!(ki == ki)) ki = -FLT_MAX;
+  int64_t rank = 0;
+  for (int64_t j0 = 0; j0 < d; j0 += 256) {
+    __syncthreads();
+    float kt = j0 + threadIdx.x < d ? key[j0 + threadIdx.x] : -FLT_MAX;
+    tile[threadIdx.x] = kt == kt ? kt : -FLT_MAX;
+    __syncthreads();
+    const int n = static_cast<int>(d - j0 < 256 ? d - j0 : 256);
+    for (int t = 0; t < n; ++t) {
+      const float kj = tile[t];
+      rank += (kj > ki) || (kj == ki && j0 + t < i);
+    }
+  }
+  if (i < d) perm[rank] = static_cast<int32_t>(i);
+}
+
+// A[a][b] = H[p(d-1-a)][p(d-1-b)] (lower triangle and diagonal only).
+__global__ void __launch_bounds__(256) gather_reversed_kernel(const float *__restrict__ H,
+                                                              int64_t d,
+                                                              const int32_t *__restrict__ perm,
+                                                              float *__restrict__ A) {
+  for (int64_t a = blockIdx.y; a < d; a += gridDim.y) {
+    const int64_t sa = d - 1 - a;
+    const int64_t ra = perm ? perm[sa] : sa;
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; b <= a;
+         b += static_cast<int64_t>(gridDim.x) * 256) {
+      const int64_t sb = d - 1 - b;
+      const int64_t cb = perm ? perm[sb] : sb;
+      A[a * d + b] = H[ra * d + cb];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- panel factor
+// Cholesky of the nb x nb diagonal block at (k0, k0) of the lower matrix A
+// (in place), and the inverse of that block written to linv [NB][NB].
+// Sub-panels of 32 columns: a warp factors the 32 x 32 diagonal piece, one
+// thread per row solves the rows below, then all threads update the rest.
+constexpr int SP = NB + 1;  // padded row stride in shared memory
+
+__global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A, int64_t d,
+                                                          int64_t k0, int nb,
+                                                          float *__restrict__ linv,
+                                                          int *status) {
+  extern __shared__ float sm[];
+  float *S = sm;             // [NB][SP]  the block, then L
+  float *Li = sm + NB * SP;  // [NB][SP]  L^-1
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < NB * NB; e += 256) {
+    const int r = e / NB, c = e % NB;
+    S[r * SP + c] = (r < nb && c <= r) ? A[(k0 + r) * d + k0 + c] : (r == c ? 1.0f : 0.0f);
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < NB; c0 += 32) {
+    if (warp == 0) {
+      const int r = c0 + lane;
+      for (int j = 0; j < 32; ++j) {
+        const int cj = c0 + j;
+        float piv = S[cj * SP + cj];
+        if (!(piv > 0.0f) || !(piv < FLT_MAX)) {
+          if (lane == 0 && cj < nb) atomicMin(&status[1], static_cast<int>(k0 + cj));
+          piv = 1.0f;
+        }
+        const float dj = __fsqrt_rn(piv);
+        __syncwarp();
+        if (lane == j) S[cj * SP + cj] = dj;
+        if (lane > j) S[r * SP + cj] = __fdiv_rn(S[r * SP + cj], dj);
+        __syncwarp();
+        if (lane > j) {
+          const float lrj = S[r * SP + cj];
+          for (int k = j + 1; k <= lane; ++k) S[r * SP + c0 + k] -= lrj * S[(c0 + k) * SP + cj];
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    // rows below: x L_dd^T = a  (forward substitution per row)
+    for (int r = c0 + 32 + tid; r < NB; r += 256) {
+      float x[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float v = S[r * SP + c0 + j];
+        for (int k = 0; k < j; ++k) v -= x[k] * S[(c0 + j) * SP + c0 + k];
+        x[j] = __fdiv_rn(v, S[(c0 + j) * SP + c0 + j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) S[r * SP + c0 + j] = x[j];
+    }
+    __syncthreads();
+    // trailing update of the rest of the block
+    const int base = c0 + 32;
+    const int m = NB - base;
+    for (int e = tid; e < m * m; e += 256) {
+      const int i = base + e / m, k = base + e % m;
+      if (k > i) continue;
+      float acc = S[i * SP + k];
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) acc -= S[i * SP + c0 + j] * S[k * SP + c0 + j];
+      S[i * SP + k] = acc;
+    }
+    __syncthreads();
+  }
+  // L^-1 by forward substitution, one column per thread
+  if (tid < NB) {
+    const int c = tid;
+    for (int r = 0; r < NB; ++r) {
+      float v = (r == c) ? 1.0f : 0.0f;
+      if (r >= c) {
+        for (int k = c; k < r; ++k) v -= S[r * SP + k] * Li[k * SP + c];
+        v = __fdiv_rn(v, S[r * SP + r]);
+      } else {
+        v = 0.0f;
+      }
+      Li[r * SP + c] = v;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < NB * NB; e += 256) {
+    const int r = e / NB, c = e % NB;
+    if (r < nb && c <= r) A[(k0 + r) * d + k0 + c] = S[r * SP + c];
+    linv[e] = Li[r * SP + c];
+  }
+}
+
+// ---------------------------------------------------------------- SIMT GEMM
+// C[m][n] = beta * C[m][n] + alpha * sum_k A(m, k) B(k, n), fp32, tiles of
+// 128 x 128 x 8 with an 8 x 8 register block per thread.  A(m, k) =
+// A[m * lda + k]; B(k, n) = B_NT ? B[n * ldb + k] : B[k * ldb + n].  With
+// LOWER only the n <= m part of C is computed (tiles above the diagonal are
+// skipped).  K must be a multiple of 8.  In-place use (C overlapping A or
+// B) is safe when every tile reads all of its operands before its stores
+// and no other tile writes them.
+constexpr int GBM = 128, GBN = 128, GBK = 8;
+
+template <bool B_NT, bool LOWER>
+__global__ void __launch_bounds__(256) sgemm_kernel(int M, int N, int K, float alpha,
+                                                    const float *__restrict__ Am, int64_t lda,
+                                                    const float *__restrict__ Bm, int64_t ldb,
+                                                    float beta, float *Cm, int64_t ldc) {
+  const int tm = blockIdx.y * GBM, tn = blockIdx.x * GBN;
+  if (LOWER && tn > tm + GBM - 1) return;
+  __shared__ __align__(16) float As[2][GBK][GBM + 4];
+  __shared__ __align__(16) float Bs[2][GBK][GBN + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  // loader mapping: A: row = tid / 2, k = (tid % 2) * 4 (float4 along k)
+  const int la_r = tid >> 1, la_k = (tid & 1) * 4;
+  // B NT: same as A; B NN: k = tid / 32, n = (tid % 32) * 4
+  const int lb_r = B_NT ? (tid >> 1) : (tid >> 5);
+  const int lb_c = B_NT ? ((tid & 1) * 4) : ((tid & 31) * 4);
+  float4 ra, rb;
+  auto load = [&](int k0) {
+    const int am = tm + la_r;
+    ra = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (am < M) ra = *reinterpret_cast<const float4 *>(Am + am * lda + k0 + la_k);
+    rb = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (B_NT) {
+      const int bn = tn + lb_r;
+      if (bn < N) rb = *reinterpret_cast<const float4 *>(Bm + bn * ldb + k0 + lb_c);
+    } else {
+      const int bk = k0 + lb_r, bn = tn + lb_c;
+      const float *p = Bm + bk * ldb + bn;
+      if (bn + 3 < N) {
+        rb = *reinterpret_cast<const float4 *>(p);
+      } else {
+        rb.x = bn < N ? p[0] : 0.f;
+        rb.y = bn + 1 < N ? p[1] : 0.f;
+        rb.z = bn + 2 < N ? p[2] : 0.f;
+        rb.w = 0.f;
+      }
+    }
+  };
+  auto store = [&](int buf) {
+    As[buf][la_k + 0][la_r] = ra.x;
+    As[buf][la_k + 1][la_r] = ra.y;
+    As[buf][la_k + 2][la_r] = ra.z;
+    As[buf][la_k + 3][la_r] = ra.w;
+    if (B_NT) {
+      Bs[buf][lb_c + 0][lb_r] = rb.x;
+      Bs[buf][lb_c + 1][lb_r] = rb.y;
+      Bs[buf][lb_c + 2][lb_r] = rb.z;
+      Bs[buf][lb_c + 3][lb_r] = rb.w;
+    } else {
+      *reinterpret_cast<float4 *>(&Bs[buf][lb_r][lb_c]) = rb;
+    }
+  };
+  load(0);
+  store(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < K; k0 += GBK) {
+    const bool more = k0 + GBK < K;
+    if (more) load(k0 + GBK);
+#pragma unroll
+    for (int kk = 0; kk < GBK; ++kk) {
+      float a[8], b[8];
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
+      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+      a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
+      b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (more) {
+      store(buf ^ 1);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+  // every tile has read all of its operands before any store below
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = tm + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = tn + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (n >= N || (LOWER && n > m)) continue;
+      float *c = Cm + m * ldc + n;
+      const float v = alpha * acc[i][j];
+      *c = beta == 0.0f ? v : fmaf(beta, *c, v);
+    }
+  }
+}
+
+template <bool B_NT, bool LOWER>
+void sgemm(int M, int N, int K, float alpha, const float *A, int64_t lda, const float *B,
+           int64_t ldb, float beta, float *C, int64_t ldc, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0) return;
+  dim3 grid((N + GBN - 1) / GBN, (M + GBM - 1) / GBM);
+  sgemm_kernel<B_NT, LOWER><<<grid, 256, 0, st>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc);
+  count_launch();
+}
+
+// X := I on the lower triangle and on the whole NB x NB diagonal blocks
+// (the right-hand side of L X = I); the rest of the upper part is never read.
+__global__ void __launch_bounds__(256) eye_lower_kernel(float *__restrict__ X, int64_t d) {
+  for (int64_t r = blockIdx.y; r < d; r += gridDim.y) {
+    int64_t end = (r / NB + 1) * NB;
+    if (end > d) end = d;
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; c < end;
+         c += static_cast<int64_t>(gridDim.x) * 256)
+      X[r * d + c] = r == c ? 1.0f : 0.0f;
+  }
+}
+
+// U[a][b] = X[d-1-a][d-1-b] for a <= b, 0 below the diagonal; also turns
+// the recorded pivot failure into the info value.
+__global__ void __launch_bounds__(256) reverse_upper_kernel(const float *__restrict__ X,
+                                                            int64_t d, float *__restrict__ U) {
+  for (int64_t a = blockIdx.y; a < d; a += gridDim.y)
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; b < d;
+         b += static_cast<int64_t>(gridDim.x) * 256)
+      U[a * d + b] = b >= a ? X[(d - 1 - a) * d + (d - 1 - b)] : 0.0f;
+}
+
+// The factorisation runs on the reversed matrix: reversed pivot k is column
+// d-1-k in processing order.
+__global__ void finish_info_kernel(int *status, int64_t d, int32_t *info_dev) {
+  const int v = status[1] == INT_MAX ? -1 : static_cast<int>(d - 1 - status[1]);
+  status[1] = v;
+  if (info_dev) *info_dev = v;
+}
+
+}  // namespace
+
+// W[:, end:] -= Err * U[blk, end:] for the GPTQ trailing update (fp32).
+void trailing_update_sgemm(int M, int N, int K, const float *Err, int64_t lde, const float *Urow,
+                           int64_t ldu, float *Wk, int64_t ldw, cudaStream_t st) {
+  sgemm<false, false>(M, N, K, -1.0f, Err, lde, Urow, ldu, 1.0f, Wk, ldw, st);
+}
+
+size_t chol_ws_bytes(int64_t d) {
+  const int64_t n_panels = (d + NB - 1) / NB;
+  return kWsHeader + round_up(static_cast<size_t>(d) * sizeof(float), 256) +
+         static_cast<size_t>(n_panels) * NB * NB * sizeof(float);
+}
+
+gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32_t *perm_out,
+                           uint8_t *dead_out, float *U, int32_t *info_dev, void *ws,
+                           cudaStream_t st) {
+  CholWs w = carve(ws, d);
+  damp_kernel<<<1, 1024, 0, st>>>(H, d, damp, dead_out, w.key, w.status);
+  count_launch();
+  if (act_order) {
+    rank_kernel<<<static_cast<unsigned>((d + 255) / 256), 256, 0, st>>>(w.key, d, perm_out);
+    count_launch();
+  }
+  const unsigned gx = static_cast<unsigned>((d + 255) / 256);
+  const unsigned gy = static_cast<unsigned>(d < 65535 ? d : 65535);
+  float *A = U;  // the factorisation lives in the U buffer
+  float *X = H;  // L^-1 is built in the H buffer
+  gather_reversed_kernel<<<dim3(gx, gy), 256, 0, st>>>(
+      H, d, act_order ? perm_out : nullptr, A);
+  count_launch();
+  {
+    const gq_status s = check_launch("damp/gather");
+    if (s != GQ_OK) return s;
+  }
+  const size_t pot_smem = 2 * NB * SP * sizeof(float);
+  cudaFuncSetAttribute(potrf_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(pot_smem));
+  const int64_t n_panels = (d + NB - 1) / NB;
+  // ---- Cholesky, right-looking
+  for (int64_t p = 0; p < n_panels; ++p) {
+    const int64_t k0 = p * NB;
+    const int nb = static_cast<int>(d - k0 < NB ? d - k0 : NB);
+    float *lp = w.linv + p * NB * NB;
+    potrf_panel_kernel<<<1, 256, pot_smem, st>>>(A, d, k0, nb, lp, w.status);
+    count_launch();
+    const int64_t k1 = k0 + nb;
+    const int rest = static_cast<int>(d - k1);
+    if (rest > 0) {
+      // panel rows below: A[k1:, k0:k1] := A[k1:, k0:k1] L_pp^-T
+      sgemm<true, false>(rest, nb, NB, 1.0f, A + k1 * d + k0, d, lp, NB, 0.0f, A + k1 * d + k0,
+                         d, st);
+      // trailing: A[k1:, k1:] -= P P^T (lower part)
+      sgemm<true, true>(rest, rest, NB, -1.0f, A + k1 * d + k0, d, A + k1 * d + k0, d, 1.0f,
+                        A + k1 * d + k1, d, st);
+    }
+  }
+  // ---- X = L^-1 by blocked forward substitution on the identity
+  eye_lower_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d);
+  count_launch();
+  for (int64_t p = 0; p < n_panels; ++p) {
+    const int64_t r0 = p * NB;
+    const int nb = static_cast<int>(d - r0 < NB ? d - r0 : NB);
+    const int cols = static_cast<int>(r0 + nb);
+    float *lp = w.linv + p * NB * NB;
+    // X[r0:r0+nb, 0:cols] := L_pp^-1 X[r0:r0+nb, 0:cols]
+    sgemm<false, false>(nb, cols, nb, 1.0f, lp, NB, X + r0 * d, d, 0.0f, X + r0 * d, d, st);
+    const int64_t r1 = r0 + nb;
+    const int rest = static_cast<int>(d - r1);
+    if (rest > 0) {
+      // X[r1:, 0:cols] -= L[r1:, r0:r1] X[r0:r1, 0:cols]
+      sgemm<false, false>(rest, cols, nb, -1.0f, A + r1 * d + r0, d, X + r0 * d, d, 1.0f,
+                          X + r1 * d, d, st);
+    }
+  }
+  reverse_upper_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d, U);
+  count_launch();
+  finish_info_kernel<<<1, 1, 0, st>>>(w.status, d, info_dev);
+  count_launch();
+  return check_launch("damp_cholesky_inverse");
+}
+
+}  // namespace gq

@@ -1,0 +1,228 @@
+// GPTQ on one layer: the column-block kernel and the lazy trailing update.
+//
+// "GPTQ: Post-Training INT4" -- "The GPTQ Algorithm": columns in a fixed
+// order, blocks of B columns; inside a block, for each column j the code of
+// the current weight, delta = (w - q) / U_jj and w[j+1:end] -= delta *
+// U[j, j+1:end]; after the block one batched update W[:, end:] -= Err *
+// U[blk, end:].  "Group Quantization": a group's scale (and zero) comes
+// from its current weights when its first column is reached.
+//
+// Layout: W is copied once to an fp32 working matrix Wk [d_out][d_in] in
+// processing order (act-order gather and dead-column zeroing fused into the
+// copy).  The block kernel keeps the B x B block of U in shared memory and
+// gives every output row to one thread, whose B weights live in registers
+// for the whole block: the in-block update is register FMAs against
+// broadcast shared-memory reads, with no shuffles and no synchronisation.
+// A processed weight's register is reused for its scaled error delta, so
+// the Err block leaves the kernel in one contiguous store per row.  The
+// trailing update is a GEMM of d_out x (d_in - end) x B.
+#include "gptq_block.cuh"
+
+namespace gq {
+
+GQ_GPTQ_BLOCK_INSTANCES(GQ_DECLARE_BLOCK)
+
+namespace {
+
+struct GptqWs {
+  float *Wk;        // [d_out][d_in] fp32 working copy, processing order
+  float *Err;       // [d_out][B]
+  uint8_t *codes;   // [d_out][d_in] codes in processing order (act-order only)
+  int32_t *inv;     // [d_in] processing position of each original column
+};
+
+GptqWs carve(void *ws, int64_t d_out, int64_t d_in, int B, bool with_perm) {
+  uint8_t *p = static_cast<uint8_t *>(ws) + kWsHeader;
+  GptqWs w{};
+  w.Wk = reinterpret_cast<float *>(p);
+  p += round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256);
+  w.Err = reinterpret_cast<float *>(p);
+  p += round_up(static_cast<size_t>(d_out) * B * sizeof(float), 256);
+  if (with_perm) {
+    w.codes = p;
+    p += round_up(static_cast<size_t>(d_out) * d_in, 256);
+    w.inv = reinterpret_cast<int32_t *>(p);
+  }
+  return w;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// Wk[r][p] = dead[src] ? 0 : W[r][src], src = perm ? perm[p] : p.
+template <typename T>
+__global__ void __launch_bounds__(256) prep_kernel(const T *__restrict__ W, int64_t d_out,
+                                                   int64_t d_in, const int32_t *__restrict__ perm,
+                                                   const uint8_t *__restrict__ dead,
+                                                   float *__restrict__ Wk) {
+  const int64_t n = d_out * d_in;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t r = e / d_in, p = e % d_in;
+    int64_t src = perm ? perm[p] : p;
+    src = src < 0 ? 0 : (src >= d_in ? d_in - 1 : src);  // never read outside the row
+    float v = to_f32(W[r * d_in + src]);
+    if (dead && dead[src]) v = 0.0f;
+    Wk[e] = v;
+  }
+}
+
+// Per-channel grid from the initial (working) row: one warp per row.
+__global__ void __launch_bounds__(256) row_params_kernel(const float *__restrict__ Wk,
+                                                         int64_t d_out, int64_t d_in, int sym,
+                                                         uint16_t *__restrict__ scales,
+                                                         uint16_t *__restrict__ zeros) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = warp; r < d_out; r += n_warps) {
+    float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+    for (int64_t c = lane; c < d_in; c += 32) {
+      const float v = Wk[r * d_in + c];
+      amax = fmaxf(amax, fabsf(v));
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    if (lane == 0) {
+      const GridParams g = sym ? grid_sym(amax) : grid_affine(mn, mx);
+      scales[r] = g.s_bits;
+      if (zeros) zeros[r] = sym ? 0 : g.z_bits;
+    }
+  }
+}
+
+__global__ void invert_perm_kernel(const int32_t *__restrict__ perm, int64_t d,
+                                   int32_t *__restrict__ inv) {
+  for (int64_t p = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; p < d;
+       p += static_cast<int64_t>(gridDim.x) * 256)
+  {
+    const int32_t q = perm[p];
+    if (q >= 0 && q < d) inv[q] = static_cast<int32_t>(p);
+  }
+}
+
+// qpacked[r][w] from the processing-order codes: nibble k <- codes[r][inv[8w+k]].
+__global__ void __launch_bounds__(256) pack_perm_kernel(const uint8_t *__restrict__ codes,
+                                                        int64_t d_out, int64_t d_in,
+                                                        const int32_t *__restrict__ inv,
+                                                        uint32_t *__restrict__ qpacked) {
+  const int64_t words = d_in / 8;
+  const int64_t n = d_out * words;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t r = e / words, wd = e % words;
+    uint32_t v = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      int64_t pos = inv[wd * 8 + k];
+      pos = pos < 0 ? 0 : (pos >= d_in ? d_in - 1 : pos);
+      v |= static_cast<uint32_t>(codes[r * d_in + pos]) << (4 * k);
+    }
+    qpacked[e] = v;
+  }
+}
+
+__global__ void g_idx_kernel(const int32_t *__restrict__ inv, int64_t d, int g,
+                             int32_t *__restrict__ g_idx) {
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; c < d;
+       c += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t pos = inv ? inv[c] : c;
+    g_idx[c] = g < 0 ? 0 : static_cast<int32_t>(pos / g);
+  }
+}
+
+GptqBlockLaunch pick_block(int B, int G) {
+#define GQ_PICK(b, g) \
+  if (B == b && G == g) return launch_gptq_block<b, g>;
+  GQ_GPTQ_BLOCK_INSTANCES(GQ_PICK)
+#undef GQ_PICK
+  return nullptr;
+}
+
+}  // namespace
+
+// fp32 GEMM of chol.cu, reused for the trailing update.
+void trailing_update_sgemm(int M, int N, int K, const float *Err, int64_t lde, const float *Urow,
+                           int64_t ldu, float *Wk, int64_t ldw, cudaStream_t st);
+
+size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size) {
+  return kWsHeader + round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256) +
+         round_up(static_cast<size_t>(d_out) * block_size * sizeof(float), 256) +
+         round_up(static_cast<size_t>(d_out) * d_in, 256) +
+         round_up(static_cast<size_t>(d_in) * sizeof(int32_t), 256);
+}
+
+gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,
+                      int group_size, int block_size, int sym, const int32_t *perm,
+                      const uint8_t *dead, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
+                      int32_t *g_idx, void *ws, cudaStream_t st) {
+  const int B = block_size;
+  GptqBlockLaunch blk = pick_block(B, group_size);
+  if (!blk) return fail(GQ_ERR_ARG, "unsupported (block_size, group_size) combination");
+  GptqWs w = carve(ws, d_out, d_in, B, perm != nullptr);
+  const int64_t n = d_out * d_in;
+  unsigned grid = static_cast<unsigned>((n + 255) / 256);
+  const unsigned cap = static_cast<unsigned>(num_sms()) * 16;
+  if (grid > cap) grid = cap;
+  switch (dt) {
+    case GQ_F32:
+      prep_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(W), d_out, d_in, perm,
+                                               dead, w.Wk);
+      break;
+    case GQ_F16:
+      prep_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half *>(W), d_out, d_in,
+                                                perm, dead, w.Wk);
+      break;
+    case GQ_BF16:
+      prep_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(W),
+                                                       d_out, d_in, perm, dead, w.Wk);
+      break;
+  }
+  count_launch();
+  const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
+  if (group_size == -1) {
+    unsigned g2 = static_cast<unsigned>((d_out + 7) / 8);
+    if (g2 > cap) g2 = cap;
+    row_params_kernel<<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros);
+    count_launch();
+  }
+  for (int64_t c0 = 0; c0 < d_in; c0 += B) {
+    const int bw = static_cast<int>(d_in - c0 < B ? d_in - c0 : B);
+    blk(w.Wk, d_out, d_in, c0, bw, U, sym, w.Err, perm ? nullptr : qpacked, w.codes, scales,
+        zeros, n_groups, st);
+    const int64_t c1 = c0 + bw;
+    if (c1 < d_in)
+      trailing_update_sgemm(static_cast<int>(d_out), static_cast<int>(d_in - c1), bw, w.Err, B,
+                            U + c0 * d_in + c1, d_in, w.Wk + c1, d_in, st);
+  }
+  const unsigned gd = static_cast<unsigned>((d_in + 255) / 256);
+  if (perm) {
+    invert_perm_kernel<<<gd, 256, 0, st>>>(perm, d_in, w.inv);
+    count_launch();
+    unsigned gp = static_cast<unsigned>((d_out * (d_in / 8) + 255) / 256);
+    if (gp > cap) gp = cap;
+    pack_perm_kernel<<<gp, 256, 0, st>>>(w.codes, d_out, d_in, w.inv, qpacked);
+    count_launch();
+  }
+  if (g_idx) {
+    g_idx_kernel<<<gd, 256, 0, st>>>(perm ? w.inv : nullptr, d_in, group_size, g_idx);
+    count_launch();
+  }
+  return check_launch("gptq_quantize_layer");
+}
+
+}  // namespace gq

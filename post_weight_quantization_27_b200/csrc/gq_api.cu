@@ -192,7 +192,9 @@ gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent, i
 }
 
 size_t gq_gptq_workspace_size(int64_t d_out, int64_t d_in, int block_size) {
-  if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || block_size < 32 || block_size % 32 != 0) return 0;
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || block_size < 32 || block_size > 128 ||
+      block_size % 32 != 0)
+    return 0;
   return gptq_ws_bytes(d_out, d_in, block_size);
 }
 
@@ -209,10 +211,10 @@ gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out,
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
-  if (block_size < 32 || block_size % 32 != 0 || block_size > 256)
-    return fail(GQ_ERR_ARG, "block_size must be a multiple of 32 in [32, 256]");
-  if (group_size != -1 && block_size % group_size != 0)
-    return fail(GQ_ERR_ARG, "group_size must divide block_size");
+  if (block_size != 32 && block_size != 64 && block_size != 128)
+    return fail(GQ_ERR_ARG, "block_size must be 32, 64 or 128");
+  if (group_size != -1 && (group_size < 32 || block_size % group_size != 0))
+    return fail(GQ_ERR_ARG, "GPTQ group_size must be -1, 32, 64 or 128 and divide block_size");
   if (!aligned(W, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
   GQ_TRY(check_ws(ws, ws_bytes, gptq_ws_bytes(d_out, d_in, block_size)));
   return launch_gptq(W, w_dtype, d_out, d_in, U, group_size, block_size, sym, perm, dead,

@@ -29,7 +29,14 @@
 namespace gq {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, CHUNK_KB = 16;
+#ifndef GQ_HESS_CHUNK_KB
+#define GQ_HESS_CHUNK_KB 2
+#endif
+// K-blocks (of 64 tokens) accumulated inside TMEM before the partial is
+// drained into fp32 registers.  The tensor core's fp32 accumulation error
+// grows with the length of this chain; 2 (128 tokens) keeps H within a few
+// fp32 ulps of the exact sum while the drain still overlaps the MMAs.
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, CHUNK_KB = GQ_HESS_CHUNK_KB;
 constexpr int A_BYTES = BM * BK * 2;  // two 64x64 boxes
 constexpr int B_BYTES = BN * BK * 2;  // four 64x64 boxes
 constexpr int BOX_BYTES = 64 * BK * 2;

@@ -1,0 +1,320 @@
+// Layer reconstruction error SSE = ||(W - W^) X^T||_F^2 on the tensor cores.
+//
+// "Model Quantization Mechanics", section 2.1 and "GPTQ: Post-Training
+// INT4", "OBQ Foundation": the layer-wise objective ||W X - W^ X||^2;
+// "GPT-2 Quantization Reconstruction Error" reports it per layer as an MSE.
+//
+// 1. dW = W - W^ in fp32 from the packed codes and the 16-bit scales, split
+//    into bf16 hi + lo (dW = hi + lo to ~2^-17 relative); X is exactly bf16.
+// 2. A persistent tcgen05 GEMM over 128 (rows) x 256 (tokens) output tiles:
+//    TMA loads hi, lo and X boxes (K-major, 128-byte swizzle, no
+//    multicast); two MMAs per K step (hi and lo) accumulate into one of two
+//    TMEM accumulators; the epilogue warps square and sum their rows while
+//    the next tile is already being multiplied.  The d_out x n_tok product
+//    never leaves the SM.
+// 3. Per-warp fp64 partials are added in a fixed order: deterministic.
+#include "gq_device.cuh"
+#include "gq_internal.h"
+
+namespace gq {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB (one box of 64 x 128)
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB (one box of 64 x 256)
+constexpr int STAGE_BYTES = 2 * A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 320;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+struct ReconArgs {
+  int n_mt, n_nt, nkb;
+  double *partials;  // [n_tiles][8]
+  int *status;
+};
+
+// dW = W - s (c - z), split into bf16 hi + lo.
+template <typename T>
+__device__ __forceinline__ float ld_w(const T *p);
+template <>
+__device__ __forceinline__ float ld_w<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ld_w<__half>(const __half *p) { return __half2float(*p); }
+template <>
+__device__ __forceinline__ float ld_w<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  return __bfloat162float(*p);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) dequant_diff_kernel(
+    const T *__restrict__ W, const uint32_t *__restrict__ q, const uint16_t *__restrict__ scales,
+    const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx, int64_t d_out,
+    int64_t d_in, int group_size, int sym, __nv_bfloat16 *__restrict__ hi,
+    __nv_bfloat16 *__restrict__ lo) {
+  const int64_t words = d_in / 8;
+  const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
+  const int64_t n = d_out * words;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t r = e / words, wd = e % words;
+    const uint32_t word = q[e];
+    __align__(16) __nv_bfloat16 h[8], l[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int64_t c = wd * 8 + k;
+      int64_t gi = g_idx ? g_idx[c] : (group_size == -1 ? 0 : c / group_size);
+      gi = gi < 0 ? 0 : (gi >= n_groups ? n_groups - 1 : gi);
+      const float s = __half2float(__ushort_as_half(scales[r * n_groups + gi]));
+      const float z = sym ? 0.0f : __half2float(__ushort_as_half(zeros[r * n_groups + gi]));
+      const int nib = static_cast<int>((word >> (4 * k)) & 0xFu);
+      const float code = static_cast<float>(sym ? nib - 8 : nib);
+      const float what = s * (code - z);
+      const float dw = ld_w(W + r * d_in + c) - what;
+      const __nv_bfloat16 hb = __float2bfloat16_rn(dw);
+      h[k] = hb;
+      l[k] = __float2bfloat16_rn(dw - __bfloat162float(hb));
+    }
+    *reinterpret_cast<uint4 *>(hi + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(h);
+    *reinterpret_cast<uint4 *>(lo + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(l);
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    recon_mma_kernel(const __grid_constant__ CUtensorMap tmHi,
+                     const __grid_constant__ CUtensorMap tmLo,
+                     const __grid_constant__ CUtensorMap tmX, ReconArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + STAGES;
+  uint64_t *acc_full = bars + 2 * STAGES;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmHi);
+    tma_prefetch_desc(&tmLo);
+    tma_prefetch_desc(&tmX);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_tiles = a.n_mt * a.n_nt;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int mt = t % a.n_mt, nt = t / a.n_mt;
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          uint8_t *st = smem + s * STAGE_BYTES;
+          tma_load_2d(st, &tmHi, &full[s], kb * BK, mt * BM);
+          tma_load_2d(st + A_BYTES, &tmLo, &full[s], kb * BK, mt * BM);
+          tma_load_2d(st + 2 * A_BYTES, &tmX, &full[s], kb * BK, nt * BN);
+        }
+      }
+      const uint32_t n_wait = it < STAGES ? it : STAGES;
+      for (uint32_t k = 0; k < n_wait; ++k) {
+        const uint32_t j = it - 1 - k;
+        if (!mbar_wait(&full[j % STAGES], (j / STAGES) & 1)) ok = false;
+      }
+      if (!ok) set_status(a.status, kDevTimeout);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0, ch = 0;
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, false);
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++ch) {
+        const uint32_t buf = ch & 1, use = ch >> 1;
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * BN;
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&full[s], r & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sh = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t sl = sh + A_BYTES;
+          const uint32_t sx = sh + 2 * A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // K-major: 16 elements = 32 bytes along the swizzled 128-byte row
+            const uint64_t bd = smem_desc_sw128(sx + kk * 32, 16, 1024);
+            mma_bf16(d_tmem, smem_desc_sw128(sh + kk * 32, 16, 1024), bd, idesc,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(d_tmem, smem_desc_sw128(sl + kk * 32, 16, 1024), bd, idesc, 1u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+      }
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) ok = false;
+      if (!ok) set_status(a.status, kDevTimeout);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int ew = warp - 2;
+    uint32_t ch = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++ch) {
+      const uint32_t buf = ch & 1, use = ch >> 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t taddr =
+          tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN + half * 128;
+      float ssq = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ssq = fmaf(v[i], v[i], ssq);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      double dsum = static_cast<double>(ssq);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+      if (lane == 0) a.partials[static_cast<size_t>(t) * 8 + ew] = dsum;
+    }
+    if (!ok && lane == 0) set_status(a.status, kDevTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+__global__ void __launch_bounds__(1024) recon_reduce_kernel(const double *__restrict__ partials,
+                                                            int64_t n, const int *status,
+                                                            double *__restrict__ sse) {
+  __shared__ double red[1024];
+  double s = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += 1024) s += partials[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 512; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *sse = (status && *status) ? __longlong_as_double(0x7ff8000000000000ll) : red[0];
+}
+
+struct ReconLayout {
+  int n_mt, n_nt, nkb;
+  size_t off_partials, off_hi, off_lo, total;
+};
+
+ReconLayout recon_layout(int64_t d_out, int64_t d_in, int64_t n_tok) {
+  ReconLayout L{};
+  L.n_mt = static_cast<int>((d_out + BM - 1) / BM);
+  L.n_nt = static_cast<int>((n_tok + BN - 1) / BN);
+  L.nkb = static_cast<int>((d_in + BK - 1) / BK);
+  L.off_partials = kWsHeader;
+  size_t off = L.off_partials + round_up(static_cast<size_t>(L.n_mt) * L.n_nt * 8 * sizeof(double), 256);
+  L.off_hi = off;
+  off += round_up(static_cast<size_t>(d_out) * d_in * 2, 256);
+  L.off_lo = off;
+  off += round_up(static_cast<size_t>(d_out) * d_in * 2, 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+size_t recon_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok) {
+  return recon_layout(d_out, d_in, n_tok).total;
+}
+
+gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
+                       const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
+                       int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
+                       int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st) {
+  const ReconLayout L = recon_layout(d_out, d_in, n_tok);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  int *status = reinterpret_cast<int *>(base);
+  double *partials = reinterpret_cast<double *>(base + L.off_partials);
+  __nv_bfloat16 *hi = reinterpret_cast<__nv_bfloat16 *>(base + L.off_hi);
+  __nv_bfloat16 *lo = reinterpret_cast<__nv_bfloat16 *>(base + L.off_lo);
+  if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
+  const int64_t n_tiles = static_cast<int64_t>(L.n_mt) * L.n_nt;
+  if (n_tok == 0) {
+    recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, 0, status, sse_dev);
+    count_launch();
+    return check_launch("recon_reduce_kernel");
+  }
+  unsigned g = static_cast<unsigned>((d_out * (d_in / 8) + 255) / 256);
+  const unsigned cap = static_cast<unsigned>(num_sms()) * 16;
+  if (g > cap) g = cap;
+  switch (dt) {
+    case GQ_F32:
+      dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
+                                                    scales, zeros, g_idx, d_out, d_in,
+                                                    group_size, sym, hi, lo);
+      break;
+    case GQ_F16:
+      dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
+                                                     scales, zeros, g_idx, d_out, d_in,
+                                                     group_size, sym, hi, lo);
+      break;
+    case GQ_BF16:
+      dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, d_out, d_in,
+          group_size, sym, hi, lo);
+      break;
+  }
+  count_launch();
+  CUtensorMap tHi, tLo, tX;
+  gq_status s = make_tmap_2d(&tHi, hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d_in, d_out, d_in, BK, BM);
+  if (s == GQ_OK) s = make_tmap_2d(&tLo, lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d_in, d_out, d_in, BK, BM);
+  if (s == GQ_OK) s = make_tmap_2d(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d_in, n_tok, d_in, BK, BN);
+  if (s != GQ_OK) return s;
+  cudaFuncSetAttribute(recon_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(SMEM_BYTES));
+  ReconArgs a{L.n_mt, L.n_nt, L.nkb, partials, status};
+  const int grid = static_cast<int>(n_tiles < num_sms() ? n_tiles : num_sms());
+  recon_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tHi, tLo, tX, a);
+  count_launch();
+  s = check_launch("recon_mma_kernel");
+  if (s != GQ_OK) return s;
+  recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, n_tiles * 8, status, sse_dev);
+  count_launch();
+  return check_launch("recon_reduce_kernel");
+}
+
+}  // namespace gq

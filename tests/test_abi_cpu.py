@@ -78,7 +78,7 @@ def test_other_argument_errors():
     assert L.gq_damp_cholesky_inverse(FAKE, 64, -1.0, 0, None, None, FAKE, None, None,
                                       FAKE, 1 << 30, None) == 1
     # group_size must divide block_size
-    assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 192, FAKE, 4, 96, 128, 1, None, None,
+    assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 192, FAKE, 4, 48, 96, 1, None, None,
                                     FAKE, FAKE, None, None, FAKE, 1 << 40, None) == 1
     # misaligned workspace
     assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 128, FAKE, 4, 128, 128, 1, None, None, FAKE,

@@ -377,3 +377,32 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # the lazy trailing update dropped (only the 2-column in-block updates kept)
     blockdiag = np.kron(np.eye(d // 2), np.ones((2, 2))) * U
     assert not matches(blockdiag, 2)
+
+
+def test_tie_follow_only_at_ties():
+    """The replay mode adopts another implementation's code only where the
+    oracle's own value is a rounding tie; elsewhere it changes nothing."""
+    rng = np.random.default_rng(17)
+    d = 16
+    X = rng.standard_normal((40, d))
+    W = (rng.standard_normal((4, d)) * 0.1).astype(np.float64)
+    H, _ = O.damp_hessian(O.hessian(X), 0.01)
+    U = np.diag(1.0 / np.sqrt(np.diag(H)))         # diagonal: no feedback
+    base = O.gptq_quantize(W, U, group_size=-1)
+    same = O.gptq_quantize(W, U, group_size=-1, follow=dict(codes=base.codes, scales=base.scales))
+    assert same.n_followed == 0 and np.array_equal(same.codes, base.codes)
+    other = base.codes.copy()
+    other[0, 3] += 1 if other[0, 3] < 7 else -1     # not a tie: must be ignored
+    r = O.gptq_quantize(W, U, group_size=-1, follow=dict(codes=other, scales=base.scales))
+    assert r.n_followed == 0 and np.array_equal(r.codes, base.codes)
+    # plant an exact tie: w = 2.5 s rounds to 2 (half to even); 3 is also correct
+    s = float(base.scales[1, 0])
+    W2 = W.copy()
+    W2[1, 5] = 2.5 * s
+    b2 = O.gptq_quantize(W2, U, group_size=-1)
+    assert b2.scales[1, 0] == base.scales[1, 0] and b2.codes[1, 5] == 2
+    tie = b2.codes.copy()
+    tie[1, 5] = 3
+    r2 = O.gptq_quantize(W2, U, group_size=-1, follow=dict(codes=tie, scales=b2.scales))
+    assert r2.n_followed == 1 and r2.codes[1, 5] == 3
+    assert np.array_equal(np.delete(r2.codes.ravel(), 1 * d + 5), np.delete(b2.codes.ravel(), 1 * d + 5))
