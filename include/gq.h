@@ -135,6 +135,31 @@ gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent,
                                    void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * gq_damp_cholesky_inverse without a workspace.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory and so cannot supply `ws`: code whose
+ * device memory is all owned by a host framework's pool or fixed budget
+ * (an extra cudaMalloc would bypass its accounting, or fail because the
+ * memory is already reserved), and code that must not stall on cudaMalloc /
+ * cudaFree, which can synchronise the whole device.
+ *
+ * Arguments and results are those of gq_damp_cholesky_inverse without
+ * (ws, ws_bytes).  Limit: d_in <= 4096; larger d_in returns GQ_ERR_SHAPE
+ * before any launch.  The scratch is a fixed ~2 MiB array in device memory
+ * that every GPU using this library holds until the process exits; the
+ * call allocates nothing.  The first call on a device looks up that
+ * array's device address (once per device, for the current device); make
+ * that first call before any stream capture.  All calls share the one
+ * array: calls whose GPU work may overlap (other streams, other host
+ * threads on the same device) race on it and must be serialised by the
+ * caller.
+ * ---------------------------------------------------------------------- */
+gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, float damp_percent,
+                                           int act_order, int32_t *perm_out,
+                                           uint8_t *dead_out, float *U, int32_t *info_dev,
+                                           int32_t *info_host, void *stream);
+
+/* ------------------------------------------------------------------------
  * GPTQ on one layer.
  * "GPTQ: Post-Training INT4", "The GPTQ Algorithm": columns in a fixed
  * left-to-right order (the act-order permutation if given) in blocks of

@@ -20,6 +20,8 @@
 // updates run as tiled fp32 GEMMs over the whole GPU.
 #include <cfloat>
 #include <climits>
+#include <mutex>
+#include <string>
 
 #include "gq_device.cuh"
 #include "gq_internal.h"
@@ -452,3 +454,87 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
 }
 
 }  // namespace gq
+
+// ---------------------------------------------------------------------------
+// gq_damp_cholesky_inverse_noalloc: the same computation for callers that
+// cannot allocate device memory, so cannot hand in a workspace either.  Its
+// scratch is the file-scope array below, a fixed part of every GPU context
+// that loads this library (it stays there until the process exits).
+namespace gq {
+namespace {
+
+constexpr int64_t kNoAllocMaxDin = 4096;
+constexpr size_t kNoAllocScratchBytes =
+    kWsHeader + ((static_cast<size_t>(kNoAllocMaxDin) * sizeof(float) + 255) / 256) * 256 +
+    static_cast<size_t>((kNoAllocMaxDin + NB - 1) / NB) * NB * NB * sizeof(float);
+
+static __device__ __align__(256) uint8_t g_noalloc_chol_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// The array's device address on the current device, looked up once per
+// device.  The array's name is only a host-side handle in host code; the
+// kernels need this address.
+gq_status noalloc_scratch(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(GQ_ERR_CUDA, "no current CUDA device (or device index >= 64)");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_chol_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(GQ_ERR_CUDA, std::string("cudaGetSymbolAddress failed: ") +
+                                   cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GQ_OK;
+}
+
+}  // namespace
+}  // namespace gq
+
+extern "C" gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, float damp_percent,
+                                                      int act_order, int32_t *perm_out,
+                                                      uint8_t *dead_out, float *U,
+                                                      int32_t *info_dev, int32_t *info_host,
+                                                      void *stream) {
+  using namespace gq;
+  clear_error();
+  if (!H || !U) return fail(GQ_ERR_ARG, "null pointer");
+  if (act_order != 0 && !perm_out) return fail(GQ_ERR_ARG, "act_order needs perm_out");
+  if (!(damp_percent >= 0.0f) || !(damp_percent < 1e30f))
+    return fail(GQ_ERR_ARG, "damp_percent must be finite and >= 0");
+  if (d_in < 8 || d_in % 8 != 0)
+    return fail(GQ_ERR_SHAPE, "d_in must be a positive multiple of 8");
+  if (d_in > kNoAllocMaxDin)
+    return fail(GQ_ERR_SHAPE, "d_in " + std::to_string(d_in) +
+                                  " exceeds the no-allocation limit of " +
+                                  std::to_string(kNoAllocMaxDin) +
+                                  "; use gq_damp_cholesky_inverse with a workspace");
+  void *scratch = nullptr;
+  const gq_status s0 = noalloc_scratch(&scratch);
+  if (s0 != GQ_OK) return s0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every buffer in the scratch is written before it is read within the call
+  // (damp_kernel resets the status words), so earlier calls' leftovers are
+  // harmless.
+  const gq_status s = launch_damp_chol(H, d_in, damp_percent, act_order, perm_out, dead_out, U,
+                                       info_dev, scratch, st);
+  if (s != GQ_OK) return s;
+  if (info_host) {
+    int32_t info = -1;
+    const int32_t *src = info_dev ? info_dev : reinterpret_cast<const int32_t *>(scratch) + 1;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpy(&info, src, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return check_launch("damp_cholesky_noalloc sync");
+    *info_host = info;
+    if (info >= 0)
+      return fail(GQ_ERR_NOT_PD, "damped Hessian not positive definite at column " +
+                                     std::to_string(info));
+  }
+  return GQ_OK;
+}

@@ -12,6 +12,8 @@ namespace gq {
 std::atomic<uint64_t> g_launches{0};
 static thread_local std::string t_last_error;
 
+void clear_error() { t_last_error.clear(); }
+
 gq_status fail(gq_status s, const std::string &msg) {
   t_last_error = msg;
   return s;

@@ -16,6 +16,8 @@ namespace gq {
 extern std::atomic<uint64_t> g_launches;
 inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+// Clears the thread-local error text (start of every entry point).
+void clear_error();
 // Sets the thread-local error text and returns `s`.
 gq_status fail(gq_status s, const std::string &msg);
 // GQ_ERR_CUDA with the text of the pending CUDA error, or GQ_OK.

@@ -54,6 +54,9 @@ def lib() -> ctypes.CDLL:
     L.gq_damp_cholesky_inverse.restype = _c_int
     L.gq_damp_cholesky_inverse.argtypes = [_c_vp, _c_i64, _c_f32, _c_int, _c_vp, _c_vp, _c_vp,
                                            _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_damp_cholesky_inverse_noalloc.restype = _c_int
+    L.gq_damp_cholesky_inverse_noalloc.argtypes = [_c_vp, _c_i64, _c_f32, _c_int, _c_vp, _c_vp,
+                                                   _c_vp, _c_vp, _c_vp, _c_vp]
     L.gq_gptq_workspace_size.restype = _c_sz
     L.gq_gptq_workspace_size.argtypes = [_c_i64, _c_i64, _c_int]
     L.gq_gptq_quantize_layer.restype = _c_int
@@ -75,6 +78,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_workspace_size",
            "gq_hessian_accumulate", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
+           "gq_damp_cholesky_inverse_noalloc",
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
            "gq_recon_workspace_size", "gq_recon_error")
 
@@ -168,6 +172,28 @@ def damp_cholesky_inverse(H: torch.Tensor, damp_percent: float = 0.01, act_order
                                         ctypes.byref(info_host) if check else None,
                                         _p(ws), ws.numel(), _stream(stream))
     _check(st, "gq_damp_cholesky_inverse")
+    return U, perm, dead, info
+
+
+def damp_cholesky_inverse_noalloc(H: torch.Tensor, damp_percent: float = 0.01,
+                                  act_order: bool = False, U: torch.Tensor | None = None,
+                                  check: bool = True, stream=None):
+    """As damp_cholesky_inverse, through the entry point that takes no
+    workspace (for callers that cannot allocate device memory; d_in <= 4096).
+    The output tensors here are still allocated by torch for convenience."""
+    _dev(H, "H", torch.float32)
+    d = H.shape[0]
+    dev = H.device
+    U = torch.empty((d, d), dtype=torch.float32, device=dev) if U is None else _dev(U, "U", torch.float32, (d, d))
+    perm = torch.empty(d, dtype=torch.int32, device=dev) if act_order else None
+    dead = torch.empty(d, dtype=torch.uint8, device=dev)
+    info = torch.empty(1, dtype=torch.int32, device=dev)
+    info_host = ctypes.c_int32(-1)
+    st = lib().gq_damp_cholesky_inverse_noalloc(_p(H), d, float(damp_percent),
+                                                int(bool(act_order)), _p(perm), _p(dead), _p(U),
+                                                _p(info), ctypes.byref(info_host) if check else None,
+                                                _stream(stream))
+    _check(st, "gq_damp_cholesky_inverse_noalloc")
     return U, perm, dead, info
 
 
