@@ -130,87 +130,206 @@ __global__ void __launch_bounds__(256) gather_reversed_kernel(const float *__res
 // ---------------------------------------------------------------- panel factor
 // Cholesky of the nb x nb diagonal block at (k0, k0) of the lower matrix A
 // (in place), and the inverse of that block written to linv [NB][NB].
-// Sub-panels of 32 columns: a warp factors the 32 x 32 diagonal piece, one
-// thread per row solves the rows below, then all threads update the rest.
-constexpr int SP = NB + 1;  // padded row stride in shared memory
+// The 128 columns are done in sub-panels of 32:
+//   (a) one warp factors the 32 x 32 diagonal piece with a row per lane in
+//       registers (pivot and column broadcast by shuffles);
+//   (b) one thread per row below solves x L^T = a with the row in registers;
+//   (c) all threads apply the sub-panel to the rest of the block in 4 x 4
+//       register tiles.
+// The inverse: each warp inverts one 32 x 32 diagonal block (a column per
+// lane), then X_ij = -X_ii (sum_k L_ik X_kj) for the blocks below, one
+// diagonal band at a time.
+constexpr int SP = NB + 1;  // padded row stride in shared memory (bank-conflict free columns)
+
+// Column J of the warp's 32 x 32 Cholesky (lane = row, w = the row), unrolled
+// by template recursion so every register index is a constant.
+template <int J>
+__device__ __forceinline__ void chol32_column(float (&w)[32], float &my_rd, int lane, int64_t col0,
+                                              int nb_left, int *status) {
+  if constexpr (J < 32) {
+    float piv = __shfl_sync(0xffffffffu, w[J], J);
+    if (!(piv > 0.0f) || !(piv < FLT_MAX)) {
+      if (lane == 0 && J < nb_left) atomicMin(&status[1], static_cast<int>(col0 + J));
+      piv = 1.0f;
+    }
+    const float dj = __fsqrt_rn(piv);
+    const float rj = __fdiv_rn(1.0f, dj);
+    const float lij = lane > J ? w[J] * rj : (lane == J ? dj : 0.0f);
+    w[J] = lij;
+    if (lane == J) my_rd = rj;
+#pragma unroll
+    for (int k = J + 1; k < 32; ++k) {
+      const float lkj = __shfl_sync(0xffffffffu, lij, k);
+      if (k <= lane) w[k] = fmaf(-lij, lkj, w[k]);
+    }
+    chol32_column<J + 1>(w, my_rd, lane, col0, nb_left, status);
+  }
+}
+constexpr int TP = 33;      // stride of the 32 x 32 temporaries
+constexpr size_t POTRF_SMEM = (2 * NB * SP + NB + 3 * 32 * TP) * sizeof(float);
 
 __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A, int64_t d,
                                                           int64_t k0, int nb,
                                                           float *__restrict__ linv,
                                                           int *status) {
   extern __shared__ float sm[];
-  float *S = sm;             // [NB][SP]  the block, then L
-  float *Li = sm + NB * SP;  // [NB][SP]  L^-1
+  float *S = sm;                // [NB][SP]  the block, then L (lower)
+  float *Li = S + NB * SP;      // [NB][SP]  L^-1 (lower)
+  float *rd = Li + NB * SP;     // [NB]      1 / L_jj
+  float *T = rd + NB;           // [3][32][TP] temporaries of the inverse
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int e = tid; e < NB * NB; e += 256) {
-    const int r = e / NB, c = e % NB;
-    S[r * SP + c] = (r < nb && c <= r) ? A[(k0 + r) * d + k0 + c] : (r == c ? 1.0f : 0.0f);
+  // the block's lower part, 16 float4 loads per thread in flight at once;
+  // identity padding past the matrix edge (only the lower part is ever read)
+  {
+    float4 v[NB * NB / 4 / 256];
+#pragma unroll
+    for (int u = 0; u < NB * NB / 4 / 256; ++u) {
+      const int idx = tid + 256 * u;
+      const int r = idx >> 5, c = (idx & 31) * 4;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nb && c < nb && c <= r)
+        v[u] = *reinterpret_cast<const float4 *>(A + (k0 + r) * d + k0 + c);
+    }
+#pragma unroll
+    for (int u = 0; u < NB * NB / 4 / 256; ++u) {
+      const int idx = tid + 256 * u;
+      const int r = idx >> 5, c = (idx & 31) * 4;
+      const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float x = e[q];
+        if (r >= nb) x = (r == c + q) ? 1.0f : 0.0f;
+        S[r * SP + c + q] = x;
+        Li[r * SP + c + q] = 0.0f;
+      }
+    }
   }
   __syncthreads();
+
   for (int c0 = 0; c0 < NB; c0 += 32) {
+    // (a) diagonal 32 x 32 piece
     if (warp == 0) {
-      const int r = c0 + lane;
-      for (int j = 0; j < 32; ++j) {
-        const int cj = c0 + j;
-        float piv = S[cj * SP + cj];
-        if (!(piv > 0.0f) || !(piv < FLT_MAX)) {
-          if (lane == 0 && cj < nb) atomicMin(&status[1], static_cast<int>(k0 + cj));
-          piv = 1.0f;
-        }
-        const float dj = __fsqrt_rn(piv);
-        __syncwarp();
-        if (lane == j) S[cj * SP + cj] = dj;
-        if (lane > j) S[r * SP + cj] = __fdiv_rn(S[r * SP + cj], dj);
-        __syncwarp();
-        if (lane > j) {
-          const float lrj = S[r * SP + cj];
-          for (int k = j + 1; k <= lane; ++k) S[r * SP + c0 + k] -= lrj * S[(c0 + k) * SP + cj];
-        }
-        __syncwarp();
-      }
+      float w[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) w[k] = (k <= lane) ? S[(c0 + lane) * SP + c0 + k] : 0.0f;
+      float my_rd = 1.0f;
+      chol32_column<0>(w, my_rd, lane, k0 + c0, nb - c0, status);
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        if (k <= lane) S[(c0 + lane) * SP + c0 + k] = w[k];
+      rd[c0 + lane] = my_rd;
     }
     __syncthreads();
-    // rows below: x L_dd^T = a  (forward substitution per row)
+    // (b) rows below the piece: x = a L_dd^-T, right-looking within the row
     for (int r = c0 + 32 + tid; r < NB; r += 256) {
-      float x[32];
+      float a[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) a[k] = S[r * SP + c0 + k];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float v = S[r * SP + c0 + j];
-        for (int k = 0; k < j; ++k) v -= x[k] * S[(c0 + j) * SP + c0 + k];
-        x[j] = __fdiv_rn(v, S[(c0 + j) * SP + c0 + j]);
+        const float x = a[j] * rd[c0 + j];
+        a[j] = x;
+#pragma unroll
+        for (int k = j + 1; k < 32; ++k) a[k] = fmaf(-x, S[(c0 + k) * SP + c0 + j], a[k]);
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) S[r * SP + c0 + j] = x[j];
+      for (int k = 0; k < 32; ++k) S[r * SP + c0 + k] = a[k];
     }
     __syncthreads();
-    // trailing update of the rest of the block
+    // (c) rest of the block: S[i][k] -= sum_j S[i][c0+j] S[k][c0+j], base <= k <= i
     const int base = c0 + 32;
-    const int m = NB - base;
-    for (int e = tid; e < m * m; e += 256) {
-      const int i = base + e / m, k = base + e % m;
-      if (k > i) continue;
-      float acc = S[i * SP + k];
+    const int mt = (NB - base) / 4;  // 4 x 4 tiles per side
+    const int n_tiles = mt * (mt + 1) / 2;
+    for (int t = tid; t < n_tiles; t += 256) {
+      int ti = 0;
+      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+      const int tk = t - ti * (ti + 1) / 2;
+      const int i0 = base + 4 * ti, kk0 = base + 4 * tk;
+      float acc[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
 #pragma unroll 8
-      for (int j = 0; j < 32; ++j) acc -= S[i * SP + c0 + j] * S[k * SP + c0 + j];
-      S[i * SP + k] = acc;
+      for (int j = 0; j < 32; ++j) {
+        float pi[4], pk[4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          pi[a] = S[(i0 + a) * SP + c0 + j];
+          pk[a] = S[(kk0 + a) * SP + c0 + j];
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(pi[a], pk[b], acc[a][b]);
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          if (kk0 + b <= i0 + a) S[(i0 + a) * SP + kk0 + b] -= acc[a][b];
     }
     __syncthreads();
   }
-  // L^-1 by forward substitution, one column per thread
-  if (tid < NB) {
-    const int c = tid;
-    for (int r = 0; r < NB; ++r) {
-      float v = (r == c) ? 1.0f : 0.0f;
-      if (r >= c) {
-        for (int k = c; k < r; ++k) v -= S[r * SP + k] * Li[k * SP + c];
-        v = __fdiv_rn(v, S[r * SP + r]);
-      } else {
-        v = 0.0f;
-      }
-      Li[r * SP + c] = v;
+
+  // inverse, diagonal blocks: warp q, lane = column
+  if (warp < 4) {
+    const int q0 = 32 * warp;
+    float v[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) v[r] = (r == lane) ? 1.0f : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float x = v[j] * rd[q0 + j];
+      v[j] = x;
+#pragma unroll
+      for (int r = j + 1; r < 32; ++r) v[r] = fmaf(-S[(q0 + r) * SP + q0 + j], x, v[r]);
     }
+#pragma unroll
+    for (int r = 0; r < 32; ++r) Li[(q0 + r) * SP + q0 + lane] = v[r];
   }
   __syncthreads();
+  // bands below the diagonal: X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj, i - j = lvl
+  // (each thread: one row r, four consecutive columns 4*c4 .. 4*c4+3)
+  for (int lvl = 1; lvl < 4; ++lvl) {
+    const int nblk = 4 - lvl;
+    for (int e = tid; e < nblk * 256; e += 256) {
+      const int b = e >> 8, r = (e >> 3) & 31, c = (e & 7) * 4;
+      const int j = b, i = b + lvl;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      const float *srow = S + (32 * i + r) * SP;
+#pragma unroll 4
+      for (int k = 32 * j; k < 32 * i; ++k) {
+        const float l = srow[k];
+        const float *x = Li + k * SP + 32 * j + c;
+        a0 = fmaf(l, x[0], a0);
+        a1 = fmaf(l, x[1], a1);
+        a2 = fmaf(l, x[2], a2);
+        a3 = fmaf(l, x[3], a3);
+      }
+      float *t = T + (b * 32 + r) * TP + c;
+      t[0] = a0; t[1] = a1; t[2] = a2; t[3] = a3;
+    }
+    __syncthreads();
+    for (int e = tid; e < nblk * 256; e += 256) {
+      const int b = e >> 8, r = (e >> 3) & 31, c = (e & 7) * 4;
+      const int j = b, i = b + lvl;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      const float *xrow = Li + (32 * i + r) * SP + 32 * i;
+      for (int k = 0; k <= r; ++k) {
+        const float xv = xrow[k];
+        const float *t = T + (b * 32 + k) * TP + c;
+        a0 = fmaf(xv, t[0], a0);
+        a1 = fmaf(xv, t[1], a1);
+        a2 = fmaf(xv, t[2], a2);
+        a3 = fmaf(xv, t[3], a3);
+      }
+      float *o = Li + (32 * i + r) * SP + 32 * j + c;
+      o[0] = -a0; o[1] = -a1; o[2] = -a2; o[3] = -a3;
+    }
+    __syncthreads();
+  }
+
   for (int e = tid; e < NB * NB; e += 256) {
     const int r = e / NB, c = e % NB;
     if (r < nb && c <= r) A[(k0 + r) * d + k0 + c] = S[r * SP + c];
@@ -406,7 +525,7 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
     const gq_status s = check_launch("damp/gather");
     if (s != GQ_OK) return s;
   }
-  const size_t pot_smem = 2 * NB * SP * sizeof(float);
+  const size_t pot_smem = POTRF_SMEM;
   cudaFuncSetAttribute(potrf_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(pot_smem));
   const int64_t n_panels = (d + NB - 1) / NB;

@@ -200,10 +200,18 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
     row_params_kernel<<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros);
     count_launch();
   }
+  int *status = static_cast<int *>(ws);
+  if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
+  CUtensorMap tmU;
+  {
+    const gq_status s = make_tmap_2d(&tmU, U, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d_in, d_in,
+                                     d_in, B, B, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (s != GQ_OK) return s;
+  }
   for (int64_t c0 = 0; c0 < d_in; c0 += B) {
     const int bw = static_cast<int>(d_in - c0 < B ? d_in - c0 : B);
-    blk(w.Wk, d_out, d_in, c0, bw, U, sym, w.Err, perm ? nullptr : qpacked, w.codes, scales,
-        zeros, n_groups, st);
+    blk(tmU, w.Wk, d_out, d_in, c0, bw, sym, w.Err, perm ? nullptr : qpacked, w.codes, scales,
+        zeros, n_groups, status, st);
     const int64_t c1 = c0 + bw;
     if (c1 < d_in)
       trailing_update_sgemm(static_cast<int>(d_out), static_cast<int>(d_in - c1), bw, w.Err, B,

@@ -1,17 +1,24 @@
 // The GPTQ column-block kernel ("GPTQ: Post-Training INT4", "The GPTQ
 // Algorithm": the loop over the columns of one block of B columns).
 //
-// One output row per thread.  The row's B weights stay in registers for the
-// whole block; the B x B block of U is in shared memory and every thread
-// reads the same element at the same time (broadcast, no bank conflicts).
-// The column loop is unrolled by template recursion so that every register
-// index is a compile-time constant (a plain loop of this size is not fully
-// unrolled and would put the weights in local memory).
+// One output row per thread.  The block's columns are taken in sub-blocks
+// of SB (32, or 64 when the group size is 64): the SB current weights of the
+// row live in registers; the updates that the block's earlier columns owe
+// them are applied first by a compact loop over those columns (their scaled
+// errors delta are kept in shared memory, one column of a [B][rows] array
+// per thread, so the accesses are conflict free); then the SB columns are
+// quantised one after another with the in-sub-block updates in registers.
+// Only the SB-step loop is unrolled (by template recursion, so every
+// register index is a constant): the kernel's code stays small enough for
+// the instruction cache, which a fully unrolled 128-step loop is not.
+// The B x B block of U is in shared memory (one TMA copy); every thread
+// reads the same element at the same time (broadcast).
 //
 // Column j:  group start -> scale (and zero) from the current weights of
-//            the group (a warp-free register reduction over G values);
-//            c = code(w_j), q = s (c - z), delta = (w_j - q) / U_jj;
-//            w_k -= delta * U_jk for k > j;  w_j := delta (the Err entry).
+//            the group; c = code(w_j), q = s (c - z), delta = (w_j - q) /
+//            U_jj; w_k -= delta * U_jk for k > j;  w_j := delta (the Err
+//            entry).  Divisions use a correctly rounded reciprocal and one
+//            FMA correction.
 #pragma once
 
 #include "gq_device.cuh"
@@ -19,23 +26,24 @@
 
 namespace gq {
 
-constexpr int GPTQ_ROWS_PER_CTA = 64;
-
-template <int B, int G>
-struct BlockCtx {
-  const float *Ub;
-  int bw;
+struct SubCtx {
+  const float *Ub;   // [B][B]
+  const float *rU;   // [B]  RN(1 / U_jj)
+  float *D;          // [B][rows] scaled errors of this block
+  int B, rows, tid, bw;
   bool sym;
   int64_t row, c0, n_groups;
   uint16_t *scales, *zeros;
 };
 
-template <int B, int G, int J>
-__device__ __forceinline__ void gptq_column(float (&w)[B], uint32_t (&packed)[B / 8],
-                                            GridParams &gp, const BlockCtx<B, G> &cx) {
-  if constexpr (J < B) {
-    if (J < cx.bw) {
-      if constexpr (G > 0 && J % G == 0) {
+template <int SB, int G, int J>
+__device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[SB / 8],
+                                            GridParams &gp, float &rs, const SubCtx &cx,
+                                            int jb) {
+  if constexpr (J < SB) {
+    const int j = jb + J;  // column within the block
+    if (j < cx.bw) {
+      if constexpr (G > 0 && G <= SB && J % G == 0) {
         float amax = 0.0f, mn = 0.0f, mx = 0.0f;
 #pragma unroll
         for (int k = J; k < J + G; ++k) {
@@ -44,115 +52,169 @@ __device__ __forceinline__ void gptq_column(float (&w)[B], uint32_t (&packed)[B 
           mx = fmaxf(mx, w[k]);
         }
         gp = cx.sym ? grid_sym(amax) : grid_affine(mn, mx);
-        const int64_t gi = (cx.c0 + J) / G;
+        rs = __fdiv_rn(1.0f, gp.s);
+        const int64_t gi = (cx.c0 + j) / G;
         cx.scales[cx.row * cx.n_groups + gi] = gp.s_bits;
         if (cx.zeros) cx.zeros[cx.row * cx.n_groups + gi] = cx.sym ? 0 : gp.z_bits;
       }
-      const float c = grid_code(w[J], gp, cx.sym);
+      const float *urow = cx.Ub + j * cx.B + jb;
+      const float c = grid_code_r(w[J], gp, rs, cx.sym);
       const float q = gp.s * (c - gp.z);
-      const float delta = __fdiv_rn(w[J] - q, cx.Ub[J * B + J]);
+      const float delta = div_by_recip(w[J] - q, urow[J], cx.rU[j]);
       packed[J / 8] |= grid_nibble(c, cx.sym) << (4 * (J % 8));
 #pragma unroll
-      for (int k = J + 1; k < B; ++k) w[k] = fmaf(-delta, cx.Ub[J * B + k], w[k]);
+      for (int k = J + 1; k < SB; ++k) w[k] = fmaf(-delta, urow[k], w[k]);
       w[J] = delta;
+      cx.D[j * cx.rows + cx.tid] = delta;
     }
-    gptq_column<B, G, J + 1>(w, packed, gp, cx);
+    gptq_column<SB, G, J + 1>(w, packed, gp, rs, cx, jb);
   }
 }
 
 // Wk: fp32 working weights [d_out][d_in] (processing order); the block is
 // columns c0 .. c0+bw-1.  Writes Err [d_out][B], and either the packed
 // codes (qpacked, no act-order) or one code byte per column (codes).
+// The B x B block of U arrives by one TMA copy (entries past the matrix
+// edge read as zero; only the upper triangle is used).
 template <int B, int G>
-__global__ void __launch_bounds__(GPTQ_ROWS_PER_CTA) gptq_block_kernel(
-    const float *__restrict__ Wk, int64_t d_out, int64_t d_in, int64_t c0, int bw,
-    const float *__restrict__ U, int sym, float *__restrict__ Err,
+__global__ void __launch_bounds__(128) gptq_block_kernel(
+    const __grid_constant__ CUtensorMap tmU, const float *__restrict__ Wk, int64_t d_out,
+    int64_t d_in, int64_t c0, int bw, int sym, float *__restrict__ Err,
     uint32_t *__restrict__ qpacked, uint8_t *__restrict__ codes, uint16_t *__restrict__ scales,
-    uint16_t *__restrict__ zeros, int64_t n_groups) {
-  extern __shared__ __align__(16) float Ub[];  // [B][B], upper triangle of the block
-  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
-    const int r = e / B, c = e % B;
-    Ub[e] = (r < bw && c < bw && c >= r) ? U[(c0 + r) * d_in + c0 + c] : 0.0f;
+    uint16_t *__restrict__ zeros, int64_t n_groups, int *status) {
+  constexpr int SB = (G == 64) ? 64 : 32;
+  static_assert(B % SB == 0, "sub-block must divide the block");
+  extern __shared__ __align__(128) float Ub[];  // [B][B], rU[B], D[B][rows], mbarrier
+  const int rows = blockDim.x, tid = threadIdx.x;
+  float *rU = Ub + B * B;
+  float *D = rU + B;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(D + B * rows);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
   }
   __syncthreads();
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, B * B * sizeof(float));
+    tma_load_2d(Ub, &tmU, bar, static_cast<int32_t>(c0), static_cast<int32_t>(c0));
+  }
+  if (!mbar_wait(bar, 0)) {
+    if (tid == 0) set_status(status, kDevTimeout);
+    return;
+  }
+  for (int j = tid; j < B; j += rows) rU[j] = j < bw ? __fdiv_rn(1.0f, Ub[j * B + j]) : 1.0f;
+  __syncthreads();
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows + tid;
   if (row >= d_out) return;
 
-  float w[B];
-  const float *src = Wk + row * d_in + c0;
-#pragma unroll
-  for (int k = 0; k < B; k += 4) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (k < bw) v = *reinterpret_cast<const float4 *>(src + k);
-    w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
-  }
   const bool s = sym != 0;
+  const float *src = Wk + row * d_in + c0;
   GridParams gp{};
+  float rs = 1.0f;
   if (G < 0) {  // per-channel scale, computed once from the initial row
     gp.s = __half2float(__ushort_as_half(scales[row]));
     gp.z = s ? 0.0f : __half2float(__ushort_as_half(zeros[row]));
+    rs = __fdiv_rn(1.0f, gp.s);
+  } else if (G == B) {  // one group per block: its first column sees the initial values
+    float amax = 0.0f, mn = 0.0f, mx = 0.0f;
+    for (int k = 0; k < bw; k += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src + k);
+      amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
+      mn = fminf(fminf(mn, fminf(v.x, v.y)), fminf(v.z, v.w));
+      mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+    }
+    gp = s ? grid_sym(amax) : grid_affine(mn, mx);
+    rs = __fdiv_rn(1.0f, gp.s);
+    scales[row * n_groups + c0 / B] = gp.s_bits;
+    if (zeros) zeros[row * n_groups + c0 / B] = s ? 0 : gp.z_bits;
   }
-  uint32_t packed[B / 8];
-#pragma unroll
-  for (int i = 0; i < B / 8; ++i) packed[i] = 0;
-  const BlockCtx<B, G> cx{Ub, bw, s, row, c0, n_groups, scales, zeros};
-  gptq_column<B, G, 0>(w, packed, gp, cx);
+  const SubCtx cx{Ub, rU, D, B, rows, tid, bw, s, row, c0, n_groups, scales, zeros};
+  constexpr int GS = (G == B) ? -1 : G;  // group handled above when it spans the block
 
-  float *err = Err + row * B;
+  for (int jb = 0; jb < bw; jb += SB) {
+    float w[SB];
 #pragma unroll
-  for (int k = 0; k < B; k += 4)
-    *reinterpret_cast<float4 *>(err + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
-  if (qpacked) {
-    uint32_t *dst = qpacked + row * (d_in / 8) + c0 / 8;
+    for (int k = 0; k < SB; k += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (jb + k < bw) v = *reinterpret_cast<const float4 *>(src + jb + k);
+      w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
+    }
+    // updates owed by the block's earlier columns
+    for (int j = 0; j < jb; ++j) {
+      const float dj = D[j * rows + tid];
+      const float *u = Ub + j * B + jb;
 #pragma unroll
-    for (int i = 0; i < B / 8; ++i)
-      if (i * 8 < bw) dst[i] = packed[i];
-  } else {
-    uint8_t *dst = codes + row * d_in + c0;
-#pragma unroll
-    for (int i = 0; i < B / 8; ++i)
-      if (i * 8 < bw) {
-        uint2 v;
-        v.x = (packed[i] & 0xFu) | ((packed[i] >> 4) & 0xFu) << 8 |
-              ((packed[i] >> 8) & 0xFu) << 16 | ((packed[i] >> 12) & 0xFu) << 24;
-        v.y = ((packed[i] >> 16) & 0xFu) | ((packed[i] >> 20) & 0xFu) << 8 |
-              ((packed[i] >> 24) & 0xFu) << 16 | ((packed[i] >> 28) & 0xFu) << 24;
-        *reinterpret_cast<uint2 *>(dst + i * 8) = v;
+      for (int k = 0; k < SB; k += 4) {
+        const float4 uv = *reinterpret_cast<const float4 *>(u + k);
+        w[k] = fmaf(-dj, uv.x, w[k]);
+        w[k + 1] = fmaf(-dj, uv.y, w[k + 1]);
+        w[k + 2] = fmaf(-dj, uv.z, w[k + 2]);
+        w[k + 3] = fmaf(-dj, uv.w, w[k + 3]);
       }
+    }
+    uint32_t packed[SB / 8];
+#pragma unroll
+    for (int i = 0; i < SB / 8; ++i) packed[i] = 0;
+    gptq_column<SB, GS, 0>(w, packed, gp, rs, cx, jb);
+
+    float *err = Err + row * B + jb;
+#pragma unroll
+    for (int k = 0; k < SB; k += 4)
+      *reinterpret_cast<float4 *>(err + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+    if (qpacked) {
+      uint32_t *dst = qpacked + row * (d_in / 8) + (c0 + jb) / 8;
+#pragma unroll
+      for (int i = 0; i < SB / 8; ++i)
+        if (jb + i * 8 < bw) dst[i] = packed[i];
+    } else {
+      uint8_t *dst = codes + row * d_in + c0 + jb;
+#pragma unroll
+      for (int i = 0; i < SB / 8; ++i)
+        if (jb + i * 8 < bw) {
+          uint2 v;
+          v.x = (packed[i] & 0xFu) | ((packed[i] >> 4) & 0xFu) << 8 |
+                ((packed[i] >> 8) & 0xFu) << 16 | ((packed[i] >> 12) & 0xFu) << 24;
+          v.y = ((packed[i] >> 16) & 0xFu) | ((packed[i] >> 20) & 0xFu) << 8 |
+                ((packed[i] >> 24) & 0xFu) << 16 | ((packed[i] >> 28) & 0xFu) << 24;
+          *reinterpret_cast<uint2 *>(dst + i * 8) = v;
+        }
+    }
   }
 }
 
-typedef void (*GptqBlockLaunch)(const float *, int64_t, int64_t, int64_t, int, const float *,
-                                int, float *, uint32_t *, uint8_t *, uint16_t *, uint16_t *,
-                                int64_t, cudaStream_t);
+typedef gq_status (*GptqBlockLaunch)(const CUtensorMap &, const float *, int64_t, int64_t,
+                                     int64_t, int, int, float *, uint32_t *, uint8_t *,
+                                     uint16_t *, uint16_t *, int64_t, int *, cudaStream_t);
 
+// tmU: fp32 tensor map over U with a B x B box and no swizzle.  Rows per
+// CTA shrink for short layers so that more SMs take part.
 template <int B, int G>
-void launch_gptq_block(const float *Wk, int64_t d_out, int64_t d_in, int64_t c0, int bw,
-                       const float *U, int sym, float *Err, uint32_t *qp, uint8_t *codes,
-                       uint16_t *scales, uint16_t *zeros, int64_t n_groups, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(B) * B * sizeof(float);
+gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_out,
+                            int64_t d_in, int64_t c0, int bw, int sym, float *Err,
+                            uint32_t *qp, uint8_t *codes, uint16_t *scales, uint16_t *zeros,
+                            int64_t n_groups, int *status, cudaStream_t st) {
+  const int sms = num_sms();
+  const int rows = d_out >= 4 * 128 * sms ? 128 : (d_out >= 2 * 64 * sms ? 64 : 32);
+  const size_t smem = (static_cast<size_t>(B) * (B + 1) + static_cast<size_t>(B) * rows) *
+                          sizeof(float) + 16;
   cudaFuncSetAttribute(gptq_block_kernel<B, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(smem));
-  const unsigned grid =
-      static_cast<unsigned>((d_out + GPTQ_ROWS_PER_CTA - 1) / GPTQ_ROWS_PER_CTA);
-  gptq_block_kernel<B, G><<<grid, GPTQ_ROWS_PER_CTA, smem, st>>>(
-      Wk, d_out, d_in, c0, bw, U, sym, Err, qp, codes, scales, zeros, n_groups);
+  const unsigned grid = static_cast<unsigned>((d_out + rows - 1) / rows);
+  gptq_block_kernel<B, G><<<grid, rows, smem, st>>>(tmU, Wk, d_out, d_in, c0, bw, sym, Err, qp,
+                                                    codes, scales, zeros, n_groups, status);
   count_launch();
+  return GQ_OK;
 }
 
 // Instantiated in gptq_b*.cu (one translation unit each, compiled in parallel).
 #define GQ_GPTQ_BLOCK_INSTANCES(X) \
   X(128, -1) X(128, 128) X(128, 64) X(128, 32) X(64, -1) X(64, 64) X(64, 32) X(32, -1) X(32, 32)
 
-#define GQ_DECLARE_BLOCK(b, g)                                                               \
-  extern template void launch_gptq_block<b, g>(const float *, int64_t, int64_t, int64_t, int, \
-                                               const float *, int, float *, uint32_t *,       \
-                                               uint8_t *, uint16_t *, uint16_t *, int64_t,    \
-                                               cudaStream_t);
-#define GQ_DEFINE_BLOCK(b, g)                                                         \
-  template void launch_gptq_block<b, g>(const float *, int64_t, int64_t, int64_t, int, \
-                                        const float *, int, float *, uint32_t *,       \
-                                        uint8_t *, uint16_t *, uint16_t *, int64_t,    \
-                                        cudaStream_t);
+#define GQ_BLOCK_SIG(b, g)                                                                  \
+  gq_status launch_gptq_block<b, g>(const CUtensorMap &, const float *, int64_t, int64_t,      \
+                                    int64_t, int, int, float *, uint32_t *, uint8_t *,         \
+                                    uint16_t *, uint16_t *, int64_t, int *, cudaStream_t);
+#define GQ_DECLARE_BLOCK(b, g) extern template GQ_BLOCK_SIG(b, g)
+#define GQ_DEFINE_BLOCK(b, g) template GQ_BLOCK_SIG(b, g)
 
 }  // namespace gq

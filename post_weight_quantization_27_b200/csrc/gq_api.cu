@@ -60,7 +60,7 @@ static EncodeTiledFn encode_fn() {
 
 gq_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt,
                        size_t elem_bytes, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
-                       uint32_t box_inner, uint32_t box_outer) {
+                       uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(GQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {inner, outer};
@@ -68,7 +68,7 @@ gq_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType d
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(GQ_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   return GQ_OK;
@@ -217,7 +217,7 @@ gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out,
     return fail(GQ_ERR_ARG, "block_size must be 32, 64 or 128");
   if (group_size != -1 && (group_size < 32 || block_size % group_size != 0))
     return fail(GQ_ERR_ARG, "GPTQ group_size must be -1, 32, 64 or 128 and divide block_size");
-  if (!aligned(W, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
+  if (!aligned(W, 16) || !aligned(U, 16)) return fail(GQ_ERR_ARG, "W and U must be 16-byte aligned");
   GQ_TRY(check_ws(ws, ws_bytes, gptq_ws_bytes(d_out, d_in, block_size)));
   return launch_gptq(W, w_dtype, d_out, d_in, U, group_size, block_size, sym, perm, dead,
                      qpacked, scales, zeros, g_idx, ws, static_cast<cudaStream_t>(stream));

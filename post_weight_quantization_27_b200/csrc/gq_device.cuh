@@ -214,6 +214,22 @@ __device__ __forceinline__ float grid_code(float w, const GridParams &g, bool sy
   float c = __fadd_rn(rintf(__fdiv_rn(w, g.s)), g.z);
   return sym ? fminf(fmaxf(c, -7.0f), 7.0f) : fminf(fmaxf(c, 0.0f), 15.0f);
 }
+// Correctly rounded fp32 quotient a / b given r = RN(1 / b): q0 = RN(a r) is
+// within one ulp of a / b, and one FMA correction q0 + r (a - b q0) gives the
+// round-to-nearest quotient (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990).  Used where the divisor is fixed for many quotients; checked
+// against __fdiv_rn by the GPTQ == RTN tests on diagonal Hessians.
+__device__ __forceinline__ float div_by_recip(float a, float b, float r) {
+  const float q0 = __fmul_rn(a, r);
+  const float e = __fmaf_rn(-q0, b, a);
+  return __fmaf_rn(e, r, q0);
+}
+// Code of w with the group's reciprocal scale rs = RN(1 / s).
+__device__ __forceinline__ float grid_code_r(float w, const GridParams &g, float rs, bool sym) {
+  float c = __fadd_rn(rintf(div_by_recip(w, g.s, rs)), g.z);
+  return sym ? fminf(fmaxf(c, -7.0f), 7.0f) : fminf(fmaxf(c, 0.0f), 15.0f);
+}
 // Stored nibble of a code.
 __device__ __forceinline__ uint32_t grid_nibble(float c, bool sym) {
   return static_cast<uint32_t>(static_cast<int>(c) + (sym ? 8 : 0)) & 0xFu;

@@ -30,7 +30,8 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // `pitch_elems` elements; box of box_inner x box_outer.
 gq_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt,
                        size_t elem_bytes, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
-                       uint32_t box_inner, uint32_t box_outer);
+                       uint32_t box_inner, uint32_t box_outer,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 
 int num_sms();
 

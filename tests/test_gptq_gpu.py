@@ -150,3 +150,29 @@ def test_gptq_workload_layers(workload, idx):
     Wn, Xn = W.float().numpy(), X.float().numpy()
     check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=spec.group_size, sym=spec.sym,
                                            follow=f)[0], spec.d_in, spec.sym)
+
+
+def test_gptq_division_matches_ieee_at_midpoints():
+    """The column loop divides by a reciprocal plus one FMA correction; with
+    a diagonal Hessian GPTQ must still reproduce RTN (IEEE division) bit for
+    bit, on weights packed with exact rounding midpoints k + 1/2 of the
+    row's step and their fp32 neighbours."""
+    d_in, d_out = 512, 2048
+    g = torch.Generator().manual_seed(31)
+    W = torch.randn((d_out, d_in), generator=g) * 0.02
+    amax = W.abs().amax(1, keepdim=True)
+    s16 = (amax / 7).to(torch.float16).float()
+    k = torch.randint(-7, 7, (d_out, d_in), generator=g).float()
+    mid = (k + 0.5) * s16
+    pick = torch.randint(0, 4, (d_out, d_in), generator=g)
+    W = torch.where(pick == 0, mid, W)
+    W = torch.where(pick == 1, torch.nextafter(mid, torch.full_like(mid, 1e9)), W)
+    W = torch.where(pick == 2, torch.nextafter(mid, torch.full_like(mid, -1e9)), W)
+    W = torch.clamp(W, -amax, amax)
+    X = torch.zeros((d_in, d_in), dtype=torch.bfloat16)
+    X[torch.arange(d_in), torch.arange(d_in)] = torch.linspace(0.5, 2.0, d_in).to(torch.bfloat16)
+    for gs, sym in ((-1, True), (128, True), (64, False)):
+        out, _ = _run_gpu(W, X, gs, sym)
+        rtn = gq.rtn_quantize_pack(W.cuda(), 4, gs, sym)
+        torch.cuda.synchronize()
+        assert np.array_equal(u32(out["qpacked"]), u32(rtn["qpacked"])), (gs, sym)
