@@ -16,8 +16,9 @@
 // and factored in place; X = L^-1 is built in the H buffer (the caller's H
 // is scratch); the last kernel writes U = J X J back into the U buffer.
 // Blocked right-looking algorithms with 128-wide panels; one CTA factors a
-// diagonal block in shared memory, the panel solve and the trailing
-// updates run as tiled fp32 GEMMs over the whole GPU.
+// diagonal block in shared memory (and inverts it), the panel solve, the
+// trailing updates and the inverse's block steps are fp32 GEMMs on the
+// tensor cores (3 x TF32 split, gemm_tc.cu).
 #include <cfloat>
 #include <climits>
 #include <mutex>
@@ -152,8 +153,10 @@ __device__ __forceinline__ void chol32_column(float (&w)[32], float &my_rd, int 
       if (lane == 0 && J < nb_left) atomicMin(&status[1], static_cast<int>(col0 + J));
       piv = 1.0f;
     }
-    const float dj = __fsqrt_rn(piv);
-    const float rj = __fdiv_rn(1.0f, dj);
+    // 1 / sqrt(piv): hardware estimate plus one Newton step r (3 - piv r^2) / 2
+    float rj = rsqrtf(piv);
+    rj = rj * fmaf(-0.5f * piv, rj * rj, 1.5f);
+    const float dj = piv * rj;
     const float lij = lane > J ? w[J] * rj : (lane == J ? dj : 0.0f);
     w[J] = lij;
     if (lane == J) my_rd = rj;
@@ -337,129 +340,6 @@ __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A,
   }
 }
 
-// ---------------------------------------------------------------- SIMT GEMM
-// C[m][n] = beta * C[m][n] + alpha * sum_k A(m, k) B(k, n), fp32, tiles of
-// 128 x 128 x 8 with an 8 x 8 register block per thread.  A(m, k) =
-// A[m * lda + k]; B(k, n) = B_NT ? B[n * ldb + k] : B[k * ldb + n].  With
-// LOWER only the n <= m part of C is computed (tiles above the diagonal are
-// skipped).  K must be a multiple of 8.  In-place use (C overlapping A or
-// B) is safe when every tile reads all of its operands before its stores
-// and no other tile writes them.
-constexpr int GBM = 128, GBN = 128, GBK = 8;
-
-template <bool B_NT, bool LOWER>
-__global__ void __launch_bounds__(256) sgemm_kernel(int M, int N, int K, float alpha,
-                                                    const float *__restrict__ Am, int64_t lda,
-                                                    const float *__restrict__ Bm, int64_t ldb,
-                                                    float beta, float *Cm, int64_t ldc) {
-  const int tm = blockIdx.y * GBM, tn = blockIdx.x * GBN;
-  if (LOWER && tn > tm + GBM - 1) return;
-  __shared__ __align__(16) float As[2][GBK][GBM + 4];
-  __shared__ __align__(16) float Bs[2][GBK][GBN + 4];
-  const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-
-  // loader mapping: A: row = tid / 2, k = (tid % 2) * 4 (float4 along k)
-  const int la_r = tid >> 1, la_k = (tid & 1) * 4;
-  // B NT: same as A; B NN: k = tid / 32, n = (tid % 32) * 4
-  const int lb_r = B_NT ? (tid >> 1) : (tid >> 5);
-  const int lb_c = B_NT ? ((tid & 1) * 4) : ((tid & 31) * 4);
-  float4 ra, rb;
-  auto load = [&](int k0) {
-    const int am = tm + la_r;
-    ra = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (am < M) ra = *reinterpret_cast<const float4 *>(Am + am * lda + k0 + la_k);
-    rb = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (B_NT) {
-      const int bn = tn + lb_r;
-      if (bn < N) rb = *reinterpret_cast<const float4 *>(Bm + bn * ldb + k0 + lb_c);
-    } else {
-      const int bk = k0 + lb_r, bn = tn + lb_c;
-      const float *p = Bm + bk * ldb + bn;
-      if (bn + 3 < N) {
-        rb = *reinterpret_cast<const float4 *>(p);
-      } else {
-        rb.x = bn < N ? p[0] : 0.f;
-        rb.y = bn + 1 < N ? p[1] : 0.f;
-        rb.z = bn + 2 < N ? p[2] : 0.f;
-        rb.w = 0.f;
-      }
-    }
-  };
-  auto store = [&](int buf) {
-    As[buf][la_k + 0][la_r] = ra.x;
-    As[buf][la_k + 1][la_r] = ra.y;
-    As[buf][la_k + 2][la_r] = ra.z;
-    As[buf][la_k + 3][la_r] = ra.w;
-    if (B_NT) {
-      Bs[buf][lb_c + 0][lb_r] = rb.x;
-      Bs[buf][lb_c + 1][lb_r] = rb.y;
-      Bs[buf][lb_c + 2][lb_r] = rb.z;
-      Bs[buf][lb_c + 3][lb_r] = rb.w;
-    } else {
-      *reinterpret_cast<float4 *>(&Bs[buf][lb_r][lb_c]) = rb;
-    }
-  };
-  load(0);
-  store(0);
-  __syncthreads();
-  int buf = 0;
-  for (int k0 = 0; k0 < K; k0 += GBK) {
-    const bool more = k0 + GBK < K;
-    if (more) load(k0 + GBK);
-#pragma unroll
-    for (int kk = 0; kk < GBK; ++kk) {
-      float a[8], b[8];
-      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
-      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
-      a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
-      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
-      b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    if (more) {
-      store(buf ^ 1);
-      __syncthreads();
-      buf ^= 1;
-    }
-  }
-  // every tile has read all of its operands before any store below
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int m = tm + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-    if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int n = tn + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
-      if (n >= N || (LOWER && n > m)) continue;
-      float *c = Cm + m * ldc + n;
-      const float v = alpha * acc[i][j];
-      *c = beta == 0.0f ? v : fmaf(beta, *c, v);
-    }
-  }
-}
-
-template <bool B_NT, bool LOWER>
-void sgemm(int M, int N, int K, float alpha, const float *A, int64_t lda, const float *B,
-           int64_t ldb, float beta, float *C, int64_t ldc, cudaStream_t st) {
-  if (M <= 0 || N <= 0 || K <= 0) return;
-  dim3 grid((N + GBN - 1) / GBN, (M + GBM - 1) / GBM);
-  sgemm_kernel<B_NT, LOWER><<<grid, 256, 0, st>>>(M, N, K, alpha, A, lda, B, ldb, beta, C, ldc);
-  count_launch();
-}
-
 // X := I on the lower triangle and on the whole NB x NB diagonal blocks
 // (the right-hand side of L X = I); the rest of the upper part is never read.
 __global__ void __launch_bounds__(256) eye_lower_kernel(float *__restrict__ X, int64_t d) {
@@ -491,12 +371,6 @@ __global__ void finish_info_kernel(int *status, int64_t d, int32_t *info_dev) {
 }
 
 }  // namespace
-
-// W[:, end:] -= Err * U[blk, end:] for the GPTQ trailing update (fp32).
-void trailing_update_sgemm(int M, int N, int K, const float *Err, int64_t lde, const float *Urow,
-                           int64_t ldu, float *Wk, int64_t ldw, cudaStream_t st) {
-  sgemm<false, false>(M, N, K, -1.0f, Err, lde, Urow, ldu, 1.0f, Wk, ldw, st);
-}
 
 size_t chol_ws_bytes(int64_t d) {
   const int64_t n_panels = (d + NB - 1) / NB;
@@ -539,12 +413,15 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
     const int64_t k1 = k0 + nb;
     const int rest = static_cast<int>(d - k1);
     if (rest > 0) {
-      // panel rows below: A[k1:, k0:k1] := A[k1:, k0:k1] L_pp^-T
-      sgemm<true, false>(rest, nb, NB, 1.0f, A + k1 * d + k0, d, lp, NB, 0.0f, A + k1 * d + k0,
-                         d, st);
+      // panel rows below: A[k1:, k0:k1] := A[k1:, k0:k1] L_pp^-T (in place:
+      // each output tile owns its rows)
+      gq_status s = launch_gemm_tf32x3(rest, nb, NB, 1.0f, A + k1 * d + k0, d, lp, NB, true,
+                                       0.0f, A + k1 * d + k0, d, false, w.status, st);
+      if (s != GQ_OK) return s;
       // trailing: A[k1:, k1:] -= P P^T (lower part)
-      sgemm<true, true>(rest, rest, NB, -1.0f, A + k1 * d + k0, d, A + k1 * d + k0, d, 1.0f,
-                        A + k1 * d + k1, d, st);
+      s = launch_gemm_tf32x3(rest, rest, NB, -1.0f, A + k1 * d + k0, d, A + k1 * d + k0, d,
+                             true, 1.0f, A + k1 * d + k1, d, true, w.status, st);
+      if (s != GQ_OK) return s;
     }
   }
   // ---- X = L^-1 by blocked forward substitution on the identity
@@ -555,14 +432,18 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
     const int nb = static_cast<int>(d - r0 < NB ? d - r0 : NB);
     const int cols = static_cast<int>(r0 + nb);
     float *lp = w.linv + p * NB * NB;
-    // X[r0:r0+nb, 0:cols] := L_pp^-1 X[r0:r0+nb, 0:cols]
-    sgemm<false, false>(nb, cols, nb, 1.0f, lp, NB, X + r0 * d, d, 0.0f, X + r0 * d, d, st);
+    // X[r0:r0+nb, 0:cols] := L_pp^-1 X[r0:r0+nb, 0:cols] (in place: each
+    // output tile owns its columns)
+    gq_status s = launch_gemm_tf32x3(nb, cols, nb, 1.0f, lp, NB, X + r0 * d, d, false, 0.0f,
+                                     X + r0 * d, d, false, w.status, st);
+    if (s != GQ_OK) return s;
     const int64_t r1 = r0 + nb;
     const int rest = static_cast<int>(d - r1);
     if (rest > 0) {
       // X[r1:, 0:cols] -= L[r1:, r0:r1] X[r0:r1, 0:cols]
-      sgemm<false, false>(rest, cols, nb, -1.0f, A + r1 * d + r0, d, X + r0 * d, d, 1.0f,
-                          X + r1 * d, d, st);
+      s = launch_gemm_tf32x3(rest, cols, nb, -1.0f, A + r1 * d + r0, d, X + r0 * d, d, false,
+                             1.0f, X + r1 * d, d, false, w.status, st);
+      if (s != GQ_OK) return s;
     }
   }
   reverse_upper_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d, U);

@@ -1,0 +1,348 @@
+// fp32 GEMM on the tensor cores: C = beta C + alpha A B with fp32 A, B, C.
+//
+// Used for the GPTQ lazy trailing update W[:, end:] -= Err U[blk, end:]
+// ("GPTQ: Post-Training INT4" -- "The GPTQ Algorithm", block-wise
+// processing) and for the blocked Cholesky's panel solves and trailing
+// updates.  Those updates decide later rounding decisions, so they need
+// fp32-level accuracy: each operand element a is split into a TF32-exact
+// high part h = a with the low 13 mantissa bits cleared and the remainder
+// l = a - h (exact in fp32), and the product is h_a h_b + h_a l_b + l_a h_b
+// (three tcgen05.mma kind::tf32; the dropped l_a l_b and the TF32 rounding
+// of l are ~2^-20 relative).
+//
+// Persistent kernel, one CTA per SM, 128 x 128 output tiles, K in steps of
+// 32 (one 128-byte swizzle row of fp32):
+//   warp 0     TMA loads of the fp32 A and B tiles (no multicast)
+//   warps 2-5  split each staged element in place into h and l (l into a
+//              second buffer), then make the writes visible to the async
+//              proxy before releasing the stage to the MMA warp
+//   warp 1     three MMAs per 8-wide K step into one of two TMEM
+//              accumulators (the epilogue of one tile overlaps the next)
+//   warps 6-9  C = beta C + alpha acc from TMEM, one row per thread
+// A is K-major (A(m, k) = A[m lda + k]); B is either K-major (B(k, n) =
+// B[n ldb + k]) or N-major (B(k, n) = B[k ldb + n]); an N-major TF32 operand
+// must be staged with the 32-byte-atom variant of the 128-byte swizzle.  With `lower` only
+// tiles and elements with n <= m are computed and stored.
+#include "gq_device.cuh"
+#include "gq_internal.h"
+
+namespace gq {
+namespace {
+
+constexpr int TM = 128, TN = 128, TK = 32, STAGES = 3;
+constexpr int TILE_BYTES = TM * TK * 4;         // 16 KB, A or B tile
+constexpr int STAGE_BYTES = 4 * TILE_BYTES;     // A_h, A_l, B_h, B_l
+constexpr int NUM_THREADS = 320;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+
+struct TcArgs {
+  int M, N, K;
+  float alpha, beta;
+  float *C;
+  int64_t ldc;
+  int n_mt, n_nt, nkb, n_tiles;
+  int b_kmajor, lower;
+  int *status;
+};
+
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool b_mn) {
+  return (1u << 4)                     // D f32
+         | (2u << 7)                   // A tf32
+         | (2u << 10)                  // B tf32
+         | ((b_mn ? 1u : 0u) << 16)    // B major
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Tile t -> (mt, nt); lower: only nt <= mt, enumerated row by row.
+__device__ __forceinline__ void tile_of(const TcArgs &a, int t, int &mt, int &nt) {
+  if (!a.lower) {
+    mt = t % a.n_mt;
+    nt = t / a.n_mt;
+    return;
+  }
+  int r = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
+  while (r * (r + 1) / 2 > t) --r;
+  while ((r + 1) * (r + 2) / 2 <= t) ++r;
+  mt = r;
+  nt = t - r * (r + 1) / 2;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint64_t *full = bars;                  // TMA landed
+  uint64_t *split = bars + STAGES;        // h / l split done
+  uint64_t *empty = bars + 2 * STAGES;    // MMAs done with the stage
+  uint64_t *acc_full = bars + 3 * STAGES;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&split[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < a.n_tiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_of(a, t, mt, nt);
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], 2 * TILE_BYTES);
+          uint8_t *st = smem + s * STAGE_BYTES;
+          tma_load_2d(st, &tmA, &full[s], kb * TK, mt * TM);
+          if (a.b_kmajor) {
+            tma_load_2d(st + 2 * TILE_BYTES, &tmB, &full[s], kb * TK, nt * TN);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tma_load_2d(st + 2 * TILE_BYTES + q * (TILE_BYTES / 4), &tmB, &full[s],
+                          nt * TN + 32 * q, kb * TK);
+          }
+        }
+      }
+      const uint32_t n_wait = it < STAGES ? it : STAGES;
+      for (uint32_t k = 0; k < n_wait; ++k) {
+        const uint32_t j = it - 1 - k;
+        if (!mbar_wait(&full[j % STAGES], (j / STAGES) & 1)) ok = false;
+      }
+      if (!ok) set_status(a.status, kDevTimeout);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ---------------- h / l split of each staged tile
+    const int ct = threadIdx.x - 64;  // 0..127
+    bool ok = true;
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < a.n_tiles && ok; t += gridDim.x) {
+      for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+        const uint32_t s = it % STAGES, r = it / STAGES;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], r & 1));
+        if (!ok) break;
+        uint8_t *st = smem + s * STAGE_BYTES;
+#pragma unroll
+        for (int op = 0; op < 2; ++op) {
+          float4 *hp = reinterpret_cast<float4 *>(st + op * 2 * TILE_BYTES);
+          float4 *lp = reinterpret_cast<float4 *>(st + op * 2 * TILE_BYTES + TILE_BYTES);
+#pragma unroll
+          for (int i = 0; i < TILE_BYTES / 16 / 128; ++i) {
+            const int idx = ct + 128 * i;
+            float4 v = hp[idx];
+            float4 h, l;
+            h.x = __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
+            h.y = __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
+            h.z = __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
+            h.w = __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+            l.x = v.x - h.x;
+            l.y = v.y - h.y;
+            l.z = v.z - h.z;
+            l.w = v.w - h.w;
+            hp[idx] = h;
+            lp[idx] = l;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&split[s]);
+      }
+    }
+    if (!ok && lane == 0) set_status(a.status, kDevTimeout);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      uint32_t it = 0, ch = 0;
+      const uint32_t idesc = idesc_tf32(TM, TN, a.b_kmajor == 0);
+      for (int t = blockIdx.x; t < a.n_tiles && ok; t += gridDim.x, ++ch) {
+        const uint32_t buf = ch & 1, use = ch >> 1;
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * TN;
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const uint32_t s = it % STAGES, r = it / STAGES;
+          if (!mbar_wait(&split[s], r & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ah = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t al = ah + TILE_BYTES;
+          const uint32_t bh = ah + 2 * TILE_BYTES;
+          const uint32_t bl = ah + 3 * TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TK / 8; ++kk) {
+            // A: K-major, 8 fp32 = 32 bytes along the swizzled row
+            const uint64_t dah = smem_desc_sw128(ah + kk * 32, 16, 1024);
+            const uint64_t dal = smem_desc_sw128(al + kk * 32, 16, 1024);
+            uint64_t dbh, dbl;
+            if (a.b_kmajor) {
+              dbh = smem_desc_sw128(bh + kk * 32, 16, 1024);
+              dbl = smem_desc_sw128(bl + kk * 32, 16, 1024);
+            } else {
+              // N-major: 32-wide N chunks of 4 KB, 32-byte-atom swizzle,
+              // 4-row atoms of 512 bytes; 8 K rows per MMA = 1 KB
+              dbh = smem_desc_sw128(bh + kk * 1024, TILE_BYTES / 4, 512, kLayoutSw128Atom32);
+              dbl = smem_desc_sw128(bl + kk * 1024, TILE_BYTES / 4, 512, kLayoutSw128Atom32);
+            }
+            mma_tf32(d_tmem, dal, dbh, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_tf32(d_tmem, dah, dbl, idesc, 1u);
+            mma_tf32(d_tmem, dah, dbh, idesc, 1u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+      }
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) ok = false;
+      if (!ok) set_status(a.status, kDevTimeout);
+    }
+  } else {
+    // ---------------- epilogue: warps 6..9
+    const int quarter = warp & 3;
+    uint32_t ch = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++ch) {
+      int mt, nt;
+      tile_of(a, t, mt, nt);
+      const uint32_t buf = ch & 1, use = ch >> 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1));
+      if (!ok) break;
+      tc_fence_after();
+      const int m = mt * TM + quarter * 32 + lane;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * TN;
+      float *crow = a.C + static_cast<int64_t>(m) * a.ldc + nt * TN;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        if (m < a.M) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const int n = nt * TN + c * 32 + i;
+            if (n + 3 < a.N && (!a.lower || n + 3 <= m)) {
+              float4 *p = reinterpret_cast<float4 *>(crow + c * 32 + i);
+              float4 o = make_float4(a.alpha * v[i], a.alpha * v[i + 1], a.alpha * v[i + 2],
+                                     a.alpha * v[i + 3]);
+              if (a.beta != 0.0f) {
+                const float4 old = *p;
+                o.x = fmaf(a.beta, old.x, o.x);
+                o.y = fmaf(a.beta, old.y, o.y);
+                o.z = fmaf(a.beta, old.z, o.z);
+                o.w = fmaf(a.beta, old.w, o.w);
+              }
+              *p = o;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int ne = n + e;
+                if (ne < a.N && (!a.lower || ne <= m)) {
+                  float *p = crow + c * 32 + i + e;
+                  const float o = a.alpha * v[i + e];
+                  *p = a.beta != 0.0f ? fmaf(a.beta, *p, o) : o;
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+    if (!ok && lane == 0) set_status(a.status, kDevTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+// C (M x N, ldc) = beta C + alpha A B; see the file comment for layouts.
+// All pointers 16-byte aligned, lda / ldb / ldc multiples of 4.
+gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
+                             const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
+                             int64_t ldc, bool lower, int *status, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0) return GQ_OK;
+  CUtensorMap tA, tB;
+  gq_status s = make_tmap_2d(&tA, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K, M, lda, TK, TM);
+  if (s != GQ_OK) return s;
+  if (b_kmajor)
+    s = make_tmap_2d(&tB, B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K, N, ldb, TK, TN);
+  else
+    s = make_tmap_2d(&tB, B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, K, ldb, 32, TK,
+                     CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+  if (s != GQ_OK) return s;
+  TcArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.C = C;
+  a.ldc = ldc;
+  a.n_mt = (M + TM - 1) / TM;
+  a.n_nt = (N + TN - 1) / TN;
+  a.nkb = (K + TK - 1) / TK;
+  a.b_kmajor = b_kmajor ? 1 : 0;
+  a.lower = lower ? 1 : 0;
+  a.n_tiles = lower ? a.n_mt * (a.n_mt + 1) / 2 : a.n_mt * a.n_nt;
+  a.status = status;
+  cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(SMEM_BYTES));
+  const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();
+  gemm_tf32x3_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tA, tB, a);
+  count_launch();
+  return check_launch("gemm_tf32x3_kernel");
+}
+
+}  // namespace gq

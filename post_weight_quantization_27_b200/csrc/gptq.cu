@@ -15,7 +15,8 @@
 // broadcast shared-memory reads, with no shuffles and no synchronisation.
 // A processed weight's register is reused for its scaled error delta, so
 // the Err block leaves the kernel in one contiguous store per row.  The
-// trailing update is a GEMM of d_out x (d_in - end) x B.
+// trailing update is a d_out x (d_in - end) x B GEMM on the tensor cores
+// (gemm_tc.cu).
 #include "gptq_block.cuh"
 
 namespace gq {
@@ -155,10 +156,6 @@ GptqBlockLaunch pick_block(int B, int G) {
 
 }  // namespace
 
-// fp32 GEMM of chol.cu, reused for the trailing update.
-void trailing_update_sgemm(int M, int N, int K, const float *Err, int64_t lde, const float *Urow,
-                           int64_t ldu, float *Wk, int64_t ldw, cudaStream_t st);
-
 size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size) {
   return kWsHeader + round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256) +
          round_up(static_cast<size_t>(d_out) * block_size * sizeof(float), 256) +
@@ -213,9 +210,13 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
     blk(tmU, w.Wk, d_out, d_in, c0, bw, sym, w.Err, perm ? nullptr : qpacked, w.codes, scales,
         zeros, n_groups, status, st);
     const int64_t c1 = c0 + bw;
-    if (c1 < d_in)
-      trailing_update_sgemm(static_cast<int>(d_out), static_cast<int>(d_in - c1), bw, w.Err, B,
-                            U + c0 * d_in + c1, d_in, w.Wk + c1, d_in, st);
+    if (c1 < d_in) {
+      // W[:, c1:] -= Err U[c0:c1, c1:] on the tensor cores
+      const gq_status s = launch_gemm_tf32x3(static_cast<int>(d_out), static_cast<int>(d_in - c1),
+                                             bw, -1.0f, w.Err, B, U + c0 * d_in + c1, d_in,
+                                             false, 1.0f, w.Wk + c1, d_in, false, status, st);
+      if (s != GQ_OK) return s;
+    }
   }
   const unsigned gd = static_cast<unsigned>((d_in + 255) / 256);
   if (perm) {

@@ -110,15 +110,20 @@ __device__ __forceinline__ void tc_fence_after() {
 // groups of 8 rows along K; for a K-major tile sbo is the stride between
 // groups of 8 rows along M (or N) and lbo is unused (one swizzle atom
 // spans the whole 64-element K extent).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                                    uint32_t layout = 2) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)layout << 61;
   return d;
 }
+// Layout type 1: 128-byte swizzle with 32-byte atoms, the one layout the
+// tensor core accepts for MN-major 32-bit (TF32) operands; atoms are 4 rows
+// of 128 bytes, so sbo is the stride between groups of 4 K rows.
+constexpr uint32_t kLayoutSw128Atom32 = 1;
 
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B and an
 // fp32 accumulator; a_mn / b_mn select MN-major operands.

@@ -53,6 +53,11 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
                            uint8_t *dead_out, float *U, int32_t *info_dev, void *ws,
                            cudaStream_t st);
 
+// C = beta C + alpha A B in fp32 on the tensor cores (3 x TF32 split).
+gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
+                             const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
+                             int64_t ldc, bool lower, int *status, cudaStream_t st);
+
 size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size);
 gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,
                       int group_size, int block_size, int sym, const int32_t *perm,

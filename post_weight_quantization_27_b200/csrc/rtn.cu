@@ -56,10 +56,14 @@ struct Vec8<__nv_bfloat16> {
   }
 };
 
-__device__ __forceinline__ uint32_t pack_word(const float (&v)[8], const GridParams &g, bool sym) {
+// rs = RN(1 / s): the quotient w / s is formed as a correctly rounded
+// division from the reciprocal (gq_device.cuh), three instructions instead
+// of a full division per weight, so the kernel stays memory-bound.
+__device__ __forceinline__ uint32_t pack_word(const float (&v)[8], const GridParams &g, float rs,
+                                              bool sym) {
   uint32_t word = 0;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) word |= grid_nibble(grid_code(v[k], g, sym), sym) << (4 * k);
+  for (int k = 0; k < 8; ++k) word |= grid_nibble(grid_code_r(v[k], g, rs, sym), sym) << (4 * k);
   return word;
 }
 
@@ -78,9 +82,10 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
   const int64_t total = d_out * n_groups;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t words_per_row = d_in / 8;
   const bool s = sym != 0;
 
+  // segment s = row * n_groups + group; every segment starts seg_words * 8
+  // weights after the previous one, so its address needs no division
   for (int64_t base = warp * SPW * UNROLL; base < total; base += n_warps * SPW * UNROLL) {
     float v[UNROLL][WPL][8];
     bool act[UNROLL];
@@ -89,9 +94,7 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
     for (int u = 0; u < UNROLL; ++u) {
       seg[u] = base + u * SPW + lane / TEAM;
       act[u] = seg[u] < total;
-      const int64_t row = act[u] ? seg[u] / n_groups : 0;
-      const int64_t gi = act[u] ? seg[u] % n_groups : 0;
-      const T *src = W + row * d_in + gi * seg_words * 8;
+      const T *src = W + (act[u] ? seg[u] : 0) * seg_words * 8;
 #pragma unroll
       for (int k = 0; k < WPL; ++k) {
         const int64_t w = tl + static_cast<int64_t>(k) * TEAM;
@@ -124,17 +127,16 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
       }
       if (!act[u]) continue;
       const GridParams g = s ? grid_sym(amax) : grid_affine(vmin, vmax);
-      const int64_t row = seg[u] / n_groups;
-      const int64_t gi = seg[u] % n_groups;
+      const float rs = __fdiv_rn(1.0f, g.s);
       if (tl == 0) {
-        scales[row * n_groups + gi] = g.s_bits;
-        if (zeros) zeros[row * n_groups + gi] = s ? 0 : g.z_bits;
+        scales[seg[u]] = g.s_bits;
+        if (zeros) zeros[seg[u]] = s ? 0 : g.z_bits;
       }
-      uint32_t *dst = q + row * words_per_row + gi * seg_words;
+      uint32_t *dst = q + seg[u] * seg_words;
 #pragma unroll
       for (int k = 0; k < WPL; ++k) {
         const int64_t w = tl + static_cast<int64_t>(k) * TEAM;
-        if (w < seg_words) dst[w] = pack_word(v[u][k], g, s);
+        if (w < seg_words) dst[w] = pack_word(v[u][k], g, rs, s);
       }
     }
   }
@@ -155,6 +157,7 @@ __global__ void __launch_bounds__(256) rtn_stream_kernel(const T *__restrict__ W
   for (int64_t row = warp; row < d_out; row += n_warps) {
     const T *src = W + row * d_in;
     float amax = 0.0f, vmin = 0.0f, vmax = 0.0f;
+#pragma unroll 4
     for (int64_t w = lane; w < words; w += 32) {
       float v[8];
       Vec8<T>::load(src + w * 8, v);
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(256) rtn_stream_kernel(const T *__restrict__ W
       vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
     }
     const GridParams g = s ? grid_sym(amax) : grid_affine(vmin, vmax);
+    const float rs = __fdiv_rn(1.0f, g.s);
     if (lane == 0) {
       scales[row] = g.s_bits;
       if (zeros) zeros[row] = s ? 0 : g.z_bits;
@@ -179,7 +183,7 @@ __global__ void __launch_bounds__(256) rtn_stream_kernel(const T *__restrict__ W
     for (int64_t w = lane; w < words; w += 32) {
       float v[8];
       Vec8<T>::load(src + w * 8, v);
-      q[row * words + w] = pack_word(v, g, s);
+      q[row * words + w] = pack_word(v, g, rs, s);
     }
   }
 }

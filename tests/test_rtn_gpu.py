@@ -79,3 +79,34 @@ def test_rtn_full_size_layers(workload, idx):
     if spec.d_out * spec.d_in > 50_000_000:
         rows = np.sort(np.random.default_rng(idx).choice(spec.d_out, 96, replace=False))
     _check(W, spec.group_size, spec.sym, rows)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("group_size,sym", [(-1, True), (128, True), (128, False), (32, False)])
+def test_rtn_dense_midpoints(dt, group_size, sym):
+    """Weights packed with exact rounding midpoints (k + 1/2) s of each
+    group's step and their neighbours one ulp away, where a division that
+    is not correctly rounded would change the code."""
+    d_out, d_in = 1024, 512
+    g = torch.Generator().manual_seed(77 + group_size)
+    W = (torch.randn((d_out, d_in), generator=g) * 0.02).to(DT[dt]).float()
+    gs = d_in if group_size == -1 else group_size
+    Wg = W.view(d_out, d_in // gs, gs)
+    amax = Wg.abs().amax(2, keepdim=True)
+    s16 = (amax / 7).to(torch.float16).float() if sym else \
+        ((Wg.amax(2, keepdim=True).clamp(min=0) - Wg.amin(2, keepdim=True).clamp(max=0)) / 15).to(torch.float16).float()
+    k = torch.randint(-6, 6, Wg.shape, generator=g).float()
+    mid = ((k + 0.5) * s16).to(DT[dt]).float()
+    pick = torch.randint(0, 4, Wg.shape, generator=g)
+    up = torch.nextafter(mid, torch.full_like(mid, 1e9))
+    dn = torch.nextafter(mid, torch.full_like(mid, -1e9))
+    Wm = torch.where(pick == 0, mid, torch.where(pick == 1, up, torch.where(pick == 2, dn, Wg)))
+    if sym:
+        Wm = torch.maximum(torch.minimum(Wm, amax), -amax)
+        keep = [Wg.abs().argmax(2, keepdim=True)]
+    else:
+        Wm = torch.maximum(torch.minimum(Wm, Wg.amax(2, keepdim=True)), Wg.amin(2, keepdim=True))
+        keep = [Wg.argmax(2, keepdim=True), Wg.argmin(2, keepdim=True)]
+    for idx in keep:                                        # the group's extremes stay,
+        Wm.scatter_(2, idx, Wg.gather(2, idx))               # so its step is s16 above
+    _check(Wm.reshape(d_out, d_in).to(DT[dt]), group_size, sym)
