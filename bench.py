@@ -230,11 +230,13 @@ def schedule(runs, n_streams):
     return lists
 
 
-def capture_step(runs, n_streams, timed=False, host=None):
+def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=0):
     """One whole step (every layer, every stage) captured as a CUDA graph:
     the layers run on ``n_streams`` streams forked from and joined back to
     one capture stream.  ``timed`` adds timing event nodes around each
-    stage call; ``host`` adds the pinned host <-> device copies of the
+    stage call; ``kernel`` adds the library's per-launch event pairs around
+    every launch of that kernel (read with gq.kernel_timer_read after the
+    replays); ``host`` adds the pinned host <-> device copies of the
     end-to-end run.  Returns (graph, stream, stage events, launches/step)."""
     import torch
     from post_weight_quantization_27_b200 import gq
@@ -243,6 +245,8 @@ def capture_step(runs, n_streams, timed=False, host=None):
     g = torch.cuda.CUDAGraph()
     events = []
     n0 = gq.launch_count()
+    if kernel is not None:
+        gq.kernel_timer_start([kernel], capacity)
     with torch.cuda.graph(g, stream=main):
         fork = torch.cuda.Event()
         fork.record(main)
@@ -275,7 +279,55 @@ def capture_step(runs, n_streams, timed=False, host=None):
             j = torch.cuda.Event()
             j.record(sd)
             main.wait_event(j)
+    if kernel is not None:
+        gq.kernel_timer_stop()
     return g, main, events, gq.launch_count() - n0
+
+
+def replay(graph, stream, n, timed=False):
+    """Launch the captured step ``n`` times on ``stream`` (the stream it was
+    captured from, so the timing events below bracket the replays); with
+    ``timed`` returns the mean ms per replay from events on that stream,
+    synchronising on both sides."""
+    import torch
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(n):
+            graph.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / max(n, 1) if timed else None
+
+
+def kernel_shares(runs):
+    """One eager pass of the whole step on one stream with every kernel's
+    launches timed: per kernel (total ms, launches), serialised like an ncu
+    launch list; picks the dominant kernel."""
+    import torch
+    from post_weight_quantization_27_b200 import gq
+    n0 = gq.launch_count()
+    for r in runs:
+        for st in LayerRun.STAGES:
+            getattr(r, st)()
+    torch.cuda.synchronize()
+    cap = int(1.2 * (gq.launch_count() - n0)) + 64
+    gq.kernel_timer_start(gq.KERNELS, cap)
+    try:
+        for r in runs:
+            for st in LayerRun.STAGES:
+                getattr(r, st)()
+        torch.cuda.synchronize()
+        recs = gq.kernel_timer_read()
+    finally:
+        gq.kernel_timer_release()
+    tot = {}
+    for k, ms, w in recs:
+        t, n, wk = tot.get(k, (0.0, 0, 0.0))
+        tot[k] = (t + ms, n + 1, wk + w)
+    return tot
 
 
 def stage_work(spec):
@@ -305,15 +357,14 @@ def gpu_arm(args, world, rank, local):
     peaks = measured_peaks()
     n_streams = max(1, min(args.streams, len(runs)))
 
-    # one eager pass (sets kernel attributes), then the captured step
-    for r in runs:
-        for st in LayerRun.STAGES:
-            getattr(r, st)()
-    torch.cuda.synchronize()
-    graph, gstream, events, launches_per_step = capture_step(runs, n_streams, timed=True)
+    # eager passes (set kernel attributes; per-kernel shares), then the
+    # captured step with the dominant kernel's launches timed
+    shares = kernel_shares(runs)
+    dom_kernel = max(shares, key=lambda k: shares[k][0])
+    graph, gstream, events, launches_per_step = capture_step(
+        runs, n_streams, timed=True, kernel=dom_kernel, capacity=shares[dom_kernel][1] + 64)
 
-    for _ in range(args.warmup):
-        graph.replay()
+    replay(graph, gstream, args.warmup)
     torch.cuda.synchronize()
     barrier(world)
 
@@ -321,15 +372,10 @@ def gpu_arm(args, world, rank, local):
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
         barrier(world)
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(gstream)
-        for _ in range(args.steps):
-            graph.replay()
-        t1.record(gstream)
-        torch.cuda.synchronize()
+        w0 = time.perf_counter()
+        ms_local = replay(graph, gstream, args.steps, timed=True)
+        wall_ms = (time.perf_counter() - w0) * 1e3 / args.steps
         barrier(world)
-    ms_local = t0.elapsed_time(t1) / args.steps
     ms = reduce_max(ms_local, world)
     clocks = clk.summary()
 
@@ -343,8 +389,9 @@ def gpu_arm(args, world, rank, local):
     n_layers = len(runs)
     value = world * n_layers / (ms / 1e3)
 
-    dom = max(stage_ms, key=stage_ms.get)
-    roof = roofline(dom, stage_ms, tot, peaks)
+    recs = [r for r in gq.kernel_timer_read() if r[0] == dom_kernel]
+    gq.kernel_timer_release()
+    roof = roofline(dom_kernel, recs, peaks, args.workload)
     del graph
 
     e2e = e2e_run(runs, args, dev, world, n_streams)
@@ -357,6 +404,7 @@ def gpu_arm(args, world, rank, local):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms, 4),
+        "wall_ms_per_step": round(wall_ms, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -369,9 +417,15 @@ def gpu_arm(args, world, rank, local):
                        sum(r.W.numel() * r.W.element_size() + r.X.numel() * 2 for r in runs) / 1e6)},
         "mweights_per_s": round(world * tot["weights"] / (ms / 1e3) / 1e6, 2),
         "stage_ms_sum_of_calls": {k: round(v, 4) for k, v in stage_ms.items()},
-        "xtx_tflops": round(tot["hessian_flops"] / (stage_ms["hessian"] / 1e3) / 1e12, 2),
-        "rtn_gbs": round(tot["rtn_bytes"] / (stage_ms["rtn"] / 1e3) / 1e9, 2),
-        "recon_tflops": round(tot["recon_flops"] / (stage_ms["recon"] / 1e3) / 1e12, 2),
+        "kernel_share_eager": {k: {"ms": round(t, 3), "launches": n,
+                                   "share": round(t / sum(v[0] for v in shares.values()), 4)}
+                               for k, (t, n, _) in sorted(shares.items(), key=lambda x: -x[1][0])},
+        # per-kernel rates from the serialised eager pass (work / event time)
+        "xtx_tflops": rate(shares, "hessian_mma", 1e12),
+        "rtn_gbs": rate(shares, "rtn", 1e9),
+        "recon_tflops": rate(shares, "recon_mma", 1e12),
+        "tf32x3_gemm_tflops": rate(shares, "gemm_tf32x3", 1e12),
+        "gptq_block_gbs": rate(shares, "gptq_block", 1e9),
         "roofline": roof,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": clocks,
@@ -380,32 +434,76 @@ def gpu_arm(args, world, rank, local):
     return out
 
 
-def roofline(dom, stage_ms, tot, peaks):
-    """Roofline of the dominant stage, from its algorithmic work and its
-    CUDA-event time inside the timed region."""
-    t = stage_ms[dom] / 1e3          # sum over the step's calls of this stage
-    if dom == "hessian":
-        a = tot["hessian_flops"] / t / 1e12
-        return {"stage": dom, "bound": "tensor", "achieved": round(a, 2),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(a / peaks["bf16_tflops"], 4), "traffic": None,
-                "peak_source": peaks["source"] + " (burst bf16)"}
-    if dom == "recon":
-        a = tot["recon_flops"] / t / 1e12
-        return {"stage": dom, "bound": "tensor", "achieved": round(a, 2),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(a / peaks["bf16_tflops"], 4), "traffic": None,
-                "peak_source": peaks["source"] + " (burst bf16)"}
-    if dom == "rtn":
-        a = tot["rtn_bytes"] / t / 1e9
-        return {"stage": dom, "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(a / peaks["hbm_gbs"], 4), "traffic": None,
-                "peak_source": peaks["source"]}
-    # gptq / solve: report the fp32 weight traffic of the stage against HBM
-    a = tot["weights"] * 4 * 2 / t / 1e9
-    return {"stage": dom, "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": round(a / peaks["hbm_gbs"], 4), "traffic": None,
-            "peak_source": peaks["source"], "note": "fp32 working-copy bytes (read+write W once)"}
+def rate(shares, kernel, scale):
+    if kernel not in shares or shares[kernel][0] <= 0:
+        return None
+    t, _, w = shares[kernel]
+    return round(w / (t / 1e3) / scale, 2)
+
+
+# Roofline ceiling per kernel: (bound, unit, ceiling name).  The tensor
+# ceilings derive from the measured bf16 GEMM rate (sustained: the kernels
+# are timed inside a long step) by the nominal dense ratios of B200
+# (tf32 1.1 / bf16 2.25 PFLOP/s) and the number of tensor passes per
+# algorithmic product (3 for the 3 x TF32 split, 2 for the bf16 hi + lo
+# split); the fp32 ALU ceiling is 148 SMs x 128 FMA lanes x 2 flops x the
+# maximum SM clock.
+KERNEL_BOUND = {
+    "hessian_mma": ("tensor", "bf16"),
+    "recon_mma": ("tensor", "bf16 hi+lo (2 passes)"),
+    "gemm_tf32x3": ("tensor", "3xTF32 (3 tf32 passes)"),
+    "potrf_trsm": ("alu", "fp32 FMA"),
+    "block_inverse": ("alu", "fp32 FMA"),
+    "gptq_block": ("hbm", "HBM copy"),
+    "rtn": ("hbm", "HBM copy"),
+}
+
+
+def kernel_peak(kernel, peaks):
+    bf16 = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    src = peaks["source"]
+    if kernel == "hessian_mma":
+        return bf16, "TFLOP/s", f"{src} bf16 sustained"
+    if kernel == "recon_mma":
+        return bf16 / 2, "TFLOP/s", f"{src} bf16 sustained / 2 passes"
+    if kernel == "gemm_tf32x3":
+        return bf16 * 1.1 / 2.25 / 3, "TFLOP/s", f"{src} bf16 sustained x 1.1/2.25 (tf32) / 3 passes"
+    if kernel in ("potrf_trsm", "block_inverse"):
+        mhz = peaks.get("sm_max_mhz") or 1965.0
+        return 148 * 128 * 2 * mhz * 1e6 / 1e12, "TFLOP/s", f"148 SMs x 128 FMA x 2 x {mhz:.0f} MHz"
+    return peaks["hbm_gbs"], "GB/s", f"{src} HBM copy"
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch of ``kernel`` on ``workload`` from the committed
+    ncu summary (profiles/traffic.txt: kernel, workload, bytes per launch),
+    or None when no capture of the current kernel is recorded."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel \
+                    and parts[1] == str(workload):
+                return float(parts[2])
+    return None
+
+
+def roofline(kernel, recs, peaks, workload):
+    """Roofline of the dominant kernel: its launches' algorithmic work (flops
+    or bytes, as the library counts them per launch) over their CUDA-event
+    durations in the last timed replay."""
+    bound, what = KERNEL_BOUND[kernel]
+    peak, unit, src = kernel_peak(kernel, peaks)
+    work = sum(w for _, _, w in recs)
+    sec = sum(ms for _, ms, _ in recs) / 1e3
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    a = work / sec / scale if sec > 0 else 0.0
+    return {"kernel": kernel, "bound": bound, "achieved": round(a, 3), "peak": round(peak, 1),
+            "unit": unit, "frac": round(a / peak, 4), "traffic": profiled_traffic(kernel, workload),
+            "launches": len(recs), "avg_launch_us": round(sec / max(len(recs), 1) * 1e6, 2),
+            "work_per_launch": work / max(len(recs), 1), "ceiling": what, "peak_source": src}
 
 
 def e2e_run(runs, args, dev, world, n_streams):
@@ -425,17 +523,10 @@ def e2e_run(runs, args, dev, world, n_streams):
     d2h = sum(h["q"].numel() * 4 + h["s"].numel() * 2 + h["qr"].numel() * 4 + 16 for h in host)
     graph, gstream, _, _ = capture_step(runs, n_streams, timed=False, host=host)
     steps = max(1, min(args.steps, 5))
-    graph.replay()
+    replay(graph, gstream, 1)
     torch.cuda.synchronize()
     barrier(world)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(gstream)
-    for _ in range(steps):
-        graph.replay()
-    t1.record(gstream)
-    torch.cuda.synchronize()
-    ms = reduce_max(t0.elapsed_time(t1) / steps, world)
+    ms = reduce_max(replay(graph, gstream, steps, timed=True), world)
     del graph
     return {"value": round(world * len(runs) / (ms / 1e3), 3), "unit": "layers/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}

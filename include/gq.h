@@ -248,6 +248,56 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
                          double *sse_host, double *mse_host, void *ws, size_t ws_bytes,
                          void *stream);
 
+/* ------------------------------------------------------------------------
+ * Per-launch kernel timing (a measurement aid; the pages describe no such
+ * facility).  A throughput figure for one kernel needs that kernel's own
+ * duration, which events around a whole entry point (several kernels) do
+ * not give.
+ *
+ *   gq_kernel_timer_start(mask, capacity)
+ *       creates `capacity` CUDA event pairs on the current device.  From
+ *       then on, every launch of a kernel whose bit (1 << gq_kernel) is set
+ *       in `mask` is bracketed by an event pair recorded on the launch's
+ *       own stream, together with the launch's algorithmic work, until
+ *       `capacity` launches have been recorded or the timer is stopped.
+ *       Inside a stream capture the pair is captured as external event
+ *       nodes: every replay of the graph records it again, so a read after
+ *       the replays gives the last replay's durations.  Launches on other
+ *       devices are not recorded.  GQ_ERR_ARG if a session is active or
+ *       capacity <= 0; GQ_ERR_CUDA if the events cannot be created.
+ *   gq_kernel_timer_stop()
+ *       no further launches are recorded (the records stay readable).
+ *   gq_kernel_timer_read(kind, ms, work, max)
+ *       after the recorded work has completed: fills up to `max` entries of
+ *       the host arrays (the gq_kernel of the launch, its duration in ms,
+ *       its algorithmic work) and returns the number of records, or -1 if
+ *       an event cannot be read (the work has not run or not finished).
+ *   gq_kernel_timer_release()
+ *       destroys the events and ends the session.
+ * The algorithmic work is counted in flops (2 per multiply-add) for
+ * HESSIAN_MMA (symmetric half of X^T X), POTRF_TRSM, BLOCK_INVERSE,
+ * GEMM_TF32X3 (the fp32 product; lower-triangle calls count the triangle)
+ * and RECON_MMA (one product (W - W^) X^T), and in bytes that must cross
+ * HBM for GPTQ_BLOCK (the block's working weights read, Err written, the U
+ * block, codes and scales) and RTN (W read, codes, scales and zeros
+ * written).  One session at a time per process; the calls are thread safe.
+ * ---------------------------------------------------------------------- */
+typedef enum {
+  GQ_KERNEL_HESSIAN_MMA = 0,
+  GQ_KERNEL_POTRF_TRSM = 1,
+  GQ_KERNEL_BLOCK_INVERSE = 2,
+  GQ_KERNEL_GEMM_TF32X3 = 3,
+  GQ_KERNEL_GPTQ_BLOCK = 4,
+  GQ_KERNEL_RTN = 5,
+  GQ_KERNEL_RECON_MMA = 6,
+  GQ_KERNEL_COUNT = 7
+} gq_kernel;
+
+gq_status gq_kernel_timer_start(uint32_t mask, int32_t capacity);
+gq_status gq_kernel_timer_stop(void);
+int32_t gq_kernel_timer_read(int32_t *kind, float *ms, double *work, int32_t max);
+gq_status gq_kernel_timer_release(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,14 +13,17 @@
 // is the upper Cholesky factor of H^-1.  Two d^3/3 steps instead of three.
 //
 // Memory: A is gathered (reversed, act-order permuted) into the U buffer
-// and factored in place; X = L^-1 is built in the H buffer (the caller's H
-// is scratch); the last kernel writes U = J X J back into the U buffer.
+// and factored in place, except that each diagonal block's factor (then its
+// inverse) goes to a [NB][NB] slot of the workspace; X = L^-1 is built in
+// the H buffer (the caller's H is scratch); the last kernel writes
+// U = J X J back into the U buffer.
 // Blocked right-looking algorithms with 128-wide panels; one CTA factors a
 // diagonal block in shared memory (and inverts it), the panel solve, the
 // trailing updates and the inverse's block steps are fp32 GEMMs on the
 // tensor cores (3 x TF32 split, gemm_tc.cu).
 #include <cfloat>
 #include <climits>
+#include <map>
 #include <mutex>
 #include <string>
 
@@ -169,20 +172,37 @@ __device__ __forceinline__ void chol32_column(float (&w)[32], float &my_rd, int 
   }
 }
 constexpr int TP = 33;      // stride of the 32 x 32 temporaries
-constexpr size_t POTRF_SMEM = (2 * NB * SP + NB + 3 * 32 * TP) * sizeof(float);
 
-__global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A, int64_t d,
-                                                          int64_t k0, int nb,
-                                                          float *__restrict__ linv,
-                                                          int *status) {
+// ---------------------------------------------------------------- panel
+// One 128-column panel of the blocked Cholesky: the 128 x 128 diagonal
+// block factored in shared memory, and the rows below it solved against
+// that factor, in one launch.  CTA t owns the panel rows k0 + 128 t .. +127;
+// every CTA factors the diagonal block itself, so the panel solve needs
+// neither a separate launch nor the block's inverse.  CTA 0 writes the
+// factor to lpp ([NB][NB], identity padded), not back into A: with more
+// CTAs than fit on the GPU at once, later CTAs still read the unfactored
+// block from A after CTA 0 has finished.
+// The 128 columns go in sub-panels of 32:
+//   (a) one warp factors the 32 x 32 diagonal piece, a row per lane in
+//       registers (pivot and column broadcast by shuffles);
+//   (b) one thread per row below the piece (in the diagonal block and in
+//       the CTA's own tile) solves x L^T = a with the row in registers;
+//   (c) all threads apply the sub-panel to the remaining columns of both,
+//       in 4 x 4 register tiles.
+constexpr size_t PANEL_SMEM = (2 * NB * SP + NB) * sizeof(float);
+
+__global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, int64_t d,
+                                                         int64_t k0, int nb,
+                                                         float *__restrict__ lpp, int *status) {
   extern __shared__ float sm[];
-  float *S = sm;                // [NB][SP]  the block, then L (lower)
-  float *Li = S + NB * SP;      // [NB][SP]  L^-1 (lower)
-  float *rd = Li + NB * SP;     // [NB]      1 / L_jj
-  float *T = rd + NB;           // [3][32][TP] temporaries of the inverse
+  float *S = sm;            // [NB][SP]  the diagonal block, then its factor L (lower)
+  float *P = S + NB * SP;   // [NB][SP]  this CTA's panel rows (CTA 0: unused)
+  float *rd = P + NB * SP;  // [NB]      1 / L_jj
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // the block's lower part, 16 float4 loads per thread in flight at once;
-  // identity padding past the matrix edge (only the lower part is ever read)
+  const bool own = blockIdx.x > 0;
+  const int64_t row0 = k0 + static_cast<int64_t>(blockIdx.x) * NB;
+  const int prows = own ? static_cast<int>(d - row0 < NB ? d - row0 : NB) : 0;
+
   {
     float4 v[NB * NB / 4 / 256];
 #pragma unroll
@@ -199,11 +219,26 @@ __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A,
       const int r = idx >> 5, c = (idx & 31) * 4;
       const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float x = e[q];
-        if (r >= nb) x = (r == c + q) ? 1.0f : 0.0f;
-        S[r * SP + c + q] = x;
-        Li[r * SP + c + q] = 0.0f;
+      for (int q = 0; q < 4; ++q)
+        S[r * SP + c + q] = r < nb ? e[q] : (r == c + q ? 1.0f : 0.0f);  // identity padding
+    }
+    if (own) {
+#pragma unroll
+      for (int u = 0; u < NB * NB / 4 / 256; ++u) {
+        const int idx = tid + 256 * u;
+        const int r = idx >> 5, c = (idx & 31) * 4;
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < prows && c < nb)
+          v[u] = *reinterpret_cast<const float4 *>(A + (row0 + r) * d + k0 + c);
+      }
+#pragma unroll
+      for (int u = 0; u < NB * NB / 4 / 256; ++u) {
+        const int idx = tid + 256 * u;
+        const int r = idx >> 5, c = (idx & 31) * 4;
+        P[r * SP + c] = v[u].x;
+        P[r * SP + c + 1] = v[u].y;
+        P[r * SP + c + 2] = v[u].z;
+        P[r * SP + c + 3] = v[u].w;
       }
     }
   }
@@ -216,18 +251,22 @@ __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A,
 #pragma unroll
       for (int k = 0; k < 32; ++k) w[k] = (k <= lane) ? S[(c0 + lane) * SP + c0 + k] : 0.0f;
       float my_rd = 1.0f;
-      chol32_column<0>(w, my_rd, lane, k0 + c0, nb - c0, status);
+      chol32_column<0>(w, my_rd, lane, k0 + c0, blockIdx.x == 0 ? nb - c0 : 0, status);
 #pragma unroll
       for (int k = 0; k < 32; ++k)
         if (k <= lane) S[(c0 + lane) * SP + c0 + k] = w[k];
       rd[c0 + lane] = my_rd;
     }
     __syncthreads();
-    // (b) rows below the piece: x = a L_dd^-T, right-looking within the row
-    for (int r = c0 + 32 + tid; r < NB; r += 256) {
+    // (b) rows below the piece -- in the block, then the CTA's tile rows:
+    //     x = a L_dd^-T, right-looking within the row
+    const int below = NB - (c0 + 32);
+    const int n_rows = below + (own ? NB : 0);
+    for (int i = tid; i < n_rows; i += 256) {
+      float *row = i < below ? S + (c0 + 32 + i) * SP : P + (i - below) * SP;
       float a[32];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) a[k] = S[r * SP + c0 + k];
+      for (int k = 0; k < 32; ++k) a[k] = row[c0 + k];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float x = a[j] * rd[c0 + j];
@@ -236,46 +275,107 @@ __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A,
         for (int k = j + 1; k < 32; ++k) a[k] = fmaf(-x, S[(c0 + k) * SP + c0 + j], a[k]);
       }
 #pragma unroll
-      for (int k = 0; k < 32; ++k) S[r * SP + c0 + k] = a[k];
+      for (int k = 0; k < 32; ++k) row[c0 + k] = a[k];
     }
     __syncthreads();
-    // (c) rest of the block: S[i][k] -= sum_j S[i][c0+j] S[k][c0+j], base <= k <= i
+    // (c) remaining columns base.. of the block (lower part) and of the tile
+    //     rows: M[i][k] -= sum_j M[i][c0+j] S[k][c0+j]
     const int base = c0 + 32;
-    const int mt = (NB - base) / 4;  // 4 x 4 tiles per side
-    const int n_tiles = mt * (mt + 1) / 2;
-    for (int t = tid; t < n_tiles; t += 256) {
-      int ti = 0;
-      while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-      const int tk = t - ti * (ti + 1) / 2;
-      const int i0 = base + 4 * ti, kk0 = base + 4 * tk;
+    const int mt = (NB - base) / 4;           // 4-wide column tiles left
+    const int n_s = mt * (mt + 1) / 2;        // lower tiles of the block
+    const int n_p = own ? (NB / 4) * mt : 0;  // tiles of the panel rows
+    for (int t = tid; t < n_s + n_p; t += 256) {
+      const float *src;
+      float *dst;
+      int i0, kk0;
+      bool tri;
+      if (t < n_s) {
+        int ti = 0;
+        while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
+        const int tk = t - ti * (ti + 1) / 2;
+        i0 = base + 4 * ti;
+        kk0 = base + 4 * tk;
+        src = S;
+        dst = S;
+        tri = true;
+      } else {
+        const int u = t - n_s;
+        i0 = 4 * (u / mt);
+        kk0 = base + 4 * (u % mt);
+        src = P;
+        dst = P;
+        tri = false;
+      }
       float acc[4][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
+        for (int y = 0; y < 4; ++y) acc[x][y] = 0.0f;
 #pragma unroll 8
       for (int j = 0; j < 32; ++j) {
         float pi[4], pk[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          pi[a] = S[(i0 + a) * SP + c0 + j];
-          pk[a] = S[(kk0 + a) * SP + c0 + j];
+        for (int x = 0; x < 4; ++x) {
+          pi[x] = src[(i0 + x) * SP + c0 + j];
+          pk[x] = S[(kk0 + x) * SP + c0 + j];
         }
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int x = 0; x < 4; ++x)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(pi[a], pk[b], acc[a][b]);
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(pi[x], pk[y], acc[x][y]);
       }
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
-          if (kk0 + b <= i0 + a) S[(i0 + a) * SP + kk0 + b] -= acc[a][b];
+        for (int y = 0; y < 4; ++y)
+          if (!tri || kk0 + y <= i0 + x) dst[(i0 + x) * SP + kk0 + y] -= acc[x][y];
     }
     __syncthreads();
   }
 
-  // inverse, diagonal blocks: warp q, lane = column
+  if (!own) {
+    for (int e = tid; e < NB * NB; e += 256) {
+      const int r = e / NB, c = e % NB;
+      lpp[e] = c <= r ? S[r * SP + c] : 0.0f;
+    }
+  } else {
+    for (int e = tid; e < NB * NB / 4; e += 256) {
+      const int r = e >> 5, c = (e & 31) * 4;
+      if (r < prows && c < nb)
+        *reinterpret_cast<float4 *>(A + (row0 + r) * d + k0 + c) =
+            make_float4(P[r * SP + c], P[r * SP + c + 1], P[r * SP + c + 2], P[r * SP + c + 3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- block inverse
+// lp := L_pp^-1, in place, for the factored diagonal block that
+// potrf_trsm_kernel left in lp ([NB][NB], lower, identity padded past the
+// matrix edge).  Each warp inverts one 32 x 32 diagonal block (a column per
+// lane), then X_ij = -X_ii (sum_k L_ik X_kj) fills the blocks below, one
+// diagonal band at a time.
+constexpr size_t INV_SMEM = (2 * NB * SP + NB + 3 * 32 * TP) * sizeof(float);
+
+__global__ void __launch_bounds__(256) block_inverse_kernel(float *__restrict__ lp) {
+  extern __shared__ float sm[];
+  float *S = sm;                // [NB][SP]  L (lower)
+  float *Li = S + NB * SP;      // [NB][SP]  L^-1 (lower)
+  float *rd = Li + NB * SP;     // [NB]
+  float *T = rd + NB;           // [3][32][TP]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < NB * NB / 4; e += 256) {
+    const int r = e >> 5, c = (e & 31) * 4;
+    const float4 v = *reinterpret_cast<const float4 *>(lp + r * NB + c);
+    const float x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      S[r * SP + c + q] = x[q];
+      Li[r * SP + c + q] = 0.0f;
+    }
+  }
+  __syncthreads();
+  if (tid < NB) rd[tid] = __frcp_rn(S[tid * SP + tid]);
+  __syncthreads();
   if (warp < 4) {
     const int q0 = 32 * warp;
     float v[32];
@@ -292,8 +392,7 @@ __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A,
     for (int r = 0; r < 32; ++r) Li[(q0 + r) * SP + q0 + lane] = v[r];
   }
   __syncthreads();
-  // bands below the diagonal: X_ij = -X_ii sum_{k=j}^{i-1} L_ik X_kj, i - j = lvl
-  // (each thread: one row r, four consecutive columns 4*c4 .. 4*c4+3)
+  // (each thread: one row r, four consecutive columns)
   for (int lvl = 1; lvl < 4; ++lvl) {
     const int nblk = 4 - lvl;
     for (int e = tid; e < nblk * 256; e += 256) {
@@ -332,12 +431,8 @@ __global__ void __launch_bounds__(256) potrf_panel_kernel(float *__restrict__ A,
     }
     __syncthreads();
   }
-
-  for (int e = tid; e < NB * NB; e += 256) {
-    const int r = e / NB, c = e % NB;
-    if (r < nb && c <= r) A[(k0 + r) * d + k0 + c] = S[r * SP + c];
-    linv[e] = Li[r * SP + c];
-  }
+  __syncthreads();  // every thread has read lp before it is overwritten
+  for (int e = tid; e < NB * NB; e += 256) lp[e] = Li[(e / NB) * SP + e % NB];
 }
 
 // X := I on the lower triangle and on the whole NB x NB diagonal blocks
@@ -378,9 +473,47 @@ size_t chol_ws_bytes(int64_t d) {
          static_cast<size_t>(n_panels) * NB * NB * sizeof(float);
 }
 
+// A second stream (and two events) per caller stream and device, created on
+// first use and kept for the life of the process.  Keyed by the caller's
+// stream so that solves issued on different streams keep independent
+// inverse chains (one shared helper stream would serialise them).  None is
+// created while the caller's stream is being captured into a graph; the
+// inverse chain then stays on the caller's stream.
+struct AuxStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t ev = nullptr, join = nullptr;
+};
+
+AuxStream *aux_stream(cudaStream_t caller) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, AuxStream> cache;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, caller);
+  auto it = cache.find(key);
+  if (it != cache.end()) return &it->second;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(caller, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  AuxStream a;
+  if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&a.ev, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return &(cache[key] = a);
+}
+
 gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32_t *perm_out,
                            uint8_t *dead_out, float *U, int32_t *info_dev, void *ws,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool use_aux) {
   CholWs w = carve(ws, d);
   damp_kernel<<<1, 1024, 0, st>>>(H, d, damp, dead_out, w.key, w.status);
   count_launch();
@@ -399,52 +532,68 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
     const gq_status s = check_launch("damp/gather");
     if (s != GQ_OK) return s;
   }
-  const size_t pot_smem = POTRF_SMEM;
-  cudaFuncSetAttribute(potrf_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(pot_smem));
+  cudaFuncSetAttribute(potrf_trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(PANEL_SMEM));
+  cudaFuncSetAttribute(block_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(INV_SMEM));
   const int64_t n_panels = (d + NB - 1) / NB;
-  // ---- Cholesky, right-looking
+  eye_lower_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d);
+  count_launch();
+  // The inverse X = L^-1 (blocked forward substitution on the identity) runs
+  // as a second chain: its step p needs the panel p of L and step p-1 only,
+  // so on a second stream it overlaps the rest of the factorisation.
+  cudaStream_t inv_st = st;
+  AuxStream *aux = nullptr;
+  if (use_aux) {
+    aux = aux_stream(st);
+    if (aux) inv_st = aux->s;
+  }
   for (int64_t p = 0; p < n_panels; ++p) {
     const int64_t k0 = p * NB;
     const int nb = static_cast<int>(d - k0 < NB ? d - k0 : NB);
-    float *lp = w.linv + p * NB * NB;
-    potrf_panel_kernel<<<1, 256, pot_smem, st>>>(A, d, k0, nb, lp, w.status);
-    count_launch();
     const int64_t k1 = k0 + nb;
     const int rest = static_cast<int>(d - k1);
+    const unsigned tiles = static_cast<unsigned>(1 + (rest + NB - 1) / NB);
+    float *lp = w.linv + p * NB * NB;
+    int slot = timer_begin(GQ_KERNEL_POTRF_TRSM, st);
+    potrf_trsm_kernel<<<tiles, 256, PANEL_SMEM, st>>>(A, d, k0, nb, lp, w.status);
+    count_launch();
+    // Cholesky of the block nb^3 / 3, the panel solve rest nb^2
+    timer_end(slot, st, static_cast<double>(nb) * nb * (nb / 3.0 + rest));
+    if (aux) {
+      if (cudaEventRecord(aux->ev, st) != cudaSuccess ||
+          cudaStreamWaitEvent(aux->s, aux->ev, 0) != cudaSuccess)
+        return check_launch("stream fork");
+    }
     if (rest > 0) {
-      // panel rows below: A[k1:, k0:k1] := A[k1:, k0:k1] L_pp^-T (in place:
-      // each output tile owns its rows)
-      gq_status s = launch_gemm_tf32x3(rest, nb, NB, 1.0f, A + k1 * d + k0, d, lp, NB, true,
-                                       0.0f, A + k1 * d + k0, d, false, w.status, st);
-      if (s != GQ_OK) return s;
       // trailing: A[k1:, k1:] -= P P^T (lower part)
-      s = launch_gemm_tf32x3(rest, rest, NB, -1.0f, A + k1 * d + k0, d, A + k1 * d + k0, d,
-                             true, 1.0f, A + k1 * d + k1, d, true, w.status, st);
+      const gq_status s = launch_gemm_tf32x3(rest, rest, NB, -1.0f, A + k1 * d + k0, d,
+                                             A + k1 * d + k0, d, true, 1.0f, A + k1 * d + k1, d,
+                                             true, w.status, st);
+      if (s != GQ_OK) return s;
+    }
+    // ---- inverse step p (on inv_st)
+    slot = timer_begin(GQ_KERNEL_BLOCK_INVERSE, inv_st);
+    block_inverse_kernel<<<1, 256, INV_SMEM, inv_st>>>(lp);
+    count_launch();
+    timer_end(slot, inv_st, static_cast<double>(nb) * nb * nb / 3.0);
+    const int cols = static_cast<int>(k1);
+    // X[k0:k1, 0:cols] := L_pp^-1 X[k0:k1, 0:cols] (in place: each output
+    // tile owns its columns)
+    gq_status s = launch_gemm_tf32x3(nb, cols, nb, 1.0f, lp, NB, X + k0 * d, d, false, 0.0f,
+                                     X + k0 * d, d, false, w.status, inv_st);
+    if (s != GQ_OK) return s;
+    if (rest > 0) {
+      // X[k1:, 0:cols] -= L[k1:, k0:k1] X[k0:k1, 0:cols]
+      s = launch_gemm_tf32x3(rest, cols, nb, -1.0f, A + k1 * d + k0, d, X + k0 * d, d, false,
+                             1.0f, X + k1 * d, d, false, w.status, inv_st);
       if (s != GQ_OK) return s;
     }
   }
-  // ---- X = L^-1 by blocked forward substitution on the identity
-  eye_lower_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d);
-  count_launch();
-  for (int64_t p = 0; p < n_panels; ++p) {
-    const int64_t r0 = p * NB;
-    const int nb = static_cast<int>(d - r0 < NB ? d - r0 : NB);
-    const int cols = static_cast<int>(r0 + nb);
-    float *lp = w.linv + p * NB * NB;
-    // X[r0:r0+nb, 0:cols] := L_pp^-1 X[r0:r0+nb, 0:cols] (in place: each
-    // output tile owns its columns)
-    gq_status s = launch_gemm_tf32x3(nb, cols, nb, 1.0f, lp, NB, X + r0 * d, d, false, 0.0f,
-                                     X + r0 * d, d, false, w.status, st);
-    if (s != GQ_OK) return s;
-    const int64_t r1 = r0 + nb;
-    const int rest = static_cast<int>(d - r1);
-    if (rest > 0) {
-      // X[r1:, 0:cols] -= L[r1:, r0:r1] X[r0:r1, 0:cols]
-      s = launch_gemm_tf32x3(rest, cols, nb, -1.0f, A + r1 * d + r0, d, X + r0 * d, d, false,
-                             1.0f, X + r1 * d, d, false, w.status, st);
-      if (s != GQ_OK) return s;
-    }
+  if (aux) {
+    if (cudaEventRecord(aux->join, aux->s) != cudaSuccess ||
+        cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)
+      return check_launch("stream join");
   }
   reverse_upper_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d, U);
   count_launch();
@@ -523,7 +672,7 @@ extern "C" gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, fl
   // (damp_kernel resets the status words), so earlier calls' leftovers are
   // harmless.
   const gq_status s = launch_damp_chol(H, d_in, damp_percent, act_order, perm_out, dead_out, U,
-                                       info_dev, scratch, st);
+                                       info_dev, scratch, st, false);
   if (s != GQ_OK) return s;
   if (info_host) {
     int32_t info = -1;

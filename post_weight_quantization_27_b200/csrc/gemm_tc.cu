@@ -340,8 +340,12 @@ gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, i
   cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(SMEM_BYTES));
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();
+  const int slot = timer_begin(GQ_KERNEL_GEMM_TF32X3, st);
   gemm_tf32x3_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tA, tB, a);
   count_launch();
+  // the fp32 product: 2 M N K flops, M (M + 1) K for the lower triangle
+  timer_end(slot, st,
+            lower ? static_cast<double>(M) * (M + 1) * K : 2.0 * M * static_cast<double>(N) * K);
   return check_launch("gemm_tf32x3_kernel");
 }
 

@@ -58,10 +58,11 @@ __device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[S
         if (cx.zeros) cx.zeros[cx.row * cx.n_groups + gi] = cx.sym ? 0 : gp.z_bits;
       }
       const float *urow = cx.Ub + j * cx.B + jb;
-      const float c = grid_code_r(w[J], gp, rs, cx.sym);
+      uint32_t nib;
+      const float c = grid_code_fast(w[J], gp, rs, cx.sym, nib);
       const float q = gp.s * (c - gp.z);
       const float delta = div_by_recip(w[J] - q, urow[J], cx.rU[j]);
-      packed[J / 8] |= grid_nibble(c, cx.sym) << (4 * (J % 8));
+      packed[J / 8] |= nib << (4 * (J % 8));
 #pragma unroll
       for (int k = J + 1; k < SB; ++k) w[k] = fmaf(-delta, urow[k], w[k]);
       w[J] = delta;
@@ -200,9 +201,16 @@ gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_o
   cudaFuncSetAttribute(gptq_block_kernel<B, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(smem));
   const unsigned grid = static_cast<unsigned>((d_out + rows - 1) / rows);
+  const int slot = timer_begin(GQ_KERNEL_GPTQ_BLOCK, st);
   gptq_block_kernel<B, G><<<grid, rows, smem, st>>>(tmU, Wk, d_out, d_in, c0, bw, sym, Err, qp,
                                                     codes, scales, zeros, n_groups, status);
   count_launch();
+  // working weights of the block read, Err written (fp32), the U block,
+  // codes (packed: half a byte, else one byte per weight), scales (+ zeros)
+  const double groups = G < 0 ? 0.0 : static_cast<double>((bw + G - 1) / G);
+  timer_end(slot, st,
+            static_cast<double>(d_out) * bw * (8.0 + (qp ? 0.5 : 1.0)) +
+                4.0 * static_cast<double>(B) * B + 2.0 * d_out * groups * (sym ? 1 : 2));
   return GQ_OK;
 }
 

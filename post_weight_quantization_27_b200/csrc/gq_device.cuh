@@ -230,6 +230,26 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float r) {
   const float e = __fmaf_rn(-q0, b, a);
   return __fmaf_rn(e, r, q0);
 }
+// Integer code of w and its stored nibble, with rs = RN(1 / s).  The
+// quotient is clamped to the code range first (equivalent, since the bounds
+// are integers), then rounded half-to-even exactly by adding 1.5 * 2^23: for
+// |q| <= 16 the sum lies in [2^23, 2^24), where the spacing is 1 and the
+// constant is even, so the rounded sum is C + rint(q) and its low mantissa
+// bits are the code.  No float-to-int conversion is needed.
+__device__ __forceinline__ float grid_code_fast(float w, const GridParams &g, float rs, bool sym,
+                                                uint32_t &nib) {
+  constexpr float C = 12582912.0f;  // 1.5 * 2^23
+  const float q = div_by_recip(w, g.s, rs);
+  if (sym) {
+    const float t = __fadd_rn(fminf(fmaxf(q, -7.0f), 7.0f), C);
+    nib = (__float_as_uint(t) + 8u) & 0xFu;  // c + 8
+    return __fsub_rn(t, C);
+  }
+  const float r = __fsub_rn(__fadd_rn(fminf(fmaxf(q, -16.0f), 16.0f), C), C);  // rint(q)
+  const float c = fminf(fmaxf(__fadd_rn(r, g.z), 0.0f), 15.0f);
+  nib = __float_as_uint(__fadd_rn(c, C)) & 0xFu;
+  return c;
+}
 // Code of w with the group's reciprocal scale rs = RN(1 / s).
 __device__ __forceinline__ float grid_code_r(float w, const GridParams &g, float rs, bool sym) {
   float c = __fadd_rn(rintf(div_by_recip(w, g.s, rs)), g.z);

@@ -16,6 +16,21 @@ namespace gq {
 extern std::atomic<uint64_t> g_launches;
 inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+// Per-launch timing (gq_kernel_timer_*): timer_begin before a launch
+// returns a record slot (or -1 when the kernel is not being timed; one
+// atomic load on that path), timer_end after it records the closing event
+// and the launch's algorithmic work.
+extern std::atomic<uint32_t> g_timer_mask;
+int timer_begin_slow(gq_kernel k, cudaStream_t st);
+void timer_end_slow(int slot, cudaStream_t st, double work);
+inline int timer_begin(gq_kernel k, cudaStream_t st) {
+  return (g_timer_mask.load(std::memory_order_relaxed) & (1u << k)) ? timer_begin_slow(k, st)
+                                                                     : -1;
+}
+inline void timer_end(int slot, cudaStream_t st, double work) {
+  if (slot >= 0) timer_end_slow(slot, st, work);
+}
+
 // Clears the thread-local error text (start of every entry point).
 void clear_error();
 // Sets the thread-local error text and returns `s`.
@@ -49,9 +64,11 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
                          const HessPlan &plan, cudaStream_t st);
 
 size_t chol_ws_bytes(int64_t d);
+// use_aux: run the inverse chain on a second stream (forked from and joined
+// back to `st` with events).
 gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32_t *perm_out,
                            uint8_t *dead_out, float *U, int32_t *info_dev, void *ws,
-                           cudaStream_t st);
+                           cudaStream_t st, bool use_aux = true);
 
 // C = beta C + alpha A B in fp32 on the tensor cores (3 x TF32 split).
 gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,

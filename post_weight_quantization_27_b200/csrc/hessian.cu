@@ -301,8 +301,11 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
     }
     HessArgs a{p.n_bj, p.n_tiles, p.n_split, p.kb_per_split, p.nkb_total, P, status};
     const int grid = n_items < num_sms() ? n_items : num_sms();
+    const int slot = timer_begin(GQ_KERNEL_HESSIAN_MMA, st);
     hessian_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, a);
     count_launch();
+    // symmetric half of X^T X: n_tok d_in (d_in + 1) flops
+    timer_end(slot, st, static_cast<double>(n_tok) * d_in * (d_in + 1));
     s = check_launch("hessian_mma_kernel");
     if (s != GQ_OK) return s;
   }

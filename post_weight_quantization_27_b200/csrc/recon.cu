@@ -308,8 +308,12 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        static_cast<int>(SMEM_BYTES));
   ReconArgs a{L.n_mt, L.n_nt, L.nkb, partials, status};
   const int grid = static_cast<int>(n_tiles < num_sms() ? n_tiles : num_sms());
+  const int slot = timer_begin(GQ_KERNEL_RECON_MMA, st);
   recon_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tHi, tLo, tX, a);
   count_launch();
+  // one product (W - W^) X^T: 2 n_tok d_out d_in flops (the hi + lo split
+  // runs it twice on the tensor cores)
+  timer_end(slot, st, 2.0 * static_cast<double>(n_tok) * d_out * d_in);
   s = check_launch("recon_mma_kernel");
   if (s != GQ_OK) return s;
   recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, n_tiles * 8, status, sse_dev);

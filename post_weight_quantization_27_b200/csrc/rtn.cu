@@ -12,6 +12,8 @@
 // 16-byte vector loads and every packed word is written by one coalesced
 // 4-byte store.  Rows longer than 32 * 8 words stream twice through L2
 // instead (second kernel).
+#include <type_traits>
+
 #include "gq_device.cuh"
 #include "gq_internal.h"
 
@@ -56,25 +58,67 @@ struct Vec8<__nv_bfloat16> {
   }
 };
 
+// Eight weights as loaded (16-bit types stay packed, 4 registers per word),
+// converted to fp32 where used, so that more words can be in flight.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *p) {
+    a = __ldg(reinterpret_cast<const float4 *>(p));
+    b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void get(float (&v)[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+template <typename H2>
+struct Raw8Half {
+  uint4 u;
+  __device__ __forceinline__ void zero() { u = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void get(float (&v)[8]) const {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f;
+      if constexpr (sizeof(H2) == 4 && std::is_same<H2, __half2>::value)
+        f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+      else
+        f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+};
+template <>
+struct Raw8<__half> : Raw8Half<__half2> {
+  __device__ __forceinline__ void load(const __half *p) {
+    u = __ldg(reinterpret_cast<const uint4 *>(p));
+  }
+};
+template <>
+struct Raw8<__nv_bfloat16> : Raw8Half<__nv_bfloat162> {
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+    u = __ldg(reinterpret_cast<const uint4 *>(p));
+  }
+};
+
 // Code word of 8 weights.  rs = RN(1 / s): the quotient w / s is formed as a
-// correctly rounded division from the reciprocal (gq_device.cuh), so the
-// decision rint(w / s) is the IEEE one in three instructions; the rest is
-// integer arithmetic (round-half-even conversion, clamp, nibble insert).
+// correctly rounded division from the reciprocal and rounded exactly with a
+// magic-constant addition (gq_device.cuh), so the decision rint(w / s) is the
+// IEEE one in a handful of full-rate instructions per weight.
 template <bool SYM>
 __device__ __forceinline__ uint32_t pack_word(const float (&v)[8], const GridParams &g,
                                               float rs) {
-  const int z = static_cast<int>(g.z);
   uint32_t word = 0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    int c = __float2int_rn(div_by_recip(v[k], g.s, rs));
-    if (SYM) {
-      c = min(max(c, -7), 7) + 8;
-    } else {
-      c = min(max(c, -16), 16) + z;
-      c = min(max(c, 0), 15);
-    }
-    word |= static_cast<uint32_t>(c) << (4 * k);
+    uint32_t nib;
+    grid_code_fast(v[k], g, rs, SYM, nib);
+    word |= nib << (4 * k);
   }
   return word;
 }
@@ -102,8 +146,28 @@ struct SegStat {
       }
     }
   }
+  // Same values as grid_sym / grid_affine, with the divisions by 7 and 15
+  // done from their correctly rounded reciprocals.
   __device__ __forceinline__ GridParams grid() const {
-    return SYM ? grid_sym(a) : grid_affine(a, b);
+    GridParams g;
+    float s32 = SYM ? div_by_recip(a, 7.0f, 1.0f / 7.0f)
+                    : div_by_recip(__fsub_rn(b, a), 15.0f, 1.0f / 15.0f);
+    __half h = __float2half_rn(fminf(s32, 65504.0f));
+    const bool degenerate = __half2float(h) == 0.0f;
+    if (degenerate) h = __float2half_rn(1.0f);
+    g.s = __half2float(h);
+    g.s_bits = __half_as_ushort(h);
+    if (SYM) {
+      g.z = 0.0f;
+      g.z_bits = 0;
+    } else {
+      float z = rintf(div_by_recip(-a, g.s, __frcp_rn(g.s)));
+      z = fminf(fmaxf(z, 0.0f), 15.0f);
+      if (degenerate) z = 0.0f;
+      g.z = __fadd_rn(z, 0.0f);
+      g.z_bits = __half_as_ushort(__float2half_rn(g.z));
+    }
+    return g;
   }
 };
 
@@ -124,7 +188,7 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
   // segment s = row * n_groups + group; every segment starts seg_words * 8
   // weights after the previous one, so its address needs no division
   for (int64_t base = warp * SPW * UNROLL; base < total; base += n_warps * SPW * UNROLL) {
-    float v[UNROLL][WPL][8];
+    Raw8<T> raw[UNROLL][WPL];
     int64_t seg[UNROLL];
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
@@ -134,21 +198,20 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
 #pragma unroll
       for (int k = 0; k < WPL; ++k) {
         const int64_t w = tl + static_cast<int64_t>(k) * TEAM;
-        if (act && w < seg_words) {
-          Vec8<T>::load(src + w * 8, v[u][k]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[u][k][e] = 0.0f;  // never changes the statistic
-        }
+        if (act && w < seg_words) raw[u][k].load(src + w * 8);
+        else raw[u][k].zero();  // zeros never change the statistic
       }
     }
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
       SegStat<SYM> st;
 #pragma unroll
-      for (int k = 0; k < WPL; ++k)
+      for (int k = 0; k < WPL; ++k) {
+        float v[8];
+        raw[u][k].get(v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) st.add(v[u][k][e]);
+        for (int e = 0; e < 8; ++e) st.add(v[e]);
+      }
       st.reduce(TEAM);
       if (seg[u] >= total) continue;
       const GridParams g = st.grid();
@@ -161,7 +224,11 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
 #pragma unroll
       for (int k = 0; k < WPL; ++k) {
         const int64_t w = tl + static_cast<int64_t>(k) * TEAM;
-        if (w < seg_words) dst[w] = pack_word<SYM>(v[u][k], g, rs);
+        if (w < seg_words) {
+          float v[8];
+          raw[u][k].get(v);
+          dst[w] = pack_word<SYM>(v, g, rs);
+        }
       }
     }
   }
@@ -222,21 +289,28 @@ void launch_reg(const void *W, int64_t d_out, int64_t seg_words, int64_t n_group
   count_launch();
 }
 
+// Team size and words per lane: as many words per lane as a small register
+// budget allows (4 for 16-bit weights, 2 for fp32), so that a warp quantises
+// several groups at once and the per-group work is amortised.
 template <typename T>
 gq_status launch_typed(const void *W, int64_t d_out, int64_t d_in, int group_size, int sym,
                        uint32_t *q, uint16_t *sc, uint16_t *z, cudaStream_t st) {
   const int64_t seg_len = group_size == -1 ? d_in : group_size;
   const int64_t n_groups = d_in / seg_len;
   const int64_t words = seg_len / 8;
-  if (words <= 1) launch_reg<T, 1, 1, 4>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 2) launch_reg<T, 2, 1, 4>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 4) launch_reg<T, 4, 1, 4>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 8) launch_reg<T, 8, 1, 4>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 16) launch_reg<T, 16, 1, 4>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 32) launch_reg<T, 32, 1, 4>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 64) launch_reg<T, 32, 2, 2>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 128) launch_reg<T, 32, 4, 1>(W, d_out, words, n_groups, sym, q, sc, z, st);
-  else if (words <= 256) launch_reg<T, 32, 8, 1>(W, d_out, words, n_groups, sym, q, sc, z, st);
+  constexpr int WL = sizeof(T) == 2 ? 4 : 2;  // target words per lane
+#define GQ_R(TEAM, WPL) launch_reg<T, TEAM, WPL, 2>(W, d_out, words, n_groups, sym, q, sc, z, st)
+  if (words <= 1) GQ_R(1, 1);
+  else if (words <= 2) GQ_R(1, 2);
+  else if (words <= WL) GQ_R(1, WL);
+  else if (words <= 2 * WL) GQ_R(2, WL);
+  else if (words <= 4 * WL) GQ_R(4, WL);
+  else if (words <= 8 * WL) GQ_R(8, WL);
+  else if (words <= 16 * WL) GQ_R(16, WL);
+  else if (words <= 32 * WL) GQ_R(32, WL);
+  else if (words <= 128) GQ_R(32, 4);
+  else if (words <= 256) GQ_R(32, 8);
+#undef GQ_R
   else {
     int64_t blocks = (d_out + 7) / 8;
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
@@ -258,16 +332,32 @@ gq_status launch_typed(const void *W, int64_t d_out, int64_t d_in, int group_siz
 gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, int group_size,
                      int sym, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
                      cudaStream_t st) {
+  int wb = 0;
+  gq_status s = GQ_OK;
+  const int slot = timer_begin(GQ_KERNEL_RTN, st);
   switch (dt) {
     case GQ_F32:
-      return launch_typed<float>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st);
+      wb = 4;
+      s = launch_typed<float>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st);
+      break;
     case GQ_F16:
-      return launch_typed<__half>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st);
+      wb = 2;
+      s = launch_typed<__half>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st);
+      break;
     case GQ_BF16:
-      return launch_typed<__nv_bfloat16>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros,
-                                         st);
+      wb = 2;
+      s = launch_typed<__nv_bfloat16>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros,
+                                      st);
+      break;
+    default:
+      s = fail(GQ_ERR_DTYPE, "unknown dtype");
   }
-  return fail(GQ_ERR_DTYPE, "unknown dtype");
+  // W read; codes (half a byte per weight), fp16 scales (and zeros) written
+  const double n_groups = group_size == -1 ? 1.0 : static_cast<double>(d_in / group_size);
+  timer_end(slot, st,
+            static_cast<double>(d_out) * d_in * (wb + 0.5) +
+                2.0 * d_out * n_groups * (sym ? 1 : 2));
+  return s;
 }
 
 }  // namespace gq

@@ -72,6 +72,14 @@ def lib() -> ctypes.CDLL:
     L.gq_recon_error.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                                  _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp,
                                  _c_sz, _c_vp]
+    L.gq_kernel_timer_start.restype = _c_int
+    L.gq_kernel_timer_start.argtypes = [ctypes.c_uint32, ctypes.c_int32]
+    L.gq_kernel_timer_stop.restype = _c_int
+    L.gq_kernel_timer_stop.argtypes = []
+    L.gq_kernel_timer_read.restype = ctypes.c_int32
+    L.gq_kernel_timer_read.argtypes = [_c_vp, _c_vp, _c_vp, ctypes.c_int32]
+    L.gq_kernel_timer_release.restype = _c_int
+    L.gq_kernel_timer_release.argtypes = []
     _lib = L
     return L
 
@@ -80,7 +88,8 @@ EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_w
            "gq_hessian_accumulate", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
            "gq_damp_cholesky_inverse_noalloc",
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
-           "gq_recon_workspace_size", "gq_recon_error")
+           "gq_recon_workspace_size", "gq_recon_error", "gq_kernel_timer_start",
+           "gq_kernel_timer_stop", "gq_kernel_timer_read", "gq_kernel_timer_release")
 
 
 def _check(status: int, where: str) -> None:
@@ -284,3 +293,46 @@ def recon_error(W: torch.Tensor, q: dict, X: torch.Tensor, group_size: int = -1,
                               _p(ws), ws.numel(), _stream(stream))
     _check(st, "gq_recon_error")
     return (sse_h.value, mse_h.value) if sync else sse
+
+
+# ------------------------------------------------------------------ per-launch kernel timing
+
+# gq_kernel values (include/gq.h) and the unit of each kernel's work figure
+KERNELS = ("hessian_mma", "potrf_trsm", "block_inverse", "gemm_tf32x3", "gptq_block", "rtn",
+           "recon_mma")
+KERNEL_UNITS = {"hessian_mma": "flop", "potrf_trsm": "flop", "block_inverse": "flop",
+                "gemm_tf32x3": "flop", "gptq_block": "byte", "rtn": "byte", "recon_mma": "flop"}
+
+
+def kernel_timer_start(kernels, capacity: int) -> None:
+    """Time every launch of the named kernels (up to ``capacity`` launches)."""
+    mask = 0
+    for k in kernels:
+        mask |= 1 << KERNELS.index(k)
+    _check(lib().gq_kernel_timer_start(mask, int(capacity)), "gq_kernel_timer_start")
+
+
+def kernel_timer_stop() -> None:
+    _check(lib().gq_kernel_timer_stop(), "gq_kernel_timer_stop")
+
+
+def kernel_timer_read() -> list:
+    """[(kernel name, ms, algorithmic work)] of the recorded launches (their
+    last execution); call after the work has finished."""
+    import numpy as np
+    L = lib()
+    n = L.gq_kernel_timer_read(None, None, None, 0)
+    if n < 0:
+        _check(8, "gq_kernel_timer_read")
+    kind = np.zeros(max(n, 1), dtype=np.int32)
+    ms = np.zeros(max(n, 1), dtype=np.float32)
+    work = np.zeros(max(n, 1), dtype=np.float64)
+    m = L.gq_kernel_timer_read(kind.ctypes.data, ms.ctypes.data, work.ctypes.data, n)
+    if m < 0:
+        _check(8, "gq_kernel_timer_read")
+    return [(KERNELS[k], float(t), float(w)) for k, t, w in zip(kind[:n], ms[:n], work[:n])
+            if k >= 0]
+
+
+def kernel_timer_release() -> None:
+    _check(lib().gq_kernel_timer_release(), "gq_kernel_timer_release")

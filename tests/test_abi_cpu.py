@@ -87,3 +87,13 @@ def test_other_argument_errors():
     # recon: null sse_dev
     assert L.gq_recon_error(FAKE, 0, FAKE, FAKE, None, None, 8, 64, -1, 1, FAKE, 16, None,
                             None, None, FAKE, 1 << 30, None) == 1
+
+
+def test_kernel_timer_without_session():
+    L = gq.lib()
+    assert L.gq_kernel_timer_start(1, 0) == 1       # capacity must be positive
+    assert L.gq_kernel_timer_start(1, -5) == 1
+    assert L.gq_kernel_timer_read(None, None, None, 0) == 0
+    assert L.gq_kernel_timer_stop() == 0
+    assert L.gq_kernel_timer_release() == 0
+    assert set(gq.KERNEL_UNITS) == set(gq.KERNELS)
