@@ -1,0 +1,87 @@
+"""Run the path on one layer of a workload once, on the GPU, through the
+C-ABI library -- a fixed, small case for profilers (ncu) and for timing one
+stage by hand.
+
+    python -m post_weight_quantization_27_b200.cases --workload 2 --layer 3
+           [--tokens N] [--repeat R] [--stages hessian,solve,gptq,rtn,recon]
+
+The stages always run in path order (H -> damp/U -> GPTQ -> RTN -> recon),
+each as many times as --repeat says; a stage that is not listed still runs
+once if a later listed stage needs its output.  Prints one line per stage
+with its CUDA-event time.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import gq
+from . import inputs as I
+
+ORDER = ("hessian", "solve", "gptq", "rtn", "recon")
+
+
+def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) -> dict:
+    spec = I.workload_layers(workload)[layer]
+    if tokens is not None:
+        spec = spec.with_tokens(tokens)
+    W = I.make_weights(spec).cuda()
+    X = I.make_x_device(spec, "cuda")
+    last = max(ORDER.index(s) for s in stages)
+    need = set(stages) | set(ORDER[:last])
+    if "recon" in stages:
+        need |= {"gptq"}
+    times = {}
+
+    def timed(name, fn):
+        n = repeat if name in stages else 1
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        out = None
+        e0.record()
+        for _ in range(n):
+            out = fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times[name] = e0.elapsed_time(e1) / n
+        return out
+
+    H = U = perm = dead = q = None
+    if "hessian" in need:
+        H = timed("hessian", lambda: gq.hessian(X))
+    if "solve" in need:
+        Hs = H.clone()
+        U, perm, dead, _ = timed("solve", lambda: gq.damp_cholesky_inverse(
+            Hs.copy_(H), spec.damp, act_order=spec.act_order))
+    if "gptq" in need:
+        q = timed("gptq", lambda: gq.gptq_quantize_layer(
+            W, U, 4, spec.group_size, spec.block_size, spec.sym, perm=perm, dead=dead))
+    if "rtn" in need:
+        timed("rtn", lambda: gq.rtn_quantize_pack(W, 4, spec.group_size, spec.sym))
+    if "recon" in need:
+        timed("recon", lambda: gq.recon_error(W, q, X, spec.group_size, spec.sym))
+    return {"spec": spec, "ms": times}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--layer", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--repeat", type=int, default=1)
+    ap.add_argument("--stages", default=",".join(ORDER))
+    a = ap.parse_args()
+    stages = [s for s in a.stages.split(",") if s]
+    for s in stages:
+        if s not in ORDER:
+            raise SystemExit(f"unknown stage {s!r}; stages are {', '.join(ORDER)}")
+    r = run(a.workload, a.layer, a.tokens, stages, a.repeat)
+    sp = r["spec"]
+    print(f"workload {a.workload} layer {a.layer} ({sp.name}: {sp.d_in} -> {sp.d_out}, "
+          f"{sp.n_tok} tokens)")
+    for k, v in r["ms"].items():
+        print(f"  {k:8s} {v:10.3f} ms")
+
+
+if __name__ == "__main__":
+    main()

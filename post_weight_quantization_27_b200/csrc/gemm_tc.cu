@@ -8,17 +8,24 @@
 // high part h = a with the low 13 mantissa bits cleared and the remainder
 // l = a - h (exact in fp32), and the product is h_a h_b + h_a l_b + l_a h_b
 // (three tcgen05.mma kind::tf32; the dropped l_a l_b and the TF32 rounding
-// of l are ~2^-20 relative).
+// of l are ~2^-20 relative).  The tensor core reads only the high 19 bits of
+// each 32-bit TF32 operand (results are bit-identical whether the low 13
+// bits are cleared or not), so the staged fp32 tile itself serves as h and
+// only l is written.
 //
 // Persistent kernel, one CTA per SM, 128 x 128 output tiles, K in steps of
 // 32 (one 128-byte swizzle row of fp32):
 //   warp 0     TMA loads of the fp32 A and B tiles (no multicast)
-//   warps 2-5  split each staged element in place into h and l (l into a
-//              second buffer), then make the writes visible to the async
-//              proxy before releasing the stage to the MMA warp
+//   warps 2-5  write l = a - h of each staged element into a second buffer,
+//              then make the writes visible to the async proxy before
+//              releasing the stage to the MMA warp
 //   warp 1     three MMAs per 8-wide K step into one of two TMEM
 //              accumulators (the epilogue of one tile overlaps the next)
-//   warps 6-9  C = beta C + alpha acc from TMEM, one row per thread
+//   warps 6-9  epilogue: the C tile is fetched by TMA into a staging buffer
+//              while the tile's MMAs run; each thread (one accumulator row)
+//              forms beta C + alpha acc in the staging buffer, and TMA
+//              stores it (clipped at the matrix edge).  Global memory is
+//              only touched by whole-tile TMA copies.
 // A is K-major (A(m, k) = A[m lda + k]); B is either K-major (B(k, n) =
 // B[n ldb + k]) or N-major (B(k, n) = B[k ldb + n]); an N-major TF32 operand
 // must be staged with the 32-byte-atom variant of the 128-byte swizzle.  With `lower` only
@@ -29,12 +36,13 @@
 namespace gq {
 namespace {
 
-constexpr int TM = 128, TN = 128, TK = 32, STAGES = 3;
+constexpr int TM = 128, TN = 128, TK = 32, STAGES = 2;
 constexpr int TILE_BYTES = TM * TK * 4;         // 16 KB, A or B tile
 constexpr int STAGE_BYTES = 4 * TILE_BYTES;     // A_h, A_l, B_h, B_l
+constexpr int C_BYTES = TM * TN * 4;            // C staging: 4 boxes [128 rows][32 fp32]
 constexpr int NUM_THREADS = 320;
 constexpr uint32_t TMEM_COLS = 256;
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + C_BYTES + 1024 + 256;
 
 struct TcArgs {
   int M, N, K;
@@ -65,10 +73,6 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Tile t -> (mt, nt); lower: only nt <= mt, enumerated row by row.
 __device__ __forceinline__ void tile_of(const TcArgs &a, int t, int &mt, int &nt) {
   if (!a.lower) {
@@ -85,18 +89,21 @@ __device__ __forceinline__ void tile_of(const TcArgs &a, int t, int &mt, int &nt
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA,
-                       const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmC, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint8_t *cs = smem + STAGES * STAGE_BYTES;  // C staging, 1024-byte aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(cs + C_BYTES);
   uint64_t *full = bars;                  // TMA landed
   uint64_t *split = bars + STAGES;        // h / l split done
   uint64_t *empty = bars + 2 * STAGES;    // MMAs done with the stage
   uint64_t *acc_full = bars + 3 * STAGES;
   uint64_t *acc_empty = acc_full + 2;
   uint64_t *drain = acc_empty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  uint64_t *c_full = drain + 1;           // C tile landed in the staging buffer
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -110,6 +117,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&acc_empty[b], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(c_full, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -119,6 +127,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
   }
   tc_fence_before();
   __syncthreads();
@@ -173,7 +182,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < TILE_BYTES / 16 / 128; ++i) {
             const int idx = ct + 128 * i;
-            float4 v = hp[idx];
+            const float4 v = hp[idx];
             float4 h, l;
             h.x = __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
             h.y = __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
@@ -183,7 +192,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             l.y = v.y - h.y;
             l.z = v.z - h.z;
             l.w = v.w - h.w;
-            hp[idx] = h;
             lp[idx] = l;
           }
         }
@@ -241,58 +249,78 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) set_status(a.status, kDevTimeout);
     }
   } else {
-    // ---------------- epilogue: warps 6..9
+    // ---------------- epilogue: warps 6..9 (thread = accumulator row)
     const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;               // row within the tile
+    const bool leader = threadIdx.x == 192;          // issues the C copies
+    const bool need_c = a.beta != 0.0f || a.lower != 0;
     uint32_t ch = 0;
     bool ok = true;
+    auto load_c = [&](int t) {
+      int mt, nt;
+      tile_of(a, t, mt, nt);
+      mbar_arrive_expect_tx(c_full, C_BYTES);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tma_load_2d(cs + q * (C_BYTES / 4), &tmC, c_full, nt * TN + 32 * q, mt * TM);
+    };
+    if (leader && need_c && static_cast<int>(blockIdx.x) < a.n_tiles) load_c(blockIdx.x);
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++ch) {
       int mt, nt;
       tile_of(a, t, mt, nt);
       const uint32_t buf = ch & 1, use = ch >> 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1));
+      bool got = true;
+      if (need_c) got = mbar_wait(c_full, ch & 1);
+      got = mbar_wait(&acc_full[buf], use & 1) && got;
+      ok = __all_sync(0xffffffffu, got);
       if (!ok) break;
       tc_fence_after();
-      const int m = mt * TM + quarter * 32 + lane;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * TN;
-      float *crow = a.C + static_cast<int64_t>(m) * a.ldc + nt * TN;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      const int m = mt * TM + r;
+      const bool diag = a.lower && mt == nt;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
         float v[32];
-        tmem_ld32(taddr + c * 32, v);
-        if (m < a.M) {
+        tmem_ld32(taddr + q * 32, v);
+        uint8_t *row = cs + q * (C_BYTES / 4) + r * 128;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const int n = nt * TN + c * 32 + i;
-            if (n + 3 < a.N && (!a.lower || n + 3 <= m)) {
-              float4 *p = reinterpret_cast<float4 *>(crow + c * 32 + i);
-              float4 o = make_float4(a.alpha * v[i], a.alpha * v[i + 1], a.alpha * v[i + 2],
-                                     a.alpha * v[i + 3]);
-              if (a.beta != 0.0f) {
-                const float4 old = *p;
-                o.x = fmaf(a.beta, old.x, o.x);
-                o.y = fmaf(a.beta, old.y, o.y);
-                o.z = fmaf(a.beta, old.z, o.z);
-                o.w = fmaf(a.beta, old.w, o.w);
-              }
-              *p = o;
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int ne = n + e;
-                if (ne < a.N && (!a.lower || ne <= m)) {
-                  float *p = crow + c * 32 + i + e;
-                  const float o = a.alpha * v[i + e];
-                  *p = a.beta != 0.0f ? fmaf(a.beta, *p, o) : o;
-                }
-              }
-            }
+        for (int c = 0; c < 8; ++c) {
+          // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+          float4 *p = reinterpret_cast<float4 *>(row + ((c ^ (r & 7)) << 4));
+          const float4 old = need_c ? *p : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 o;
+          o.x = fmaf(a.beta, old.x, a.alpha * v[4 * c]);
+          o.y = fmaf(a.beta, old.y, a.alpha * v[4 * c + 1]);
+          o.z = fmaf(a.beta, old.z, a.alpha * v[4 * c + 2]);
+          o.w = fmaf(a.beta, old.w, a.alpha * v[4 * c + 3]);
+          if (diag) {  // keep the strict upper part of a diagonal tile
+            const int n = nt * TN + 32 * q + 4 * c;
+            if (n > m) o.x = old.x;
+            if (n + 1 > m) o.y = old.y;
+            if (n + 2 > m) o.z = old.z;
+            if (n + 3 > m) o.w = old.w;
           }
+          *p = o;
         }
       }
+      // the accumulator buffer is free once its columns are in registers
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (leader) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tma_store_2d(&tmC, cs + q * (C_BYTES / 4), nt * TN + 32 * q, mt * TM);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // staging buffer reusable
+        const int tn = t + static_cast<int>(gridDim.x);
+        if (need_c && tn < a.n_tiles) load_c(tn);
+      }
+      named_bar_sync(1, 128);
     }
+    if (leader) bulk_wait_group0();
     if (!ok && lane == 0) set_status(a.status, kDevTimeout);
   }
 
@@ -308,7 +336,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace
 
 // C (M x N, ldc) = beta C + alpha A B; see the file comment for layouts.
-// All pointers 16-byte aligned, lda / ldb / ldc multiples of 4.
+// All pointers 16-byte aligned, lda / ldb / ldc multiples of 4.  C may
+// overlap A or B only when beta == 0 and every C tile is the B tile of its
+// own columns (an in-place left multiplication); tiles of C are read (beta
+// != 0 or lower) and written whole, so with `lower` the strict upper part of
+// a diagonal tile is written back unchanged.
 gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
                              const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
                              int64_t ldc, bool lower, int *status, cudaStream_t st) {
@@ -321,6 +353,9 @@ gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, i
   else
     s = make_tmap_2d(&tB, B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, K, ldb, 32, TK,
                      CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+  if (s != GQ_OK) return s;
+  CUtensorMap tC;
+  s = make_tmap_2d(&tC, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, M, ldc, 32, TM);
   if (s != GQ_OK) return s;
   TcArgs a{};
   a.M = M;
@@ -341,7 +376,7 @@ gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, i
                        static_cast<int>(SMEM_BYTES));
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();
   const int slot = timer_begin(GQ_KERNEL_GEMM_TF32X3, st);
-  gemm_tf32x3_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tA, tB, a);
+  gemm_tf32x3_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tA, tB, tC, a);
   count_launch();
   // the fp32 product: 2 M N K flops, M (M + 1) K for the lower triangle
   timer_end(slot, st,
