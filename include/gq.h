@@ -192,7 +192,13 @@ gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, float damp_pe
  *   g_idx      [d_in] int32 (out) or NULL: the group of each original
  *              column (position in perm / group_size)
  *   ws         >= gq_gptq_workspace_size(d_out, d_in, block_size) bytes;
- *              holds the fp32 working copy of W.
+ *              holds the fp32 working copy of W (4 d_out d_in bytes) and
+ *              the scaled errors of one super-block (4 d_out S bytes).
+ * The lazy update is applied on two levels with the same terms: after a
+ * block, to the rest of its super-block of S columns (S = block_size times
+ * a power of two near sqrt(d_in / block_size)); after a super-block, to all
+ * columns beyond it at once.  Only the order of the fp32 sums differs from
+ * the one-level form.
  * ---------------------------------------------------------------------- */
 size_t gq_gptq_workspace_size(int64_t d_out, int64_t d_in, int block_size);
 gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,

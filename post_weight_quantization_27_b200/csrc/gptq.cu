@@ -14,9 +14,20 @@
 // for the whole block: the in-block update is register FMAs against
 // broadcast shared-memory reads, with no shuffles and no synchronisation.
 // A processed weight's register is reused for its scaled error delta, so
-// the Err block leaves the kernel in one contiguous store per row.  The
-// trailing update is a d_out x (d_in - end) x B GEMM on the tensor cores
+// the Err block leaves the kernel in one contiguous store per row.
+//
+// The lazy trailing update is done on two levels.  Columns are grouped in
+// super-blocks of S columns (S a power-of-two multiple of B near
+// sqrt(B d_in)); after each block only the rest of its super-block is
+// updated (K = B), and after each super-block the columns beyond it get
+// the whole super-block's update in one GEMM (K = S) from the scaled errors
+// of all its blocks.  Every update the single-level scheme applies is
+// applied, only summed in another order; the traffic over the trailing
+// weights drops from about d_in / 2B to about S / 2B + d_in / 2S fp32
+// read-writes per weight.  Both GEMMs are fp32 on the tensor cores
 // (gemm_tc.cu).
+#include <cmath>
+
 #include "gptq_block.cuh"
 
 namespace gq {
@@ -25,9 +36,19 @@ GQ_GPTQ_BLOCK_INSTANCES(GQ_DECLARE_BLOCK)
 
 namespace {
 
+// Super-block width: B times the power of two nearest (on a log scale)
+// sqrt(d_in / B), at most the block-rounded width of the layer.
+int64_t super_cols(int64_t d_in, int B) {
+  const double target = std::sqrt(static_cast<double>(B) * static_cast<double>(d_in));
+  int64_t S = B;
+  while (static_cast<double>(2 * S) <= target * 1.4142135623730951) S *= 2;
+  const int64_t full = (d_in + B - 1) / B * B;
+  return S < full ? S : full;
+}
+
 struct GptqWs {
   float *Wk;        // [d_out][d_in] fp32 working copy, processing order
-  float *Err;       // [d_out][B]
+  float *Err;       // [d_out][S] scaled errors of the current super-block
   uint8_t *codes;   // [d_out][d_in] codes in processing order (act-order only)
   int32_t *inv;     // [d_in] processing position of each original column
 };
@@ -38,7 +59,7 @@ GptqWs carve(void *ws, int64_t d_out, int64_t d_in, int B, bool with_perm) {
   w.Wk = reinterpret_cast<float *>(p);
   p += round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256);
   w.Err = reinterpret_cast<float *>(p);
-  p += round_up(static_cast<size_t>(d_out) * B * sizeof(float), 256);
+  p += round_up(static_cast<size_t>(d_out) * super_cols(d_in, B) * sizeof(float), 256);
   if (with_perm) {
     w.codes = p;
     p += round_up(static_cast<size_t>(d_out) * d_in, 256);
@@ -158,7 +179,8 @@ GptqBlockLaunch pick_block(int B, int G) {
 
 size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size) {
   return kWsHeader + round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256) +
-         round_up(static_cast<size_t>(d_out) * block_size * sizeof(float), 256) +
+         round_up(static_cast<size_t>(d_out) * super_cols(d_in, block_size) * sizeof(float),
+                  256) +
          round_up(static_cast<size_t>(d_out) * d_in, 256) +
          round_up(static_cast<size_t>(d_in) * sizeof(int32_t), 256);
 }
@@ -205,16 +227,28 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
                                      d_in, B, B, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (s != GQ_OK) return s;
   }
-  for (int64_t c0 = 0; c0 < d_in; c0 += B) {
-    const int bw = static_cast<int>(d_in - c0 < B ? d_in - c0 : B);
-    blk(tmU, w.Wk, d_out, d_in, c0, bw, sym, w.Err, perm ? nullptr : qpacked, w.codes, scales,
-        zeros, n_groups, status, st);
-    const int64_t c1 = c0 + bw;
-    if (c1 < d_in) {
-      // W[:, c1:] -= Err U[c0:c1, c1:] on the tensor cores
-      const gq_status s = launch_gemm_tf32x3(static_cast<int>(d_out), static_cast<int>(d_in - c1),
-                                             bw, -1.0f, w.Err, B, U + c0 * d_in + c1, d_in,
-                                             false, 1.0f, w.Wk + c1, d_in, false, status, st);
+  const int64_t S = super_cols(d_in, B);
+  for (int64_t s0 = 0; s0 < d_in; s0 += S) {
+    const int64_t s1 = s0 + S < d_in ? s0 + S : d_in;
+    for (int64_t c0 = s0; c0 < s1; c0 += B) {
+      const int bw = static_cast<int>(s1 - c0 < B ? s1 - c0 : B);
+      float *err = w.Err + (c0 - s0);
+      blk(tmU, w.Wk, d_out, d_in, c0, bw, sym, err, S, perm ? nullptr : qpacked, w.codes,
+          scales, zeros, n_groups, status, st);
+      const int64_t c1 = c0 + bw;
+      if (c1 < s1) {
+        // W[:, c1:s1] -= Err_blk U[c0:c1, c1:s1]
+        const gq_status s = launch_gemm_tf32x3(
+            static_cast<int>(d_out), static_cast<int>(s1 - c1), bw, -1.0f, err, S,
+            U + c0 * d_in + c1, d_in, false, 1.0f, w.Wk + c1, d_in, false, status, st);
+        if (s != GQ_OK) return s;
+      }
+    }
+    if (s1 < d_in) {
+      // W[:, s1:] -= Err_super U[s0:s1, s1:]
+      const gq_status s = launch_gemm_tf32x3(
+          static_cast<int>(d_out), static_cast<int>(d_in - s1), static_cast<int>(s1 - s0), -1.0f,
+          w.Err, S, U + s0 * d_in + s1, d_in, false, 1.0f, w.Wk + s1, d_in, false, status, st);
       if (s != GQ_OK) return s;
     }
   }

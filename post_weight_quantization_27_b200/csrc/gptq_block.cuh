@@ -73,14 +73,15 @@ __device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[S
 }
 
 // Wk: fp32 working weights [d_out][d_in] (processing order); the block is
-// columns c0 .. c0+bw-1.  Writes Err [d_out][B], and either the packed
-// codes (qpacked, no act-order) or one code byte per column (codes).
+// columns c0 .. c0+bw-1.  Writes the block's scaled errors to Err (row
+// stride err_ld >= B), and either the packed codes (qpacked, no act-order)
+// or one code byte per column (codes).
 // The B x B block of U arrives by one TMA copy (entries past the matrix
 // edge read as zero; only the upper triangle is used).
 template <int B, int G>
 __global__ void __launch_bounds__(128) gptq_block_kernel(
     const __grid_constant__ CUtensorMap tmU, const float *__restrict__ Wk, int64_t d_out,
-    int64_t d_in, int64_t c0, int bw, int sym, float *__restrict__ Err,
+    int64_t d_in, int64_t c0, int bw, int sym, float *__restrict__ Err, int64_t err_ld,
     uint32_t *__restrict__ qpacked, uint8_t *__restrict__ codes, uint16_t *__restrict__ scales,
     uint16_t *__restrict__ zeros, int64_t n_groups, int *status) {
   constexpr int SB = (G == 64) ? 64 : 32;
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(128) gptq_block_kernel(
     for (int i = 0; i < SB / 8; ++i) packed[i] = 0;
     gptq_column<SB, GS, 0>(w, packed, gp, rs, cx, jb);
 
-    float *err = Err + row * B + jb;
+    float *err = Err + row * err_ld + jb;
 #pragma unroll
     for (int k = 0; k < SB; k += 4)
       *reinterpret_cast<float4 *>(err + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(128) gptq_block_kernel(
 }
 
 typedef gq_status (*GptqBlockLaunch)(const CUtensorMap &, const float *, int64_t, int64_t,
-                                     int64_t, int, int, float *, uint32_t *, uint8_t *,
+                                     int64_t, int, int, float *, int64_t, uint32_t *, uint8_t *,
                                      uint16_t *, uint16_t *, int64_t, int *, cudaStream_t);
 
 // tmU: fp32 tensor map over U with a B x B box and no swizzle.  Rows per
@@ -192,8 +193,8 @@ typedef gq_status (*GptqBlockLaunch)(const CUtensorMap &, const float *, int64_t
 template <int B, int G>
 gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_out,
                             int64_t d_in, int64_t c0, int bw, int sym, float *Err,
-                            uint32_t *qp, uint8_t *codes, uint16_t *scales, uint16_t *zeros,
-                            int64_t n_groups, int *status, cudaStream_t st) {
+                            int64_t err_ld, uint32_t *qp, uint8_t *codes, uint16_t *scales,
+                            uint16_t *zeros, int64_t n_groups, int *status, cudaStream_t st) {
   const int sms = num_sms();
   const int rows = d_out >= 4 * 128 * sms ? 128 : (d_out >= 2 * 64 * sms ? 64 : 32);
   const size_t smem = (static_cast<size_t>(B) * (B + 1) + static_cast<size_t>(B) * rows) *
@@ -202,8 +203,9 @@ gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_o
                        static_cast<int>(smem));
   const unsigned grid = static_cast<unsigned>((d_out + rows - 1) / rows);
   const int slot = timer_begin(GQ_KERNEL_GPTQ_BLOCK, st);
-  gptq_block_kernel<B, G><<<grid, rows, smem, st>>>(tmU, Wk, d_out, d_in, c0, bw, sym, Err, qp,
-                                                    codes, scales, zeros, n_groups, status);
+  gptq_block_kernel<B, G><<<grid, rows, smem, st>>>(tmU, Wk, d_out, d_in, c0, bw, sym, Err,
+                                                    err_ld, qp, codes, scales, zeros, n_groups,
+                                                    status);
   count_launch();
   // working weights of the block read, Err written (fp32), the U block,
   // codes (packed: half a byte, else one byte per weight), scales (+ zeros)
@@ -220,8 +222,9 @@ gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_o
 
 #define GQ_BLOCK_SIG(b, g)                                                                  \
   gq_status launch_gptq_block<b, g>(const CUtensorMap &, const float *, int64_t, int64_t,      \
-                                    int64_t, int, int, float *, uint32_t *, uint8_t *,         \
-                                    uint16_t *, uint16_t *, int64_t, int *, cudaStream_t);
+                                    int64_t, int, int, float *, int64_t, uint32_t *,           \
+                                    uint8_t *, uint16_t *, uint16_t *, int64_t, int *,         \
+                                    cudaStream_t);
 #define GQ_DECLARE_BLOCK(b, g) extern template GQ_BLOCK_SIG(b, g)
 #define GQ_DEFINE_BLOCK(b, g) template GQ_BLOCK_SIG(b, g)
 
