@@ -132,46 +132,91 @@ __global__ void __launch_bounds__(256) gather_reversed_kernel(const float *__res
 }
 
 // ---------------------------------------------------------------- panel factor
-// Cholesky of the nb x nb diagonal block at (k0, k0) of the lower matrix A
-// (in place), and the inverse of that block written to linv [NB][NB].
-// The 128 columns are done in sub-panels of 32:
-//   (a) one warp factors the 32 x 32 diagonal piece with a row per lane in
-//       registers (pivot and column broadcast by shuffles);
-//   (b) one thread per row below solves x L^T = a with the row in registers;
-//   (c) all threads apply the sub-panel to the rest of the block in 4 x 4
-//       register tiles.
-// The inverse: each warp inverts one 32 x 32 diagonal block (a column per
-// lane), then X_ij = -X_ii (sum_k L_ik X_kj) for the blocks below, one
-// diagonal band at a time.
 constexpr int SP = NB + 1;  // padded row stride in shared memory (bank-conflict free columns)
+constexpr int TT = 2 * NB + 4;  // row stride of the transposed sub-panel (float4 aligned)
 
-// Column J of the warp's 32 x 32 Cholesky (lane = row, w = the row), unrolled
-// by template recursion so every register index is a constant.
-template <int J>
-__device__ __forceinline__ void chol32_column(float (&w)[32], float &my_rd, int lane, int64_t col0,
-                                              int nb_left, int *status) {
-  if constexpr (J < 32) {
-    float piv = __shfl_sync(0xffffffffu, w[J], J);
-    if (!(piv > 0.0f) || !(piv < FLT_MAX)) {
-      if (lane == 0 && J < nb_left) atomicMin(&status[1], static_cast<int>(col0 + J));
-      piv = 1.0f;
-    }
+// Factor the 32 x 32 piece at (c0, c0) of S in place with one warp (lane =
+// row, the row in registers); rd gets the reciprocals of its diagonal.
+// Column J: the pivot is broadcast by a shuffle, the column of L goes
+// through colbuf (32 floats, read back as broadcast float4s) to every
+// row's update.  The column loop is not unrolled (the body selects the
+// registers of column J by predicated moves), which keeps the code small:
+// a fully unrolled factor is large enough that its instruction fetches
+// dominate on an SM that has not run it recently.  Entries right of a
+// lane's diagonal are updated too; they are never read.  A pivot that is
+// not positive and finite is replaced by 1; returns the first such column
+// (32 if none).
+__device__ __forceinline__ int chol32_piece(float *S, float *rd, float *colbuf, int c0,
+                                            int lane) {
+  float w[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) w[k] = (k <= lane) ? S[(c0 + lane) * SP + c0 + k] : 0.0f;
+  float my_rd = 1.0f;
+  int bad = 32;
+#pragma unroll 1
+  for (int J = 0; J < 32; ++J) {
+    float wj = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) wj = (k == J) ? w[k] : wj;
+    float piv = __shfl_sync(0xffffffffu, wj, J);
+    const bool ill = !(piv > 0.0f) || !(piv < FLT_MAX);
+    bad = (ill && bad == 32) ? J : bad;
+    piv = ill ? 1.0f : piv;
     // 1 / sqrt(piv): hardware estimate plus one Newton step r (3 - piv r^2) / 2
     float rj = rsqrtf(piv);
     rj = rj * fmaf(-0.5f * piv, rj * rj, 1.5f);
-    const float dj = piv * rj;
-    const float lij = lane > J ? w[J] * rj : (lane == J ? dj : 0.0f);
-    w[J] = lij;
-    if (lane == J) my_rd = rj;
+    const float lij = lane > J ? wj * rj : (lane == J ? piv * rj : 0.0f);
+    my_rd = lane == J ? rj : my_rd;
+    colbuf[lane] = lij;
+    __syncwarp();
 #pragma unroll
-    for (int k = J + 1; k < 32; ++k) {
-      const float lkj = __shfl_sync(0xffffffffu, lij, k);
-      if (k <= lane) w[k] = fmaf(-lij, lkj, w[k]);
+    for (int k4 = 0; k4 < 8; ++k4) {
+      const float4 l4 = reinterpret_cast<const float4 *>(colbuf)[k4];
+      const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = 4 * k4 + e;
+        w[k] = (k == J) ? lij : fmaf(-lij, lk[e], w[k]);
+      }
     }
-    chol32_column<J + 1>(w, my_rd, lane, col0, nb_left, status);
+    __syncwarp();
   }
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    if (k <= lane) S[(c0 + lane) * SP + c0 + k] = w[k];
+  rd[c0 + lane] = my_rd;
+  return bad;
 }
-constexpr int TP = 33;      // stride of the 32 x 32 temporaries
+
+// One 8 x 8 register tile of the rank-32 update M[i][k] -= sum_j L[i][j] L[k][j]
+// from the transposed sub-panel T (T[j][q] = L of source row q, column j):
+// target rows are sources qi .. qi+7, target columns sources qk .. qk+7.
+__device__ __forceinline__ void update_tile8(const float *__restrict__ T, int qi, int qk,
+                                             float *dst, int dst_ld, bool tri, int i0, int k0) {
+  float acc[8][8];
+#pragma unroll
+  for (int x = 0; x < 8; ++x)
+#pragma unroll
+    for (int y = 0; y < 8; ++y) acc[x][y] = 0.0f;
+#pragma unroll 4
+  for (int j = 0; j < 32; ++j) {
+    const float4 a0 = *reinterpret_cast<const float4 *>(T + j * TT + qi);
+    const float4 a1 = *reinterpret_cast<const float4 *>(T + j * TT + qi + 4);
+    const float4 b0 = *reinterpret_cast<const float4 *>(T + j * TT + qk);
+    const float4 b1 = *reinterpret_cast<const float4 *>(T + j * TT + qk + 4);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+#pragma unroll
+      for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < 8; ++x)
+#pragma unroll
+    for (int y = 0; y < 8; ++y)
+      if (!tri || k0 + y <= i0 + x) dst[(i0 + x) * dst_ld + k0 + y] -= acc[x][y];
+}
 
 // ---------------------------------------------------------------- panel
 // One 128-column panel of the blocked Cholesky: the 128 x 128 diagonal
@@ -182,14 +227,18 @@ constexpr int TP = 33;      // stride of the 32 x 32 temporaries
 // factor to lpp ([NB][NB], identity padded), not back into A: with more
 // CTAs than fit on the GPU at once, later CTAs still read the unfactored
 // block from A after CTA 0 has finished.
-// The 128 columns go in sub-panels of 32:
+// The 128 columns go in sub-panels of 32 (c0 = 0, 32, 64, 96):
 //   (a) one warp factors the 32 x 32 diagonal piece, a row per lane in
 //       registers (pivot and column broadcast by shuffles);
 //   (b) one thread per row below the piece (in the diagonal block and in
-//       the CTA's own tile) solves x L^T = a with the row in registers;
-//   (c) all threads apply the sub-panel to the remaining columns of both,
-//       in 4 x 4 register tiles.
-constexpr size_t PANEL_SMEM = (2 * NB * SP + NB) * sizeof(float);
+//       the CTA's own rows) solves x L^T = a with the row in registers and
+//       also stores it transposed (T[j][q], q < 128: block row, q >= 128:
+//       own row q - 128), so that the update reads whole float4 runs;
+//   (c) the rank-32 update of the remaining columns in 8 x 8 register
+//       tiles, in two parts: first the next sub-panel's 32 columns (all
+//       warps), then the rest (warps 1-7) while warp 0 already factors the
+//       next diagonal piece, which only needs the first part.
+constexpr size_t PANEL_SMEM = (2 * NB * SP + NB + 32 * TT + 32) * sizeof(float);
 
 __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, int64_t d,
                                                          int64_t k0, int nb,
@@ -198,6 +247,8 @@ __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, 
   float *S = sm;            // [NB][SP]  the diagonal block, then its factor L (lower)
   float *P = S + NB * SP;   // [NB][SP]  this CTA's panel rows (CTA 0: unused)
   float *rd = P + NB * SP;  // [NB]      1 / L_jj
+  float *T = rd + NB;       // [32][TT]  the current sub-panel, transposed
+  float *colbuf = T + 32 * TT;  // [32]    one column of a 32 x 32 piece
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool own = blockIdx.x > 0;
   const int64_t row0 = k0 + static_cast<int64_t>(blockIdx.x) * NB;
@@ -244,26 +295,23 @@ __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, 
   }
   __syncthreads();
 
+  int bad = 32 * 4;  // first bad pivot column of the block (warp 0 lanes), 128 if none
+  if (warp == 0) {
+    const int b = chol32_piece(S, rd, colbuf, 0, lane);
+    bad = b < 32 ? b : bad;
+  }
   for (int c0 = 0; c0 < NB; c0 += 32) {
-    // (a) diagonal 32 x 32 piece
-    if (warp == 0) {
-      float w[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) w[k] = (k <= lane) ? S[(c0 + lane) * SP + c0 + k] : 0.0f;
-      float my_rd = 1.0f;
-      chol32_column<0>(w, my_rd, lane, k0 + c0, blockIdx.x == 0 ? nb - c0 : 0, status);
-#pragma unroll
-      for (int k = 0; k < 32; ++k)
-        if (k <= lane) S[(c0 + lane) * SP + c0 + k] = w[k];
-      rd[c0 + lane] = my_rd;
-    }
-    __syncthreads();
-    // (b) rows below the piece -- in the block, then the CTA's tile rows:
-    //     x = a L_dd^-T, right-looking within the row
-    const int below = NB - (c0 + 32);
+    __syncthreads();  // piece c0 factored; the previous update finished
+    // (b) rows below the piece -- in the block, then the CTA's rows:
+    //     x = a L_dd^-T, right-looking within the row; stored back and
+    //     transposed into T
+    const int base = c0 + 32;
+    const int below = NB - base;
     const int n_rows = below + (own ? NB : 0);
     for (int i = tid; i < n_rows; i += 256) {
-      float *row = i < below ? S + (c0 + 32 + i) * SP : P + (i - below) * SP;
+      const bool in_s = i < below;
+      float *row = in_s ? S + (base + i) * SP : P + (i - below) * SP;
+      const int q = in_s ? base + i : NB + (i - below);
       float a[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) a[k] = row[c0 + k];
@@ -275,63 +323,86 @@ __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, 
         for (int k = j + 1; k < 32; ++k) a[k] = fmaf(-x, S[(c0 + k) * SP + c0 + j], a[k]);
       }
 #pragma unroll
-      for (int k = 0; k < 32; ++k) row[c0 + k] = a[k];
+      for (int k = 0; k < 32; ++k) {
+        row[c0 + k] = a[k];
+        T[k * TT + q] = a[k];
+      }
     }
     __syncthreads();
-    // (c) remaining columns base.. of the block (lower part) and of the tile
-    //     rows: M[i][k] -= sum_j M[i][c0+j] S[k][c0+j]
-    const int base = c0 + 32;
-    const int mt = (NB - base) / 4;           // 4-wide column tiles left
-    const int n_s = mt * (mt + 1) / 2;        // lower tiles of the block
-    const int n_p = own ? (NB / 4) * mt : 0;  // tiles of the panel rows
-    for (int t = tid; t < n_s + n_p; t += 256) {
-      const float *src;
-      float *dst;
-      int i0, kk0;
-      bool tri;
-      if (t < n_s) {
-        int ti = 0;
-        while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-        const int tk = t - ti * (ti + 1) / 2;
-        i0 = base + 4 * ti;
-        kk0 = base + 4 * tk;
-        src = S;
-        dst = S;
-        tri = true;
-      } else {
-        const int u = t - n_s;
-        i0 = 4 * (u / mt);
-        kk0 = base + 4 * (u % mt);
-        src = P;
-        dst = P;
-        tri = false;
-      }
-      float acc[4][4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = 0.0f;
-#pragma unroll 8
-      for (int j = 0; j < 32; ++j) {
-        float pi[4], pk[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          pi[x] = src[(i0 + x) * SP + c0 + j];
-          pk[x] = S[(kk0 + x) * SP + c0 + j];
+    if (base >= NB) break;
+    // (c) 8 x 8 tiles over the remaining columns k >= base.  Column tile
+    //     tk (columns base + 8 tk ..), row tile ti of the block (rows base +
+    //     8 ti .., only tk <= ti) or tp of the own rows.
+    const int m8 = below / 8;
+    const int p8 = own ? NB / 8 : 0;
+    // part 1: the next sub-panel's columns (tk < 4), all warps
+    {
+      const int n_s = 4 * m8 - 6;       // block tiles with tk < 4 and tk <= ti
+      const int n_t = n_s + p8 * 4;
+      for (int t = tid; t < n_t; t += 256) {
+        int qi, tk;
+        bool tri;
+        float *dst;
+        int dld, i0;
+        if (t < n_s) {
+          // rows ti = 0..3 hold ti + 1 tiles, the rest 4
+          int ti, u = t;
+          if (u < 10) {
+            ti = u < 1 ? 0 : (u < 3 ? 1 : (u < 6 ? 2 : 3));
+            tk = u - ti * (ti + 1) / 2;
+          } else {
+            ti = 4 + (u - 10) / 4;
+            tk = (u - 10) % 4;
+          }
+          i0 = base + 8 * ti;
+          qi = i0;
+          dst = S;
+          dld = SP;
+          tri = ti == tk;
+        } else {
+          const int u = t - n_s;
+          const int tp = u / 4;
+          tk = u % 4;
+          i0 = 8 * tp;
+          qi = NB + i0;
+          dst = P;
+          dld = SP;
+          tri = false;
         }
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(pi[x], pk[y], acc[x][y]);
+        update_tile8(T, qi, base + 8 * tk, dst, dld, tri, i0, base + 8 * tk);
       }
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y)
-          if (!tri || kk0 + y <= i0 + x) dst[(i0 + x) * SP + kk0 + y] -= acc[x][y];
     }
     __syncthreads();
+    // part 2: columns beyond the next sub-panel (tk >= 4), warps 1-7, while
+    //         warp 0 factors the next diagonal piece
+    if (warp == 0) {
+      const int b = chol32_piece(S, rd, colbuf, base, lane);
+      bad = (b < 32 && bad == 128) ? base + b : bad;
+    } else if (m8 > 4) {
+      const int mr = m8 - 4;                      // column tiles tk = 4 .. m8-1
+      const int n_s = mr * (mr + 1) / 2;          // block tiles with 4 <= tk <= ti
+      const int n_t = n_s + p8 * mr;
+      for (int t = tid - 32; t < n_t; t += 224) {
+        int ti, tk;
+        if (t < n_s) {
+          int r = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
+          while (r * (r + 1) / 2 > t) --r;
+          while ((r + 1) * (r + 2) / 2 <= t) ++r;
+          ti = 4 + r;
+          tk = 4 + (t - r * (r + 1) / 2);
+          const int i0 = base + 8 * ti;
+          update_tile8(T, i0, base + 8 * tk, S, SP, ti == tk, i0, base + 8 * tk);
+        } else {
+          const int u = t - n_s;
+          const int tp = u / mr;
+          tk = 4 + u % mr;
+          update_tile8(T, NB + 8 * tp, base + 8 * tk, P, SP, false, 8 * tp, base + 8 * tk);
+        }
+      }
+    }
   }
+  if (blockIdx.x == 0 && warp == 0 && lane == 0 && bad < nb)
+    atomicMin(&status[1], static_cast<int>(k0 + bad));
 
   if (!own) {
     for (int e = tid; e < NB * NB; e += 256) {
@@ -347,6 +418,8 @@ __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, 
     }
   }
 }
+
+constexpr int TP = 33;      // stride of the 32 x 32 temporaries
 
 // ---------------------------------------------------------------- block inverse
 // lp := L_pp^-1, in place, for the factored diagonal block that

@@ -19,10 +19,15 @@
 //     lane = one tile row per thread).  Short accumulation chains inside
 //     the tensor core keep the fp32 error small at 262144 tokens.
 //   * tiles are split over token ranges when there are too few tiles for
-//     the SMs; each (split, tile) writes its raw partial tile to the
-//     workspace and a second kernel adds the splits in a fixed order,
-//     scales by 2, adds the incoming H and mirrors the upper triangle:
-//     the result is deterministic and exactly symmetric.
+//     the SMs, or when a split makes the last wave of tiles less ragged;
+//     each (split, tile) writes its raw partial tile to the workspace and
+//     a second kernel adds the splits in a fixed order, scales by 2, adds
+//     the incoming H and mirrors the upper triangle: the result is
+//     deterministic and exactly symmetric.
+//   * tiles are taken in groups of 8 row blocks, column block by column
+//     block inside a group, so that the tiles in flight at one time share
+//     few X column slabs (the L2 then serves most of the operand traffic;
+//     row-major order would stream a new 256-column slab per tile).
 #include "gq_device.cuh"
 #include "gq_internal.h"
 
@@ -46,7 +51,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 
 struct HessArgs {
-  int n_bj, n_tiles, n_split, kb_per_split, nkb_total;
+  int n_bi, n_bj, n_tiles, n_split, kb_per_split, nkb_total;
   float *P;
   int *status;
 };
@@ -57,14 +62,40 @@ __host__ __device__ __forceinline__ int64_t tile_row_start(int64_t b, int64_t n_
   const int64_t k = b >> 1;
   return b * n_bj - (k * (k - 1) + (b & 1) * k);
 }
-__device__ __forceinline__ void tile_coords(int t, int n_bj, int &bi, int &bj) {
-  int lo = 0, hi = 2 * n_bj;  // row_start is increasing in b
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (tile_row_start(mid, n_bj) <= t) lo = mid; else hi = mid;
+constexpr int RASTER_G = 8;  // row blocks per raster group
+
+// Processing position r -> tile (bi, bj): groups of RASTER_G row blocks;
+// inside a group, column block j holds the group's row blocks b with
+// b <= 2j + 1 (the tiles of j that touch the upper triangle).
+__device__ __forceinline__ void raster_tile(int r, int n_bi, int n_bj, int &bi, int &bj) {
+  for (int b0 = 0; b0 < n_bi; b0 += RASTER_G) {
+    const int b1 = min(b0 + RASTER_G, n_bi);
+    const int jlo = b0 >> 1;
+    // column blocks jlo .. jm-1 hold 2j + 2 - b0 row blocks, jm .. n_bj-1 all b1 - b0
+    const int jm = max(jlo, min(n_bj, (b1 - 1) >> 1));
+    const int count = (jm - jlo) * (2 - b0) + (jm - jlo) * (jm + jlo - 1) + (n_bj - jm) * (b1 - b0);
+    if (r >= count) {
+      r -= count;
+      continue;
+    }
+    for (int j = jlo; j < n_bj; ++j) {
+      const int c = min(b1, 2 * j + 2) - b0;
+      if (r < c) {
+        bi = b0 + r;
+        bj = j;
+        return;
+      }
+      r -= c;
+    }
   }
-  bi = lo;
-  bj = (lo >> 1) + (t - static_cast<int>(tile_row_start(lo, n_bj)));
+  bi = 0;
+  bj = 0;
+}
+
+// Index of tile (bi, bj) in row-major order over the upper tiles (the
+// layout of the partial tiles in the workspace).
+__device__ __forceinline__ int natural_tile(int bi, int bj, int n_bj) {
+  return static_cast<int>(tile_row_start(bi, n_bj)) + (bj - (bi >> 1));
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -112,7 +143,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         const int split = item / a.n_tiles, t = item % a.n_tiles;
         int bi, bj;
-        tile_coords(t, a.n_bj, bi, bj);
+        raster_tile(t, a.n_bi, a.n_bj, bi, bj);
         const int kb0 = split * a.kb_per_split;
         const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
@@ -207,7 +238,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
       }
       if (!ok) break;
-      float *dst = a.P + (static_cast<size_t>(item) * BM + row) * BN + half * 128;
+      int bi, bj;
+      raster_tile(item % a.n_tiles, a.n_bi, a.n_bj, bi, bj);
+      const size_t slot = static_cast<size_t>(split) * a.n_tiles + natural_tile(bi, bj, a.n_bj);
+      float *dst = a.P + (slot * BM + row) * BN + half * 128;
 #pragma unroll
       for (int c = 0; c < 128; c += 4)
         *reinterpret_cast<float4 *>(dst + c) = make_float4(m[c], m[c + 1], m[c + 2], m[c + 3]);
@@ -265,11 +299,26 @@ HessPlan hessian_plan(int64_t n_tok, int64_t d_in) {
   p.n_tiles = static_cast<int>(tile_row_start(p.n_bi, p.n_bj));
   p.nkb_total = static_cast<int>((n_tok + BK - 1) / BK);
   int split = 1;
-  const int target = 2 * num_sms();
+  const int sms = num_sms();
+  const int target = 2 * sms;
   if (p.nkb_total > 0 && p.n_tiles < target) {
     const int want = (target + p.n_tiles - 1) / p.n_tiles;
     const int most = p.nkb_total / 4 > 1 ? p.nkb_total / 4 : 1;
     split = want < most ? want : most;
+  } else if (p.nkb_total > 0) {
+    // enough tiles: split (2..4 ways, each split >= 256 k-blocks) only when
+    // that fills the last wave of the persistent grid noticeably better
+    auto fill = [&](int sp) {
+      const int64_t items = static_cast<int64_t>(p.n_tiles) * sp;
+      const int64_t waves = (items + sms - 1) / sms;
+      return static_cast<double>(items) / static_cast<double>(waves * sms);
+    };
+    double best = fill(1);
+    for (int sp = 2; sp <= 4; ++sp)
+      if (p.nkb_total / sp >= 256 && fill(sp) > best + 0.02) {
+        best = fill(sp);
+        split = sp;
+      }
   }
   if (p.nkb_total == 0) {
     p.n_split = 0;
@@ -299,7 +348,7 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
                            static_cast<int>(SMEM_BYTES));
       attr_set = true;
     }
-    HessArgs a{p.n_bj, p.n_tiles, p.n_split, p.kb_per_split, p.nkb_total, P, status};
+    HessArgs a{p.n_bi, p.n_bj, p.n_tiles, p.n_split, p.kb_per_split, p.nkb_total, P, status};
     const int grid = n_items < num_sms() ? n_items : num_sms();
     const int slot = timer_begin(GQ_KERNEL_HESSIAN_MMA, st);
     hessian_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, a);
