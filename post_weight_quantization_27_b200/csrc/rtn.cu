@@ -123,6 +123,31 @@ __device__ __forceinline__ uint32_t pack_word(const float (&v)[8], const GridPar
   return word;
 }
 
+// The same codes for a group whose quotients are known to be small (see
+// RtnGrid::fast): q = w / s needs no clamp before the magic-constant
+// rounding, C + rint(q) is exact, and the code is read from the bits of
+// that sum as an integer (symmetric: the range -7..7 is already guaranteed;
+// affine: rint(q) + z clamped to 0..15 in integer arithmetic).
+template <bool SYM>
+__device__ __forceinline__ uint32_t pack_word_small(const float (&v)[8], const GridParams &g,
+                                                    float rs, int zi) {
+  constexpr float C = 12582912.0f;  // 1.5 * 2^23; its low mantissa bits are 0
+  uint32_t word = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t t = __float_as_uint(__fadd_rn(div_by_recip(v[k], g.s, rs), C));
+    uint32_t nib;
+    if (SYM) {
+      nib = (t + 8u) & 0xFu;
+    } else {
+      const int c = static_cast<int>(t - __float_as_uint(C)) + zi;
+      nib = static_cast<uint32_t>(min(max(c, 0), 15));
+    }
+    word |= nib << (4 * k);
+  }
+  return word;
+}
+
 // Running statistic of a segment: max |w| (symmetric) or min and max (affine;
 // both start at 0, which is what the grid's range widening needs).
 template <bool SYM>
@@ -147,17 +172,24 @@ struct SegStat {
     }
   }
   // Same values as grid_sym / grid_affine, with the divisions by 7 and 15
-  // done from their correctly rounded reciprocals.
-  __device__ __forceinline__ GridParams grid() const {
+  // done from their correctly rounded reciprocals.  small: every finite
+  // weight of the segment has |w / s| < 7.5 (symmetric: the fp16 scale is
+  // a normal number, or the group is all but zero) or < 2^22 (affine: the
+  // scale did not saturate), so pack_word_small gives the same codes.
+  __device__ __forceinline__ GridParams grid(bool &small) const {
     GridParams g;
     float s32 = SYM ? div_by_recip(a, 7.0f, 1.0f / 7.0f)
                     : div_by_recip(__fsub_rn(b, a), 15.0f, 1.0f / 15.0f);
+    small = s32 <= 65504.0f;
     __half h = __float2half_rn(fminf(s32, 65504.0f));
     const bool degenerate = __half2float(h) == 0.0f;
     if (degenerate) h = __float2half_rn(1.0f);
     g.s = __half2float(h);
     g.s_bits = __half_as_ushort(h);
     if (SYM) {
+      // a normal fp16 scale is within 2^-11 of s32; a group whose s32 rounds
+      // to 0 in fp16 has |w| < 7 * 2^-25 and uses s = 1
+      small = small && ((g.s_bits & 0x7C00u) != 0 || degenerate);
       g.z = 0.0f;
       g.z_bits = 0;
     } else {
@@ -214,8 +246,10 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
       }
       st.reduce(TEAM);
       if (seg[u] >= total) continue;
-      const GridParams g = st.grid();
+      bool small;
+      const GridParams g = st.grid(small);
       const float rs = __frcp_rn(g.s);
+      const int zi = static_cast<int>(g.z);
       if (tl == 0) {
         scales[seg[u]] = g.s_bits;
         if (zeros) zeros[seg[u]] = SYM ? 0 : g.z_bits;
@@ -227,7 +261,7 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
         if (w < seg_words) {
           float v[8];
           raw[u][k].get(v);
-          dst[w] = pack_word<SYM>(v, g, rs);
+          dst[w] = small ? pack_word_small<SYM>(v, g, rs, zi) : pack_word<SYM>(v, g, rs);
         }
       }
     }
@@ -256,7 +290,8 @@ __global__ void __launch_bounds__(256) rtn_stream_kernel(const T *__restrict__ W
       for (int e = 0; e < 8; ++e) st.add(v[e]);
     }
     st.reduce(32);
-    const GridParams g = st.grid();
+    bool small;
+    const GridParams g = st.grid(small);
     const float rs = __frcp_rn(g.s);
     if (lane == 0) {
       scales[row] = g.s_bits;

@@ -110,3 +110,20 @@ def test_rtn_dense_midpoints(dt, group_size, sym):
     for idx in keep:                                        # the group's extremes stay,
         Wm.scatter_(2, idx, Wg.gather(2, idx))               # so its step is s16 above
     _check(Wm.reshape(d_out, d_in).to(DT[dt]), group_size, sym)
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+@pytest.mark.parametrize("group_size,sym", [(-1, True), (-1, False), (32, True), (32, False),
+                                            (128, True), (128, False)])
+def test_rtn_extreme_scales(dt, group_size, sym):
+    """Rows whose fp16 scale is subnormal, saturates at 65504, or is zero
+    (all-zero rows and rows that underflow), next to ordinary rows: the
+    kernels' short path for groups with small quotients and their general
+    path must both match the oracle."""
+    d_out, d_in = 60, 256
+    g = torch.Generator().manual_seed(5 + group_size + (0 if sym else 1))
+    W = torch.randn((d_out, d_in), generator=g)
+    mags = torch.tensor([1e-30, 1e-9, 3e-7, 2e-6, 1e-5, 0.02, 1.0, 3e5, 1e6, 1e9, 0.0, 6e4])
+    W = W * mags[torch.arange(d_out) % len(mags)][:, None]
+    W[5, :128] *= 1e-12                     # one row mixing tiny and ordinary groups
+    _check(W.to(DT[dt]), group_size, sym)
