@@ -33,6 +33,20 @@ struct ReconArgs {
   int *status;
 };
 
+// Tile t -> (row tile, token tile) in groups of 16 row tiles, token tile by
+// token tile inside a group: the tiles in flight at one time share a few
+// slabs of W - W^ and of X (row-tile-first order cycled all of W - W^
+// through the L2 for every couple of token tiles).
+constexpr int RASTER_GM = 16;
+__device__ __forceinline__ void recon_tile(int t, int n_mt, int n_nt, int &mt, int &nt) {
+  const int per_group = RASTER_GM * n_nt;
+  const int g = t / per_group;
+  const int r = t - g * per_group;
+  const int rows = min(RASTER_GM, n_mt - g * RASTER_GM);
+  mt = g * RASTER_GM + r % rows;
+  nt = r / rows;
+}
+
 // dW = W - s (c - z), split into bf16 hi + lo.
 template <typename T>
 __device__ __forceinline__ float ld_w(const T *p);
@@ -127,7 +141,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       uint32_t it = 0;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int mt = t % a.n_mt, nt = t / a.n_mt;
+        int mt, nt;
+        recon_tile(t, a.n_mt, a.n_nt, mt, nt);
         for (int kb = 0; kb < a.nkb; ++kb, ++it) {
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { ok = false; break; }
