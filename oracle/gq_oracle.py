@@ -50,6 +50,17 @@ Readings taken where the pages are silent, ambiguous or garbled:
 9. Act-order: perm = stable argsort(-diag H) after damping; groups are
    consecutive columns in permuted order; g_idx[c] is the group of original
    column c; codes are returned in original column order.
+10. Activation-aware scaling ("Model Quantization Mechanics", section 2.2;
+   "GPT-2 Quantization Reconstruction Error", "Possible extensions"): the
+   pages say only that input channel c's weights are multiplied by a
+   per-channel s_c chosen from the magnitude of that channel's activations,
+   and the activations divided by it.  Read as: magnitude a_c = the RMS of
+   x_c, taken from the undamped Hessian (H_cc = 2 sum_t x_tc^2); s_c =
+   (a_c / a_bar)^alpha with a_bar the geometric mean of the non-zero a_c
+   (s_c = 1 for a dead channel); alpha from the grid k / n_grid, k = 0 ..
+   n_grid - 1, the one with the smallest layer MSE (first on ties); the
+   quantised weights are RTN(W diag(s)) and the layer's effective weights
+   W^ = dequant(RTN(W diag(s))) diag(s)^-1.  alpha = 0 is plain RTN.
 """
 from __future__ import annotations
 
@@ -68,7 +79,7 @@ __all__ = [
     "GptqResult", "gptq_quantize", "dequantize_packed", "recon_sse",
     "recon_sse_trace", "bits_per_weight", "obs_quantize", "bruteforce_row",
     "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
-    "gptq_layer",
+    "gptq_layer", "awq_channel_scales", "awq_apply", "awq_rtn_search",
 ]
 
 
@@ -454,6 +465,56 @@ def recon_sse_trace(W, W_hat, H_undamped) -> float:
     undamped H = 2 X^T X (pin only)."""
     dW = np.asarray(W, dtype=np.float64) - np.asarray(W_hat, dtype=np.float64)
     return float(np.sum((dW @ H_undamped) * dW) / 2.0)
+
+
+# --------------------------------------------------------------------------
+# Activation-aware scaling before RTN (reading 10)
+# --------------------------------------------------------------------------
+
+def awq_channel_scales(H_diag, alpha) -> np.ndarray:
+    """s_c = (a_c / a_bar)^alpha in fp64 with a_c = sqrt(H_cc / 2N): the 2N
+    cancels, so s_c = (H_cc / H_bar)^(alpha / 2), H_bar the geometric mean of
+    the positive H_cc; s_c = 1 where H_cc <= 0 ("Model Quantization
+    Mechanics", section 2.2: per-channel scale from activation magnitude)."""
+    h = np.asarray(H_diag, dtype=np.float64)
+    pos = h > 0
+    s = np.ones_like(h)
+    if pos.any():
+        logbar = np.mean(np.log(h[pos]))
+        s[pos] = np.exp(0.5 * alpha * (np.log(h[pos]) - logbar))
+    return s
+
+
+def awq_apply(W, s32, group_size=-1, sym=True):
+    """RTN of W diag(s) (the product taken in fp32, as stored), and the
+    effective weights dequant(...) diag(s)^-1 in fp64."""
+    s32 = np.asarray(s32, dtype=F32)
+    Wp = (np.asarray(W, dtype=F32) * s32[None, :]).astype(F32)
+    r = rtn_quantize(Wp, group_size, sym)
+    g = Wp.shape[1] if group_size == -1 else group_size
+    gi = np.arange(Wp.shape[1]) // g
+    What = dequantize_codes(r["codes"], r["scales"][:, gi].astype(np.float64),
+                            r["zeros"][:, gi].astype(np.float64))
+    return r, What / s32.astype(np.float64)[None, :]
+
+
+def awq_rtn_search(W, X, group_size=-1, sym=True, n_grid=20):
+    """Grid search of alpha (reading 10): for each alpha = k / n_grid the layer
+    MSE ||(W - W^) X^T||^2 / (N d_out) of RTN after scaling; returns
+    dict(best, alpha, mse [n_grid], s (fp32, of the best alpha), rtn (the
+    RTN result of the best alpha: codes, scales, zeros, qpacked), W_hat)."""
+    X = np.asarray(X, dtype=np.float64)
+    hd = 2.0 * np.sum(X * X, axis=0)
+    n, d_out = X.shape[0], np.asarray(W).shape[0]
+    mse, keep = [], []
+    for k in range(n_grid):
+        s32 = awq_channel_scales(hd, k / n_grid).astype(F32)
+        r, What = awq_apply(W, s32, group_size, sym)
+        mse.append(recon_sse(W, What, X) / (n * d_out))
+        keep.append((s32, r, What))
+    best = int(np.argmin(mse))
+    s32, r, What = keep[best]
+    return dict(best=best, alpha=best / n_grid, mse=np.array(mse), s=s32, rtn=r, W_hat=What)
 
 
 # --------------------------------------------------------------------------

@@ -406,3 +406,65 @@ def test_tie_follow_only_at_ties():
     r2 = O.gptq_quantize(W2, U, group_size=-1, follow=dict(codes=tie, scales=b2.scales))
     assert r2.n_followed == 1 and r2.codes[1, 5] == 3
     assert np.array_equal(np.delete(r2.codes.ravel(), 1 * d + 5), np.delete(b2.codes.ravel(), 1 * d + 5))
+
+
+# ---------------------------------------------------------------- activation-aware scaling
+
+def _awq_case(seed=0, d_in=64, d_out=32, n=512):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((n, d_in))
+    X[:, 3] *= 50.0                       # two channels with large activations
+    X[:, 10] *= 20.0
+    W = rng.standard_normal((d_out, d_in)) * 0.02
+    return W, X
+
+
+def test_awq_scales_closed_form():
+    """s_c = (H_cc / H_bar)^(alpha/2): the geometric mean of the scales of the
+    live channels is 1, a dead channel gets 1, alpha = 0 gives all ones, and
+    the ratio of two channels' scales is (H_aa / H_bb)^(alpha/2)."""
+    h = np.array([4.0, 1.0, 0.0, 16.0, 0.25])
+    s = O.awq_channel_scales(h, 0.5)
+    live = h > 0
+    assert abs(np.exp(np.mean(np.log(s[live])))) == pytest.approx(1.0, rel=1e-14)
+    assert s[2] == 1.0
+    assert s[0] / s[1] == pytest.approx((4.0 / 1.0) ** 0.25, rel=1e-14)
+    assert np.all(O.awq_channel_scales(h, 0.0) == 1.0)
+
+
+def test_awq_alpha_zero_is_rtn():
+    """alpha = 0 scales nothing: the codes are plain RTN's and the curve's first
+    point is RTN's MSE, computed here by the trace route."""
+    W, X = _awq_case()
+    H = O.hessian(X)
+    for g, sym in ((-1, True), (32, False)):
+        res = O.awq_rtn_search(W, X, group_size=g, sym=sym, n_grid=10)
+        ref = O.rtn_quantize(W, g, sym)
+        Wr = O.dequantize_packed(ref["qpacked"], ref["scales"], ref["zeros"], W.shape[1], g, sym)
+        mse_rtn = O.recon_sse_trace(W, Wr, H) / (X.shape[0] * W.shape[0])
+        assert res["mse"][0] == pytest.approx(mse_rtn, rel=1e-9)
+        r0, _ = O.awq_apply(W, np.ones(W.shape[1], dtype=np.float32), g, sym)
+        assert np.array_equal(r0["codes"], ref["codes"])
+
+
+def test_awq_best_is_consistent_and_helps():
+    """The returned effective weights give the curve's minimum (trace route);
+    on inputs with outlier channels a positive alpha beats RTN clearly."""
+    W, X = _awq_case()
+    H = O.hessian(X)
+    res = O.awq_rtn_search(W, X, group_size=-1, sym=True, n_grid=10)
+    assert res["best"] == int(np.argmin(res["mse"]))
+    mse_best = O.recon_sse_trace(W, res["W_hat"], H) / (X.shape[0] * W.shape[0])
+    assert mse_best == pytest.approx(res["mse"][res["best"]], rel=1e-9)
+    assert res["best"] > 0 and res["mse"][res["best"]] < 0.5 * res["mse"][0]
+
+
+def test_awq_invariant_to_activation_scale():
+    """Scaling every activation by a constant leaves the scales and the choice
+    of alpha unchanged and multiplies the MSE curve by the constant squared."""
+    W, X = _awq_case(seed=3)
+    a = O.awq_rtn_search(W, X, group_size=32, sym=True, n_grid=8)
+    b = O.awq_rtn_search(W, 3.0 * X, group_size=32, sym=True, n_grid=8)
+    assert a["best"] == b["best"]
+    assert np.allclose(a["s"], b["s"], rtol=1e-6)
+    assert np.allclose(b["mse"], 9.0 * a["mse"], rtol=1e-6)
