@@ -255,6 +255,49 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
                          void *stream);
 
 /* ------------------------------------------------------------------------
+ * Activation-aware per-channel scaling before RTN.
+ * "Model Quantization Mechanics", section 2.2: a per-channel factor s
+ * multiplies the weights of input channels whose activations are large and
+ * divides those activations, so the layer's output is unchanged while its
+ * salient weights lose less to rounding; "GPT-2 Quantization Reconstruction
+ * Error", "Possible extensions": scale important channels, judged by
+ * activation magnitude, before quantising.  The pages give no formula; this
+ * call takes s_c = (H_cc / H_bar)^(alpha / 2) from the diagonal of the
+ * undamped Hessian H = 2 X^T X (the channel RMS over its geometric mean,
+ * to the power alpha; s_c = 1 where H_cc <= 0), tries alpha = k / n_grid
+ * for k = 0 .. n_grid - 1, measures each as the layer error
+ * ||(W - W^) X^T||^2 with W^ = dequant(RTN(W diag(s))) diag(s)^-1, and
+ * quantises the layer with the alpha of the smallest error (the first on
+ * ties).  alpha = 0 is plain RTN.
+ *
+ *   W, w_dtype   [d_out][d_in] (device, read only, 16-byte aligned)
+ *   H            [d_in][d_in] fp32 undamped Hessian (device; only the
+ *                diagonal is read), e.g. from gq_hessian_accumulate
+ *   X            [n_tok][d_in] bf16 calibration inputs (device, 16-byte
+ *                aligned), n_tok >= 1
+ *   bits, group_size, sym   as for gq_rtn_quantize_pack
+ *   n_grid       1 .. 256 (20 tries alpha = 0, 0.05, .., 0.95)
+ *   qpacked, scales, zeros  (out) RTN of W diag(s) for the chosen alpha, in
+ *                the layout of gq_rtn_quantize_pack; the dequantised
+ *                weights must be divided by col_scale per input column
+ *   col_scale    [d_in] fp32 (device, out) s of the chosen alpha, or NULL
+ *   mse_host     [n_grid] double (host, out) the error per alpha divided by
+ *                n_tok * d_out, or NULL
+ *   best_host    int32 (host, out) the chosen k, or NULL
+ *   ws           >= gq_awq_workspace_size(d_out, d_in, n_tok, group_size,
+ *                sym) bytes, 256-byte aligned
+ * Synchronises the stream once (the choice of alpha is made on the host).
+ * ---------------------------------------------------------------------- */
+size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size,
+                             int sym);
+gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
+                            const float *H, const void *X_bf16, int64_t n_tok, int bits,
+                            int group_size, int sym, int n_grid, uint32_t *qpacked,
+                            uint16_t *scales, uint16_t *zeros, float *col_scale,
+                            double *mse_host, int32_t *best_host, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/* ------------------------------------------------------------------------
  * Per-launch kernel timing (a measurement aid; the pages describe no such
  * facility).  A throughput figure for one kernel needs that kernel's own
  * duration, which events around a whole entry point (several kernels) do

@@ -3,12 +3,13 @@ C-ABI library -- a fixed, small case for profilers (ncu) and for timing one
 stage by hand.
 
     python -m post_weight_quantization_27_b200.cases --workload 2 --layer 3
-           [--tokens N] [--repeat R] [--stages hessian,solve,gptq,rtn,recon]
+           [--tokens N] [--repeat R] [--stages hessian,solve,gptq,rtn,recon,awq]
 
 The stages always run in path order (H -> damp/U -> GPTQ -> RTN -> recon),
 each as many times as --repeat says; a stage that is not listed still runs
 once if a later listed stage needs its output.  Prints one line per stage
-with its CUDA-event time.
+with its CUDA-event time.  "awq" is the activation-aware scaling search
+before RTN (20 values of alpha), which needs only H.
 """
 from __future__ import annotations
 
@@ -19,7 +20,7 @@ import torch
 from . import gq
 from . import inputs as I
 
-ORDER = ("hessian", "solve", "gptq", "rtn", "recon")
+ORDER = ("hessian", "solve", "gptq", "rtn", "recon", "awq")
 
 
 def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) -> dict:
@@ -32,6 +33,8 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
     need = set(stages) | set(ORDER[:last])
     if "recon" in stages:
         need |= {"gptq"}
+    if stages == ["awq"]:  # needs only H
+        need = {"hessian", "awq"}
     times = {}
 
     def timed(name, fn):
@@ -60,6 +63,8 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
         timed("rtn", lambda: gq.rtn_quantize_pack(W, 4, spec.group_size, spec.sym))
     if "recon" in need:
         timed("recon", lambda: gq.recon_error(W, q, X, spec.group_size, spec.sym))
+    if "awq" in need:
+        timed("awq", lambda: gq.awq_rtn_search(W, H, X, 4, spec.group_size, spec.sym, 20))
     return {"spec": spec, "ms": times}
 
 

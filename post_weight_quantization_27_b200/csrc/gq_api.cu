@@ -276,4 +276,36 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
   return GQ_OK;
 }
 
+size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size,
+                             int sym) {
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || n_tok < 1) return 0;
+  if (group_size != -1 && (group_size < 8 || group_size % 8 != 0 || d_in % group_size != 0))
+    return 0;
+  return awq_ws_bytes(d_out, d_in, n_tok, group_size, sym);
+}
+
+gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
+                            const float *H, const void *X_bf16, int64_t n_tok, int bits,
+                            int group_size, int sym, int n_grid, uint32_t *qpacked,
+                            uint16_t *scales, uint16_t *zeros, float *col_scale,
+                            double *mse_host, int32_t *best_host, void *ws, size_t ws_bytes,
+                            void *stream) {
+  t_last_error.clear();
+  GQ_TRY(check_dtype(w_dtype));
+  if (!W || !H || !X_bf16 || !qpacked || !scales) return fail(GQ_ERR_ARG, "null pointer");
+  if (bits != 4) return fail(GQ_ERR_ARG, "only bits == 4 is implemented");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
+  if (n_grid < 1 || n_grid > 256) return fail(GQ_ERR_ARG, "n_grid must be 1 .. 256");
+  GQ_TRY(check_layer(d_out, d_in));
+  GQ_TRY(check_group(group_size, d_in));
+  if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
+  if (!aligned(W, 16) || !aligned(X_bf16, 16))
+    return fail(GQ_ERR_ARG, "W and X must be 16-byte aligned");
+  GQ_TRY(check_ws(ws, ws_bytes, awq_ws_bytes(d_out, d_in, n_tok, group_size, sym)));
+  return launch_awq_rtn_search(W, w_dtype, d_out, d_in, H, X_bf16, n_tok, group_size, sym,
+                               n_grid, qpacked, scales, zeros, col_scale, mse_host, best_host,
+                               ws, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

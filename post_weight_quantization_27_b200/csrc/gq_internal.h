@@ -85,6 +85,15 @@ size_t recon_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok);
 gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
-                       int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st);
+                       int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
+                       const float *col_inv = nullptr);
+
+// Activation-aware scaling before RTN (awq.cu).
+size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int sym);
+gq_status launch_awq_rtn_search(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in,
+                                const float *H, const void *X, int64_t n_tok, int group_size,
+                                int sym, int n_grid, uint32_t *qpacked, uint16_t *scales,
+                                uint16_t *zeros, float *col_scale, double *mse_host,
+                                int32_t *best_host, void *ws, cudaStream_t st);
 
 }  // namespace gq

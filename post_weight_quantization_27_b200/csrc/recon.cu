@@ -47,7 +47,8 @@ __device__ __forceinline__ void recon_tile(int t, int n_mt, int n_nt, int &mt, i
   nt = r / rows;
 }
 
-// dW = W - s (c - z), split into bf16 hi + lo.
+// dW = W - s (c - z) (times col_inv[c] when given: the codes quantise
+// W diag(s_col) and col_inv = 1 / s_col), split into bf16 hi + lo.
 template <typename T>
 __device__ __forceinline__ float ld_w(const T *p);
 template <>
@@ -62,9 +63,9 @@ __device__ __forceinline__ float ld_w<__nv_bfloat16>(const __nv_bfloat16 *p) {
 template <typename T>
 __global__ void __launch_bounds__(256) dequant_diff_kernel(
     const T *__restrict__ W, const uint32_t *__restrict__ q, const uint16_t *__restrict__ scales,
-    const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx, int64_t d_out,
-    int64_t d_in, int group_size, int sym, __nv_bfloat16 *__restrict__ hi,
-    __nv_bfloat16 *__restrict__ lo) {
+    const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx,
+    const float *__restrict__ col_inv, int64_t d_out, int64_t d_in, int group_size, int sym,
+    __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo) {
   const int64_t words = d_in / 8;
   const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
   const int64_t n = d_out * words;
@@ -82,7 +83,8 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
       const float z = sym ? 0.0f : __half2float(__ushort_as_half(zeros[r * n_groups + gi]));
       const int nib = static_cast<int>((word >> (4 * k)) & 0xFu);
       const float code = static_cast<float>(sym ? nib - 8 : nib);
-      const float what = s * (code - z);
+      float what = s * (code - z);
+      if (col_inv) what *= col_inv[c];  // effective weight of a scaled layer
       const float dw = ld_w(W + r * d_in + c) - what;
       const __nv_bfloat16 hb = __float2bfloat16_rn(dw);
       h[k] = hb;
@@ -279,7 +281,8 @@ size_t recon_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok) {
 gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
-                       int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st) {
+                       int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
+                       const float *col_inv) {
   const ReconLayout L = recon_layout(d_out, d_in, n_tok);
   uint8_t *base = static_cast<uint8_t *>(ws);
   int *status = reinterpret_cast<int *>(base);
@@ -299,18 +302,18 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
   switch (dt) {
     case GQ_F32:
       dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
-                                                    scales, zeros, g_idx, d_out, d_in,
+                                                    scales, zeros, g_idx, col_inv, d_out, d_in,
                                                     group_size, sym, hi, lo);
       break;
     case GQ_F16:
       dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
-                                                     scales, zeros, g_idx, d_out, d_in,
-                                                     group_size, sym, hi, lo);
+                                                     scales, zeros, g_idx, col_inv, d_out,
+                                                     d_in, group_size, sym, hi, lo);
       break;
     case GQ_BF16:
       dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, d_out, d_in,
-          group_size, sym, hi, lo);
+          static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, col_inv, d_out,
+          d_in, group_size, sym, hi, lo);
       break;
   }
   count_launch();

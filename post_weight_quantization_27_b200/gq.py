@@ -72,6 +72,12 @@ def lib() -> ctypes.CDLL:
     L.gq_recon_error.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                                  _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp,
                                  _c_sz, _c_vp]
+    L.gq_awq_workspace_size.restype = _c_sz
+    L.gq_awq_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64, _c_int, _c_int]
+    L.gq_awq_rtn_search.restype = _c_int
+    L.gq_awq_rtn_search.argtypes = [_c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int,
+                                    _c_int, _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
+                                    _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_kernel_timer_start.restype = _c_int
     L.gq_kernel_timer_start.argtypes = [ctypes.c_uint32, ctypes.c_int32]
     L.gq_kernel_timer_stop.restype = _c_int
@@ -88,7 +94,8 @@ EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_w
            "gq_hessian_accumulate", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
            "gq_damp_cholesky_inverse_noalloc",
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
-           "gq_recon_workspace_size", "gq_recon_error", "gq_kernel_timer_start",
+           "gq_recon_workspace_size", "gq_recon_error", "gq_awq_workspace_size",
+           "gq_awq_rtn_search", "gq_kernel_timer_start",
            "gq_kernel_timer_stop", "gq_kernel_timer_read", "gq_kernel_timer_release")
 
 
@@ -293,6 +300,40 @@ def recon_error(W: torch.Tensor, q: dict, X: torch.Tensor, group_size: int = -1,
                               _p(ws), ws.numel(), _stream(stream))
     _check(st, "gq_recon_error")
     return (sse_h.value, mse_h.value) if sync else sse
+
+
+# ------------------------------------------------------------------ activation-aware scaling
+
+def awq_workspace_size(d_out: int, d_in: int, n_tok: int, group_size: int = -1,
+                       sym: bool = True) -> int:
+    return int(lib().gq_awq_workspace_size(d_out, d_in, n_tok, group_size, int(bool(sym))))
+
+
+def awq_rtn_search(W: torch.Tensor, H: torch.Tensor, X: torch.Tensor, bits: int = 4,
+                   group_size: int = -1, sym: bool = True, n_grid: int = 20,
+                   ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Per-channel activation-aware scaling before RTN (include/gq.h).
+    Returns the RTN outputs for the chosen alpha plus ``col_scale`` (device
+    fp32 [d_in]), ``mse`` (list of the error per alpha) and ``best`` (k)."""
+    import numpy as np
+    _dev(W, "W")
+    _dev(H, "H", torch.float32)
+    _dev(X, "X", torch.bfloat16)
+    d_out, d_in = W.shape
+    n_tok = X.shape[0]
+    o = _outputs(d_out, d_in, group_size, sym, W.device, False)
+    col = torch.empty(d_in, dtype=torch.float32, device=W.device)
+    mse = np.zeros(n_grid, dtype=np.float64)
+    best = ctypes.c_int32(-1)
+    ws = workspace(awq_workspace_size(d_out, d_in, n_tok, group_size, sym), W.device) \
+        if ws is None else ws
+    st = lib().gq_awq_rtn_search(_p(W), _DTYPES[W.dtype], d_out, d_in, _p(H), _p(X), n_tok, bits,
+                                 group_size, int(bool(sym)), n_grid, _p(o["qpacked"]),
+                                 _p(o["scales"]), _p(o["zeros"]), _p(col), mse.ctypes.data,
+                                 ctypes.byref(best), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_awq_rtn_search")
+    o.update(col_scale=col, mse=mse, best=int(best.value))
+    return o
 
 
 # ------------------------------------------------------------------ per-launch kernel timing
