@@ -33,10 +33,15 @@
  *     [d_out][d_in/8]; nibble k (bits 4k..4k+3) of word j is column 8j+k.
  *     Symmetric codes c in -7..7 are stored as c+8; affine codes 0..15 as is.
  *   - Scales and zeros are IEEE fp16 bit patterns (uint16), [d_out][n_groups]
- *     with n_groups = d_in / group_size, or 1 for group_size == -1.  Zeros
+ *     with n_groups = d_in / group_size, or 1 for group_size -1 and 0.  Zeros
  *     hold the integer zero-point 0..15 (0 for symmetric).
- *   - group_size is -1 (one group per output row) or a multiple of 8 that
- *     divides d_in; for GPTQ it is -1, 32, 64 or 128 and divides block_size.
+ *   - group_size is -1 (one group per output row), 0 (one scale for the
+ *     whole matrix -- "GPT-2 Quantization Reconstruction Error", "Possible
+ *     extensions": per-tensor scaling -- stored once per row, so the output
+ *     has the per-row layout and every consumer treats it like -1) or a
+ *     multiple of 8 that divides d_in; for GPTQ it is -1, 0, 32, 64 or 128
+ *     and divides block_size.  A per-tensor GPTQ scale comes from the whole
+ *     initial matrix, as a per-row one comes from the initial row.
  *   - Inputs must be finite; non-finite values give unspecified codes.
  */
 #ifndef GQ_H
@@ -180,7 +185,7 @@ gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, float damp_pe
  *   U          [d_in][d_in] fp32 upper factor from gq_damp_cholesky_inverse
  *              (in processing order)
  *   bits       4
- *   group_size -1, 32, 64 or 128, dividing d_in and block_size
+ *   group_size -1, 0 (per tensor), 32, 64 or 128, dividing d_in and block_size
  *   block_size 32, 64 or 128 (the pages' value is 128)
  *   sym        1 symmetric, 0 affine
  *   perm       [d_in] int32 processing order (act-order) or NULL

@@ -247,13 +247,22 @@ def bits_per_weight(d_out, d_in, group_size, sym, act_order=False):
 # --------------------------------------------------------------------------
 
 def rtn_quantize(W, group_size=-1, sym=True, bits=4):
-    """Round-to-nearest on the raw weights, per channel (group_size = -1) or
-    per group of consecutive weights in a row.
+    """Round-to-nearest on the raw weights, per channel (group_size = -1),
+    per tensor (group_size = 0: one scale for the whole matrix, "GPT-2
+    Quantization Reconstruction Error", "Possible extensions"; stored once
+    per row) or per group of consecutive weights in a row.
 
     Returns dict(codes [d_out, d_in] int, scales fp16 [d_out, n_groups],
     zeros fp16 [d_out, n_groups], qpacked uint32 [d_out, d_in / 8])."""
     W32 = np.asarray(W, dtype=F32)
     d_out, d_in = W32.shape
+    if group_size == 0:
+        s, z = (sym_params if sym else affine_params)(W32.reshape(1, -1), bits)
+        scales = np.full((d_out, 1), s[0], dtype=np.float16)
+        zeros = np.full((d_out, 1), z[0], dtype=np.float16)
+        codes = quantize_codes(W32, scales, zeros, sym, bits)
+        return dict(codes=codes, scales=scales, zeros=zeros,
+                    qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None)
     g = d_in if group_size == -1 else group_size
     n_groups = d_in // g
     codes = np.zeros((d_out, d_in), dtype=np.int64)
@@ -331,6 +340,9 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     if perm is not None:
         perm = np.asarray(perm, dtype=np.int64)
         W = W[:, perm]
+    per_tensor = group_size == 0   # one scale from the whole initial matrix
+    if per_tensor:
+        group_size = -1
     g = d_in if group_size == -1 else group_size
     if group_size != -1:
         assert d_in % g == 0 and block_size % g == 0
@@ -371,7 +383,10 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
             n_followed += int(take.sum())
         return s, z
 
-    if group_size == -1:
+    if per_tensor:
+        s, z = params(W.astype(F32).reshape(1, -1), bits)
+        scales[:, 0], zeros[:, 0] = s[0], z[0]
+    elif group_size == -1:
         s, z = group(W.astype(F32), 0)
         scales[:, 0], zeros[:, 0] = s, z
     for b0 in range(0, d_in, block_size):
@@ -439,7 +454,7 @@ def dequantize_packed(qpacked, scales, zeros, d_in, group_size, sym,
     """W^ from packed codes and the stored 16-bit scales / zeros."""
     c = unpack_nibbles(qpacked, d_in, sym, bits)
     if g_idx is None:
-        g = d_in if group_size == -1 else group_size
+        g = d_in if group_size <= 0 else group_size
         g_idx = np.arange(d_in) // g
     g_idx = np.asarray(g_idx, dtype=np.int64)
     s = np.asarray(scales)[:, g_idx]

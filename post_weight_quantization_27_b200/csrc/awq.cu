@@ -111,7 +111,7 @@ struct AwqWs {
 };
 
 AwqWs carve(void *ws, int64_t d_out, int64_t d_in, int group_size) {
-  const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
+  const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   uint8_t *p = static_cast<uint8_t *>(ws) + kWsHeader;
   AwqWs w{};
   auto take = [&](size_t bytes) {
@@ -134,7 +134,7 @@ AwqWs carve(void *ws, int64_t d_out, int64_t d_in, int group_size) {
 
 // Bytes that carve() lays out before the reconstruction workspace.
 size_t carve_bytes(int64_t d_out, int64_t d_in, int group_size) {
-  const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
+  const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   return kWsHeader + 3 * round_up(static_cast<size_t>(d_in) * 4, 256) + round_up(4, 256) +
          round_up(static_cast<size_t>(d_out) * d_in * 4, 256) +
          round_up(static_cast<size_t>(d_out) * (d_in / 8) * 4, 256) +

@@ -190,6 +190,8 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
                       const uint8_t *dead, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
                       int32_t *g_idx, void *ws, cudaStream_t st) {
   const int B = block_size;
+  const bool per_tensor = group_size == 0;  // one scale for the matrix, stored per row
+  if (per_tensor) group_size = -1;
   GptqBlockLaunch blk = pick_block(B, group_size);
   if (!blk) return fail(GQ_ERR_ARG, "unsupported (block_size, group_size) combination");
   GptqWs w = carve(ws, d_out, d_in, B, perm != nullptr);
@@ -213,7 +215,12 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
   }
   count_launch();
   const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
-  if (group_size == -1) {
+  if (per_tensor) {
+    const gq_status s = launch_tensor_params_f32(
+        w.Wk, d_out, d_in, sym, scales, zeros, w.Err,
+        d_out * super_cols(d_in, B), st);
+    if (s != GQ_OK) return s;
+  } else if (group_size == -1) {
     unsigned g2 = static_cast<unsigned>((d_out + 7) / 8);
     if (g2 > cap) g2 = cap;
     row_params_kernel<<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros);

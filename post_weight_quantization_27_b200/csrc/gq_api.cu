@@ -96,9 +96,9 @@ gq_status check_layer(int64_t d_out, int64_t d_in) {
 }
 
 gq_status check_group(int group_size, int64_t d_in) {
-  if (group_size == -1) return GQ_OK;
+  if (group_size == -1 || group_size == 0) return GQ_OK;
   if (group_size < 8 || group_size % 8 != 0 || d_in % group_size != 0)
-    return fail(GQ_ERR_SHAPE, "group_size must be -1 or a multiple of 8 dividing d_in");
+    return fail(GQ_ERR_SHAPE, "group_size must be -1, 0 or a multiple of 8 dividing d_in");
   return GQ_OK;
 }
 
@@ -215,8 +215,8 @@ gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out,
   GQ_TRY(check_group(group_size, d_in));
   if (block_size != 32 && block_size != 64 && block_size != 128)
     return fail(GQ_ERR_ARG, "block_size must be 32, 64 or 128");
-  if (group_size != -1 && (group_size < 32 || block_size % group_size != 0))
-    return fail(GQ_ERR_ARG, "GPTQ group_size must be -1, 32, 64 or 128 and divide block_size");
+  if (group_size > 0 && (group_size < 32 || block_size % group_size != 0))
+    return fail(GQ_ERR_ARG, "GPTQ group_size must be -1, 0, 32, 64 or 128 and divide block_size");
   if (!aligned(W, 16) || !aligned(U, 16)) return fail(GQ_ERR_ARG, "W and U must be 16-byte aligned");
   GQ_TRY(check_ws(ws, ws_bytes, gptq_ws_bytes(d_out, d_in, block_size)));
   return launch_gptq(W, w_dtype, d_out, d_in, U, group_size, block_size, sym, perm, dead,
@@ -279,8 +279,9 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
 size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size,
                              int sym) {
   if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || n_tok < 1) return 0;
-  if (group_size != -1 && (group_size < 8 || group_size % 8 != 0 || d_in % group_size != 0))
+  if (group_size > 0 && (group_size < 8 || group_size % 8 != 0 || d_in % group_size != 0))
     return 0;
+  if (group_size < -1) return 0;
   return awq_ws_bytes(d_out, d_in, n_tok, group_size, sym);
 }
 

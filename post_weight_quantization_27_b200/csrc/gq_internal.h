@@ -51,6 +51,10 @@ gq_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType d
 int num_sms();
 
 // ---- kernels (each returns GQ_OK or GQ_ERR_CUDA after launching) ----
+// group_size: -1 per row, 0 per tensor (one scale, stored once per row), else per group.
+gq_status launch_tensor_params_f32(const float *W, int64_t d_out, int64_t d_in, int sym,
+                                   uint16_t *scales, uint16_t *zeros, float *scratch,
+                                   int64_t scratch_floats, cudaStream_t st);
 gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, int group_size,
                      int sym, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
                      cudaStream_t st);

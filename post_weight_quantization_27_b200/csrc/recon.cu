@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
     const float *__restrict__ col_inv, int64_t d_out, int64_t d_in, int group_size, int sym,
     __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo) {
   const int64_t words = d_in / 8;
-  const int64_t n_groups = group_size == -1 ? 1 : d_in / group_size;
+  const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   const int64_t n = d_out * words;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * 256) {
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int64_t c = wd * 8 + k;
-      int64_t gi = g_idx ? g_idx[c] : (group_size == -1 ? 0 : c / group_size);
+      int64_t gi = g_idx ? g_idx[c] : (group_size <= 0 ? 0 : c / group_size);
       gi = gi < 0 ? 0 : (gi >= n_groups ? n_groups - 1 : gi);
       const float s = __half2float(__ushort_as_half(scales[r * n_groups + gi]));
       const float z = sym ? 0.0f : __half2float(__ushort_as_half(zeros[r * n_groups + gi]));
@@ -283,6 +283,7 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
                        int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
                        const float *col_inv) {
+  if (group_size == 0) group_size = -1;  // per-tensor scales are stored per row
   const ReconLayout L = recon_layout(d_out, d_in, n_tok);
   uint8_t *base = static_cast<uint8_t *>(ws);
   int *status = reinterpret_cast<int *>(base);

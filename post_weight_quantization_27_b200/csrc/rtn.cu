@@ -306,6 +306,131 @@ __global__ void __launch_bounds__(256) rtn_stream_kernel(const T *__restrict__ W
   }
 }
 
+// ---------------------------------------------------------------- per-tensor
+// One scale (and zero) for the whole matrix ("GPT-2 Quantization
+// Reconstruction Error", "Possible extensions": per-tensor, a single global
+// scale), stored once per row so that the output has the per-channel
+// layout.  Statistic of all weights (block partials, then one block), the
+// parameters, then the codes.
+template <bool SYM>
+__device__ __forceinline__ void block_combine(SegStat<SYM> &st, float *sa, float *sb) {
+  st.reduce(32);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    sa[warp] = st.a;
+    sb[warp] = st.b;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    st.a = lane < nw ? sa[lane] : 0.0f;
+    st.b = lane < nw ? sb[lane] : 0.0f;
+    st.reduce(32);
+  }
+}
+
+template <typename T, bool SYM>
+__global__ void __launch_bounds__(256) tensor_stat_kernel(const T *__restrict__ W, int64_t words,
+                                                          float *__restrict__ part) {
+  __shared__ float sa[8], sb[8];
+  SegStat<SYM> st;
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; w < words;
+       w += static_cast<int64_t>(gridDim.x) * 256) {
+    float v[8];
+    Vec8<T>::load(W + w * 8, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) st.add(v[e]);
+  }
+  block_combine<SYM>(st, sa, sb);
+  if (threadIdx.x == 0) {
+    part[2 * blockIdx.x] = st.a;
+    part[2 * blockIdx.x + 1] = st.b;
+  }
+}
+
+// part: n_part (a, b) pairs, or W itself (n_part == 0: a small tensor is
+// reduced here directly).
+template <typename T, bool SYM>
+__global__ void __launch_bounds__(256) tensor_params_kernel(const float *__restrict__ part,
+                                                            int n_part, const T *__restrict__ W,
+                                                            int64_t words, int64_t d_out,
+                                                            uint16_t *__restrict__ scales,
+                                                            uint16_t *__restrict__ zeros) {
+  __shared__ float sa[8], sb[8];
+  __shared__ uint16_t ps, pz;
+  SegStat<SYM> st;
+  if (n_part > 0) {
+    for (int i = threadIdx.x; i < n_part; i += 256) {
+      if (SYM) {
+        st.a = fmaxf(st.a, part[2 * i]);
+      } else {
+        st.a = fminf(st.a, part[2 * i]);
+        st.b = fmaxf(st.b, part[2 * i + 1]);
+      }
+    }
+  } else {
+    for (int64_t w = threadIdx.x; w < words; w += 256) {
+      float v[8];
+      Vec8<T>::load(W + w * 8, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) st.add(v[e]);
+    }
+  }
+  block_combine<SYM>(st, sa, sb);
+  if (threadIdx.x == 0) {
+    bool small;
+    const GridParams g = st.grid(small);
+    ps = g.s_bits;
+    pz = SYM ? 0 : g.z_bits;
+  }
+  __syncthreads();
+  for (int64_t r = threadIdx.x; r < d_out; r += 256) {
+    scales[r] = ps;
+    if (zeros) zeros[r] = pz;
+  }
+}
+
+template <typename T, bool SYM>
+__global__ void __launch_bounds__(256) tensor_pack_kernel(const T *__restrict__ W, int64_t words,
+                                                          const uint16_t *__restrict__ scales,
+                                                          const uint16_t *__restrict__ zeros,
+                                                          uint32_t *__restrict__ q) {
+  GridParams g{};
+  g.s = __half2float(__ushort_as_half(scales[0]));
+  g.z = SYM ? 0.0f : __half2float(__ushort_as_half(zeros[0]));
+  const float rs = __frcp_rn(g.s);
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; w < words;
+       w += static_cast<int64_t>(gridDim.x) * 256) {
+    float v[8];
+    Vec8<T>::load(W + w * 8, v);
+    q[w] = pack_word<SYM>(v, g, rs);
+  }
+}
+
+template <typename T, bool SYM>
+void launch_tensor_typed(const T *W, int64_t d_out, int64_t d_in, uint32_t *q, uint16_t *sc,
+                         uint16_t *z, float *scratch, int64_t scratch_floats, cudaStream_t st) {
+  const int64_t words = d_out * d_in / 8;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+  int64_t nb = (words + 255) / 256;
+  if (nb > cap) nb = cap;
+  if (nb > scratch_floats / 2) nb = scratch_floats / 2;
+  if (words <= 8192 || nb < 2) {  // small: one block reads the tensor itself
+    tensor_params_kernel<T, SYM><<<1, 256, 0, st>>>(nullptr, 0, W, words, d_out, sc, z);
+    count_launch();
+  } else {
+    tensor_stat_kernel<T, SYM><<<static_cast<unsigned>(nb), 256, 0, st>>>(W, words, scratch);
+    tensor_params_kernel<T, SYM><<<1, 256, 0, st>>>(scratch, static_cast<int>(nb), W, words,
+                                                    d_out, sc, z);
+    count_launch(2);
+  }
+  int64_t gp = (words + 255) / 256;
+  const int64_t gcap = static_cast<int64_t>(num_sms()) * 8;
+  if (gp > gcap) gp = gcap;
+  tensor_pack_kernel<T, SYM><<<static_cast<unsigned>(gp), 256, 0, st>>>(W, words, sc, z, q);
+  count_launch();
+}
+
 template <typename T, int TEAM, int WPL, int UNROLL>
 void launch_reg(const void *W, int64_t d_out, int64_t seg_words, int64_t n_groups, int sym,
                 uint32_t *q, uint16_t *sc, uint16_t *z, cudaStream_t st) {
@@ -330,6 +455,16 @@ void launch_reg(const void *W, int64_t d_out, int64_t seg_words, int64_t n_group
 template <typename T>
 gq_status launch_typed(const void *W, int64_t d_out, int64_t d_in, int group_size, int sym,
                        uint32_t *q, uint16_t *sc, uint16_t *z, cudaStream_t st) {
+  if (group_size == 0) {  // per-tensor; the packed output is the block partials' scratch
+    const T *w = static_cast<const T *>(W);
+    const int64_t scratch = d_out * d_in / 8;
+    float *part = reinterpret_cast<float *>(q);
+    if (sym)
+      launch_tensor_typed<T, true>(w, d_out, d_in, q, sc, z, part, scratch, st);
+    else
+      launch_tensor_typed<T, false>(w, d_out, d_in, q, sc, z, part, scratch, st);
+    return check_launch("rtn per-tensor");
+  }
   const int64_t seg_len = group_size == -1 ? d_in : group_size;
   const int64_t n_groups = d_in / seg_len;
   const int64_t words = seg_len / 8;
@@ -364,6 +499,33 @@ gq_status launch_typed(const void *W, int64_t d_out, int64_t d_in, int group_siz
 
 }  // namespace
 
+// Per-tensor grid parameters of an fp32 matrix (the GPTQ working copy),
+// written once per row; scratch holds the block partials.
+gq_status launch_tensor_params_f32(const float *W, int64_t d_out, int64_t d_in, int sym,
+                                   uint16_t *scales, uint16_t *zeros, float *scratch,
+                                   int64_t scratch_floats, cudaStream_t st) {
+  const int64_t words = d_out * d_in / 8;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+  int64_t nb = (words + 255) / 256;
+  if (nb > cap) nb = cap;
+  if (nb > scratch_floats / 2) nb = scratch_floats / 2;
+  const bool small = words <= 8192 || nb < 2;
+  if (!small) {
+    if (sym)
+      tensor_stat_kernel<float, true><<<static_cast<unsigned>(nb), 256, 0, st>>>(W, words, scratch);
+    else
+      tensor_stat_kernel<float, false><<<static_cast<unsigned>(nb), 256, 0, st>>>(W, words, scratch);
+    count_launch();
+  }
+  const int n_part = small ? 0 : static_cast<int>(nb);
+  if (sym)
+    tensor_params_kernel<float, true><<<1, 256, 0, st>>>(scratch, n_part, W, words, d_out, scales, zeros);
+  else
+    tensor_params_kernel<float, false><<<1, 256, 0, st>>>(scratch, n_part, W, words, d_out, scales, zeros);
+  count_launch();
+  return check_launch("per-tensor parameters");
+}
+
 gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, int group_size,
                      int sym, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
                      cudaStream_t st) {
@@ -388,7 +550,7 @@ gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, in
       s = fail(GQ_ERR_DTYPE, "unknown dtype");
   }
   // W read; codes (half a byte per weight), fp16 scales (and zeros) written
-  const double n_groups = group_size == -1 ? 1.0 : static_cast<double>(d_in / group_size);
+  const double n_groups = group_size <= 0 ? 1.0 : static_cast<double>(d_in / group_size);
   timer_end(slot, st,
             static_cast<double>(d_out) * d_in * (wb + 0.5) +
                 2.0 * d_out * n_groups * (sym ? 1 : 2));

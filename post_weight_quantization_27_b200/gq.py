@@ -220,7 +220,7 @@ def gptq_workspace_size(d_out: int, d_in: int, block_size: int = 128) -> int:
 
 
 def _n_groups(d_in: int, group_size: int) -> int:
-    return 1 if group_size == -1 else d_in // group_size
+    return 1 if group_size <= 0 else d_in // group_size
 
 
 def _outputs(d_out, d_in, group_size, sym, dev, with_g_idx):

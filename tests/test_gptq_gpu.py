@@ -68,6 +68,8 @@ def _run_gpu(W, X, group_size, sym, act_order=False, block_size=128, damp=0.01):
     (33, 200, 800, -1, True, "f32"),          # ragged last block (72 columns)
     (50, 512, 1500, 64, True, "f16"),
     (40, 512, 1500, 32, False, "f32"),
+    (96, 256, 512, 0, True, "f32"),           # per-tensor scale
+    (64, 384, 1000, 0, False, "bf16"),
 ])
 def test_gptq_end_to_end(d_out, d_in, n_tok, group_size, sym, dt):
     W, X = _layer(d_out, d_in, n_tok, d_out + d_in, dt)
@@ -134,7 +136,7 @@ def test_gptq_diagonal_hessian_is_rtn():
     X = torch.zeros((d_in, d_in), dtype=torch.bfloat16)
     X[torch.arange(d_in), torch.arange(d_in)] = torch.linspace(0.5, 3.0, d_in).to(torch.bfloat16)
     W, _ = _layer(48, d_in, 10, 13)
-    for gs, sym in ((-1, True), (128, False), (32, True)):
+    for gs, sym in ((-1, True), (128, False), (32, True), (0, True), (0, False)):
         out, _ = _run_gpu(W, X, gs, sym)
         rtn = gq.rtn_quantize_pack(W.cuda(), 4, gs, sym)
         torch.cuda.synchronize()

@@ -468,3 +468,38 @@ def test_awq_invariant_to_activation_scale():
     assert a["best"] == b["best"]
     assert np.allclose(a["s"], b["s"], rtol=1e-6)
     assert np.allclose(b["mse"], 9.0 * a["mse"], rtol=1e-6)
+
+
+
+# ---------------------------------------------------------------- per-tensor scales
+
+def test_per_tensor_closed_form():
+    """group_size 0: one scale s = max |w| / 7 (symmetric) or (max' - min') / 15
+    (affine) over the whole matrix, stored in every row; when every row has
+    the same extremes it equals the per-channel result, and a single-row
+    matrix is per-channel by definition."""
+    rng = np.random.default_rng(7)
+    W = np.clip(rng.standard_normal((6, 32)) * 0.02, -0.04, 0.04).astype(np.float32)
+    W[:, 0] = 0.1                                  # every row's max
+    W[:, 1] = -0.05                                # every row's min
+    for sym in (True, False):
+        pt = O.rtn_quantize(W, 0, sym)
+        pc = O.rtn_quantize(W, -1, sym)
+        assert np.array_equal(pt["codes"], pc["codes"])
+        assert np.array_equal(pt["scales"], pc["scales"])
+        one = O.rtn_quantize(W[2:3] * 3.0, 0, sym)
+        assert np.array_equal(one["codes"], O.rtn_quantize(W[2:3] * 3.0, -1, sym)["codes"])
+    W[4, 7] = 0.7
+    pt = O.rtn_quantize(W, 0, True)
+    assert np.all(pt["scales"] == np.float16(np.float32(0.7) / np.float32(7)))
+
+
+def test_per_tensor_gptq_diagonal_is_rtn():
+    """With orthogonal inputs (diagonal H) GPTQ with one scale per tensor
+    equals RTN with one scale per tensor."""
+    d = 64
+    X = np.diag(np.linspace(0.5, 3.0, d))
+    W = np.random.default_rng(8).standard_normal((10, d)) * 0.02
+    for sym in (True, False):
+        res, *_ = O.gptq_layer(W, X, group_size=0, sym=sym)
+        assert np.array_equal(res.codes, O.rtn_quantize(W, 0, sym)["codes"])

@@ -36,7 +36,8 @@ def _check(W: torch.Tensor, group_size: int, sym: bool, rows=None):
 
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("group_size,sym", [(-1, True), (-1, False), (128, True), (128, False),
-                                            (32, True), (8, False), (64, True), (256, False)])
+                                            (32, True), (8, False), (64, True), (256, False),
+                                            (0, True), (0, False)])
 @pytest.mark.parametrize("shape", [(7, 256), (33, 768), (130, 1024)])
 def test_rtn_bit_exact(dt, group_size, sym, shape):
     d_out, d_in = shape
@@ -127,3 +128,15 @@ def test_rtn_extreme_scales(dt, group_size, sym):
     W = W * mags[torch.arange(d_out) % len(mags)][:, None]
     W[5, :128] *= 1e-12                     # one row mixing tiny and ordinary groups
     _check(W.to(DT[dt]), group_size, sym)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("shape", [(1, 8), (3, 16), (2048, 4096)])
+def test_rtn_per_tensor(dt, shape):
+    """One scale for the whole matrix (group_size 0): a one-block path for
+    small matrices and block partials for large ones."""
+    g = torch.Generator().manual_seed(shape[0] + shape[1])
+    W = (torch.randn(shape, generator=g) * 0.02).to(DT[dt])
+    W.view(-1)[shape[0] * shape[1] // 2] = 0.3      # the extreme sits in the middle
+    _check(W, 0, True)
+    _check(W, 0, False)
