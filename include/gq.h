@@ -260,6 +260,29 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
                          void *stream);
 
 /* ------------------------------------------------------------------------
+ * W4A16 product: a consumer of the packed format.
+ * "GPTQ: Post-Training INT4", "Group Quantization" and "Running GPTQ with
+ * AutoGPTQ": the 4-bit codes with 16-bit scales (and zeros) are what a
+ * quantised model is served from; this call multiplies them with 16-bit
+ * activations: Y = W^ X^T with W^ = s (c - z) per group.
+ *
+ *   qpacked, scales, zeros, g_idx, d_out, d_in, group_size, sym
+ *              the quantised layer as produced by the calls above
+ *   X          [n_tok][d_in] bf16 (device, 16-byte aligned)
+ *   Y          [d_out][n_tok] fp32 (device, out, 16-byte aligned;
+ *              n_tok a multiple of 4): the layer's outputs, feature-major
+ *   ws         >= gq_w4a16_workspace_size(d_out, d_in, n_tok) bytes
+ * W^ is formed in fp32 (exact: an fp16 scale times a 4-bit integer) and fed
+ * to the tensor cores as a bf16 hi + lo pair, which holds it exactly; the
+ * products accumulate in fp32.
+ * ---------------------------------------------------------------------- */
+size_t gq_w4a16_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok);
+gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
+                          const uint16_t *zeros, const int32_t *g_idx, int64_t d_out,
+                          int64_t d_in, int group_size, int sym, const void *X_bf16,
+                          int64_t n_tok, float *Y, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * Activation-aware per-channel scaling before RTN.
  * "Model Quantization Mechanics", section 2.2: a per-channel factor s
  * multiplies the weights of input channels whose activations are large and

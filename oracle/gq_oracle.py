@@ -79,7 +79,7 @@ __all__ = [
     "GptqResult", "gptq_quantize", "dequantize_packed", "recon_sse",
     "recon_sse_trace", "bits_per_weight", "obs_quantize", "bruteforce_row",
     "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
-    "gptq_layer", "awq_channel_scales", "awq_apply", "awq_rtn_search",
+    "gptq_layer", "awq_channel_scales", "awq_apply", "awq_rtn_search", "w4a16_matmul",
 ]
 
 
@@ -480,6 +480,18 @@ def recon_sse_trace(W, W_hat, H_undamped) -> float:
     undamped H = 2 X^T X (pin only)."""
     dW = np.asarray(W, dtype=np.float64) - np.asarray(W_hat, dtype=np.float64)
     return float(np.sum((dW @ H_undamped) * dW) / 2.0)
+
+
+# --------------------------------------------------------------------------
+# Consumer of the packed format
+# --------------------------------------------------------------------------
+
+def w4a16_matmul(qpacked, scales, zeros, d_in, group_size, sym, X, g_idx=None):
+    """Y = W^ X^T in fp64 with W^ = s (c - z) from the packed codes ("GPTQ:
+    Post-Training INT4", "Group Quantization": 4-bit codes with 16-bit
+    scales are what the quantised model is run from)."""
+    What = dequantize_packed(qpacked, scales, zeros, d_in, group_size, sym, g_idx)
+    return What @ np.asarray(X, dtype=np.float64).T
 
 
 # --------------------------------------------------------------------------

@@ -3,13 +3,14 @@ C-ABI library -- a fixed, small case for profilers (ncu) and for timing one
 stage by hand.
 
     python -m post_weight_quantization_27_b200.cases --workload 2 --layer 3
-           [--tokens N] [--repeat R] [--stages hessian,solve,gptq,rtn,recon,awq]
+           [--tokens N] [--repeat R] [--stages hessian,solve,gptq,rtn,recon,awq,w4a16]
 
 The stages always run in path order (H -> damp/U -> GPTQ -> RTN -> recon),
 each as many times as --repeat says; a stage that is not listed still runs
 once if a later listed stage needs its output.  Prints one line per stage
 with its CUDA-event time.  "awq" is the activation-aware scaling search
-before RTN (20 values of alpha), which needs only H.
+before RTN (20 values of alpha), which needs only H; "w4a16" multiplies the
+RTN layer with the first (at most 8192) tokens.
 """
 from __future__ import annotations
 
@@ -20,7 +21,7 @@ import torch
 from . import gq
 from . import inputs as I
 
-ORDER = ("hessian", "solve", "gptq", "rtn", "recon", "awq")
+ORDER = ("hessian", "solve", "gptq", "rtn", "recon", "awq", "w4a16")
 
 
 def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) -> dict:
@@ -35,6 +36,8 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
         need |= {"gptq"}
     if stages == ["awq"]:  # needs only H
         need = {"hessian", "awq"}
+    if stages == ["w4a16"]:  # needs only the RTN output
+        need = {"rtn", "w4a16"}
     times = {}
 
     def timed(name, fn):
@@ -59,12 +62,16 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
     if "gptq" in need:
         q = timed("gptq", lambda: gq.gptq_quantize_layer(
             W, U, 4, spec.group_size, spec.block_size, spec.sym, perm=perm, dead=dead))
+    r = None
     if "rtn" in need:
-        timed("rtn", lambda: gq.rtn_quantize_pack(W, 4, spec.group_size, spec.sym))
+        r = timed("rtn", lambda: gq.rtn_quantize_pack(W, 4, spec.group_size, spec.sym))
     if "recon" in need:
         timed("recon", lambda: gq.recon_error(W, q, X, spec.group_size, spec.sym))
     if "awq" in need:
         timed("awq", lambda: gq.awq_rtn_search(W, H, X, 4, spec.group_size, spec.sym, 20))
+    if "w4a16" in need:  # the RTN layer times the first (at most 8192) tokens
+        Xs = X[:min(X.shape[0], 8192) // 4 * 4]
+        timed("w4a16", lambda: gq.w4a16_matmul(r, spec.d_in, Xs, spec.group_size, spec.sym))
     return {"spec": spec, "ms": times}
 
 

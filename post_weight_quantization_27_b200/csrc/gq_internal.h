@@ -90,7 +90,7 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
                        int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
-                       const float *col_inv = nullptr);
+                       const float *col_inv = nullptr, float *Y = nullptr);
 
 // Activation-aware scaling before RTN (awq.cu).
 size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int sym);

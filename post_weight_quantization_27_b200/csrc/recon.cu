@@ -31,6 +31,9 @@ struct ReconArgs {
   int n_mt, n_nt, nkb;
   double *partials;  // [n_tiles][8]
   int *status;
+  float *Y;          // store mode (W4A16 product): Y [M][ldy] = the GEMM itself, else NULL
+  int64_t ldy;
+  int M, N;
 };
 
 // Tile t -> (row tile, token tile) in groups of 16 row tiles, token tile by
@@ -85,7 +88,7 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
       const float code = static_cast<float>(sym ? nib - 8 : nib);
       float what = s * (code - z);
       if (col_inv) what *= col_inv[c];  // effective weight of a scaled layer
-      const float dw = ld_w(W + r * d_in + c) - what;
+      const float dw = W ? ld_w(W + r * d_in + c) - what : what;  // W NULL: W^ itself
       const __nv_bfloat16 hb = __float2bfloat16_rn(dw);
       h[k] = hb;
       l[k] = __float2bfloat16_rn(dw - __bfloat162float(hb));
@@ -209,6 +212,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t taddr =
           tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * BN + half * 128;
+      if (a.Y) {  // store mode: row m of the tile, 128 of its token columns
+        int mt, nt;
+        recon_tile(t, a.n_mt, a.n_nt, mt, nt);
+        const int m = mt * BM + quarter * 32 + lane;
+        const int n0 = nt * BN + half * 128;
+        float *yrow = a.Y + static_cast<int64_t>(m) * a.ldy + n0;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
+          if (m < a.M) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const int n = n0 + c * 32 + i;
+              if (n + 3 < a.N) {
+                *reinterpret_cast<float4 *>(yrow + c * 32 + i) =
+                    make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (n + e < a.N) yrow[c * 32 + i + e] = v[i + e];
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        continue;
+      }
       float ssq = 0.0f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -282,7 +315,7 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
                        int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
-                       const float *col_inv) {
+                       const float *col_inv, float *Y) {
   if (group_size == 0) group_size = -1;  // per-tensor scales are stored per row
   const ReconLayout L = recon_layout(d_out, d_in, n_tok);
   uint8_t *base = static_cast<uint8_t *>(ws);
@@ -292,6 +325,11 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
   __nv_bfloat16 *lo = reinterpret_cast<__nv_bfloat16 *>(base + L.off_lo);
   if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
   const int64_t n_tiles = static_cast<int64_t>(L.n_mt) * L.n_nt;
+  if (Y) {  // W4A16 product: dequantise W^ itself (no W), no reduction
+    W = nullptr;
+    dt = GQ_F32;
+    if (n_tok == 0) return GQ_OK;
+  }
   if (n_tok == 0) {
     recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, 0, status, sse_dev);
     count_launch();
@@ -325,7 +363,8 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
   if (s != GQ_OK) return s;
   cudaFuncSetAttribute(recon_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(SMEM_BYTES));
-  ReconArgs a{L.n_mt, L.n_nt, L.nkb, partials, status};
+  ReconArgs a{L.n_mt, L.n_nt, L.nkb, partials, status, Y, n_tok, static_cast<int>(d_out),
+              static_cast<int>(n_tok)};
   const int grid = static_cast<int>(n_tiles < num_sms() ? n_tiles : num_sms());
   const int slot = timer_begin(GQ_KERNEL_RECON_MMA, st);
   recon_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tHi, tLo, tX, a);
@@ -334,7 +373,7 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
   // runs it twice on the tensor cores)
   timer_end(slot, st, 2.0 * static_cast<double>(n_tok) * d_out * d_in);
   s = check_launch("recon_mma_kernel");
-  if (s != GQ_OK) return s;
+  if (s != GQ_OK || Y) return s;
   recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, n_tiles * 8, status, sse_dev);
   count_launch();
   return check_launch("recon_reduce_kernel");

@@ -72,6 +72,11 @@ def lib() -> ctypes.CDLL:
     L.gq_recon_error.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                                  _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp,
                                  _c_sz, _c_vp]
+    L.gq_w4a16_workspace_size.restype = _c_sz
+    L.gq_w4a16_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64]
+    L.gq_w4a16_matmul.restype = _c_int
+    L.gq_w4a16_matmul.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_int, _c_int,
+                                  _c_vp, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_awq_workspace_size.restype = _c_sz
     L.gq_awq_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64, _c_int, _c_int]
     L.gq_awq_rtn_search.restype = _c_int
@@ -94,7 +99,8 @@ EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_w
            "gq_hessian_accumulate", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
            "gq_damp_cholesky_inverse_noalloc",
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
-           "gq_recon_workspace_size", "gq_recon_error", "gq_awq_workspace_size",
+           "gq_recon_workspace_size", "gq_recon_error", "gq_w4a16_workspace_size",
+           "gq_w4a16_matmul", "gq_awq_workspace_size",
            "gq_awq_rtn_search", "gq_kernel_timer_start",
            "gq_kernel_timer_stop", "gq_kernel_timer_read", "gq_kernel_timer_release")
 
@@ -300,6 +306,29 @@ def recon_error(W: torch.Tensor, q: dict, X: torch.Tensor, group_size: int = -1,
                               _p(ws), ws.numel(), _stream(stream))
     _check(st, "gq_recon_error")
     return (sse_h.value, mse_h.value) if sync else sse
+
+
+# ------------------------------------------------------------------ W4A16 product
+
+def w4a16_workspace_size(d_out: int, d_in: int, n_tok: int) -> int:
+    return int(lib().gq_w4a16_workspace_size(d_out, d_in, n_tok))
+
+
+def w4a16_matmul(q: dict, d_in: int, X: torch.Tensor, group_size: int = -1, sym: bool = True,
+                 Y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """Y = W^ X^T (fp32 [d_out][n_tok]) from a quantised layer ``q`` (dict as
+    returned by the quantisers) and bf16 activations X [n_tok][d_in]."""
+    _dev(X, "X", torch.bfloat16)
+    d_out = q["qpacked"].shape[0]
+    n_tok = X.shape[0]
+    Y = torch.empty((d_out, n_tok), dtype=torch.float32, device=X.device) if Y is None else Y
+    ws = workspace(w4a16_workspace_size(d_out, d_in, n_tok), X.device) if ws is None else ws
+    st = lib().gq_w4a16_matmul(_p(q["qpacked"]), _p(q["scales"]), _p(q.get("zeros")),
+                               _p(q.get("g_idx")), d_out, d_in, group_size, int(bool(sym)), _p(X),
+                               n_tok, _p(Y), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_w4a16_matmul")
+    return Y
 
 
 # ------------------------------------------------------------------ activation-aware scaling

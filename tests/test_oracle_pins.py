@@ -503,3 +503,28 @@ def test_per_tensor_gptq_diagonal_is_rtn():
     for sym in (True, False):
         res, *_ = O.gptq_layer(W, X, group_size=0, sym=sym)
         assert np.array_equal(res.codes, O.rtn_quantize(W, 0, sym)["codes"])
+
+
+# ---------------------------------------------------------------- W4A16 product
+
+def test_w4a16_grouped_route_and_error_bound():
+    """Y = W^ X^T against a second route that never forms W^: per group,
+    s (sum_k c_k x_k - z sum_k x_k); and |Y - W X^T| stays within the
+    rounding bound sum_k |x_k| s_k / 2 of RTN."""
+    rng = np.random.default_rng(9)
+    d_out, d_in, n, g = 12, 64, 20, 16
+    W = rng.standard_normal((d_out, d_in)) * 0.02
+    X = rng.standard_normal((n, d_in))
+    for sym in (True, False):
+        r = O.rtn_quantize(W, g, sym)
+        Y = O.w4a16_matmul(r["qpacked"], r["scales"], r["zeros"], d_in, g, sym, X)
+        c = r["codes"].astype(np.float64)
+        Y2 = np.zeros((d_out, n))
+        for gi in range(d_in // g):
+            sl = slice(gi * g, (gi + 1) * g)
+            s = r["scales"][:, gi].astype(np.float64)[:, None]
+            z = (np.zeros(d_out) if sym else r["zeros"][:, gi].astype(np.float64))[:, None]
+            Y2 += s * (c[:, sl] @ X[:, sl].T - z * X[:, sl].sum(axis=1)[None, :])
+        assert np.allclose(Y, Y2, rtol=1e-12, atol=1e-12)
+        bound = 0.5 * np.abs(X) @ np.repeat(r["scales"].astype(np.float64), g, axis=1).T
+        assert np.all(np.abs(Y - W @ X.T) <= bound.T + 1e-12)
