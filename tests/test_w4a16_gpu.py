@@ -19,8 +19,12 @@ def _check(q, d_in, X, group_size, sym, g_idx=None):
                          X.float().numpy(), g_idx)
     got = Y.cpu().numpy().astype(np.float64)
     assert got.shape == ref.shape
-    assert rel_fro(got, ref) <= 1e-6
-    assert np.max(np.abs(got - ref)) <= 1e-5 * np.max(np.abs(ref))
+    # The products s (c - z) x are exact (W^ is held exactly by the bf16 pair
+    # and X is bf16); the error is the tensor core's fp32 accumulation over
+    # the d_in terms, about sqrt(d_in) * 2^-24 relative: 1e-5 bounds it for
+    # d_in up to a few thousand.
+    assert rel_fro(got, ref) <= 1e-5
+    assert np.max(np.abs(got - ref)) <= 1e-4 * np.max(np.abs(ref))
 
 
 @pytest.mark.parametrize("d_out,d_in,n_tok,group_size,sym,dt", [
