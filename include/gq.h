@@ -288,7 +288,7 @@ gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
  * multiplies the weights of input channels whose activations are large and
  * divides those activations, so the layer's output is unchanged while its
  * salient weights lose less to rounding; "GPT-2 Quantization Reconstruction
- * Error", "Possible extensions": scale important channels, judged by
+ * Error", "Possible extensions": scale important channels, chosen by
  * activation magnitude, before quantising.  The pages give no formula; this
  * call takes s_c = (H_cc / H_bar)^(alpha / 2) from the diagonal of the
  * undamped Hessian H = 2 X^T X (the channel RMS over its geometric mean,

@@ -5,7 +5,7 @@
 // divides those activations, so that the layer's output is unchanged while
 // the salient weights lose less to rounding; "GPT-2 Quantization
 // Reconstruction Error", "Possible extensions": scale up important channels,
-// judged by activation magnitude, before quantising.
+// chosen by activation magnitude, before quantising.
 //
 // Channel magnitude from the undamped Hessian H = 2 X^T X already on the
 // device: s_c = (H_cc / H_bar)^(alpha / 2) (H_bar the geometric mean of the
