@@ -97,3 +97,28 @@ def test_kernel_timer_without_session():
     assert L.gq_kernel_timer_stop() == 0
     assert L.gq_kernel_timer_release() == 0
     assert set(gq.KERNEL_UNITS) == set(gq.KERNELS)
+
+
+def test_header_is_c_and_links_from_c(tmp_path):
+    """include/gq.h compiles as C99 and a C program links libgq.so and calls
+    it (the calls below need no GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_gq.c"
+    src.write_text(
+        '#include "gq.h"\n#include <stdio.h>\n'
+        "int main(void) {\n"
+        '  printf("%s %zu %zu\\n", gq_status_string(GQ_ERR_NOT_PD),\n'
+        "         gq_hessian_workspace_size(2048, 768), gq_awq_workspace_size(8, 64, 16, -1, 1));\n"
+        "  return gq_rtn_quantize_pack(0, GQ_F32, 8, 64, 4, -1, 1, 0, 0, 0, 0) == GQ_ERR_ARG ? 0 : 1;\n"
+        "}\n")
+    libdir = os.path.dirname(gq.LIB_PATH)
+    exe = tmp_path / "use_gq"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lgq", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[0] == "GQ_ERR_NOT_PD" and int(out[1]) > 0 and int(out[2]) > 0
