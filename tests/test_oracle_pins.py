@@ -528,3 +528,49 @@ def test_w4a16_grouped_route_and_error_bound():
         assert np.allclose(Y, Y2, rtol=1e-12, atol=1e-12)
         bound = 0.5 * np.abs(X) @ np.repeat(r["scales"].astype(np.float64), g, axis=1).T
         assert np.all(np.abs(Y - W @ X.T) <= bound.T + 1e-12)
+
+
+# ---------------------------------------------------------------- two-level lazy update
+
+def _gptq_two_level(W, U, S, B=128):
+    """Per-channel symmetric GPTQ with the lazy trailing update on two levels
+    (the kernels' order): after a block of B columns only the rest of its
+    super-block of S columns is updated; after a super-block, every column
+    beyond it at once.  Plain numpy, written for this pin."""
+    W = np.array(W, dtype=np.float64, copy=True)
+    d_out, d_in = W.shape
+    s16, z16 = O.sym_params(W.astype(np.float32))
+    codes = np.zeros((d_out, d_in), dtype=np.int64)
+    for s0 in range(0, d_in, S):
+        s1 = min(s0 + S, d_in)
+        Err = np.zeros((d_out, s1 - s0))
+        for b0 in range(s0, s1, B):
+            b1 = min(b0 + B, s1)
+            for j in range(b0, b1):
+                w = W[:, j]
+                c = O.quantize_codes(w, s16, z16, True)
+                q = O.dequantize_codes(c, s16, z16)
+                codes[:, j] = c
+                delta = (w - q) / U[j, j]
+                Err[:, j - s0] = delta
+                W[:, j + 1:b1] -= np.outer(delta, U[j, j + 1:b1])
+            W[:, b1:s1] -= Err[:, b0 - s0:b1 - s0] @ U[b0:b1, b1:s1]
+        W[:, s1:] -= Err @ U[s0:s1, s1:]
+    return codes
+
+
+def test_two_level_lazy_update_is_the_same_method():
+    """The two-level order of the lazy trailing update (the kernels') gives
+    the codes of the one-level form the pages describe: the same terms
+    summed in another order."""
+    rng = np.random.default_rng(12)
+    d_in, d_out, n = 512, 48, 2048
+    X = rng.standard_normal((n, d_in)) * np.exp(0.5 * rng.standard_normal(d_in))[None, :]
+    W = rng.standard_normal((d_out, d_in)) * 0.02
+    H, _ = O.damp_hessian(O.hessian(X), 0.01)
+    U = O.upper_factor_of_inverse(H)
+    one = O.gptq_quantize(W, U, group_size=-1, block_size=128, sym=True).codes
+    for S in (256, 512):
+        two = _gptq_two_level(W, U, S)
+        assert np.mean(two == one) >= 0.9999
+        assert np.max(np.abs(two - one)) <= 1
