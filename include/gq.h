@@ -131,7 +131,13 @@ gq_status gq_hessian_accumulate(const void *X_bf16, int64_t n_tok, int64_t d_in,
  *              value there and returns GQ_ERR_NOT_PD on failure.
  *   ws         >= gq_damp_cholesky_workspace_size(d_in) bytes.
  * Computed in fp32: a blocked Cholesky of the index-reversed matrix, whose
- * reversed inverse is U (no separate inverse of H is formed).
+ * reversed inverse is U (no separate inverse of H is formed).  The
+ * inverse's block steps run on a second stream forked from and joined back
+ * to `stream` with events; that helper stream is created on first use for
+ * each (device, caller stream) pair and kept until the process exits (none
+ * is created while `stream` is being captured into a graph: the whole call
+ * then stays on `stream`).  Callers that create many short-lived streams
+ * should reuse a few instead.
  * ---------------------------------------------------------------------- */
 size_t gq_damp_cholesky_workspace_size(int64_t d_in);
 gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent,
