@@ -291,6 +291,7 @@ class GptqResult:
     qpacked: np.ndarray    # [d_out, d_in / 8] uint32 (None unless d_in % 8 == 0)
     W_hat: np.ndarray      # [d_out, d_in] fp64 dequantised, original column order
     n_followed: int = 0    # tie decisions adopted from ``follow``
+    max_follow_dist: float = 0.0   # largest boundary distance among them
 
 
 def _tie_dist(x):
@@ -299,20 +300,33 @@ def _tie_dist(x):
     return np.abs(f - np.floor(f) - 0.5)
 
 
-def _fp16_tie_dist(s32):
-    """Distance (in fp16 ulps) of an fp32 scale from the nearest fp16
-    rounding boundary."""
+def _fp16_tie_rel(s32):
+    """Relative distance of an fp32 scale from the nearest fp16 rounding
+    boundary (the midpoint between the two fp16 values around it)."""
     s = np.asarray(s32, dtype=np.float64)
     lo = s.astype(np.float16).astype(np.float64)
     up = np.nextafter(lo.astype(np.float16), np.float16(np.inf)).astype(np.float64)
     dn = np.nextafter(lo.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
-    ulp = np.where(s >= lo, up - lo, lo - dn)
     mid = np.where(s >= lo, (lo + up) / 2, (lo + dn) / 2)
-    return np.abs(s - mid) / np.where(ulp > 0, ulp, 1.0)
+    return np.abs(s - mid) / np.where(s > 0, s, 1.0)
+
+
+# Width of the rounding-tie window of the replay mode, in quantisation steps.
+# The other implementation computes each weight at its decision point in
+# fp32 after up to d_in accumulated updates; with unit roundoff u = 2^-24 and
+# error growth ~ sqrt(d_in) over sums whose terms are a few steps in size, its
+# value differs from the fp64 one by ~ sqrt(28672) * 6e-8 * (a few) ~ 1e-5
+# steps at the widest layer (measured: <= 2e-6 steps at d_in = 3072).  A
+# decision closer than this to a boundary k + 1/2 may go either way.  A scale
+# is a tie when its fp32 value lies within this relative distance of an fp16
+# rounding boundary (an error of eps steps in the group's extreme weight,
+# which spans 7 or 15 steps, moves the scale by at most eps relative), the
+# affine zero-point when -min'/s lies within this many steps of k + 1/2.
+TIE_TOL = 1e-5
 
 
 def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
-                  perm=None, dead=None, follow=None, tie_tol=1e-3) -> GptqResult:
+                  perm=None, dead=None, follow=None, tie_tol=TIE_TOL) -> GptqResult:
     """GPTQ on one layer given U (upper, H^-1 = U^T U, in the column order
     the layer is processed in).
 
@@ -328,11 +342,12 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     order and "scales"/"zeros" [d_out, n_groups]) is the output of another
     implementation.  Where the oracle's own decision is a rounding tie --
     the value w/s lies within ``tie_tol`` steps of k + 1/2, or the fp32
-    scale within ``tie_tol`` fp16 ulps of an fp16 rounding boundary -- both
-    roundings are correct, and the oracle takes the other implementation's
-    choice so that the rest of the row can be checked along it.  Nowhere
-    else does ``follow`` change anything; ``n_followed`` counts the
-    adopted decisions."""
+    scale within a relative ``tie_tol`` of an fp16 rounding boundary (see
+    TIE_TOL) -- both roundings are correct, and the oracle takes the other
+    implementation's choice so that the rest of the row can be checked
+    along it.  Nowhere else does ``follow`` change anything; ``n_followed``
+    counts the adopted decisions and ``max_follow_dist`` is the largest
+    distance from a boundary among them (steps, or relative for a scale)."""
     W = np.array(W, dtype=np.float64, copy=True)
     d_out, d_in = W.shape
     if dead is not None:
@@ -355,6 +370,7 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     scales = np.zeros((d_out, n_groups), dtype=np.float16)
     zeros = np.zeros((d_out, n_groups), dtype=np.float16)
     n_followed = 0
+    max_dist = 0.0
     if follow is not None:
         f_codes = np.asarray(follow["codes"], dtype=np.int64)
         if perm is not None:
@@ -364,23 +380,25 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                    if not sym else np.zeros_like(f_scales))
 
     def group(vals, gi):
-        nonlocal n_followed
+        nonlocal n_followed, max_dist
         s, z = params(vals, bits)
         if follow is not None:
             v = np.asarray(vals, dtype=F32)
             if sym:
                 s32 = np.max(np.abs(v), axis=-1) / F32(2 ** (bits - 1) - 1)
-                ztie = np.zeros(len(s), dtype=bool)
+                zdist = np.full(len(s), np.inf)
             else:
                 mn = np.minimum(np.min(v, axis=-1), F32(0))
                 mx = np.maximum(np.max(v, axis=-1), F32(0))
                 s32 = (mx - mn) / F32(2 ** bits - 1)
-                ztie = _tie_dist(-mn.astype(np.float64) / s.astype(np.float64)) < tie_tol
-            tie = (_fp16_tie_dist(s32) < tie_tol) | ztie
-            take = tie & ((f_scales[:, gi] != s) | (f_zeros[:, gi] != z))
+                zdist = _tie_dist(-mn.astype(np.float64) / s.astype(np.float64))
+            dist = np.minimum(_fp16_tie_rel(s32), zdist)
+            take = (dist < tie_tol) & ((f_scales[:, gi] != s) | (f_zeros[:, gi] != z))
             s = np.where(take, f_scales[:, gi], s)
             z = np.where(take, f_zeros[:, gi], z)
             n_followed += int(take.sum())
+            if take.any():
+                max_dist = max(max_dist, float(dist[take].max()))
         return s, z
 
     if per_tensor:
@@ -404,10 +422,13 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
             c = quantize_codes(w, s, z, sym, bits)
             if follow is not None:
                 r = w.astype(F32).astype(np.float64) / s.astype(np.float64)
-                take = ((_tie_dist(r) < tie_tol) & (f_codes[:, col] != c)
+                dist = _tie_dist(r)
+                take = ((dist < tie_tol) & (f_codes[:, col] != c)
                         & (np.abs(f_codes[:, col] - c) == 1))
                 c = np.where(take, f_codes[:, col], c)
                 n_followed += int(take.sum())
+                if take.any():
+                    max_dist = max(max_dist, float(dist[take].max()))
             q = dequantize_codes(c, s, z)
             codes[:, col] = c
             Q[:, col] = q
@@ -429,12 +450,13 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     assert codes.min() >= lo
     return GptqResult(codes=codes, scales=scales, zeros=zeros,
                       g_idx=g_idx.astype(np.int32), n_followed=n_followed,
+                      max_follow_dist=max_dist,
                       qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None,
                       W_hat=Q)
 
 
 def gptq_layer(W, X, bits=4, group_size=-1, block_size=128, sym=True,
-               damp_percent=0.01, act_order=False, follow=None, tie_tol=1e-3):
+               damp_percent=0.01, act_order=False, follow=None, tie_tol=TIE_TOL):
     """The whole per-layer path: H = 2 X^T X, dead columns and damping,
     optional act-order, U, then GPTQ.  Returns (GptqResult, H_undamped,
     U, perm, dead)."""
@@ -552,15 +574,17 @@ def obs_quantize(w, H, quantize):
     """Per-step OBS on one row with the Hessian re-inverted on the remaining
     set F at every step ("GPTQ: Post-Training INT4", "Hessian-Based Weight
     Update", read with H_F^-1 as in reading 5), columns taken left to right.
-    ``quantize(col, value) -> dequantised value``.  Returns the dequantised
-    row."""
+    ``quantize(col, row) -> dequantised value of row[col]``, where ``row`` is
+    the whole current row (entries at col and beyond carry every OBS update
+    so far), so that a quantiser can take a group's parameters from the
+    group's current weights.  Returns the dequantised row."""
     w = np.array(w, dtype=np.float64, copy=True)
     d = w.shape[0]
     out = np.zeros(d)
     for q in range(d):
         F = np.arange(q, d)
         HinvF = np.linalg.inv(H[np.ix_(F, F)])
-        qhat = quantize(q, w[q])
+        qhat = quantize(q, w.copy())
         out[q] = qhat
         err = w[q] - qhat
         w[F] -= err * HinvF[:, 0] / HinvF[0, 0]
@@ -588,14 +612,17 @@ def round_to_grid(w, step):
 
 
 def round_error_carried_forward(w, step):
-    """Round left to right, removing the previous rounding error from the
-    next weight before rounding it ("GPTQ and AWQ", "Example 1.1")."""
-    out, carry = [], 0.0
-    for v in w:
-        t = v + carry
-        q = np.rint(t / step) * step
-        carry = t - q
-        out.append(q)
+    """Round left to right so that every partial sum of the rounded weights
+    stays as close as the grid allows to the same partial sum of the
+    originals ("GPTQ and AWQ", "Example 1.1": the error left by one weight is
+    taken off the next before it is rounded).  In closed form, with S_k the
+    sum of w_0..w_k and Q_k that of q_0..q_k: q_k = step * rint((S_k -
+    Q_{k-1}) / step)."""
+    S = np.cumsum(np.asarray(w, dtype=np.float64))
+    out = []
+    for k in range(len(S)):
+        prev = sum(out)
+        out.append(np.rint((S[k] - prev) / step) * step)
     return out
 
 

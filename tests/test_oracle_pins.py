@@ -199,10 +199,30 @@ def test_storage_bits_per_weight(golden):
 # -------------------------------------------------------------- GPTQ
 
 def _row_quantizer(w_row, sym):
+    """Per-channel quantiser for obs_quantize: one scale from the initial row."""
     s, z = O.sym_params(w_row[None].astype(F32)) if sym else O.affine_params(w_row[None].astype(F32))
 
-    def q(col, v):
-        c = O.quantize_codes(np.array([[v]]), s[:, None], z[:, None], sym)
+    def q(col, row):
+        c = O.quantize_codes(np.array([[row[col]]]), s[:, None], z[:, None], sym)
+        return float(O.dequantize_codes(c, s[:, None], z[:, None])[0, 0])
+    return q
+
+
+def _group_quantizer(g, sym, params_from_initial=None):
+    """Group quantiser for obs_quantize written from "Group Quantization":
+    when column col starts a group (col % g == 0), the group's scale and zero
+    are taken from the row's current values of the group's g columns; later
+    columns of the group reuse them.  ``params_from_initial`` (a row) plants
+    the mistake of taking them from the initial weights instead."""
+    state = {}
+
+    def q(col, row):
+        if col % g == 0:
+            src = row if params_from_initial is None else params_from_initial
+            vals = np.asarray(src[col:col + g], dtype=np.float64)[None].astype(F32)
+            state["p"] = O.sym_params(vals) if sym else O.affine_params(vals)
+        s, z = state["p"]
+        c = O.quantize_codes(np.array([[row[col]]]), s[:, None], z[:, None], sym)
         return float(O.dequantize_codes(c, s[:, None], z[:, None])[0, 0])
     return q
 
@@ -226,6 +246,36 @@ def test_cholesky_form_equals_per_step_obs(sym):
         for i in range(4):
             ref = O.obs_quantize(W[i], H, _row_quantizer(W[i], sym))
             assert np.array_equal(ref, r.W_hat[i]), (t, i)
+
+
+@pytest.mark.parametrize("sym", [True, False])
+@pytest.mark.parametrize("g", [2, 4])
+def test_grouped_cholesky_form_equals_per_step_obs(g, sym):
+    """With groups, GPTQ's Cholesky form equals per-step OBS whose quantiser
+    takes each group's parameters from the group's current (OBS-updated)
+    weights at the group's first column (reading 6), for d_in <= 8 and every
+    lazy block size that the group divides."""
+    rng = np.random.default_rng(100 + 10 * g + sym)
+    n_diff_groups = 0
+    for t in range(40):
+        d = g * int(rng.integers(2, 8 // g + 1))
+        n = int(rng.integers(1, 3 * d))
+        X = rng.standard_normal((n, d)) * rng.lognormal(0, 0.5, d)
+        W = rng.standard_normal((6, d)) * 0.1
+        H, _ = O.damp_hessian(O.hessian(X), 0.01)
+        U = O.upper_factor_of_inverse(H)
+        r = O.gptq_quantize(W, U, group_size=g, block_size=128, sym=sym)
+        for bs in (g, 2 * g):
+            rb = O.gptq_quantize(W, U, group_size=g, block_size=bs, sym=sym)
+            assert np.array_equal(rb.codes, r.codes) and np.array_equal(rb.scales, r.scales)
+        for i in range(6):
+            ref = O.obs_quantize(W[i], H, _group_quantizer(g, sym))
+            assert np.array_equal(ref, r.W_hat[i]), (t, i)
+            init = O.rtn_quantize(W[i:i + 1].astype(F32), g, sym)["scales"]
+            n_diff_groups += int(np.sum(init != r.scales[i]))
+    # the later groups' parameters do move with the updates (else this pin
+    # could not tell current from initial weights)
+    assert n_diff_groups >= 20
 
 
 def _fixed_scale_levels(s, z, sym, d):
@@ -377,6 +427,29 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # the lazy trailing update dropped (only the 2-column in-block updates kept)
     blockdiag = np.kron(np.eye(d // 2), np.ones((2, 2))) * U
     assert not matches(blockdiag, 2)
+
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_planted_group_params_from_initial_weights_is_caught(sym):
+    """Taking each group's scale (and zero) from the initial weights instead
+    of the current ones at the group's start is a plausible mistake; the
+    grouped OBS pin must tell the two apart.  The mistake is planted in the
+    OBS quantiser (a copy of the method on the CPU): the oracle must agree
+    with the correct quantiser and disagree with the planted one."""
+    rng = np.random.default_rng(18 + sym)
+    d, g, rows = 8, 4, 48
+    X = rng.standard_normal((12, d)) * rng.lognormal(0, 0.5, d)
+    W = rng.standard_normal((rows, d)) * 0.1
+    H, _ = O.damp_hessian(O.hessian(X), 0.01)
+    U = O.upper_factor_of_inverse(H)
+    r = O.gptq_quantize(W, U, group_size=g, block_size=8, sym=sym)
+    good = bad = 0
+    for i in range(rows):
+        good += np.array_equal(O.obs_quantize(W[i], H, _group_quantizer(g, sym)), r.W_hat[i])
+        bad += np.array_equal(O.obs_quantize(W[i], H, _group_quantizer(g, sym, W[i])),
+                              r.W_hat[i])
+    assert good == rows
+    assert bad <= rows // 2
 
 
 def test_tie_follow_only_at_ties():
