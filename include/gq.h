@@ -25,6 +25,16 @@
  *   - Argument errors are detected on the host and returned before any
  *     launch; nothing is written then.  GQ_ERR_CUDA reports a launch or
  *     runtime error (gq_last_error() gives the text).
+ *   - Device-side failures: every wait inside a kernel (on a tensor-memory
+ *     accelerator copy or a tensor-core result) gives up after 2 s instead
+ *     of spinning forever and records GQ_ERR_TIMEOUT (7) in the call's
+ *     device status word, the first int32 of its workspace (0 = no failure;
+ *     the call resets it).  Calls that synchronise (the Cholesky call with
+ *     info_host, the reconstruction error with sse_host or mse_host, the
+ *     scaling search) read that word and return GQ_ERR_TIMEOUT; an
+ *     asynchronous caller reads it with gq_workspace_status() after the
+ *     work, before reusing the workspace.  The Hessian and reconstruction
+ *     error write NaN into their result when a wait gave up.
  *   - Shapes: W is d_out x d_in; X (calibration activations) is
  *     n_tok x d_in in bf16.  d_in must be a positive multiple of 8;
  *     d_out >= 1; n_tok >= 0 (an empty calibration batch adds nothing).
@@ -330,6 +340,27 @@ gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int6
                             uint16_t *scales, uint16_t *zeros, float *col_scale,
                             double *mse_host, int32_t *best_host, void *ws, size_t ws_bytes,
                             void *stream);
+
+/* ------------------------------------------------------------------------
+ * Device status of a call (a facility of this library; the pages have no
+ * counterpart).
+ *
+ *   gq_workspace_status(ws, status_host, stream)
+ *       synchronises `stream`, reads the device status word (the first
+ *       int32 of the workspace `ws` that a call on that stream was given)
+ *       into *status_host (if non-NULL) and returns GQ_OK, GQ_ERR_TIMEOUT
+ *       if a device-side wait of that call gave up, or GQ_ERR_CUDA.
+ *   gq_selftest_bounded_wait(arrive, limit_ns, ws, ws_bytes, stream)
+ *       exercises the bounded wait itself: one thread waits on a
+ *       shared-memory barrier (no copy, no tensor-core work); with arrive
+ *       != 0 it arrives on the barrier first, else nothing ever arrives and
+ *       the wait gives up after limit_ns (at most 1 s).  Records the result
+ *       in word 0 of ws (>= 256 bytes, 256-byte aligned), synchronises, and
+ *       returns GQ_OK or GQ_ERR_TIMEOUT like gq_workspace_status.
+ * ---------------------------------------------------------------------- */
+gq_status gq_workspace_status(const void *ws, int32_t *status_host, void *stream);
+gq_status gq_selftest_bounded_wait(int arrive, uint64_t limit_ns, void *ws, size_t ws_bytes,
+                                   void *stream);
 
 /* ------------------------------------------------------------------------
  * Per-launch kernel timing (a measurement aid; the pages describe no such

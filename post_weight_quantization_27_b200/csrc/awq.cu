@@ -195,10 +195,14 @@ gq_status launch_awq_rtn_search(const void *W, gq_dtype dt, int64_t d_out, int64
     if (s != GQ_OK) return s;
   }
   std::vector<double> sse(static_cast<size_t>(n_grid));
+  int32_t word = 0;  // device status of the reconstruction calls
   if (cudaMemcpyAsync(sse.data(), w.sse, sizeof(double) * n_grid, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess ||
+      cudaMemcpyAsync(&word, w.recon, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return check_launch("awq sync");
+  if (word == kDevTimeout)
+    return fail(GQ_ERR_TIMEOUT, "awq_rtn_search: a device-side wait gave up");
   int best = 0;
   for (int k = 1; k < n_grid; ++k)
     if (sse[k] < sse[best]) best = k;

@@ -748,15 +748,19 @@ extern "C" gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, fl
                                        info_dev, scratch, st, false);
   if (s != GQ_OK) return s;
   if (info_host) {
-    int32_t info = -1;
-    const int32_t *src = info_dev ? info_dev : reinterpret_cast<const int32_t *>(scratch) + 1;
-    if (cudaStreamSynchronize(st) != cudaSuccess ||
-        cudaMemcpy(&info, src, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    // words 0 and 1 of the scratch: device status, info; read on the
+    // caller's stream only (a synchronous copy could wait on other streams)
+    int32_t words[2] = {0, -1};
+    if (cudaMemcpyAsync(words, scratch, sizeof(words), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
       return check_launch("damp_cholesky_noalloc sync");
-    *info_host = info;
-    if (info >= 0)
+    *info_host = words[1];
+    if (words[0] == kDevTimeout)
+      return fail(GQ_ERR_TIMEOUT, "damp_cholesky_inverse_noalloc: a device-side wait gave up");
+    if (words[1] >= 0)
       return fail(GQ_ERR_NOT_PD, "damped Hessian not positive definite at column " +
-                                     std::to_string(info));
+                                     std::to_string(words[1]));
   }
   return GQ_OK;
 }

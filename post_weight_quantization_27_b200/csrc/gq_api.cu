@@ -117,6 +117,26 @@ gq_status check_ws(const void *ws, size_t have, size_t need) {
     if (_s != GQ_OK) return _s;           \
   } while (0)
 
+// GQ_ERR_TIMEOUT if a device status word (read after the stream has been
+// synchronised) records a wait that gave up, else GQ_OK.
+gq_status device_status(int32_t word, const char *what) {
+  if (word == kDevTimeout)
+    return fail(GQ_ERR_TIMEOUT, std::string(what) + ": a device-side wait gave up");
+  if (word != kDevOk)
+    return fail(GQ_ERR_CUDA, std::string(what) + ": device status " + std::to_string(word));
+  return GQ_OK;
+}
+
+// One thread waits on an mbarrier; with `arrive` it arrives on it first.
+// The wait gives up after limit_ns and records kDevTimeout in *status.
+__global__ void bounded_wait_kernel(int arrive, uint64_t limit_ns, int *status) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (arrive) mbar_arrive(&bar);
+  if (!mbar_wait(&bar, 0, limit_ns)) set_status(status, kDevTimeout);
+}
+
 }  // namespace
 
 extern "C" {
@@ -180,15 +200,16 @@ gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent, i
   GQ_TRY(launch_damp_chol(H, d_in, damp_percent, act_order, perm_out, dead_out, U, info_dev, ws,
                           st));
   if (info_host) {
-    int32_t info = -1;
-    const int32_t *src = info_dev ? info_dev : reinterpret_cast<const int32_t *>(ws) + 1;
-    if (cudaMemcpyAsync(&info, src, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+    // words 0 and 1 of the workspace: device status, info
+    int32_t words[2] = {0, -1};
+    if (cudaMemcpyAsync(words, ws, sizeof(words), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
       return check_launch("damp_cholesky sync");
-    *info_host = info;
-    if (info >= 0)
+    *info_host = words[1];
+    GQ_TRY(device_status(words[0], "damp_cholesky_inverse"));
+    if (words[1] >= 0)
       return fail(GQ_ERR_NOT_PD, "damped Hessian not positive definite at column " +
-                                     std::to_string(info));
+                                     std::to_string(words[1]));
   }
   return GQ_OK;
 }
@@ -266,12 +287,15 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
                       X_bf16, n_tok, sse_dev, ws, st));
   if (sse_host || mse_host) {
     double sse = 0.0;
+    int32_t word = 0;
     if (cudaMemcpyAsync(&sse, sse_dev, sizeof(double), cudaMemcpyDeviceToHost, st) !=
             cudaSuccess ||
+        cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
       return check_launch("recon_error sync");
     if (sse_host) *sse_host = sse;
     if (mse_host) *mse_host = n_tok > 0 ? sse / (static_cast<double>(n_tok) * d_out) : 0.0;
+    GQ_TRY(device_status(word, "recon_error"));
   }
   return GQ_OK;
 }
@@ -333,6 +357,31 @@ gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int6
   return launch_awq_rtn_search(W, w_dtype, d_out, d_in, H, X_bf16, n_tok, group_size, sym,
                                n_grid, qpacked, scales, zeros, col_scale, mse_host, best_host,
                                ws, static_cast<cudaStream_t>(stream));
+}
+
+gq_status gq_workspace_status(const void *ws, int32_t *status_host, void *stream) {
+  t_last_error.clear();
+  if (!ws) return fail(GQ_ERR_ARG, "null workspace");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return check_launch("workspace_status sync");
+  if (status_host) *status_host = word;
+  return device_status(word, "workspace_status");
+}
+
+gq_status gq_selftest_bounded_wait(int arrive, uint64_t limit_ns, void *ws, size_t ws_bytes,
+                                   void *stream) {
+  t_last_error.clear();
+  if (limit_ns > 1000000000ull) return fail(GQ_ERR_ARG, "limit_ns must be at most 1 s");
+  GQ_TRY(check_ws(ws, ws_bytes, kWsHeader));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
+  bounded_wait_kernel<<<1, 1, 0, st>>>(arrive ? 1 : 0, limit_ns, static_cast<int *>(ws));
+  count_launch();
+  GQ_TRY(check_launch("bounded_wait_kernel"));
+  return gq_workspace_status(ws, nullptr, stream);
 }
 
 }  // extern "C"

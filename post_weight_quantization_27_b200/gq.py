@@ -83,6 +83,10 @@ def lib() -> ctypes.CDLL:
     L.gq_awq_rtn_search.argtypes = [_c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int,
                                     _c_int, _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
                                     _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_workspace_status.restype = _c_int
+    L.gq_workspace_status.argtypes = [_c_vp, _c_vp, _c_vp]
+    L.gq_selftest_bounded_wait.restype = _c_int
+    L.gq_selftest_bounded_wait.argtypes = [_c_int, ctypes.c_uint64, _c_vp, _c_sz, _c_vp]
     L.gq_kernel_timer_start.restype = _c_int
     L.gq_kernel_timer_start.argtypes = [ctypes.c_uint32, ctypes.c_int32]
     L.gq_kernel_timer_stop.restype = _c_int
@@ -101,7 +105,8 @@ EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_w
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
            "gq_recon_workspace_size", "gq_recon_error", "gq_w4a16_workspace_size",
            "gq_w4a16_matmul", "gq_awq_workspace_size",
-           "gq_awq_rtn_search", "gq_kernel_timer_start",
+           "gq_awq_rtn_search", "gq_workspace_status", "gq_selftest_bounded_wait",
+           "gq_kernel_timer_start",
            "gq_kernel_timer_stop", "gq_kernel_timer_read", "gq_kernel_timer_release")
 
 
@@ -140,6 +145,25 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 def launch_count() -> int:
     return int(lib().gq_launch_count())
+
+
+def workspace_status(ws: torch.Tensor, stream=None) -> int:
+    """Device status word of the last call given ``ws`` (synchronises the
+    stream).  Raises GQError(GQ_ERR_TIMEOUT) if a device-side wait of that
+    call gave up; returns the word (0) otherwise."""
+    word = ctypes.c_int32(-1)
+    st = lib().gq_workspace_status(_p(ws), ctypes.byref(word), _stream(stream))
+    _check(st, "gq_workspace_status")
+    return int(word.value)
+
+
+def selftest_bounded_wait(arrive: bool, limit_ns: int, stream=None) -> int:
+    """Runs the bounded-wait self test and returns its status code (0, or 7
+    when the wait gave up) without raising."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = workspace(256, dev)
+    return int(lib().gq_selftest_bounded_wait(int(bool(arrive)), int(limit_ns), _p(ws),
+                                              ws.numel(), _stream(stream)))
 
 
 # ------------------------------------------------------------------ Hessian
