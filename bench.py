@@ -2,13 +2,14 @@
 
 A step runs the complete per-layer path on every layer of the workload:
 H = 2 X^T X, damping + dead columns + U (H^-1 = U^T U), GPTQ, RTN, and the
-reconstruction error of both quantised layers.  Default workload: the 49
-weight-bearing layers of GPT-2 small (768 -> 2304 / 768 / 3072, 3072 -> 768
-per block, x12, plus the 768 -> 50257 head) with 2560 calibration tokens
-per layer, per-channel symmetric 4-bit, block 128, damp 0.01.  Inputs are
-seeded synthetic data (no dataset or trained weights), resident in HBM.
+reconstruction error of both quantised layers.  Default workload: the
+three Llama-2-70B-shaped layers (8192 -> 8192, 8192 -> 28672, 28672 -> 8192;
+fp16 weights) with 262144 calibration tokens each, symmetric 4-bit, group
+128, block 128, damp 0.01.  Workload 2 is the 49 weight-bearing layers of
+GPT-2 small with 2560 tokens each.  Inputs are seeded synthetic data (no
+dataset or trained weights), resident in HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2|1|3|4|5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5|1|2|3|4]
                     [--impl reference]
 
 Prints one JSON line (rank 0).  Under torchrun every rank quantises its own
@@ -405,7 +406,7 @@ def gpu_arm(args, world, rank, local):
 
     recs = [r for r in gq.kernel_timer_read() if r[0] == dom_kernel]
     gq.kernel_timer_release()
-    roof = roofline(dom_kernel, recs, peaks, args.workload)
+    roof = roofline(dom_kernel, recs, peaks, args.workload, ms)
     del graph
 
     e2e = e2e_run(runs, args, dev, world, n_streams)
@@ -455,34 +456,39 @@ def rate(shares, kernel, scale):
     return round(w / (t / 1e3) / scale, 2)
 
 
-# Roofline ceiling per kernel: (bound, unit, ceiling name).  The tensor
-# ceilings derive from the measured bf16 GEMM rate (sustained: the kernels
-# are timed inside a long step) by the nominal dense ratios of B200
-# (tf32 1.1 / bf16 2.25 PFLOP/s) and the number of tensor passes per
-# algorithmic product (3 for the 3 x TF32 split, 2 for the bf16 hi + lo
-# split); the fp32 ALU ceiling is 148 SMs x 128 FMA lanes x 2 flops x the
-# maximum SM clock.
+# Roofline ceiling per kernel: (bound, dtype of its arithmetic, tensor-core
+# passes per algorithmic product).  The peak is the measured one of the
+# kernel's own arithmetic: bf16 for the bf16 contractions, TF32 (the
+# measured bf16 rate x the nominal dense TF32 / bf16 ratio of B200, 1.1 /
+# 2.25) for the 3 x TF32 GEMM, the fp32 FMA rate of the SMs (148 SMs x 128
+# lanes x 2 flops x the maximum SM clock) for the SIMT factor kernels, the
+# measured copy bandwidth for the memory-bound ones.  The fraction is
+# algorithmic work / time / that peak; the tensor pipe's own utilisation is
+# that fraction times the passes (the bf16 hi + lo split runs two products,
+# the 3 x TF32 split three), reported beside it.
 KERNEL_BOUND = {
-    "hessian_mma": ("tensor", "bf16"),
-    "recon_mma": ("tensor", "bf16 hi+lo (2 passes)"),
-    "gemm_tf32x3": ("tensor", "3xTF32 (3 tf32 passes)"),
-    "potrf_trsm": ("alu", "fp32 FMA"),
-    "block_inverse": ("alu", "fp32 FMA"),
-    "gptq_block": ("hbm", "HBM copy"),
-    "rtn": ("hbm", "HBM copy"),
+    "hessian_mma": ("tensor", "bf16", 1),
+    "recon_mma": ("tensor", "bf16", 2),
+    "gemm_tf32x3": ("tensor", "tf32", 3),
+    "potrf_trsm": ("alu", "fp32 FMA", 1),
+    "block_inverse": ("alu", "fp32 FMA", 1),
+    "gptq_block": ("hbm", "HBM copy", 1),
+    "rtn": ("hbm", "HBM copy", 1),
 }
 
 
-def kernel_peak(kernel, peaks):
-    bf16 = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+def kernel_peak(kernel, peaks, sustained=True):
+    """(peak, unit, description) for the kernel's own arithmetic.  Kernels
+    timed inside a long step take the sustained bf16 figure."""
+    bf16 = (peaks["bf16_tflops_sustained"] if sustained else None) or peaks["bf16_tflops"]
+    which = "sustained" if sustained and peaks["bf16_tflops_sustained"] else "burst"
     src = peaks["source"]
-    if kernel == "hessian_mma":
-        return bf16, "TFLOP/s", f"{src} bf16 sustained"
-    if kernel == "recon_mma":
-        return bf16 / 2, "TFLOP/s", f"{src} bf16 sustained / 2 passes"
-    if kernel == "gemm_tf32x3":
-        return bf16 * 1.1 / 2.25 / 3, "TFLOP/s", f"{src} bf16 sustained x 1.1/2.25 (tf32) / 3 passes"
-    if kernel in ("potrf_trsm", "block_inverse"):
+    _, dtype, _ = KERNEL_BOUND[kernel]
+    if dtype == "bf16":
+        return bf16, "TFLOP/s", f"{src} bf16 dense {which}"
+    if dtype == "tf32":
+        return bf16 * 1.1 / 2.25, "TFLOP/s", f"{src} bf16 dense {which} x 1.1/2.25 (tf32)"
+    if dtype == "fp32 FMA":
         mhz = peaks.get("sm_max_mhz") or 1965.0
         return 148 * 128 * 2 * mhz * 1e6 / 1e12, "TFLOP/s", f"148 SMs x 128 FMA x 2 x {mhz:.0f} MHz"
     return peaks["hbm_gbs"], "GB/s", f"{src} HBM copy"
@@ -504,20 +510,25 @@ def profiled_traffic(kernel, workload):
     return None
 
 
-def roofline(kernel, recs, peaks, workload):
+def roofline(kernel, recs, peaks, workload, ms_per_step):
     """Roofline of the dominant kernel: its launches' algorithmic work (flops
     or bytes, as the library counts them per launch) over their CUDA-event
     durations in the last timed replay."""
-    bound, what = KERNEL_BOUND[kernel]
+    bound, dtype, passes = KERNEL_BOUND[kernel]
     peak, unit, src = kernel_peak(kernel, peaks)
     work = sum(w for _, _, w in recs)
     sec = sum(ms for _, ms, _ in recs) / 1e3
     scale = 1e12 if unit == "TFLOP/s" else 1e9
     a = work / sec / scale if sec > 0 else 0.0
-    return {"kernel": kernel, "bound": bound, "achieved": round(a, 3), "peak": round(peak, 1),
-            "unit": unit, "frac": round(a / peak, 4), "traffic": profiled_traffic(kernel, workload),
-            "launches": len(recs), "avg_launch_us": round(sec / max(len(recs), 1) * 1e6, 2),
-            "work_per_launch": work / max(len(recs), 1), "ceiling": what, "peak_source": src}
+    out = {"kernel": kernel, "bound": bound, "achieved": round(a, 3), "peak": round(peak, 1),
+           "unit": unit, "frac": round(a / peak, 4), "traffic": profiled_traffic(kernel, workload),
+           "launches": len(recs), "avg_launch_us": round(sec / max(len(recs), 1) * 1e6, 2),
+           "kernel_ms_per_step": round(sec * 1e3, 3), "step_ms": round(ms_per_step, 3),
+           "work_per_launch": work / max(len(recs), 1), "arith": dtype, "peak_source": src}
+    if bound == "tensor":
+        out["tensor_passes"] = passes
+        out["tensor_pipe_frac"] = round(a * passes / peak, 4)
+    return out
 
 
 def e2e_run(runs, args, dev, world, n_streams):
@@ -572,6 +583,98 @@ def oracle_sample_step(workload: int):
     return len(data), time.perf_counter() - t0
 
 
+# Sampled units of the oracle for the full-size layers (the whole fp64 path
+# of one 28672-wide layer would take hours on the host): tokens, rows and
+# tiles per layer, and the width of the Cholesky sample.
+SAMPLE_TOKENS, SAMPLE_ROWS, SAMPLE_TILES, SAMPLE_TILE, SAMPLE_U = 8192, 128, 16, 256, 1024
+
+
+def oracle_sampled_layer(spec, rng):
+    """Times the oracle on sampled units of one full-size layer and
+    extrapolates to the whole layer.  Units: H on SAMPLE_TILES random
+    SAMPLE_TILE^2 tiles of the upper triangle over the first SAMPLE_TOKENS
+    tokens (scaled to all tiles and all tokens); U on the damped Hessian of
+    the first SAMPLE_U channels (scaled by (d_in / SAMPLE_U)^3); GPTQ, RTN
+    and both reconstruction errors on SAMPLE_ROWS random rows at full width
+    (GPTQ given a d_in x d_in factor; errors over the sampled tokens, scaled
+    to all rows and tokens).  Returns (extrapolated seconds, measured
+    seconds)."""
+    import numpy as np
+    import oracle as O
+    from post_weight_quantization_27_b200 import inputs as I
+    d, n_rows = spec.d_in, min(SAMPLE_ROWS, spec.d_out)
+    ntok = min(SAMPLE_TOKENS, spec.n_tok)
+    X = I.make_x(spec, rows=ntok).float().numpy()
+    rows = np.sort(rng.choice(spec.d_out, size=n_rows, replace=False))
+    W = I.make_weights(spec)[torch_index(rows)].float().numpy()
+    nt = (d + SAMPLE_TILE - 1) // SAMPLE_TILE
+    tri = [(a, b) for a in range(nt) for b in range(a, nt)]
+    pick = [tri[i] for i in rng.choice(len(tri), size=min(SAMPLE_TILES, len(tri)), replace=False)]
+    uw = min(SAMPLE_U, d)
+    U_full = np.eye(d)
+    t_meas = 0.0
+    # H tiles
+    t0 = time.perf_counter()
+    for a, b in pick:
+        ra = np.arange(a * SAMPLE_TILE, min(d, (a + 1) * SAMPLE_TILE))
+        rb = np.arange(b * SAMPLE_TILE, min(d, (b + 1) * SAMPLE_TILE))
+        O.hessian_entries(X[:, np.concatenate([ra, rb])], np.arange(len(ra)),
+                          np.arange(len(ra), len(ra) + len(rb)))
+    t_h = time.perf_counter() - t0
+    # U of the leading uw channels
+    Hs = O.hessian_entries(X[:, :uw], np.arange(uw), np.arange(uw))
+    t0 = time.perf_counter()
+    Hd, _ = O.damp_hessian(Hs, spec.damp)
+    O.upper_factor_of_inverse(Hd)
+    t_u = time.perf_counter() - t0
+    # GPTQ, RTN, both reconstruction errors on the sampled rows
+    t0 = time.perf_counter()
+    res = O.gptq_quantize(W, U_full, group_size=spec.group_size, block_size=spec.block_size,
+                          sym=spec.sym)
+    t_g = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    rtn = O.rtn_quantize(W, spec.group_size, spec.sym)
+    Wr = O.dequantize_packed(rtn["qpacked"], rtn["scales"], rtn["zeros"], d, spec.group_size,
+                             spec.sym)
+    t_r = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.recon_sse(W, res.W_hat, X)
+    O.recon_sse(W, Wr, X)
+    t_m = time.perf_counter() - t0
+    t_meas = t_h + t_u + t_g + t_r + t_m
+    tok = spec.n_tok / ntok
+    est = (t_h * len(tri) / len(pick) * tok + t_u * (d / uw) ** 3
+           + (t_g + t_r + t_m * tok) * spec.d_out / n_rows)
+    return est, t_meas
+
+
+def torch_index(rows):
+    import torch
+    return torch.from_numpy(rows)
+
+
+def oracle_sampled_step(workload: int, layer_ids, seed: int):
+    """The sampled oracle on the given layers of a full-size workload;
+    returns (layers, extrapolated seconds, measured seconds)."""
+    import numpy as np
+    from post_weight_quantization_27_b200 import inputs as I
+    layers = I.workload_layers(workload)
+    rng = np.random.default_rng(seed)
+    est = meas = 0.0
+    for i in layer_ids:
+        e, m = oracle_sampled_layer(layers[i], rng)
+        est += e
+        meas += m
+    return len(layer_ids), est, meas
+
+
+SAMPLED_DESC = ("per layer: H on %d random %dx%d upper-triangle tiles over the first %d tokens, "
+                "U of the leading %d channels, GPTQ + RTN + both reconstruction errors on %d "
+                "random rows at full width; each unit timed and scaled to the whole layer "
+                "(extrapolated)" % (SAMPLE_TILES, SAMPLE_TILE, SAMPLE_TILE, SAMPLE_TOKENS,
+                                    SAMPLE_U, SAMPLE_ROWS))
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -586,39 +689,62 @@ def cpu_threads() -> int:
 def reference_arm(args, world, rank):
     if rank != 0:
         return None
-    if args.workload != 2 and args.workload != 1:
-        return {"impl": "reference", "unavailable": "oracle reference arm is sized for workloads 1-2"}
-    for _ in range(args.warmup):
-        oracle_sample_step(args.workload)
-    n, sec = 0, 0.0
-    for _ in range(args.steps):
-        k, s = oracle_sample_step(args.workload)
-        n += k
-        sec += s
-    value = n / sec
-    sample = ("block 0 of the 49-layer workload (768->2304, 768->768, 768->3072, 3072->768), "
-              "full path per layer" if args.workload == 2 else "the single layer")
+    from post_weight_quantization_27_b200 import inputs as I
     cores = cpu_threads()
-    return {"metric": METRIC, "value": round(value, 4), "unit": "layers/s", "impl": "reference",
+    if args.workload in (1, 2):
+        for _ in range(args.warmup):
+            oracle_sample_step(args.workload)
+        n, sec = 0, 0.0
+        for _ in range(args.steps):
+            k, s = oracle_sample_step(args.workload)
+            n += k
+            sec += s
+        value = n / sec
+        sample = ("block 0 of the 49-layer workload (768->2304, 768->768, 768->3072, "
+                  "3072->768), full path per layer" if args.workload == 2 else "the single layer")
+        ms_step = sec / args.steps * 1e3
+    else:
+        # one layer's sampled units per step, cycling over the workload's shapes
+        n_layers = len(I.workload_layers(args.workload))
+        shapes = list(range(n_layers if args.workload != 3 else 4))
+        for w in range(args.warmup):
+            oracle_sampled_step(args.workload, [shapes[w % len(shapes)]], 1000 + w)
+        n, est, meas = 0, 0.0, 0.0
+        for k in range(args.steps):
+            a, e, m = oracle_sampled_step(args.workload, [shapes[k % len(shapes)]], k)
+            n += a
+            est += e
+            meas += m
+        value = n / est
+        sample = SAMPLED_DESC + "; one layer per step, cycling over the workload's shapes"
+        ms_step = est / args.steps * 1e3
+    return {"metric": METRIC, "value": round(value, 6), "unit": "layers/s", "impl": "reference",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(sec / args.steps * 1e3, 2), "higher_is_better": True,
+            "ms_per_step": round(ms_step, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
             "data": "synthetic (seeded)",
             "config": {"workload": WORKLOAD_NAMES[args.workload]},
-            "cpu_baseline": {"value": round(value, 4), "unit": "layers/s", "cores": cores,
+            "cpu_baseline": {"value": round(value, 6), "unit": "layers/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
-            "e2e": {"value": round(value, 4), "unit": "layers/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": round(value, 6), "unit": "layers/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
 def cpu_baseline(workload: int) -> dict:
     """The oracle on a bounded sample, timed on the host cores (rank 0, N=1)."""
-    n, sec = oracle_sample_step(workload)
-    sample = ("block 0 of the workload (4 layers: 768->2304, 768->768, 768->3072, 3072->768), "
-              "full path each; the lm_head is not in the sample" if workload == 2
-              else "first layer of the workload")
-    return {"value": round(n / sec, 4), "unit": "layers/s", "cores": cpu_threads(),
-            "kind": "oracle", "sample": sample, "seconds": round(sec, 2)}
+    if workload in (1, 2):
+        n, sec = oracle_sample_step(workload)
+        sample = ("block 0 of the workload (4 layers: 768->2304, 768->768, 768->3072, "
+                  "3072->768), full path each; the lm_head is not in the sample"
+                  if workload == 2 else "first layer of the workload")
+        return {"value": round(n / sec, 4), "unit": "layers/s", "cores": cpu_threads(),
+                "kind": "oracle", "sample": sample, "seconds": round(sec, 2)}
+    from post_weight_quantization_27_b200 import inputs as I
+    ids = list(range(len(I.workload_layers(workload)) if workload != 3 else 4))
+    n, est, meas = oracle_sampled_step(workload, ids, 7)
+    return {"value": round(n / est, 6), "unit": "layers/s", "cores": cpu_threads(),
+            "kind": "oracle", "sample": SAMPLED_DESC + "; every layer shape of the workload once",
+            "seconds_measured": round(meas, 2), "seconds_extrapolated": round(est, 1)}
 
 
 # ----------------------------------------------------------------------------- main
@@ -626,14 +752,21 @@ def cpu_baseline(workload: int) -> dict:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 10 for the full-size workloads, 50 otherwise)")
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=5, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="gq", choices=["gq", "reference"])
-    ap.add_argument("--streams", type=int, default=32)
+    ap.add_argument("--streams", type=int, default=None,
+                    help="concurrent streams (default: one per layer up to 32 for the small "
+                         "workloads; 1 for the full-size ones, whose layers each fill the GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.steps is None:
+        args.steps = 10 if args.workload >= 3 else 50
+    if args.streams is None:
+        args.streams = 1 if args.workload >= 3 else 32
     world, rank, local = dist_env()
     if world > 1:
         import datetime
@@ -645,7 +778,7 @@ def main():
             out = reference_arm(args, world, rank)
         else:
             out = gpu_arm(args, world, rank, local)
-            if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in (1, 2):
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline(args.workload)
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)

@@ -120,10 +120,26 @@ def damp_hessian(H, damp_percent=0.01):
     return H, dead
 
 
-def act_order_perm(H_damped) -> np.ndarray:
+def act_order_perm(H_damped, follow=None, key_tol=1e-6):
     """Columns in order of descending diag H, ties by lower index first
-    (desc_act of "Running GPTQ with AutoGPTQ"; reading 9)."""
-    return np.argsort(-np.diag(H_damped), kind="stable").astype(np.int64)
+    (desc_act of "Running GPTQ with AutoGPTQ"; reading 9).
+
+    ``follow`` (optional): another implementation's order.  Keys that differ
+    by less than ``key_tol`` (relative) are ties at the precision that
+    implementation computes H in, and either order of them is correct; the
+    other order is adopted when every adjacent pair of it is descending up
+    to that tolerance.  Returns the order, or (order, adopted) with
+    ``follow``."""
+    key = np.diag(np.asarray(H_damped, dtype=np.float64))
+    perm = np.argsort(-key, kind="stable").astype(np.int64)
+    if follow is None:
+        return perm
+    f = np.asarray(follow, dtype=np.int64)
+    ok = (np.array_equal(np.sort(f), np.arange(len(key)))
+          and np.all(key[f[1:]] <= key[f[:-1]] * (1.0 + key_tol)))
+    if ok and not np.array_equal(f, perm):
+        return f.copy(), True
+    return perm, False
 
 
 def upper_factor_of_inverse(H) -> np.ndarray:
@@ -132,14 +148,27 @@ def upper_factor_of_inverse(H) -> np.ndarray:
     The route the pages describe: Cholesky of H, its inverse (the listing's
     cholesky_inverse), then the Cholesky factor of H^-1 ("Model Quantization
     Mechanics", section 2.1: "a Cholesky decomposition of the inverse
-    Hessian").  Raises numpy.linalg.LinAlgError if H is not positive
-    definite."""
-    L = np.linalg.cholesky(H)                    # H = L L^T
-    Linv = np.linalg.inv(L)
-    Hinv = Linv.T @ Linv                         # H^-1
-    Hinv = 0.5 * (Hinv + Hinv.T)
-    Lh = np.linalg.cholesky(Hinv)                # H^-1 = Lh Lh^T
-    return np.ascontiguousarray(Lh.T)            # U = Lh^T
+    Hessian").  Each step is one LAPACK routine in fp64: the Cholesky
+    factorisation, the inverse of the triangular factor, the product
+    L^-T L^-1, the Cholesky factorisation of that.  Raises
+    numpy.linalg.LinAlgError if H is not positive definite."""
+    from scipy.linalg import lapack
+    H = np.asarray(H, dtype=np.float64)
+    L, info = lapack.dpotrf(H, lower=1, clean=1)         # H = L L^T
+    if info != 0:
+        raise np.linalg.LinAlgError(f"H is not positive definite (pivot {info})")
+    Linv, info = lapack.dtrtri(L, lower=1)               # L^-1 (lower triangular)
+    if info != 0:
+        raise np.linalg.LinAlgError("singular Cholesky factor")
+    del L
+    Hinv, info = lapack.dlauum(Linv, lower=1)            # lower part of L^-T L^-1 = H^-1
+    del Linv
+    Hinv = np.tril(Hinv)
+    Hinv += np.tril(Hinv, -1).T
+    Lh, info = lapack.dpotrf(Hinv, lower=1, clean=1)     # H^-1 = Lh Lh^T
+    if info != 0:
+        raise np.linalg.LinAlgError("inverse not positive definite")
+    return np.ascontiguousarray(Lh.T)                    # U = Lh^T
 
 
 # --------------------------------------------------------------------------

@@ -40,17 +40,24 @@ PEAKS = {"hbm_gbs": 6546.9, "bf16_tflops": 1676.5, "bf16_tflops_sustained": 1374
 def test_roofline_arithmetic():
     # two launches of 1e9 flop in 1 ms each: 1 TFLOP/s
     recs = [("gemm_tf32x3", 1.0, 1e9), ("gemm_tf32x3", 1.0, 1e9)]
-    r = bench.roofline("gemm_tf32x3", recs, PEAKS, 99)
+    r = bench.roofline("gemm_tf32x3", recs, PEAKS, 99, 10.0)
     assert r["achieved"] == pytest.approx(1.0)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
-    assert r["peak"] == pytest.approx(1374.1 * 1.1 / 2.25 / 3, rel=1e-3)
+    # the peak of the kernel's own arithmetic (tf32), not divided by passes
+    assert r["peak"] == pytest.approx(1374.1 * 1.1 / 2.25, rel=1e-3)
     assert r["frac"] == pytest.approx(1.0 / r["peak"], rel=1e-2)
+    assert r["tensor_passes"] == 3
+    assert r["tensor_pipe_frac"] == pytest.approx(3 * r["frac"], rel=1e-2)
     assert r["launches"] == 2 and r["avg_launch_us"] == pytest.approx(1000.0)
+    assert r["kernel_ms_per_step"] == pytest.approx(2.0) and r["step_ms"] == 10.0
+    # a bf16 contraction against the sustained bf16 peak itself
+    r = bench.roofline("recon_mma", [("recon_mma", 1.0, 1374.1e9)], PEAKS, 99, 1.0)
+    assert r["frac"] == pytest.approx(1.0, rel=1e-4) and r["tensor_pipe_frac"] == pytest.approx(2.0, rel=1e-4)
     # bytes: 6.5469e9 bytes in 1 ms -> the copy bandwidth
-    r = bench.roofline("rtn", [("rtn", 1.0, 6.5469e9)], PEAKS, 99)
+    r = bench.roofline("rtn", [("rtn", 1.0, 6.5469e9)], PEAKS, 99, 1.0)
     assert r["bound"] == "hbm" and r["frac"] == pytest.approx(1.0, rel=1e-4)
     # fp32 ALU ceiling from the SM count, lanes and clock
-    r = bench.roofline("potrf_trsm", [("potrf_trsm", 1.0, 1e9)], PEAKS, 99)
+    r = bench.roofline("potrf_trsm", [("potrf_trsm", 1.0, 1e9)], PEAKS, 99, 1.0)
     assert r["bound"] == "alu"
     assert r["peak"] == pytest.approx(148 * 128 * 2 * 1965e6 / 1e12, rel=1e-3)
 
@@ -58,7 +65,7 @@ def test_roofline_arithmetic():
 def test_every_timed_kernel_has_a_ceiling():
     from post_weight_quantization_27_b200 import gq
     for k in gq.KERNELS:
-        bound, _ = bench.KERNEL_BOUND[k]
+        bound, _, _ = bench.KERNEL_BOUND[k]
         peak, unit, _ = bench.kernel_peak(k, PEAKS)
         assert peak > 0 and unit in ("TFLOP/s", "GB/s")
         assert (unit == "GB/s") == (bound == "hbm")

@@ -40,6 +40,8 @@ def check_gptq(out, oracle_run, d_in, sym, min_agree=0.999):
                   zeros=None if sym else f16(out["zeros"]))
     rep = oracle_run(follow)
     agree, maxdiff = code_agreement(got, rep.codes)
+    print(f"[gptq parity] raw {raw_agree:.6f} replayed {agree:.6f} followed {rep.n_followed} "
+          f"max tie distance {rep.max_follow_dist:.3g}")
     assert agree >= min_agree and maxdiff <= 1, (raw_agree, agree, maxdiff, rep.n_followed)
     assert rep.n_followed <= max(4, 1e-4 * got.size), rep.n_followed
     return raw_agree, agree, rep.n_followed

@@ -647,3 +647,22 @@ def test_two_level_lazy_update_is_the_same_method():
         two = _gptq_two_level(W, U, S)
         assert np.mean(two == one) >= 0.9999
         assert np.max(np.abs(two - one)) <= 1
+
+
+def test_act_order_follow_only_within_key_ties():
+    """The act-order sort adopts another implementation's order only where
+    the keys it swaps tie within the stated relative tolerance."""
+    key = np.array([5.0, 3.0, 3.0 * (1 + 2e-7), 1.0, 4.0])
+    H = np.diag(key)
+    own = O.act_order_perm(H)
+    assert own.tolist() == [0, 4, 2, 1, 3]
+    swapped = np.array([0, 4, 1, 2, 3])            # the near-tie taken the other way
+    p, adopted = O.act_order_perm(H, follow=swapped, key_tol=1e-6)
+    assert adopted and p.tolist() == swapped.tolist()
+    p, adopted = O.act_order_perm(H, follow=swapped, key_tol=1e-8)
+    assert not adopted and p.tolist() == own.tolist()
+    wrong = np.array([4, 0, 2, 1, 3])               # 4.0 before 5.0: not a tie
+    p, adopted = O.act_order_perm(H, follow=wrong)
+    assert not adopted and p.tolist() == own.tolist()
+    p, adopted = O.act_order_perm(H, follow=own)
+    assert not adopted and p.tolist() == own.tolist()
