@@ -147,19 +147,22 @@ def measured_peaks() -> dict:
 class LayerRun:
     """Device buffers of one layer and the calls of one step on it."""
 
-    def __init__(self, spec, dev, W, X):
+    def __init__(self, spec, dev, W, X, recon_route="hessian"):
         import torch
         from post_weight_quantization_27_b200 import gq
         self.spec = spec
         self.W, self.X = W, X
+        self.route = recon_route
         d_in, d_out, n = spec.d_in, spec.d_out, spec.n_tok
         f = dict(device=dev)
-        self.H = torch.empty((d_in, d_in), dtype=torch.float32, **f)
+        self.H0 = torch.empty((d_in, d_in), dtype=torch.float32, **f)   # undamped, kept
+        self.H = torch.empty((d_in, d_in), dtype=torch.float32, **f)    # the solve's scratch
         self.U = torch.empty((d_in, d_in), dtype=torch.float32, **f)
         self.ws_h = gq.workspace(gq.hessian_workspace_size(n, d_in), dev)
         self.ws_c = gq.workspace(gq.damp_cholesky_workspace_size(d_in), dev)
         self.ws_g = gq.workspace(gq.gptq_workspace_size(d_out, d_in, spec.block_size), dev)
-        self.ws_r = gq.workspace(gq.recon_workspace_size(d_out, d_in, n), dev)
+        self.ws_r = gq.workspace(gq.recon_workspace_size(d_out, d_in, n) if recon_route == "direct"
+                                 else gq.recon_error_hessian_workspace_size(d_out, d_in), dev)
         self.q_gptq = gq._outputs(d_out, d_in, spec.group_size, spec.sym, dev, spec.act_order)
         self.q_rtn = gq._outputs(d_out, d_in, spec.group_size, spec.sym, dev, False)
         self.perm = torch.empty(d_in, dtype=torch.int32, **f) if spec.act_order else None
@@ -170,14 +173,14 @@ class LayerRun:
     def hessian(self):
         from post_weight_quantization_27_b200 import gq
         L, s = gq.lib(), gq._stream(None)
-        self.H.zero_()
-        gq._check(L.gq_hessian_accumulate(gq._p(self.X), self.spec.n_tok, self.spec.d_in,
-                                          gq._p(self.H), gq._p(self.ws_h), self.ws_h.numel(), s),
+        gq._check(L.gq_hessian_compute(gq._p(self.X), self.spec.n_tok, self.spec.d_in,
+                                       gq._p(self.H0), gq._p(self.ws_h), self.ws_h.numel(), s),
                   "hessian")
 
     def solve(self):
         from post_weight_quantization_27_b200 import gq
         L, s, sp = gq.lib(), gq._stream(None), self.spec
+        self.H.copy_(self.H0)            # the solve uses its H as scratch; H0 stays for the error
         gq._check(L.gq_damp_cholesky_inverse(
             gq._p(self.H), sp.d_in, sp.damp, int(sp.act_order), gq._p(self.perm),
             gq._p(self.dead), gq._p(self.U), gq._p(self.info), None, gq._p(self.ws_c),
@@ -204,6 +207,14 @@ class LayerRun:
         from post_weight_quantization_27_b200 import gq
         L, s, sp = gq.lib(), gq._stream(None), self.spec
         for k, o in enumerate((self.q_gptq, self.q_rtn)):
+            if self.route == "hessian":
+                gq._check(L.gq_recon_error_hessian(
+                    gq._p(self.W), gq._DTYPES[self.W.dtype], gq._p(o["qpacked"]),
+                    gq._p(o["scales"]), gq._p(o["zeros"]), gq._p(o.get("g_idx")), sp.d_out,
+                    sp.d_in, sp.group_size, int(sp.sym), gq._p(self.H0), sp.n_tok,
+                    self.sse.data_ptr() + 8 * k, None, None, gq._p(self.ws_r),
+                    self.ws_r.numel(), s), "recon")
+                continue
             gq._check(L.gq_recon_error(
                 gq._p(self.W), gq._DTYPES[self.W.dtype], gq._p(o["qpacked"]),
                 gq._p(o["scales"]), gq._p(o["zeros"]), gq._p(o.get("g_idx")), sp.d_out,
@@ -214,7 +225,7 @@ class LayerRun:
     STAGES = ("hessian", "solve", "gptq", "rtn", "recon")
 
 
-def build_layers(workload: int, dev, generate_on_device: bool):
+def build_layers(workload: int, dev, generate_on_device: bool, recon_route: str = "hessian"):
     import torch
     from post_weight_quantization_27_b200 import inputs as I
     runs = []
@@ -226,7 +237,7 @@ def build_layers(workload: int, dev, generate_on_device: bool):
     for spec in layers:
         W = I.make_weights(spec).to(dev)
         X = I.make_x_device(spec, dev) if generate_on_device else I.make_x(spec).to(dev)
-        runs.append(LayerRun(spec, dev, W, X))
+        runs.append(LayerRun(spec, dev, W, X, recon_route))
     torch.cuda.synchronize()
     return runs
 
@@ -345,7 +356,7 @@ def kernel_shares(runs):
     return tot
 
 
-def stage_work(spec):
+def stage_work(spec, recon_route="hessian"):
     """Algorithmic work per call of each stage (bytes or flops)."""
     wb = {"f32": 4, "f16": 2, "bf16": 2}[spec.w_dtype]
     n_groups = 1 if spec.group_size == -1 else spec.d_in // spec.group_size
@@ -355,8 +366,10 @@ def stage_work(spec):
         "hessian_flops": spec.n_tok * spec.d_in * (spec.d_in + 1),
         # read W, write codes + fp16 scales (+ zeros)
         "rtn_bytes": spec.d_out * spec.d_in * (wb + 0.5) + 2 * spec.d_out * n_groups + zero_bytes,
-        # two reconstruction GEMMs, 2 N d_out d_in each
-        "recon_flops": 2 * 2 * spec.n_tok * spec.d_out * spec.d_in,
+        # two reconstruction errors: 2 N d_out d_in each (direct), or
+        # 2 d_out d_in^2 each from the Hessian
+        "recon_flops": (2 * 2 * spec.n_tok * spec.d_out * spec.d_in if recon_route == "direct"
+                        else 2 * 2 * spec.d_out * spec.d_in ** 2),
         "weights": spec.d_out * spec.d_in,
     }
 
@@ -368,7 +381,7 @@ def gpu_arm(args, world, rank, local):
     dev = torch.device("cuda", local)
     gq.lib()
     big = args.workload >= 3
-    runs = build_layers(args.workload, dev, generate_on_device=big)
+    runs = build_layers(args.workload, dev, generate_on_device=big, recon_route=args.recon)
     peaks = measured_peaks()
     n_streams = max(1, min(args.streams, len(runs)))
 
@@ -399,7 +412,7 @@ def gpu_arm(args, world, rank, local):
     for i, st, e0, e1 in events:
         calls[st].append(e0.elapsed_time(e1))
     stage_ms = {st: sum(v) for st, v in calls.items()}
-    work = [stage_work(r.spec) for r in runs]
+    work = [stage_work(r.spec, args.recon) for r in runs]
     tot = {k: sum(w[k] for w in work) for k in work[0]}
     n_layers = len(runs)
     value = world * n_layers / (ms / 1e3)
@@ -426,6 +439,7 @@ def gpu_arm(args, world, rank, local):
         "dtype": "bf16 X, fp32 H/U/GPTQ, int4 codes",
         "data": "synthetic (seeded; random-init weights of the named layer shapes)",
         "config": {"workload": WORKLOAD_NAMES[args.workload], "layers": n_layers,
+                   "recon_route": args.recon,
                    "weights_per_step": tot["weights"], "parallelism": f"layers x{world} (weak)",
                    "streams": n_streams, "cuda_graph": True,
                    "l2": "inputs larger than L2 (%.0f MB of W and X per step)" % (
@@ -760,6 +774,9 @@ def main():
     ap.add_argument("--streams", type=int, default=None,
                     help="concurrent streams (default: one per layer up to 32 for the small "
                          "workloads; 1 for the full-size ones, whose layers each fill the GPU)")
+    ap.add_argument("--recon", default="hessian", choices=["hessian", "direct"],
+                    help="reconstruction error route: from the Hessian (tr(dW H0 dW^T) / 2) "
+                         "or directly (||dW X^T||^2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -111,6 +111,10 @@ uint64_t gq_launch_count(void);
 size_t gq_hessian_workspace_size(int64_t n_tok, int64_t d_in);
 gq_status gq_hessian_accumulate(const void *X_bf16, int64_t n_tok, int64_t d_in,
                                 float *H, void *ws, size_t ws_bytes, void *stream);
+/* As gq_hessian_accumulate, but H := 2 X^T X: the incoming contents of H
+ * are neither read nor needed (no separate clearing of H). */
+gq_status gq_hessian_compute(const void *X_bf16, int64_t n_tok, int64_t d_in, float *H,
+                             void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Damping, act-order and the upper Cholesky factor of the inverse Hessian.
@@ -274,6 +278,36 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
                          const void *X_bf16, int64_t n_tok, double *sse_dev,
                          double *sse_host, double *mse_host, void *ws, size_t ws_bytes,
                          void *stream);
+
+/* ------------------------------------------------------------------------
+ * Layer reconstruction error from the Hessian (the same SSE by a second
+ * route).  With H0 = 2 X^T X (undamped, as gq_hessian_accumulate returns
+ * it), ||(W - W^) X^T||_F^2 = tr((W - W^) X^T X (W - W^)^T) = tr(dW H0
+ * dW^T) / 2 ("GPTQ: Post-Training INT4", "Hessian-Based Weight Update": the
+ * layer-wise objective is the quadratic form of H).  Costs 2 d_out d_in^2
+ * flops instead of 2 n_tok d_out d_in, so it is the cheaper route whenever
+ * the calibration set has more tokens than the layer has inputs.
+ *
+ *   W, ..., sym     as for gq_recon_error
+ *   H0              [d_in][d_in] fp32 (device, read only, 16-byte aligned),
+ *                   exactly symmetric, undamped
+ *   n_tok           the number of calibration tokens H0 was accumulated
+ *                   over (only for mse_host)
+ *   sse_dev, sse_host, mse_host   as for gq_recon_error
+ *   ws              >= gq_recon_error_hessian_workspace_size(d_out, d_in)
+ *                   bytes (holds dW in fp32: 4 d_out d_in bytes)
+ * dW is formed in fp32; the product dW H0 runs in fp32 accuracy on the
+ * tensor cores (three TF32 products per term) and is never stored: each
+ * output tile's sum of (dW H0) .* dW is kept in fp64 and the tiles are
+ * added in a fixed order (deterministic).
+ * ---------------------------------------------------------------------- */
+size_t gq_recon_error_hessian_workspace_size(int64_t d_out, int64_t d_in);
+gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
+                                 const uint16_t *scales, const uint16_t *zeros,
+                                 const int32_t *g_idx, int64_t d_out, int64_t d_in,
+                                 int group_size, int sym, const float *H0, int64_t n_tok,
+                                 double *sse_dev, double *sse_host, double *mse_host, void *ws,
+                                 size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * W4A16 product: a consumer of the packed format.

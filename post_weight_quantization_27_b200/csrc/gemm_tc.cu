@@ -52,6 +52,7 @@ struct TcArgs {
   int n_mt, n_nt, nkb, n_tiles;
   int b_kmajor, lower;
   int *status;
+  double *dot;  // dot mode: [n_tiles] sum over the tile of (alpha A B) * C; C not written
 };
 
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool b_mn) {
@@ -73,11 +74,19 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
-// Tile t -> (mt, nt); lower: only nt <= mt, enumerated row by row.
+// Tile t -> (mt, nt).  General: groups of RASTER_GM row tiles, row tile
+// fastest inside a group, so that the tiles in flight at one time share a
+// few operand slabs in L2 (a long K makes each slab larger than L2 can hold
+// for all row tiles at once).  lower: only nt <= mt, enumerated row by row.
+constexpr int RASTER_GM = 16;
 __device__ __forceinline__ void tile_of(const TcArgs &a, int t, int &mt, int &nt) {
   if (!a.lower) {
-    mt = t % a.n_mt;
-    nt = t / a.n_mt;
+    const int per_group = RASTER_GM * a.n_nt;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int rows = min(RASTER_GM, a.n_mt - g * RASTER_GM);
+    mt = g * RASTER_GM + r % rows;
+    nt = r / rows;
     return;
   }
   int r = static_cast<int>((sqrtf(8.0f * t + 1.0f) - 1.0f) * 0.5f);
@@ -104,6 +113,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *drain = acc_empty + 2;
   uint64_t *c_full = drain + 1;           // C tile landed in the staging buffer
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 1);
+  double *red = reinterpret_cast<double *>(bars + 16);  // dot mode: one per epilogue warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -253,7 +263,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;               // row within the tile
     const bool leader = threadIdx.x == 192;          // issues the C copies
-    const bool need_c = a.beta != 0.0f || a.lower != 0;
+    const bool dot = a.dot != nullptr;
+    const bool need_c = a.beta != 0.0f || a.lower != 0 || dot;
     uint32_t ch = 0;
     bool ok = true;
     auto load_c = [&](int t) {
@@ -278,6 +289,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * TN;
       const int m = mt * TM + r;
       const bool diag = a.lower && mt == nt;
+      if (dot) {
+        // sum over the tile of (alpha acc) * C: each thread its row (fp32
+        // over 32 columns, fp64 across), then the four warps in order
+        double rs = 0.0;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          float v[32];
+          tmem_ld32(taddr + q * 32, v);
+          const uint8_t *row = cs + q * (C_BYTES / 4) + r * 128;
+          float part = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
+            part = fmaf(a.alpha * v[4 * c], cv.x, part);
+            part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
+            part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
+            part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
+          }
+          rs += static_cast<double>(part);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
+        if (lane == 0) red[quarter] = rs;
+        named_bar_sync(1, 128);
+        if (leader) {
+          a.dot[t] = ((red[0] + red[1]) + red[2]) + red[3];
+          const int tn = t + static_cast<int>(gridDim.x);
+          if (tn < a.n_tiles) load_c(tn);
+        }
+        named_bar_sync(1, 128);
+        continue;
+      }
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float v[32];
@@ -341,9 +387,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // own columns (an in-place left multiplication); tiles of C are read (beta
 // != 0 or lower) and written whole, so with `lower` the strict upper part of
 // a diagonal tile is written back unchanged.
+// Dot mode (dot_partials non-NULL): nothing is written to C; instead
+// dot_partials[t] = sum over output tile t of (alpha A B) .* C (fp32 within
+// a row of the tile, fp64 across rows), for t < gemm_tf32x3_tiles(M, N).
+int gemm_tf32x3_tiles(int M, int N) { return ((M + TM - 1) / TM) * ((N + TN - 1) / TN); }
+
 gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
                              const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
-                             int64_t ldc, bool lower, int *status, cudaStream_t st) {
+                             int64_t ldc, bool lower, int *status, cudaStream_t st,
+                             double *dot_partials) {
   if (M <= 0 || N <= 0 || K <= 0) return GQ_OK;
   CUtensorMap tA, tB;
   gq_status s = make_tmap_2d(&tA, A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K, M, lda, TK, TM);
@@ -372,6 +424,7 @@ gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, i
   a.lower = lower ? 1 : 0;
   a.n_tiles = lower ? a.n_mt * (a.n_mt + 1) / 2 : a.n_mt * a.n_nt;
   a.status = status;
+  a.dot = lower ? nullptr : dot_partials;
   cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(SMEM_BYTES));
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();

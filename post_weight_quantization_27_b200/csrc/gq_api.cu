@@ -179,6 +179,20 @@ gq_status gq_hessian_accumulate(const void *X_bf16, int64_t n_tok, int64_t d_in,
   return launch_hessian(X_bf16, n_tok, d_in, H, ws, p, static_cast<cudaStream_t>(stream));
 }
 
+gq_status gq_hessian_compute(const void *X_bf16, int64_t n_tok, int64_t d_in, float *H,
+                             void *ws, size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  if (!H || (n_tok > 0 && !X_bf16)) return fail(GQ_ERR_ARG, "null pointer");
+  if (n_tok < 0 || d_in < 8 || d_in % 8 != 0)
+    return fail(GQ_ERR_SHAPE, "need n_tok >= 0 and d_in a positive multiple of 8");
+  if (d_in > 65536 || n_tok > (int64_t(1) << 31) - 64)
+    return fail(GQ_ERR_SHAPE, "d_in or n_tok too large");
+  if (n_tok > 0 && !aligned(X_bf16, 16)) return fail(GQ_ERR_ARG, "X must be 16-byte aligned");
+  const HessPlan p = hessian_plan(n_tok, d_in);
+  GQ_TRY(check_ws(ws, ws_bytes, p.ws_bytes));
+  return launch_hessian(X_bf16, n_tok, d_in, H, ws, p, static_cast<cudaStream_t>(stream), false);
+}
+
 size_t gq_damp_cholesky_workspace_size(int64_t d_in) {
   if (d_in < 8 || d_in % 8 != 0) return 0;
   return chol_ws_bytes(d_in);
@@ -296,6 +310,48 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
     if (sse_host) *sse_host = sse;
     if (mse_host) *mse_host = n_tok > 0 ? sse / (static_cast<double>(n_tok) * d_out) : 0.0;
     GQ_TRY(device_status(word, "recon_error"));
+  }
+  return GQ_OK;
+}
+
+size_t gq_recon_error_hessian_workspace_size(int64_t d_out, int64_t d_in) {
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0) return 0;
+  return recon_hessian_ws_bytes(d_out, d_in);
+}
+
+gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
+                                 const uint16_t *scales, const uint16_t *zeros,
+                                 const int32_t *g_idx, int64_t d_out, int64_t d_in,
+                                 int group_size, int sym, const float *H0, int64_t n_tok,
+                                 double *sse_dev, double *sse_host, double *mse_host, void *ws,
+                                 size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  GQ_TRY(check_dtype(w_dtype));
+  if (!W || !qpacked || !scales || !sse_dev || !H0) return fail(GQ_ERR_ARG, "null pointer");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
+  GQ_TRY(check_layer(d_out, d_in));
+  GQ_TRY(check_group(group_size, d_in));
+  if (n_tok < 0) return fail(GQ_ERR_SHAPE, "bad n_tok");
+  if (d_out > (int64_t(1) << 30) || d_in > (int64_t(1) << 30))
+    return fail(GQ_ERR_SHAPE, "layer too large");
+  if (!aligned(W, 16) || !aligned(H0, 16))
+    return fail(GQ_ERR_ARG, "W and H0 must be 16-byte aligned");
+  GQ_TRY(check_ws(ws, ws_bytes, recon_hessian_ws_bytes(d_out, d_in)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GQ_TRY(launch_recon_hessian(W, w_dtype, qpacked, scales, zeros, g_idx, d_out, d_in, group_size,
+                              sym, H0, sse_dev, ws, st));
+  if (sse_host || mse_host) {
+    double sse = 0.0;
+    int32_t word = 0;
+    if (cudaMemcpyAsync(&sse, sse_dev, sizeof(double), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return check_launch("recon_error_hessian sync");
+    if (sse_host) *sse_host = sse;
+    if (mse_host) *mse_host = n_tok > 0 ? sse / (static_cast<double>(n_tok) * d_out) : 0.0;
+    GQ_TRY(device_status(word, "recon_error_hessian"));
   }
   return GQ_OK;
 }

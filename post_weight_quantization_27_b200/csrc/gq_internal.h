@@ -65,7 +65,7 @@ struct HessPlan {
 };
 HessPlan hessian_plan(int64_t n_tok, int64_t d_in);
 gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, void *ws,
-                         const HessPlan &plan, cudaStream_t st);
+                         const HessPlan &plan, cudaStream_t st, bool accumulate = true);
 
 size_t chol_ws_bytes(int64_t d);
 // use_aux: run the inverse chain on a second stream (forked from and joined
@@ -74,10 +74,14 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
                            uint8_t *dead_out, float *U, int32_t *info_dev, void *ws,
                            cudaStream_t st, bool use_aux = true);
 
-// C = beta C + alpha A B in fp32 on the tensor cores (3 x TF32 split).
+// C = beta C + alpha A B in fp32 on the tensor cores (3 x TF32 split); with
+// dot_partials, per output tile the sum of (alpha A B) .* C instead (C is
+// read, not written; gemm_tf32x3_tiles(M, N) partials).
 gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
                              const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
-                             int64_t ldc, bool lower, int *status, cudaStream_t st);
+                             int64_t ldc, bool lower, int *status, cudaStream_t st,
+                             double *dot_partials = nullptr);
+int gemm_tf32x3_tiles(int M, int N);
 
 size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size);
 gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,
@@ -86,6 +90,13 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
                       int32_t *g_idx, void *ws, cudaStream_t st);
 
 size_t recon_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok);
+// SSE by the trace route tr(dW H0 dW^T) / 2 (H0 = 2 X^T X undamped).
+size_t recon_hessian_ws_bytes(int64_t d_out, int64_t d_in);
+gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpacked,
+                               const uint16_t *scales, const uint16_t *zeros,
+                               const int32_t *g_idx, int64_t d_out, int64_t d_in, int group_size,
+                               int sym, const float *H0, double *sse_dev, void *ws,
+                               cudaStream_t st);
 gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,

@@ -258,11 +258,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// H[i][j] (i <= j) := H[i][j] + 2 * sum_s P_s(i, j); H[j][i] := H[i][j].
+// H[i][j] (i <= j) := H[i][j] + 2 * sum_s P_s(i, j) (without the H term
+// when !accumulate); H[j][i] := H[i][j].
 __global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__ H, int d,
                                                              const float *__restrict__ P,
                                                              int n_tiles, int n_bj, int n_split,
-                                                             const int *status) {
+                                                             const int *status, int accumulate) {
   const int bi = blockIdx.y, bj = blockIdx.x;
   if (bi > bj) return;
   __shared__ float tile[32][33];
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__
       float sum = 0.0f;
       for (int s = 0; s < n_split; ++s)
         sum += P[(static_cast<size_t>(s * n_tiles + t) * BM + (i - tb * BM)) * BN + (j - tj * BN)];
-      val = H[static_cast<size_t>(i) * d + j] + 2.0f * sum;
+      val = accumulate ? H[static_cast<size_t>(i) * d + j] + 2.0f * sum : 2.0f * sum;
       if (bad) val = __int_as_float(0x7fc00000);
       H[static_cast<size_t>(i) * d + j] = val;
     }
@@ -332,7 +333,7 @@ HessPlan hessian_plan(int64_t n_tok, int64_t d_in) {
 }
 
 gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, void *ws,
-                         const HessPlan &p, cudaStream_t st) {
+                         const HessPlan &p, cudaStream_t st, bool accumulate) {
   int *status = static_cast<int *>(ws);
   float *P = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kWsHeader);
   if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
@@ -360,7 +361,8 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
   }
   const int nb = static_cast<int>((d_in + 31) / 32);
   hessian_finish_kernel<<<dim3(nb, nb), 256, 0, st>>>(H, static_cast<int>(d_in), P, p.n_tiles,
-                                                      p.n_bj, p.n_split, status);
+                                                      p.n_bj, p.n_split, status,
+                                                      accumulate ? 1 : 0);
   count_launch();
   return check_launch("hessian_finish_kernel");
 }

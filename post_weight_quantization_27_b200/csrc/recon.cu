@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
     const T *__restrict__ W, const uint32_t *__restrict__ q, const uint16_t *__restrict__ scales,
     const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx,
     const float *__restrict__ col_inv, int64_t d_out, int64_t d_in, int group_size, int sym,
-    __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo) {
+    __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo, float *__restrict__ dw32) {
   const int64_t words = d_in / 8;
   const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   const int64_t n = d_out * words;
@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
     const int64_t r = e / words, wd = e % words;
     const uint32_t word = q[e];
     __align__(16) __nv_bfloat16 h[8], l[8];
+    __align__(16) float f[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int64_t c = wd * 8 + k;
@@ -89,12 +90,19 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
       float what = s * (code - z);
       if (col_inv) what *= col_inv[c];  // effective weight of a scaled layer
       const float dw = W ? ld_w(W + r * d_in + c) - what : what;  // W NULL: W^ itself
+      f[k] = dw;
       const __nv_bfloat16 hb = __float2bfloat16_rn(dw);
       h[k] = hb;
       l[k] = __float2bfloat16_rn(dw - __bfloat162float(hb));
     }
-    *reinterpret_cast<uint4 *>(hi + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(h);
-    *reinterpret_cast<uint4 *>(lo + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(l);
+    if (dw32) {  // fp32 dW (trace route)
+      float4 *dst = reinterpret_cast<float4 *>(dw32 + r * d_in + wd * 8);
+      dst[0] = *reinterpret_cast<const float4 *>(f);
+      dst[1] = *reinterpret_cast<const float4 *>(f + 4);
+    } else {
+      *reinterpret_cast<uint4 *>(hi + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(h);
+      *reinterpret_cast<uint4 *>(lo + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(l);
+    }
   }
 }
 
@@ -272,7 +280,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 __global__ void __launch_bounds__(1024) recon_reduce_kernel(const double *__restrict__ partials,
                                                             int64_t n, const int *status,
-                                                            double *__restrict__ sse) {
+                                                            double *__restrict__ sse,
+                                                            double scale = 1.0) {
   __shared__ double red[1024];
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < n; i += 1024) s += partials[i];
@@ -282,7 +291,8 @@ __global__ void __launch_bounds__(1024) recon_reduce_kernel(const double *__rest
     if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *sse = (status && *status) ? __longlong_as_double(0x7ff8000000000000ll) : red[0];
+  if (threadIdx.x == 0)
+    *sse = (status && *status) ? __longlong_as_double(0x7ff8000000000000ll) : red[0] * scale;
 }
 
 struct ReconLayout {
@@ -342,17 +352,17 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
     case GQ_F32:
       dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
                                                     scales, zeros, g_idx, col_inv, d_out, d_in,
-                                                    group_size, sym, hi, lo);
+                                                    group_size, sym, hi, lo, nullptr);
       break;
     case GQ_F16:
       dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
                                                      scales, zeros, g_idx, col_inv, d_out,
-                                                     d_in, group_size, sym, hi, lo);
+                                                     d_in, group_size, sym, hi, lo, nullptr);
       break;
     case GQ_BF16:
       dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
           static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, col_inv, d_out,
-          d_in, group_size, sym, hi, lo);
+          d_in, group_size, sym, hi, lo, nullptr);
       break;
   }
   count_launch();
@@ -375,6 +385,77 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
   s = check_launch("recon_mma_kernel");
   if (s != GQ_OK || Y) return s;
   recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, n_tiles * 8, status, sse_dev);
+  count_launch();
+  return check_launch("recon_reduce_kernel");
+}
+
+// ---------------------------------------------------------------------------
+// The same SSE by the trace route: ||dW X^T||_F^2 = tr(dW X^T X dW^T) =
+// tr(dW H0 dW^T) / 2 with the undamped H0 = 2 X^T X.  dW in fp32, then one
+// fp32 GEMM P = dW H0 on the tensor cores (3 x TF32) whose epilogue sums
+// P .* dW over each output tile instead of storing P; fp64 partials added
+// in a fixed order.  2 d_out d_in^2 flops instead of 2 n_tok d_out d_in.
+namespace {
+struct TraceLayout {
+  size_t off_partials, off_dw, total;
+};
+TraceLayout trace_layout(int64_t d_out, int64_t d_in) {
+  TraceLayout L{};
+  L.off_partials = kWsHeader;
+  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_out), static_cast<int>(d_in));
+  L.off_dw = L.off_partials + round_up(static_cast<size_t>(tiles) * sizeof(double), 256);
+  L.total = L.off_dw + round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256);
+  return L;
+}
+}  // namespace
+
+size_t recon_hessian_ws_bytes(int64_t d_out, int64_t d_in) {
+  return trace_layout(d_out, d_in).total;
+}
+
+gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpacked,
+                               const uint16_t *scales, const uint16_t *zeros,
+                               const int32_t *g_idx, int64_t d_out, int64_t d_in, int group_size,
+                               int sym, const float *H0, double *sse_dev, void *ws,
+                               cudaStream_t st) {
+  if (group_size == 0) group_size = -1;  // per-tensor scales are stored per row
+  const TraceLayout L = trace_layout(d_out, d_in);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  int *status = reinterpret_cast<int *>(base);
+  double *partials = reinterpret_cast<double *>(base + L.off_partials);
+  float *dw = reinterpret_cast<float *>(base + L.off_dw);
+  if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
+  unsigned g = static_cast<unsigned>((d_out * (d_in / 8) + 255) / 256);
+  const unsigned cap = static_cast<unsigned>(num_sms()) * 16;
+  if (g > cap) g = cap;
+  switch (dt) {
+    case GQ_F32:
+      dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
+                                                    scales, zeros, g_idx, nullptr, d_out, d_in,
+                                                    group_size, sym, nullptr, nullptr, dw);
+      break;
+    case GQ_F16:
+      dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
+                                                     scales, zeros, g_idx, nullptr, d_out, d_in,
+                                                     group_size, sym, nullptr, nullptr, dw);
+      break;
+    case GQ_BF16:
+      dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, nullptr, d_out,
+          d_in, group_size, sym, nullptr, nullptr, dw);
+      break;
+  }
+  count_launch();
+  gq_status s = check_launch("dequant_diff_kernel");
+  if (s != GQ_OK) return s;
+  // P = dW H0 (H0 symmetric, so its rows serve as the K-major B operand);
+  // per tile sum of P .* dW
+  s = launch_gemm_tf32x3(static_cast<int>(d_out), static_cast<int>(d_in), static_cast<int>(d_in),
+                         1.0f, dw, d_in, H0, d_in, true, 0.0f, dw, d_in, false, status, st,
+                         partials);
+  if (s != GQ_OK) return s;
+  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_out), static_cast<int>(d_in));
+  recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, tiles, status, sse_dev, 0.5);
   count_launch();
   return check_launch("recon_reduce_kernel");
 }

@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
     L.gq_hessian_workspace_size.argtypes = [_c_i64, _c_i64]
     L.gq_hessian_accumulate.restype = _c_int
     L.gq_hessian_accumulate.argtypes = [_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_hessian_compute.restype = _c_int
+    L.gq_hessian_compute.argtypes = [_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_damp_cholesky_workspace_size.restype = _c_sz
     L.gq_damp_cholesky_workspace_size.argtypes = [_c_i64]
     L.gq_damp_cholesky_inverse.restype = _c_int
@@ -72,6 +74,12 @@ def lib() -> ctypes.CDLL:
     L.gq_recon_error.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                                  _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp,
                                  _c_sz, _c_vp]
+    L.gq_recon_error_hessian_workspace_size.restype = _c_sz
+    L.gq_recon_error_hessian_workspace_size.argtypes = [_c_i64, _c_i64]
+    L.gq_recon_error_hessian.restype = _c_int
+    L.gq_recon_error_hessian.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64,
+                                         _c_i64, _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp,
+                                         _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_w4a16_workspace_size.restype = _c_sz
     L.gq_w4a16_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64]
     L.gq_w4a16_matmul.restype = _c_int
@@ -100,10 +108,11 @@ def lib() -> ctypes.CDLL:
 
 
 EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_workspace_size",
-           "gq_hessian_accumulate", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
+           "gq_hessian_accumulate", "gq_hessian_compute", "gq_damp_cholesky_workspace_size", "gq_damp_cholesky_inverse",
            "gq_damp_cholesky_inverse_noalloc",
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
-           "gq_recon_workspace_size", "gq_recon_error", "gq_w4a16_workspace_size",
+           "gq_recon_workspace_size", "gq_recon_error", "gq_recon_error_hessian_workspace_size",
+           "gq_recon_error_hessian", "gq_w4a16_workspace_size",
            "gq_w4a16_matmul", "gq_awq_workspace_size",
            "gq_awq_rtn_search", "gq_workspace_status", "gq_selftest_bounded_wait",
            "gq_kernel_timer_start",
@@ -185,9 +194,18 @@ def hessian_accumulate(X: torch.Tensor, H: torch.Tensor, ws: torch.Tensor | None
     return H
 
 
-def hessian(X: torch.Tensor, stream=None) -> torch.Tensor:
-    H = torch.zeros((X.shape[1], X.shape[1]), dtype=torch.float32, device=X.device)
-    return hessian_accumulate(X, H, stream=stream)
+def hessian(X: torch.Tensor, H: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """H = 2 X^T X (overwrites H when given; nothing is cleared first)."""
+    _dev(X, "X", torch.bfloat16)
+    n_tok, d_in = X.shape
+    if H is None:
+        H = torch.empty((d_in, d_in), dtype=torch.float32, device=X.device)
+    _dev(H, "H", torch.float32, (d_in, d_in))
+    ws = workspace(hessian_workspace_size(n_tok, d_in), X.device) if ws is None else ws
+    _check(lib().gq_hessian_compute(_p(X), n_tok, d_in, _p(H), _p(ws), ws.numel(),
+                                    _stream(stream)), "gq_hessian_compute")
+    return H
 
 
 # ------------------------------------------------------------------ damp + Cholesky
@@ -329,6 +347,33 @@ def recon_error(W: torch.Tensor, q: dict, X: torch.Tensor, group_size: int = -1,
                               ctypes.byref(mse_h) if sync else None,
                               _p(ws), ws.numel(), _stream(stream))
     _check(st, "gq_recon_error")
+    return (sse_h.value, mse_h.value) if sync else sse
+
+
+def recon_error_hessian_workspace_size(d_out: int, d_in: int) -> int:
+    return int(lib().gq_recon_error_hessian_workspace_size(d_out, d_in))
+
+
+def recon_error_hessian(W: torch.Tensor, q: dict, H0: torch.Tensor, n_tok: int,
+                        group_size: int = -1, sym: bool = True, sync: bool = True,
+                        sse: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                        stream=None):
+    """The same SSE from the undamped Hessian H0 = 2 X^T X:
+    tr((W - W^) H0 (W - W^)^T) / 2.  ``n_tok`` only scales the MSE.  Returns
+    like recon_error."""
+    _dev(W, "W")
+    d_out, d_in = W.shape
+    _dev(H0, "H0", torch.float32, (d_in, d_in))
+    sse = torch.empty(1, dtype=torch.float64, device=W.device) if sse is None else sse
+    ws = workspace(recon_error_hessian_workspace_size(d_out, d_in), W.device) if ws is None else ws
+    sse_h, mse_h = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    st = lib().gq_recon_error_hessian(_p(W), _DTYPES[W.dtype], _p(q["qpacked"]),
+                                      _p(q["scales"]), _p(q.get("zeros")), _p(q.get("g_idx")),
+                                      d_out, d_in, group_size, int(bool(sym)), _p(H0), n_tok,
+                                      _p(sse), ctypes.byref(sse_h) if sync else None,
+                                      ctypes.byref(mse_h) if sync else None,
+                                      _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_recon_error_hessian")
     return (sse_h.value, mse_h.value) if sync else sse
 
 

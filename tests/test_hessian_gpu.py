@@ -80,3 +80,16 @@ def test_hessian_full_size_sampled(workload, idx):
         assert rel_fro(g_, r_) <= TOL
     del X, H
     torch.cuda.empty_cache()
+
+
+def test_compute_overwrites_without_reading():
+    """gq_hessian_compute ignores what H holds (NaN here) and gives exactly
+    what accumulating onto zeros gives; with no tokens it gives zeros."""
+    X = I.random_layer(21, 200, 8, 777)[1].cuda()
+    H_nan = torch.full((200, 200), float("nan"), device="cuda")
+    a = gq.hessian(X, H=H_nan)
+    b = gq.hessian_accumulate(X, torch.zeros(200, 200, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    z = gq.hessian(X[:0], H=torch.full((200, 200), 3.0, device="cuda"))
+    assert torch.count_nonzero(z).item() == 0
