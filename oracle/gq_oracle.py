@@ -75,7 +75,7 @@ F16_MAX = F32(65504.0)
 __all__ = [
     "hessian", "hessian_entries", "damp_hessian", "act_order_perm",
     "upper_factor_of_inverse", "sym_params", "affine_params", "quantize_codes",
-    "dequantize_codes", "pack_nibbles", "unpack_nibbles", "rtn_quantize",
+    "dequantize_codes", "code_offset", "pack_nibbles", "unpack_nibbles", "rtn_quantize",
     "GptqResult", "gptq_quantize", "dequantize_packed", "recon_sse",
     "recon_sse_trace", "bits_per_weight", "obs_quantize", "bruteforce_row",
     "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
@@ -229,41 +229,53 @@ def dequantize_codes(c, s16, z16):
         np.asarray(c, dtype=np.float64) - np.asarray(z16).astype(np.float64))
 
 
+def code_offset(sym, bits=4):
+    """Stored value of code 0: symmetric codes -q..q are stored with an
+    offset of 2^(bits-1) (8 at 4 bits, so every stored value is >= 1);
+    affine codes 0..2^bits - 1 as they are."""
+    return 2 ** (bits - 1) if sym else 0
+
+
 def pack_nibbles(codes, sym, bits=4):
-    """Pack [rows, d_in] codes into uint32 words of 8 nibbles along d_in;
-    nibble k of word j is column 8j + k (low nibble first).  Symmetric codes
-    are stored with an offset of 2^(bits-1) (so 8 is the zero level)."""
-    assert bits == 4
+    """Pack [rows, d_in] codes into uint32 words: each row is one little-
+    endian bit stream along d_in in which column k occupies bits
+    bits*k .. bits*k + bits - 1, cut into 32-bit words (word j holds stream
+    bits 32j .. 32j + 31).  At 4 bits, nibble k of word j is column 8j + k;
+    at 8 bits, byte k of word j is column 4j + k.  Needs bits * d_in to be a
+    multiple of 32."""
     c = np.asarray(codes, dtype=np.int64)
-    nib = (c + 8) if sym else c
-    assert nib.min(initial=0) >= 0 and nib.max(initial=0) <= 15
+    nib = c + code_offset(sym, bits)
+    assert nib.min(initial=0) >= 0 and nib.max(initial=0) <= 2 ** bits - 1
     rows, d_in = nib.shape
-    nib = nib.reshape(rows, d_in // 8, 8).astype(np.uint64)
-    words = np.zeros((rows, d_in // 8), dtype=np.uint64)
-    for k in range(8):
-        words |= nib[:, :, k] << np.uint64(4 * k)
+    assert (bits * d_in) % 32 == 0
+    stream = ((nib[:, :, None] >> np.arange(bits)) & 1).reshape(rows, d_in * bits)
+    stream = stream.reshape(rows, -1, 32).astype(np.uint64)
+    words = np.zeros(stream.shape[:2], dtype=np.uint64)
+    for i in range(32):
+        words |= stream[:, :, i] << np.uint64(i)
     return words.astype(np.uint32)
 
 
 def unpack_nibbles(words, d_in, sym, bits=4):
     """Inverse of ``pack_nibbles``."""
-    assert bits == 4
     w = np.asarray(words, dtype=np.uint32).astype(np.uint64)
     rows = w.shape[0]
-    out = np.zeros((rows, w.shape[1], 8), dtype=np.int64)
-    for k in range(8):
-        out[:, :, k] = ((w >> np.uint64(4 * k)) & np.uint64(0xF)).astype(np.int64)
-    out = out.reshape(rows, -1)[:, :d_in]
-    return out - 8 if sym else out
+    stream = ((w[:, :, None] >> np.arange(32, dtype=np.uint64)) & np.uint64(1)).reshape(rows, -1)
+    stream = stream[:, :d_in * bits].reshape(rows, d_in, bits).astype(np.int64)
+    out = np.zeros((rows, d_in), dtype=np.int64)
+    for i in range(bits):
+        out |= stream[:, :, i] << i
+    return out - code_offset(sym, bits)
 
 
-def bits_per_weight(d_out, d_in, group_size, sym, act_order=False):
-    """Storage cost of the packed output in bits per weight: 4 bits per code
-    plus one 16-bit scale (and one 16-bit zero unless symmetric) per group
-    ("GPTQ: Post-Training INT4", "Group Quantization"), plus a 32-bit group
-    index per input column when the columns are act-ordered."""
-    n_groups = 1 if group_size == -1 else d_in // group_size
-    bits = 4 * d_out * d_in + 16 * d_out * n_groups
+def bits_per_weight(d_out, d_in, group_size, sym, act_order=False, bits=4):
+    """Storage cost of the packed output in bits per weight: ``bits`` per
+    code plus one 16-bit scale (and one 16-bit zero unless symmetric) per
+    group ("GPTQ: Post-Training INT4", "Group Quantization"), plus a 32-bit
+    group index per input column when the columns are act-ordered."""
+    n_groups = 1 if group_size <= 0 else d_in // group_size
+    code_bits = bits
+    bits = code_bits * d_out * d_in + 16 * d_out * n_groups
     if not sym:
         bits += 16 * d_out * n_groups
     if act_order:
@@ -291,7 +303,7 @@ def rtn_quantize(W, group_size=-1, sym=True, bits=4):
         zeros = np.full((d_out, 1), z[0], dtype=np.float16)
         codes = quantize_codes(W32, scales, zeros, sym, bits)
         return dict(codes=codes, scales=scales, zeros=zeros,
-                    qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None)
+                    qpacked=pack_nibbles(codes, sym, bits) if (bits * d_in) % 32 == 0 else None)
     g = d_in if group_size == -1 else group_size
     n_groups = d_in // g
     codes = np.zeros((d_out, d_in), dtype=np.int64)
@@ -304,7 +316,7 @@ def rtn_quantize(W, group_size=-1, sym=True, bits=4):
         zeros[:, gi] = z
         codes[:, gi * g:(gi + 1) * g] = quantize_codes(blk, s[:, None], z[:, None], sym, bits)
     return dict(codes=codes, scales=scales, zeros=zeros,
-                qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None)
+                qpacked=pack_nibbles(codes, sym, bits) if (bits * d_in) % 32 == 0 else None)
 
 
 # --------------------------------------------------------------------------
@@ -317,7 +329,7 @@ class GptqResult:
     scales: np.ndarray     # [d_out, n_groups] fp16, group order of the (permuted) columns
     zeros: np.ndarray      # [d_out, n_groups] fp16
     g_idx: np.ndarray      # [d_in] int32, group of each original column
-    qpacked: np.ndarray    # [d_out, d_in / 8] uint32 (None unless d_in % 8 == 0)
+    qpacked: np.ndarray    # [d_out, bits * d_in / 32] uint32 (None unless that divides)
     W_hat: np.ndarray      # [d_out, d_in] fp64 dequantised, original column order
     n_followed: int = 0    # tie decisions adopted from ``follow``
     max_follow_dist: float = 0.0   # largest boundary distance among them
@@ -480,7 +492,7 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     return GptqResult(codes=codes, scales=scales, zeros=zeros,
                       g_idx=g_idx.astype(np.int32), n_followed=n_followed,
                       max_follow_dist=max_dist,
-                      qpacked=pack_nibbles(codes, sym, bits) if d_in % 8 == 0 else None,
+                      qpacked=pack_nibbles(codes, sym, bits) if (bits * d_in) % 32 == 0 else None,
                       W_hat=Q)
 
 
@@ -537,11 +549,11 @@ def recon_sse_trace(W, W_hat, H_undamped) -> float:
 # Consumer of the packed format
 # --------------------------------------------------------------------------
 
-def w4a16_matmul(qpacked, scales, zeros, d_in, group_size, sym, X, g_idx=None):
+def w4a16_matmul(qpacked, scales, zeros, d_in, group_size, sym, X, g_idx=None, bits=4):
     """Y = W^ X^T in fp64 with W^ = s (c - z) from the packed codes ("GPTQ:
     Post-Training INT4", "Group Quantization": 4-bit codes with 16-bit
     scales are what the quantised model is run from)."""
-    What = dequantize_packed(qpacked, scales, zeros, d_in, group_size, sym, g_idx)
+    What = dequantize_packed(qpacked, scales, zeros, d_in, group_size, sym, g_idx, bits)
     return What @ np.asarray(X, dtype=np.float64).T
 
 

@@ -666,3 +666,107 @@ def test_act_order_follow_only_within_key_ties():
     assert not adopted and p.tolist() == own.tolist()
     p, adopted = O.act_order_perm(H, follow=own)
     assert not adopted and p.tolist() == own.tolist()
+
+
+# ---------------------------------------------------------------- other bit widths
+
+@pytest.mark.parametrize("bits,sym_levels", [(2, 3), (3, 7), (4, 15), (8, 255)])
+def test_grid_levels_at_other_widths(bits, sym_levels):
+    """Symmetric grid -q..q with q = 2^(bits-1) - 1 (2^bits - 1 levels, the
+    15 of "GPT-2 Quantization Reconstruction Error" at 4 bits); affine grid
+    0..2^bits - 1 (2^bits levels); the absolute maximum maps to the end."""
+    rng = np.random.default_rng(30 + bits)
+    v = np.concatenate([np.linspace(-1.0, 1.0, 2001), rng.uniform(-1, 1, 20000)])[None].astype(F32)
+    s, z = O.sym_params(v, bits)
+    c = O.quantize_codes(v, s[:, None], z[:, None], True, bits)
+    assert len(np.unique(c)) == sym_levels and c.max() == sym_levels // 2
+    s, z = O.affine_params(v, bits)
+    c = O.quantize_codes(v, s[:, None], z[:, None], False, bits)
+    assert len(np.unique(c)) == 2 ** bits and c.min() == 0 and c.max() == 2 ** bits - 1
+
+
+def test_packing_bit_positions():
+    """Column k of a row occupies stream bits bits*k .. bits*k + bits - 1,
+    words little endian: checked against positions worked out by hand."""
+    # 8 bits: byte k of word j is column 4j + k
+    assert O.pack_nibbles(np.array([[1, 2, 3, 4]]), False, 8).tolist() == [[0x04030201]]
+    assert O.pack_nibbles(np.array([[-127, 0, 127, 1]]), True, 8).tolist() == [[0x81FF8001]]
+    # 3 bits: column 10 straddles words 0 and 1 (stream bits 30, 31, 32)
+    c = np.zeros((1, 32), dtype=np.int64)
+    c[0, 10] = 7
+    c[0, 0] = 5
+    c[0, 31] = 6
+    w = O.pack_nibbles(c, False, 3)
+    assert w.shape == (1, 3)
+    assert w[0, 0] == (5 | (3 << 30)) and w[0, 1] == 1 and w[0, 2] == (6 << 29)
+    # 2 bits: column k at bits 2k of word 0 for k < 16 (symmetric zero is stored as 2)
+    assert O.pack_nibbles(np.array([[1, 3, 0, 2] + [0] * 12]), False, 2).tolist() == [[1 | 3 << 2 | 2 << 6]]
+    sym2 = sum(2 << (2 * k) for k in range(4, 16))
+    assert O.pack_nibbles(np.array([[1, -1, 0, 1] + [0] * 12]), True, 2).tolist() == [
+        [3 | 1 << 2 | 2 << 4 | 3 << 6 | sym2]]
+    rng = np.random.default_rng(31)
+    for bits in (2, 3, 4, 8):
+        for sym in (True, False):
+            lo, hi = (-(2 ** (bits - 1) - 1), 2 ** (bits - 1) - 1) if sym else (0, 2 ** bits - 1)
+            codes = rng.integers(lo, hi + 1, size=(5, 64))
+            assert np.array_equal(O.unpack_nibbles(O.pack_nibbles(codes, sym, bits), 64, sym, bits),
+                                  codes)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 8])
+def test_storage_bits_at_other_widths(bits):
+    """bits per code plus 16 bits of scale (and of zero) per group of 128."""
+    W = np.random.default_rng(32).standard_normal((8, 1024)).astype(F32) * 0.02
+    for sym in (True, False):
+        r = O.rtn_quantize(W, 128, sym, bits)
+        nbytes = r["qpacked"].nbytes + r["scales"].nbytes + (0 if sym else r["zeros"].nbytes)
+        expect = bits + 16 / 128 + (0 if sym else 16 / 128)
+        assert nbytes * 8 / W.size == expect == O.bits_per_weight(8, 1024, 128, sym, bits=bits)
+
+
+@pytest.mark.parametrize("bits", [3, 8])
+@pytest.mark.parametrize("sym", [True, False])
+def test_cholesky_form_equals_obs_at_other_widths(bits, sym):
+    """The OBS equivalence pin does not depend on the grid: it holds at 3
+    and 8 bits, per channel and with groups of 4."""
+    rng = np.random.default_rng(40 + bits + sym)
+    for t in range(20):
+        d = 8
+        X = rng.standard_normal((int(rng.integers(2, 20)), d)) * rng.lognormal(0, 0.5, d)
+        W = rng.standard_normal((4, d)) * 0.1
+        H, _ = O.damp_hessian(O.hessian(X), 0.01)
+        U = O.upper_factor_of_inverse(H)
+        r = O.gptq_quantize(W, U, bits=bits, group_size=-1, sym=sym)
+        rg = O.gptq_quantize(W, U, bits=bits, group_size=4, sym=sym)
+        for i in range(4):
+            s, z = (O.sym_params if sym else O.affine_params)(W[i][None].astype(F32), bits)
+
+            def q(col, row):
+                c = O.quantize_codes(np.array([[row[col]]]), s[:, None], z[:, None], sym, bits)
+                return float(O.dequantize_codes(c, s[:, None], z[:, None])[0, 0])
+            assert np.array_equal(O.obs_quantize(W[i], H, q), r.W_hat[i])
+
+            state = {}
+
+            def qg(col, row):
+                if col % 4 == 0:
+                    state["p"] = (O.sym_params if sym else O.affine_params)(
+                        np.asarray(row[col:col + 4])[None].astype(F32), bits)
+                s2, z2 = state["p"]
+                c = O.quantize_codes(np.array([[row[col]]]), s2[:, None], z2[:, None], sym, bits)
+                return float(O.dequantize_codes(c, s2[:, None], z2[:, None])[0, 0])
+            assert np.array_equal(O.obs_quantize(W[i], H, qg), rg.W_hat[i])
+
+
+def test_eight_bit_error_scales_with_the_step():
+    """Rounding error is uniform within half a step, so at a fixed range the
+    RTN error variance scales with the squared step: 8-bit against 4-bit
+    per channel is (7 / 127)^2 of it, within sampling noise."""
+    rng = np.random.default_rng(33)
+    W = rng.standard_normal((256, 4096)).astype(F32) * 0.02
+    err = {}
+    for bits in (4, 8):
+        r = O.rtn_quantize(W, -1, True, bits)
+        Wh = O.dequantize_packed(r["qpacked"], r["scales"], r["zeros"], 4096, -1, True, bits=bits)
+        err[bits] = np.mean((Wh - W) ** 2)
+    assert err[8] / err[4] == pytest.approx((7 / 127) ** 2, rel=0.1)
