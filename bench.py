@@ -211,14 +211,14 @@ class LayerRun:
                 gq._check(L.gq_recon_error_hessian(
                     gq._p(self.W), gq._DTYPES[self.W.dtype], gq._p(o["qpacked"]),
                     gq._p(o["scales"]), gq._p(o["zeros"]), gq._p(o.get("g_idx")), sp.d_out,
-                    sp.d_in, sp.group_size, int(sp.sym), gq._p(self.H0), sp.n_tok,
+                    sp.d_in, 4, sp.group_size, int(sp.sym), gq._p(self.H0), sp.n_tok,
                     self.sse.data_ptr() + 8 * k, None, None, gq._p(self.ws_r),
                     self.ws_r.numel(), s), "recon")
                 continue
             gq._check(L.gq_recon_error(
                 gq._p(self.W), gq._DTYPES[self.W.dtype], gq._p(o["qpacked"]),
                 gq._p(o["scales"]), gq._p(o["zeros"]), gq._p(o.get("g_idx")), sp.d_out,
-                sp.d_in, sp.group_size, int(sp.sym), gq._p(self.X), sp.n_tok,
+                sp.d_in, 4, sp.group_size, int(sp.sym), gq._p(self.X), sp.n_tok,
                 self.sse.data_ptr() + 8 * k, None, None, gq._p(self.ws_r),
                 self.ws_r.numel(), s), "recon")
 

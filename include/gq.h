@@ -38,13 +38,20 @@
  *   - Shapes: W is d_out x d_in; X (calibration activations) is
  *     n_tok x d_in in bf16.  d_in must be a positive multiple of 8;
  *     d_out >= 1; n_tok >= 0 (an empty calibration batch adds nothing).
- *     Only bits == 4 is implemented.
- *   - Packed codes: uint32 words of 8 nibbles along d_in, qpacked is
- *     [d_out][d_in/8]; nibble k (bits 4k..4k+3) of word j is column 8j+k.
- *     Symmetric codes c in -7..7 are stored as c+8; affine codes 0..15 as is.
+ *   - Code width `bits`: 4 (the pages' INT4), or 2, 3 or 8 ("GPT-2
+ *     Quantization Reconstruction Error", "Possible extensions": 4-bit
+ *     against 8-bit; "Quantization sweep: perplexity vs compression": INT8
+ *     and INT4).  Widths other than 4 need d_in and the group size to be
+ *     multiples of 32, and GPTQ block_size 128.
+ *   - Packed codes: each row is one little-endian bit stream along d_in in
+ *     which column k occupies bits `bits`*k .. `bits`*k + bits - 1, cut into
+ *     uint32 words: qpacked is [d_out][bits * d_in / 32].  At 4 bits nibble
+ *     k of word j is column 8j+k; at 8 bits byte k of word j is column 4j+k.
+ *     Symmetric codes -q..q (q = 2^(bits-1) - 1: 15 levels at 4 bits) are
+ *     stored as c + 2^(bits-1); affine codes 0..2^bits - 1 as they are.
  *   - Scales and zeros are IEEE fp16 bit patterns (uint16), [d_out][n_groups]
  *     with n_groups = d_in / group_size, or 1 for group_size -1 and 0.  Zeros
- *     hold the integer zero-point 0..15 (0 for symmetric).
+ *     hold the integer zero-point 0..2^bits - 1 (0 for symmetric).
  *   - group_size is -1 (one group per output row), 0 (one scale for the
  *     whole matrix -- "GPT-2 Quantization Reconstruction Error", "Possible
  *     extensions": per-tensor scaling -- stored once per row, so the output
@@ -194,23 +201,24 @@ gq_status gq_damp_cholesky_inverse_noalloc(float *H, int64_t d_in, float damp_pe
  * update W[:, end:] -= Err * U[blk, end:].  A group's scale (and zero) is
  * taken from that group's current (already updated) weights when its first
  * column is reached ("Group Quantization"); per-channel (group_size == -1)
- * scales come from the initial row.  Symmetric grid: s = absmax / 7, codes
- * -7..7; affine ("Model Quantization Mechanics", section 1): s = (max' -
- * min') / 15 with the range widened to contain 0, z = rint(-min'/s),
- * codes 0..15.  The fp16-rounded scale is the one used; a scale that is 0
+ * scales come from the initial row.  Symmetric grid: s = absmax / q, codes
+ * -q..q (q = 7 at 4 bits); affine ("Model Quantization Mechanics", section
+ * 1): s = (max' - min') / m with the range widened to contain 0, z =
+ * rint(-min'/s), codes 0..m (m = 15 at 4 bits).  The fp16-rounded scale is
+ * the one used; a scale that is 0
  * in fp16 becomes 1 (and z = 0); codes are rint(w / s) + z clamped, with
  * IEEE division and round-half-to-even, in fp32.
  *
  *   W          [d_out][d_in] in w_dtype (device, read only; not modified)
  *   U          [d_in][d_in] fp32 upper factor from gq_damp_cholesky_inverse
  *              (in processing order)
- *   bits       4
+ *   bits       2, 3, 4 or 8 (see the conventions above)
  *   group_size -1, 0 (per tensor), 32, 64 or 128, dividing d_in and block_size
- *   block_size 32, 64 or 128 (the pages' value is 128)
+ *   block_size 32, 64 or 128 (the pages' value is 128; 128 unless bits is 4)
  *   sym        1 symmetric, 0 affine
  *   perm       [d_in] int32 processing order (act-order) or NULL
  *   dead       [d_in] uint8 dead-column mask or NULL
- *   qpacked    [d_out][d_in/8] uint32 (out), original column order
+ *   qpacked    [d_out][bits*d_in/32] uint32 (out), original column order
  *   scales     [d_out][n_groups] fp16 bits (out); with perm, group k holds
  *              processing positions k*g .. k*g+g-1
  *   zeros      [d_out][n_groups] fp16 bits (out) or NULL (sym)
@@ -233,7 +241,7 @@ gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out,
                                  int32_t *g_idx, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
- * Round-to-nearest baseline with int4 packing.
+ * Round-to-nearest baseline with packing (int4, and the other widths).
  * "GPT-2 Quantization Reconstruction Error", "What this project does"
  * (per output row scale, 15 levels), "Model Quantization Mechanics",
  * section 1 (affine; groups of g consecutive weights), "GPTQ: Post-Training
@@ -242,7 +250,8 @@ gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out,
  * with no feedback.  Bit-exact and deterministic.
  *
  *   W        [d_out][d_in] in w_dtype (device, read only, 16-byte aligned)
- *   qpacked  [d_out][d_in/8] uint32 (out)
+ *   bits     2, 3, 4 or 8
+ *   qpacked  [d_out][bits*d_in/32] uint32 (out)
  *   scales   [d_out][n_groups] fp16 bits (out)
  *   zeros    [d_out][n_groups] fp16 bits (out) or NULL (written with 0
  *            when sym and non-NULL)
@@ -261,6 +270,8 @@ gq_status gq_rtn_quantize_pack(const void *W, gq_dtype w_dtype, int64_t d_out, i
  *   W, w_dtype         original weights [d_out][d_in] (device)
  *   qpacked, scales,   the quantised layer (device), as produced above;
  *   zeros, g_idx       zeros NULL when sym; g_idx NULL unless act-order
+ *   bits, group_size,  as the layer was quantised with
+ *   sym
  *   X                  [n_tok][d_in] bf16 (device, 16-byte aligned)
  *   sse_dev            double (device, out): SSE = ||(W - W^) X^T||_F^2
  *   sse_host, mse_host double (host, out) or NULL; if either is non-NULL
@@ -274,7 +285,7 @@ gq_status gq_rtn_quantize_pack(const void *W, gq_dtype w_dtype, int64_t d_out, i
 size_t gq_recon_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok);
 gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
                          const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
-                         int64_t d_out, int64_t d_in, int group_size, int sym,
+                         int64_t d_out, int64_t d_in, int bits, int group_size, int sym,
                          const void *X_bf16, int64_t n_tok, double *sse_dev,
                          double *sse_host, double *mse_host, void *ws, size_t ws_bytes,
                          void *stream);
@@ -304,7 +315,7 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
 size_t gq_recon_error_hessian_workspace_size(int64_t d_out, int64_t d_in);
 gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
                                  const uint16_t *scales, const uint16_t *zeros,
-                                 const int32_t *g_idx, int64_t d_out, int64_t d_in,
+                                 const int32_t *g_idx, int64_t d_out, int64_t d_in, int bits,
                                  int group_size, int sym, const float *H0, int64_t n_tok,
                                  double *sse_dev, double *sse_host, double *mse_host, void *ws,
                                  size_t ws_bytes, void *stream);
@@ -316,20 +327,20 @@ gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t
  * quantised model is served from; this call multiplies them with 16-bit
  * activations: Y = W^ X^T with W^ = s (c - z) per group.
  *
- *   qpacked, scales, zeros, g_idx, d_out, d_in, group_size, sym
+ *   qpacked, scales, zeros, g_idx, d_out, d_in, bits, group_size, sym
  *              the quantised layer as produced by the calls above
  *   X          [n_tok][d_in] bf16 (device, 16-byte aligned)
  *   Y          [d_out][n_tok] fp32 (device, out, 16-byte aligned;
  *              n_tok a multiple of 4): the layer's outputs, feature-major
  *   ws         >= gq_w4a16_workspace_size(d_out, d_in, n_tok) bytes
- * W^ is formed in fp32 (exact: an fp16 scale times a 4-bit integer) and fed
+ * W^ is formed in fp32 (exact: an fp16 scale times a small integer) and fed
  * to the tensor cores as a bf16 hi + lo pair, which holds it exactly; the
  * products accumulate in fp32.
  * ---------------------------------------------------------------------- */
 size_t gq_w4a16_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok);
 gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
                           const uint16_t *zeros, const int32_t *g_idx, int64_t d_out,
-                          int64_t d_in, int group_size, int sym, const void *X_bf16,
+                          int64_t d_in, int bits, int group_size, int sym, const void *X_bf16,
                           int64_t n_tok, float *Y, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
@@ -366,8 +377,8 @@ gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
  *                sym) bytes, 256-byte aligned
  * Synchronises the stream once (the choice of alpha is made on the host).
  * ---------------------------------------------------------------------- */
-size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size,
-                             int sym);
+size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int bits,
+                             int group_size, int sym);
 gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
                             const float *H, const void *X_bf16, int64_t n_tok, int bits,
                             int group_size, int sym, int n_grid, uint32_t *qpacked,

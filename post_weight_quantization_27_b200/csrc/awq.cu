@@ -110,7 +110,7 @@ struct AwqWs {
   void *recon;
 };
 
-AwqWs carve(void *ws, int64_t d_out, int64_t d_in, int group_size) {
+AwqWs carve(void *ws, int64_t d_out, int64_t d_in, int group_size, int bits) {
   const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   uint8_t *p = static_cast<uint8_t *>(ws) + kWsHeader;
   AwqWs w{};
@@ -124,7 +124,7 @@ AwqWs carve(void *ws, int64_t d_out, int64_t d_in, int group_size) {
   w.s = reinterpret_cast<float *>(take(static_cast<size_t>(d_in) * 4));
   w.inv = reinterpret_cast<float *>(take(static_cast<size_t>(d_in) * 4));
   w.Wp = reinterpret_cast<float *>(take(static_cast<size_t>(d_out) * d_in * 4));
-  w.q = reinterpret_cast<uint32_t *>(take(static_cast<size_t>(d_out) * (d_in / 8) * 4));
+  w.q = reinterpret_cast<uint32_t *>(take(static_cast<size_t>(d_out) * (d_in * bits / 32) * 4));
   w.sc = reinterpret_cast<uint16_t *>(take(static_cast<size_t>(d_out) * n_groups * 2));
   w.z = reinterpret_cast<uint16_t *>(take(static_cast<size_t>(d_out) * n_groups * 2));
   w.sse = reinterpret_cast<double *>(take(kMaxGrid * sizeof(double)));
@@ -133,18 +133,18 @@ AwqWs carve(void *ws, int64_t d_out, int64_t d_in, int group_size) {
 }
 
 // Bytes that carve() lays out before the reconstruction workspace.
-size_t carve_bytes(int64_t d_out, int64_t d_in, int group_size) {
+size_t carve_bytes(int64_t d_out, int64_t d_in, int group_size, int bits) {
   const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   return kWsHeader + 3 * round_up(static_cast<size_t>(d_in) * 4, 256) + round_up(4, 256) +
          round_up(static_cast<size_t>(d_out) * d_in * 4, 256) +
-         round_up(static_cast<size_t>(d_out) * (d_in / 8) * 4, 256) +
+         round_up(static_cast<size_t>(d_out) * (d_in * bits / 32) * 4, 256) +
          2 * round_up(static_cast<size_t>(d_out) * n_groups * 2, 256) +
          round_up(kMaxGrid * sizeof(double), 256);
 }
 
 gq_status scale_and_quantize(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in,
                              const AwqWs &w, float alpha, int group_size, int sym, uint32_t *q,
-                             uint16_t *sc, uint16_t *z, cudaStream_t st) {
+                             uint16_t *sc, uint16_t *z, cudaStream_t st, int bits) {
   const unsigned gd = static_cast<unsigned>((d_in + 255) / 256);
   awq_colscale_kernel<<<gd, 256, 0, st>>>(w.logd, w.logbar, d_in, alpha, w.s, w.inv);
   count_launch();
@@ -168,30 +168,32 @@ gq_status scale_and_quantize(const void *W, gq_dtype dt, int64_t d_out, int64_t 
   count_launch();
   const gq_status s = check_launch("awq scale");
   if (s != GQ_OK) return s;
-  return launch_rtn(w.Wp, GQ_F32, d_out, d_in, group_size, sym, q, sc, sym ? nullptr : z, st);
+  return launch_rtn(w.Wp, GQ_F32, d_out, d_in, group_size, sym, q, sc, sym ? nullptr : z, st,
+                    bits);
 }
 
 }  // namespace
 
-size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int) {
-  return carve_bytes(d_out, d_in, group_size) + recon_ws_bytes(d_out, d_in, n_tok);
+size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int,
+                    int bits) {
+  return carve_bytes(d_out, d_in, group_size, bits) + recon_ws_bytes(d_out, d_in, n_tok);
 }
 
 gq_status launch_awq_rtn_search(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in,
                                 const float *H, const void *X, int64_t n_tok, int group_size,
                                 int sym, int n_grid, uint32_t *qpacked, uint16_t *scales,
                                 uint16_t *zeros, float *col_scale, double *mse_host,
-                                int32_t *best_host, void *ws, cudaStream_t st) {
-  const AwqWs w = carve(ws, d_out, d_in, group_size);
+                                int32_t *best_host, void *ws, cudaStream_t st, int bits) {
+  const AwqWs w = carve(ws, d_out, d_in, group_size, bits);
   awq_logdiag_kernel<<<1, 1024, 0, st>>>(H, d_in, w.logd, w.logbar);
   count_launch();
   for (int k = 0; k < n_grid; ++k) {
     const float alpha = static_cast<float>(k) / static_cast<float>(n_grid);
     gq_status s = scale_and_quantize(W, dt, d_out, d_in, w, alpha, group_size, sym, w.q, w.sc,
-                                     w.z, st);
+                                     w.z, st, bits);
     if (s != GQ_OK) return s;
     s = launch_recon(W, dt, w.q, w.sc, sym ? nullptr : w.z, nullptr, d_out, d_in, group_size,
-                     sym, X, n_tok, w.sse + k, w.recon, st, w.inv);
+                     sym, X, n_tok, w.sse + k, w.recon, st, w.inv, nullptr, bits);
     if (s != GQ_OK) return s;
   }
   std::vector<double> sse(static_cast<size_t>(n_grid));
@@ -210,7 +212,7 @@ gq_status launch_awq_rtn_search(const void *W, gq_dtype dt, int64_t d_out, int64
     if (!(sse[k] == sse[k])) return fail(GQ_ERR_NONFINITE, "non-finite reconstruction error");
   const float alpha = static_cast<float>(best) / static_cast<float>(n_grid);
   gq_status s = scale_and_quantize(W, dt, d_out, d_in, w, alpha, group_size, sym, qpacked,
-                                   scales, zeros, st);
+                                   scales, zeros, st, bits);
   if (s != GQ_OK) return s;
   if (col_scale && cudaMemcpyAsync(col_scale, w.s, sizeof(float) * d_in,
                                    cudaMemcpyDeviceToDevice, st) != cudaSuccess)

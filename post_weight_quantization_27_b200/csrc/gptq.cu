@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const T *__restrict__ W, int6
 }
 
 // Per-channel grid from the initial (working) row: one warp per row.
+template <int BITS>
 __global__ void __launch_bounds__(256) row_params_kernel(const float *__restrict__ Wk,
                                                          int64_t d_out, int64_t d_in, int sym,
                                                          uint16_t *__restrict__ scales,
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(256) row_params_kernel(const float *__restrict
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     }
     if (lane == 0) {
-      const GridParams g = sym ? grid_sym(amax) : grid_affine(mn, mx);
+      const GridParams g = sym ? grid_sym_b<BITS>(amax) : grid_affine_b<BITS>(mn, mx);
       scales[r] = g.s_bits;
       if (zeros) zeros[r] = sym ? 0 : g.z_bits;
     }
@@ -137,24 +138,29 @@ __global__ void invert_perm_kernel(const int32_t *__restrict__ perm, int64_t d,
   }
 }
 
-// qpacked[r][w] from the processing-order codes: nibble k <- codes[r][inv[8w+k]].
+// qpacked from the processing-order stored codes: column c of row r takes
+// codes[r][inv[c]].  Each thread packs one run of columns that fills whole
+// words: 8 columns (one word) at 4 bits, else 32 columns (bits words).
 __global__ void __launch_bounds__(256) pack_perm_kernel(const uint8_t *__restrict__ codes,
                                                         int64_t d_out, int64_t d_in,
                                                         const int32_t *__restrict__ inv,
-                                                        uint32_t *__restrict__ qpacked) {
-  const int64_t words = d_in / 8;
-  const int64_t n = d_out * words;
+                                                        uint32_t *__restrict__ qpacked,
+                                                        int bits) {
+  const int run = bits == 4 ? 8 : 32;          // columns per unit
+  const int nw = run * bits / 32;              // words per unit
+  const int64_t units = d_in / run;
+  const int64_t n = d_out * units;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * 256) {
-    const int64_t r = e / words, wd = e % words;
-    uint32_t v = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      int64_t pos = inv[wd * 8 + k];
+    const int64_t r = e / units, u = e % units;
+    uint32_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int k = 0; k < run; ++k) {
+      int64_t pos = inv[u * run + k];
       pos = pos < 0 ? 0 : (pos >= d_in ? d_in - 1 : pos);
-      v |= static_cast<uint32_t>(codes[r * d_in + pos]) << (4 * k);
+      put_code_rt(v, bits, k, static_cast<uint32_t>(codes[r * d_in + pos]));
     }
-    qpacked[e] = v;
+    uint32_t *dst = qpacked + r * (d_in * bits / 32) + u * nw;
+    for (int i = 0; i < nw; ++i) dst[i] = v[i];
   }
 }
 
@@ -167,9 +173,9 @@ __global__ void g_idx_kernel(const int32_t *__restrict__ inv, int64_t d, int g,
   }
 }
 
-GptqBlockLaunch pick_block(int B, int G) {
-#define GQ_PICK(b, g) \
-  if (B == b && G == g) return launch_gptq_block<b, g>;
+GptqBlockLaunch pick_block(int B, int G, int bits) {
+#define GQ_PICK(b, g, n) \
+  if (B == b && G == g && bits == n) return launch_gptq_block<b, g, n>;
   GQ_GPTQ_BLOCK_INSTANCES(GQ_PICK)
 #undef GQ_PICK
   return nullptr;
@@ -188,12 +194,12 @@ size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size) {
 gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,
                       int group_size, int block_size, int sym, const int32_t *perm,
                       const uint8_t *dead, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
-                      int32_t *g_idx, void *ws, cudaStream_t st) {
+                      int32_t *g_idx, void *ws, cudaStream_t st, int bits) {
   const int B = block_size;
   const bool per_tensor = group_size == 0;  // one scale for the matrix, stored per row
   if (per_tensor) group_size = -1;
-  GptqBlockLaunch blk = pick_block(B, group_size);
-  if (!blk) return fail(GQ_ERR_ARG, "unsupported (block_size, group_size) combination");
+  GptqBlockLaunch blk = pick_block(B, group_size, bits);
+  if (!blk) return fail(GQ_ERR_ARG, "unsupported (block_size, group_size, bits) combination");
   GptqWs w = carve(ws, d_out, d_in, B, perm != nullptr);
   const int64_t n = d_out * d_in;
   unsigned grid = static_cast<unsigned>((n + 255) / 256);
@@ -218,12 +224,17 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
   if (per_tensor) {
     const gq_status s = launch_tensor_params_f32(
         w.Wk, d_out, d_in, sym, scales, zeros, w.Err,
-        d_out * super_cols(d_in, B), st);
+        d_out * super_cols(d_in, B), st, bits);
     if (s != GQ_OK) return s;
   } else if (group_size == -1) {
     unsigned g2 = static_cast<unsigned>((d_out + 7) / 8);
     if (g2 > cap) g2 = cap;
-    row_params_kernel<<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros);
+    switch (bits) {
+      case 2: row_params_kernel<2><<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros); break;
+      case 3: row_params_kernel<3><<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros); break;
+      case 8: row_params_kernel<8><<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros); break;
+      default: row_params_kernel<4><<<g2, 256, 0, st>>>(w.Wk, d_out, d_in, sym, scales, zeros);
+    }
     count_launch();
   }
   int *status = static_cast<int *>(ws);
@@ -263,9 +274,9 @@ gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, c
   if (perm) {
     invert_perm_kernel<<<gd, 256, 0, st>>>(perm, d_in, w.inv);
     count_launch();
-    unsigned gp = static_cast<unsigned>((d_out * (d_in / 8) + 255) / 256);
+    unsigned gp = static_cast<unsigned>((d_out * (d_in / (bits == 4 ? 8 : 32)) + 255) / 256);
     if (gp > cap) gp = cap;
-    pack_perm_kernel<<<gp, 256, 0, st>>>(w.codes, d_out, d_in, w.inv, qpacked);
+    pack_perm_kernel<<<gp, 256, 0, st>>>(w.codes, d_out, d_in, w.inv, qpacked, bits);
     count_launch();
   }
   if (g_idx) {

@@ -1,5 +1,5 @@
-// Instantiation of the GPTQ column-block kernel for block 128, group 128.
+// Instantiation of the GPTQ column-block kernel for block 128, group 128, 4-bit codes.
 #include "gptq_block.cuh"
 namespace gq {
-GQ_DEFINE_BLOCK(128, 128)
+GQ_DEFINE_BLOCK(128, 128, 4)
 }  // namespace gq

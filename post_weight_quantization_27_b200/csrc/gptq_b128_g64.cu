@@ -1,5 +1,5 @@
-// Instantiation of the GPTQ column-block kernel for block 128, group 64.
+// Instantiation of the GPTQ column-block kernel for block 128, group 64, 4-bit codes.
 #include "gptq_block.cuh"
 namespace gq {
-GQ_DEFINE_BLOCK(128, 64)
+GQ_DEFINE_BLOCK(128, 64, 4)
 }  // namespace gq

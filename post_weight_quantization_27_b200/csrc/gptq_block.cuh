@@ -36,8 +36,8 @@ struct SubCtx {
   uint16_t *scales, *zeros;
 };
 
-template <int SB, int G, int J>
-__device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[SB / 8],
+template <int SB, int G, int BITS, int J>
+__device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[SB * BITS / 32],
                                             GridParams &gp, float &rs, const SubCtx &cx,
                                             int jb) {
   if constexpr (J < SB) {
@@ -51,7 +51,7 @@ __device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[S
           mn = fminf(mn, w[k]);
           mx = fmaxf(mx, w[k]);
         }
-        gp = cx.sym ? grid_sym(amax) : grid_affine(mn, mx);
+        gp = cx.sym ? grid_sym_b<BITS>(amax) : grid_affine_b<BITS>(mn, mx);
         rs = __fdiv_rn(1.0f, gp.s);
         const int64_t gi = (cx.c0 + j) / G;
         cx.scales[cx.row * cx.n_groups + gi] = gp.s_bits;
@@ -59,16 +59,22 @@ __device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[S
       }
       const float *urow = cx.Ub + j * cx.B + jb;
       uint32_t nib;
-      const float c = grid_code_fast(w[J], gp, rs, cx.sym, nib);
+      float c;
+      if constexpr (BITS == 4) {
+        c = grid_code_fast(w[J], gp, rs, cx.sym, nib);
+        packed[J / 8] |= nib << (4 * (J % 8));
+      } else {
+        c = grid_code_b<BITS>(w[J], gp, rs, cx.sym, nib);
+        put_code<BITS, J>(packed, nib);
+      }
       const float q = gp.s * (c - gp.z);
       const float delta = div_by_recip(w[J] - q, urow[J], cx.rU[j]);
-      packed[J / 8] |= nib << (4 * (J % 8));
 #pragma unroll
       for (int k = J + 1; k < SB; ++k) w[k] = fmaf(-delta, urow[k], w[k]);
       w[J] = delta;
       cx.D[j * cx.rows + cx.tid] = delta;
     }
-    gptq_column<SB, G, J + 1>(w, packed, gp, rs, cx, jb);
+    gptq_column<SB, G, BITS, J + 1>(w, packed, gp, rs, cx, jb);
   }
 }
 
@@ -78,7 +84,7 @@ __device__ __forceinline__ void gptq_column(float (&w)[SB], uint32_t (&packed)[S
 // or one code byte per column (codes).
 // The B x B block of U arrives by one TMA copy (entries past the matrix
 // edge read as zero; only the upper triangle is used).
-template <int B, int G>
+template <int B, int G, int BITS>
 __global__ void __launch_bounds__(128) gptq_block_kernel(
     const __grid_constant__ CUtensorMap tmU, const float *__restrict__ Wk, int64_t d_out,
     int64_t d_in, int64_t c0, int bw, int sym, float *__restrict__ Err, int64_t err_ld,
@@ -125,7 +131,7 @@ __global__ void __launch_bounds__(128) gptq_block_kernel(
       mn = fminf(fminf(mn, fminf(v.x, v.y)), fminf(v.z, v.w));
       mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
     }
-    gp = s ? grid_sym(amax) : grid_affine(mn, mx);
+    gp = s ? grid_sym_b<BITS>(amax) : grid_affine_b<BITS>(mn, mx);
     rs = __fdiv_rn(1.0f, gp.s);
     scales[row * n_groups + c0 / B] = gp.s_bits;
     if (zeros) zeros[row * n_groups + c0 / B] = s ? 0 : gp.z_bits;
@@ -154,30 +160,40 @@ __global__ void __launch_bounds__(128) gptq_block_kernel(
         w[k + 3] = fmaf(-dj, uv.w, w[k + 3]);
       }
     }
-    uint32_t packed[SB / 8];
+    constexpr int NW = SB * BITS / 32;  // packed words of the sub-block
+    uint32_t packed[NW];
 #pragma unroll
-    for (int i = 0; i < SB / 8; ++i) packed[i] = 0;
-    gptq_column<SB, GS, 0>(w, packed, gp, rs, cx, jb);
+    for (int i = 0; i < NW; ++i) packed[i] = 0;
+    gptq_column<SB, GS, BITS, 0>(w, packed, gp, rs, cx, jb);
 
     float *err = Err + row * err_ld + jb;
 #pragma unroll
     for (int k = 0; k < SB; k += 4)
       *reinterpret_cast<float4 *>(err + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
     if (qpacked) {
-      uint32_t *dst = qpacked + row * (d_in / 8) + (c0 + jb) / 8;
+      // the sub-block starts on a word boundary: column c0 + jb is a
+      // multiple of 32; word i holds stream bits 32 i .. 32 i + 31
+      uint32_t *dst = qpacked + row * (d_in * BITS / 32) + (c0 + jb) * BITS / 32;
 #pragma unroll
-      for (int i = 0; i < SB / 8; ++i)
-        if (jb + i * 8 < bw) dst[i] = packed[i];
+      for (int i = 0; i < NW; ++i)
+        if (jb + (32 * i) / BITS < bw) dst[i] = packed[i];
     } else {
       uint8_t *dst = codes + row * d_in + c0 + jb;
 #pragma unroll
       for (int i = 0; i < SB / 8; ++i)
         if (jb + i * 8 < bw) {
           uint2 v;
-          v.x = (packed[i] & 0xFu) | ((packed[i] >> 4) & 0xFu) << 8 |
-                ((packed[i] >> 8) & 0xFu) << 16 | ((packed[i] >> 12) & 0xFu) << 24;
-          v.y = ((packed[i] >> 16) & 0xFu) | ((packed[i] >> 20) & 0xFu) << 8 |
-                ((packed[i] >> 24) & 0xFu) << 16 | ((packed[i] >> 28) & 0xFu) << 24;
+          if constexpr (BITS == 4) {
+            v.x = (packed[i] & 0xFu) | ((packed[i] >> 4) & 0xFu) << 8 |
+                  ((packed[i] >> 8) & 0xFu) << 16 | ((packed[i] >> 12) & 0xFu) << 24;
+            v.y = ((packed[i] >> 16) & 0xFu) | ((packed[i] >> 20) & 0xFu) << 8 |
+                  ((packed[i] >> 24) & 0xFu) << 16 | ((packed[i] >> 28) & 0xFu) << 24;
+          } else {
+            v.x = get_code(packed, BITS, 8 * i) | get_code(packed, BITS, 8 * i + 1) << 8 |
+                  get_code(packed, BITS, 8 * i + 2) << 16 | get_code(packed, BITS, 8 * i + 3) << 24;
+            v.y = get_code(packed, BITS, 8 * i + 4) | get_code(packed, BITS, 8 * i + 5) << 8 |
+                  get_code(packed, BITS, 8 * i + 6) << 16 | get_code(packed, BITS, 8 * i + 7) << 24;
+          }
           *reinterpret_cast<uint2 *>(dst + i * 8) = v;
         }
     }
@@ -190,7 +206,7 @@ typedef gq_status (*GptqBlockLaunch)(const CUtensorMap &, const float *, int64_t
 
 // tmU: fp32 tensor map over U with a B x B box and no swizzle.  Rows per
 // CTA shrink for short layers so that more SMs take part.
-template <int B, int G>
+template <int B, int G, int BITS>
 gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_out,
                             int64_t d_in, int64_t c0, int bw, int sym, float *Err,
                             int64_t err_ld, uint32_t *qp, uint8_t *codes, uint16_t *scales,
@@ -199,33 +215,38 @@ gq_status launch_gptq_block(const CUtensorMap &tmU, const float *Wk, int64_t d_o
   const int rows = d_out >= 4 * 128 * sms ? 128 : (d_out >= 2 * 64 * sms ? 64 : 32);
   const size_t smem = (static_cast<size_t>(B) * (B + 1) + static_cast<size_t>(B) * rows) *
                           sizeof(float) + 16;
-  cudaFuncSetAttribute(gptq_block_kernel<B, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(gptq_block_kernel<B, G, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(smem));
   const unsigned grid = static_cast<unsigned>((d_out + rows - 1) / rows);
   const int slot = timer_begin(GQ_KERNEL_GPTQ_BLOCK, st);
-  gptq_block_kernel<B, G><<<grid, rows, smem, st>>>(tmU, Wk, d_out, d_in, c0, bw, sym, Err,
+  gptq_block_kernel<B, G, BITS><<<grid, rows, smem, st>>>(tmU, Wk, d_out, d_in, c0, bw, sym, Err,
                                                     err_ld, qp, codes, scales, zeros, n_groups,
                                                     status);
   count_launch();
   // working weights of the block read, Err written (fp32), the U block,
-  // codes (packed: half a byte, else one byte per weight), scales (+ zeros)
+  // codes (packed: BITS / 8 bytes, else one byte per weight), scales (+ zeros)
   const double groups = G < 0 ? 0.0 : static_cast<double>((bw + G - 1) / G);
   timer_end(slot, st,
-            static_cast<double>(d_out) * bw * (8.0 + (qp ? 0.5 : 1.0)) +
+            static_cast<double>(d_out) * bw * (8.0 + (qp ? BITS / 8.0 : 1.0)) +
                 4.0 * static_cast<double>(B) * B + 2.0 * d_out * groups * (sym ? 1 : 2));
   return GQ_OK;
 }
 
-// Instantiated in gptq_b*.cu (one translation unit each, compiled in parallel).
-#define GQ_GPTQ_BLOCK_INSTANCES(X) \
-  X(128, -1) X(128, 128) X(128, 64) X(128, 32) X(64, -1) X(64, 64) X(64, 32) X(32, -1) X(32, 32)
+// Instantiated in gptq_b*.cu (one translation unit each, compiled in
+// parallel): (block, group, bits); widths other than 4 with block 128.
+#define GQ_GPTQ_BLOCK_INSTANCES(X)                                                            \
+  X(128, -1, 4) X(128, 128, 4) X(128, 64, 4) X(128, 32, 4) X(64, -1, 4) X(64, 64, 4)           \
+  X(64, 32, 4) X(32, -1, 4) X(32, 32, 4)                                                       \
+  X(128, -1, 8) X(128, 128, 8) X(128, 64, 8) X(128, 32, 8)                                     \
+  X(128, -1, 3) X(128, 128, 3) X(128, 64, 3) X(128, 32, 3)                                     \
+  X(128, -1, 2) X(128, 128, 2) X(128, 64, 2) X(128, 32, 2)
 
-#define GQ_BLOCK_SIG(b, g)                                                                  \
-  gq_status launch_gptq_block<b, g>(const CUtensorMap &, const float *, int64_t, int64_t,      \
-                                    int64_t, int, int, float *, int64_t, uint32_t *,           \
-                                    uint8_t *, uint16_t *, uint16_t *, int64_t, int *,         \
-                                    cudaStream_t);
-#define GQ_DECLARE_BLOCK(b, g) extern template GQ_BLOCK_SIG(b, g)
-#define GQ_DEFINE_BLOCK(b, g) template GQ_BLOCK_SIG(b, g)
+#define GQ_BLOCK_SIG(b, g, n)                                                               \
+  gq_status launch_gptq_block<b, g, n>(const CUtensorMap &, const float *, int64_t, int64_t,   \
+                                       int64_t, int, int, float *, int64_t, uint32_t *,        \
+                                       uint8_t *, uint16_t *, uint16_t *, int64_t, int *,      \
+                                       cudaStream_t);
+#define GQ_DECLARE_BLOCK(b, g, n) extern template GQ_BLOCK_SIG(b, g, n)
+#define GQ_DEFINE_BLOCK(b, g, n) template GQ_BLOCK_SIG(b, g, n)
 
 }  // namespace gq

@@ -102,6 +102,18 @@ gq_status check_group(int group_size, int64_t d_in) {
   return GQ_OK;
 }
 
+// Code widths: 2, 3, 4 or 8 bits.  Rows are bit streams cut into 32-bit
+// words, and widths other than 4 are packed in runs of 32 columns: d_in and
+// the group size must then be multiples of 32.
+gq_status check_bits(int bits, int64_t d_in, int group_size) {
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+    return fail(GQ_ERR_ARG, "bits must be 2, 3, 4 or 8");
+  if (bits != 4 && (d_in % 32 != 0 || (group_size > 0 && group_size % 32 != 0)))
+    return fail(GQ_ERR_SHAPE, "codes of other widths than 4 bits need d_in and group_size "
+                              "multiples of 32");
+  return GQ_OK;
+}
+
 gq_status check_ws(const void *ws, size_t have, size_t need) {
   if (need == 0) return GQ_OK;
   if (!ws || have < need)
@@ -243,19 +255,21 @@ gq_status gq_gptq_quantize_layer(const void *W, gq_dtype w_dtype, int64_t d_out,
   t_last_error.clear();
   GQ_TRY(check_dtype(w_dtype));
   if (!W || !U || !qpacked || !scales) return fail(GQ_ERR_ARG, "null pointer");
-  if (bits != 4) return fail(GQ_ERR_ARG, "only bits == 4 is implemented");
   if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
+  GQ_TRY(check_bits(bits, d_in, group_size));
   if (block_size != 32 && block_size != 64 && block_size != 128)
     return fail(GQ_ERR_ARG, "block_size must be 32, 64 or 128");
+  if (bits != 4 && block_size != 128)
+    return fail(GQ_ERR_ARG, "codes of other widths than 4 bits need block_size 128");
   if (group_size > 0 && (group_size < 32 || block_size % group_size != 0))
     return fail(GQ_ERR_ARG, "GPTQ group_size must be -1, 0, 32, 64 or 128 and divide block_size");
   if (!aligned(W, 16) || !aligned(U, 16)) return fail(GQ_ERR_ARG, "W and U must be 16-byte aligned");
   GQ_TRY(check_ws(ws, ws_bytes, gptq_ws_bytes(d_out, d_in, block_size)));
   return launch_gptq(W, w_dtype, d_out, d_in, U, group_size, block_size, sym, perm, dead,
-                     qpacked, scales, zeros, g_idx, ws, static_cast<cudaStream_t>(stream));
+                     qpacked, scales, zeros, g_idx, ws, static_cast<cudaStream_t>(stream), bits);
 }
 
 gq_status gq_rtn_quantize_pack(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
@@ -264,14 +278,14 @@ gq_status gq_rtn_quantize_pack(const void *W, gq_dtype w_dtype, int64_t d_out, i
   t_last_error.clear();
   GQ_TRY(check_dtype(w_dtype));
   if (!W || !qpacked || !scales) return fail(GQ_ERR_ARG, "null pointer");
-  if (bits != 4) return fail(GQ_ERR_ARG, "only bits == 4 is implemented");
   if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
+  GQ_TRY(check_bits(bits, d_in, group_size));
   if (!aligned(W, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
   return launch_rtn(W, w_dtype, d_out, d_in, group_size, sym, qpacked, scales, zeros,
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), bits);
 }
 
 size_t gq_recon_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok) {
@@ -281,7 +295,7 @@ size_t gq_recon_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok) {
 
 gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
                          const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
-                         int64_t d_out, int64_t d_in, int group_size, int sym,
+                         int64_t d_out, int64_t d_in, int bits, int group_size, int sym,
                          const void *X_bf16, int64_t n_tok, double *sse_dev, double *sse_host,
                          double *mse_host, void *ws, size_t ws_bytes, void *stream) {
   t_last_error.clear();
@@ -292,13 +306,14 @@ gq_status gq_recon_error(const void *W, gq_dtype w_dtype, const uint32_t *qpacke
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
+  GQ_TRY(check_bits(bits, d_in, group_size));
   if (n_tok < 0 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
   if (!aligned(W, 16) || (n_tok > 0 && !aligned(X_bf16, 16)))
     return fail(GQ_ERR_ARG, "W and X must be 16-byte aligned");
   GQ_TRY(check_ws(ws, ws_bytes, recon_ws_bytes(d_out, d_in, n_tok)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   GQ_TRY(launch_recon(W, w_dtype, qpacked, scales, zeros, g_idx, d_out, d_in, group_size, sym,
-                      X_bf16, n_tok, sse_dev, ws, st));
+                      X_bf16, n_tok, sse_dev, ws, st, nullptr, nullptr, bits));
   if (sse_host || mse_host) {
     double sse = 0.0;
     int32_t word = 0;
@@ -321,7 +336,7 @@ size_t gq_recon_error_hessian_workspace_size(int64_t d_out, int64_t d_in) {
 
 gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t *qpacked,
                                  const uint16_t *scales, const uint16_t *zeros,
-                                 const int32_t *g_idx, int64_t d_out, int64_t d_in,
+                                 const int32_t *g_idx, int64_t d_out, int64_t d_in, int bits,
                                  int group_size, int sym, const float *H0, int64_t n_tok,
                                  double *sse_dev, double *sse_host, double *mse_host, void *ws,
                                  size_t ws_bytes, void *stream) {
@@ -332,6 +347,7 @@ gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
+  GQ_TRY(check_bits(bits, d_in, group_size));
   if (n_tok < 0) return fail(GQ_ERR_SHAPE, "bad n_tok");
   if (d_out > (int64_t(1) << 30) || d_in > (int64_t(1) << 30))
     return fail(GQ_ERR_SHAPE, "layer too large");
@@ -340,7 +356,7 @@ gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t
   GQ_TRY(check_ws(ws, ws_bytes, recon_hessian_ws_bytes(d_out, d_in)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   GQ_TRY(launch_recon_hessian(W, w_dtype, qpacked, scales, zeros, g_idx, d_out, d_in, group_size,
-                              sym, H0, sse_dev, ws, st));
+                              sym, H0, sse_dev, ws, st, bits));
   if (sse_host || mse_host) {
     double sse = 0.0;
     int32_t word = 0;
@@ -363,7 +379,7 @@ size_t gq_w4a16_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok) {
 
 gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
                           const uint16_t *zeros, const int32_t *g_idx, int64_t d_out,
-                          int64_t d_in, int group_size, int sym, const void *X_bf16,
+                          int64_t d_in, int bits, int group_size, int sym, const void *X_bf16,
                           int64_t n_tok, float *Y, void *ws, size_t ws_bytes, void *stream) {
   t_last_error.clear();
   if (!qpacked || !scales || !Y || (n_tok > 0 && !X_bf16)) return fail(GQ_ERR_ARG, "null pointer");
@@ -371,6 +387,7 @@ gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
+  GQ_TRY(check_bits(bits, d_in, group_size));
   if (n_tok < 0 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
   if (d_out > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad d_out");
   if (n_tok > 0 && !aligned(X_bf16, 16)) return fail(GQ_ERR_ARG, "X must be 16-byte aligned");
@@ -379,16 +396,17 @@ gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
   GQ_TRY(check_ws(ws, ws_bytes, recon_ws_bytes(d_out, d_in, n_tok)));
   return launch_recon(nullptr, GQ_F32, qpacked, scales, zeros, g_idx, d_out, d_in, group_size,
                       sym, X_bf16, n_tok, nullptr, ws, static_cast<cudaStream_t>(stream),
-                      nullptr, Y);
+                      nullptr, Y, bits);
 }
 
-size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size,
-                             int sym) {
+size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int bits,
+                             int group_size, int sym) {
   if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || n_tok < 1) return 0;
   if (group_size > 0 && (group_size < 8 || group_size % 8 != 0 || d_in % group_size != 0))
     return 0;
   if (group_size < -1) return 0;
-  return awq_ws_bytes(d_out, d_in, n_tok, group_size, sym);
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return 0;
+  return awq_ws_bytes(d_out, d_in, n_tok, group_size, sym, bits);
 }
 
 gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int64_t d_in,
@@ -400,19 +418,19 @@ gq_status gq_awq_rtn_search(const void *W, gq_dtype w_dtype, int64_t d_out, int6
   t_last_error.clear();
   GQ_TRY(check_dtype(w_dtype));
   if (!W || !H || !X_bf16 || !qpacked || !scales) return fail(GQ_ERR_ARG, "null pointer");
-  if (bits != 4) return fail(GQ_ERR_ARG, "only bits == 4 is implemented");
   if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
   if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
   if (n_grid < 1 || n_grid > 256) return fail(GQ_ERR_ARG, "n_grid must be 1 .. 256");
   GQ_TRY(check_layer(d_out, d_in));
   GQ_TRY(check_group(group_size, d_in));
+  GQ_TRY(check_bits(bits, d_in, group_size));
   if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
   if (!aligned(W, 16) || !aligned(X_bf16, 16))
     return fail(GQ_ERR_ARG, "W and X must be 16-byte aligned");
-  GQ_TRY(check_ws(ws, ws_bytes, awq_ws_bytes(d_out, d_in, n_tok, group_size, sym)));
+  GQ_TRY(check_ws(ws, ws_bytes, awq_ws_bytes(d_out, d_in, n_tok, group_size, sym, bits)));
   return launch_awq_rtn_search(W, w_dtype, d_out, d_in, H, X_bf16, n_tok, group_size, sym,
                                n_grid, qpacked, scales, zeros, col_scale, mse_host, best_host,
-                               ws, static_cast<cudaStream_t>(stream));
+                               ws, static_cast<cudaStream_t>(stream), bits);
 }
 
 gq_status gq_workspace_status(const void *ws, int32_t *status_host, void *stream) {

@@ -294,4 +294,83 @@ __device__ __forceinline__ uint32_t grid_nibble(float c, bool sym) {
   return static_cast<uint32_t>(static_cast<int>(c) + (sym ? 8 : 0)) & 0xFu;
 }
 
+// ---------------------------------------------------------------- any width
+// The same grid with BITS-bit codes: symmetric -q..q with q = 2^(BITS-1) - 1,
+// s = absmax / q, stored as c + 2^(BITS-1); affine 0..m with m = 2^BITS - 1,
+// s = (max' - min') / m, z = rint(-min' / s) clamped to 0..m.  IEEE fp32
+// with round-to-nearest-even throughout, the operation order of the 4-bit
+// functions above (which they reproduce at BITS = 4).
+template <int BITS>
+struct BitGrid {
+  static constexpr int kQ = (1 << (BITS - 1)) - 1;   // symmetric end code
+  static constexpr int kM = (1 << BITS) - 1;         // affine end code
+  static constexpr uint32_t kMask = (1u << BITS) - 1u;
+  static constexpr uint32_t kOffset = 1u << (BITS - 1);
+};
+
+template <int BITS>
+__device__ __forceinline__ GridParams grid_from_scale_b(float s32, float mn) {
+  GridParams g;
+  __half h = __float2half_rn(fminf(s32, 65504.0f));
+  const bool degenerate = __half2float(h) == 0.0f;
+  if (degenerate) h = __float2half_rn(1.0f);
+  g.s = __half2float(h);
+  g.s_bits = __half_as_ushort(h);
+  float z = rintf(__fdiv_rn(-mn, g.s));
+  z = fminf(fmaxf(z, 0.0f), static_cast<float>(BitGrid<BITS>::kM));
+  if (degenerate) z = 0.0f;
+  z = __fadd_rn(z, 0.0f);  // -0 -> +0
+  g.z = z;
+  g.z_bits = __half_as_ushort(__float2half_rn(z));
+  return g;
+}
+template <int BITS>
+__device__ __forceinline__ GridParams grid_sym_b(float absmax) {
+  return grid_from_scale_b<BITS>(__fdiv_rn(absmax, static_cast<float>(BitGrid<BITS>::kQ)), 0.0f);
+}
+template <int BITS>
+__device__ __forceinline__ GridParams grid_affine_b(float vmin, float vmax) {
+  const float mn = fminf(vmin, 0.0f), mx = fmaxf(vmax, 0.0f);
+  return grid_from_scale_b<BITS>(
+      __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(BitGrid<BITS>::kM)), mn);
+}
+// Integer code of w (as float) and its stored value, with rs = RN(1 / s):
+// c = clamp(rint(w / s) + z) in IEEE fp32.
+template <int BITS>
+__device__ __forceinline__ float grid_code_b(float w, const GridParams &g, float rs, bool sym,
+                                             uint32_t &stored) {
+  const float r = rintf(div_by_recip(w, g.s, rs));
+  float c;
+  if (sym) {
+    c = fminf(fmaxf(r, -static_cast<float>(BitGrid<BITS>::kQ)),
+              static_cast<float>(BitGrid<BITS>::kQ));
+    stored = static_cast<uint32_t>(static_cast<int>(c) + static_cast<int>(BitGrid<BITS>::kOffset));
+  } else {
+    c = fminf(fmaxf(__fadd_rn(r, g.z), 0.0f), static_cast<float>(BitGrid<BITS>::kM));
+    stored = static_cast<uint32_t>(static_cast<int>(c));
+  }
+  return c;
+}
+// OR the stored value of column k (of a run of columns starting on a word
+// boundary) into its place in the little-endian bit stream held in words[].
+template <int BITS, int K, int NW>
+__device__ __forceinline__ void put_code(uint32_t (&words)[NW], uint32_t stored) {
+  constexpr int bit = BITS * K, w = bit / 32, off = bit % 32;
+  words[w] |= stored << off;
+  if constexpr (off + BITS > 32) words[w + 1] |= stored >> (32 - off);
+}
+// put_code with a run-time column index.
+__device__ __forceinline__ void put_code_rt(uint32_t *words, int bits, int k, uint32_t stored) {
+  const int bit = bits * k, w = bit >> 5, off = bit & 31;
+  words[w] |= stored << off;
+  if (off + bits > 32) words[w + 1] |= stored >> (32 - off);
+}
+// Stored value of column k of a run of columns starting on a word boundary.
+__device__ __forceinline__ uint32_t get_code(const uint32_t *words, int bits, int k) {
+  const int bit = bits * k, w = bit >> 5, off = bit & 31;
+  uint32_t v = words[w] >> off;
+  if (off + bits > 32) v |= words[w + 1] << (32 - off);
+  return v & ((1u << bits) - 1u);
+}
+
 }  // namespace gq

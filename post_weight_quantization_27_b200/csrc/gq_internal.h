@@ -52,12 +52,14 @@ int num_sms();
 
 // ---- kernels (each returns GQ_OK or GQ_ERR_CUDA after launching) ----
 // group_size: -1 per row, 0 per tensor (one scale, stored once per row), else per group.
+// bits: 2, 3, 4 or 8 (codes of other widths than 4 need d_in and the group a
+// multiple of 32; rows are little-endian bit streams, see include/gq.h).
 gq_status launch_tensor_params_f32(const float *W, int64_t d_out, int64_t d_in, int sym,
                                    uint16_t *scales, uint16_t *zeros, float *scratch,
-                                   int64_t scratch_floats, cudaStream_t st);
+                                   int64_t scratch_floats, cudaStream_t st, int bits = 4);
 gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, int group_size,
                      int sym, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
-                     cudaStream_t st);
+                     cudaStream_t st, int bits = 4);
 
 struct HessPlan {
   int n_bi, n_bj, n_tiles, n_split, nkb_total, kb_per_split;
@@ -87,7 +89,7 @@ size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size);
 gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,
                       int group_size, int block_size, int sym, const int32_t *perm,
                       const uint8_t *dead, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
-                      int32_t *g_idx, void *ws, cudaStream_t st);
+                      int32_t *g_idx, void *ws, cudaStream_t st, int bits = 4);
 
 size_t recon_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok);
 // SSE by the trace route tr(dW H0 dW^T) / 2 (H0 = 2 X^T X undamped).
@@ -96,19 +98,20 @@ gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpack
                                const uint16_t *scales, const uint16_t *zeros,
                                const int32_t *g_idx, int64_t d_out, int64_t d_in, int group_size,
                                int sym, const float *H0, double *sse_dev, void *ws,
-                               cudaStream_t st);
+                               cudaStream_t st, int bits = 4);
 gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
                        int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
-                       const float *col_inv = nullptr, float *Y = nullptr);
+                       const float *col_inv = nullptr, float *Y = nullptr, int bits = 4);
 
 // Activation-aware scaling before RTN (awq.cu).
-size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int sym);
+size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int sym,
+                    int bits = 4);
 gq_status launch_awq_rtn_search(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in,
                                 const float *H, const void *X, int64_t n_tok, int group_size,
                                 int sym, int n_grid, uint32_t *qpacked, uint16_t *scales,
                                 uint16_t *zeros, float *col_scale, double *mse_host,
-                                int32_t *best_host, void *ws, cudaStream_t st);
+                                int32_t *best_host, void *ws, cudaStream_t st, int bits = 4);
 
 }  // namespace gq

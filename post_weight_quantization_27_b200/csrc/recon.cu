@@ -68,40 +68,53 @@ __global__ void __launch_bounds__(256) dequant_diff_kernel(
     const T *__restrict__ W, const uint32_t *__restrict__ q, const uint16_t *__restrict__ scales,
     const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx,
     const float *__restrict__ col_inv, int64_t d_out, int64_t d_in, int group_size, int sym,
-    __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo, float *__restrict__ dw32) {
-  const int64_t words = d_in / 8;
+    __nv_bfloat16 *__restrict__ hi, __nv_bfloat16 *__restrict__ lo, float *__restrict__ dw32,
+    int bits) {
+  // a unit is a run of columns that fills whole words of the row's bit
+  // stream: 8 columns (one word) at 4 bits, else 32 columns (bits words)
+  const int run = bits == 4 ? 8 : 32;
+  const int nw = run * bits / 32;
+  const int64_t units = d_in / run;
+  const int64_t row_words = d_in * bits / 32;
   const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
-  const int64_t n = d_out * words;
+  const int64_t n = d_out * units;
+  const uint32_t mask = (1u << bits) - 1u;
+  const int offset = sym ? (1 << (bits - 1)) : 0;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * 256) {
-    const int64_t r = e / words, wd = e % words;
-    const uint32_t word = q[e];
-    __align__(16) __nv_bfloat16 h[8], l[8];
-    __align__(16) float f[8];
+    const int64_t r = e / units, u = e % units;
+    uint32_t wv[8];
+    for (int i = 0; i < nw; ++i) wv[i] = q[r * row_words + u * nw + i];
+    for (int c8 = 0; c8 < run; c8 += 8) {
+      __align__(16) __nv_bfloat16 h[8], l[8];
+      __align__(16) float f[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int64_t c = wd * 8 + k;
-      int64_t gi = g_idx ? g_idx[c] : (group_size <= 0 ? 0 : c / group_size);
-      gi = gi < 0 ? 0 : (gi >= n_groups ? n_groups - 1 : gi);
-      const float s = __half2float(__ushort_as_half(scales[r * n_groups + gi]));
-      const float z = sym ? 0.0f : __half2float(__ushort_as_half(zeros[r * n_groups + gi]));
-      const int nib = static_cast<int>((word >> (4 * k)) & 0xFu);
-      const float code = static_cast<float>(sym ? nib - 8 : nib);
-      float what = s * (code - z);
-      if (col_inv) what *= col_inv[c];  // effective weight of a scaled layer
-      const float dw = W ? ld_w(W + r * d_in + c) - what : what;  // W NULL: W^ itself
-      f[k] = dw;
-      const __nv_bfloat16 hb = __float2bfloat16_rn(dw);
-      h[k] = hb;
-      l[k] = __float2bfloat16_rn(dw - __bfloat162float(hb));
-    }
-    if (dw32) {  // fp32 dW (trace route)
-      float4 *dst = reinterpret_cast<float4 *>(dw32 + r * d_in + wd * 8);
-      dst[0] = *reinterpret_cast<const float4 *>(f);
-      dst[1] = *reinterpret_cast<const float4 *>(f + 4);
-    } else {
-      *reinterpret_cast<uint4 *>(hi + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(h);
-      *reinterpret_cast<uint4 *>(lo + r * d_in + wd * 8) = *reinterpret_cast<const uint4 *>(l);
+      for (int k = 0; k < 8; ++k) {
+        const int64_t c = u * run + c8 + k;
+        int64_t gi = g_idx ? g_idx[c] : (group_size <= 0 ? 0 : c / group_size);
+        gi = gi < 0 ? 0 : (gi >= n_groups ? n_groups - 1 : gi);
+        const float s = __half2float(__ushort_as_half(scales[r * n_groups + gi]));
+        const float z = sym ? 0.0f : __half2float(__ushort_as_half(zeros[r * n_groups + gi]));
+        const int stored = static_cast<int>(bits == 4 ? (wv[0] >> (4 * k)) & 0xFu
+                                                      : get_code(wv, bits, c8 + k) & mask);
+        const float code = static_cast<float>(stored - offset);
+        float what = s * (code - z);
+        if (col_inv) what *= col_inv[c];  // effective weight of a scaled layer
+        const float dw = W ? ld_w(W + r * d_in + c) - what : what;  // W NULL: W^ itself
+        f[k] = dw;
+        const __nv_bfloat16 hb = __float2bfloat16_rn(dw);
+        h[k] = hb;
+        l[k] = __float2bfloat16_rn(dw - __bfloat162float(hb));
+      }
+      const int64_t off = r * d_in + u * run + c8;
+      if (dw32) {  // fp32 dW (trace route)
+        float4 *dst = reinterpret_cast<float4 *>(dw32 + off);
+        dst[0] = *reinterpret_cast<const float4 *>(f);
+        dst[1] = *reinterpret_cast<const float4 *>(f + 4);
+      } else {
+        *reinterpret_cast<uint4 *>(hi + off) = *reinterpret_cast<const uint4 *>(h);
+        *reinterpret_cast<uint4 *>(lo + off) = *reinterpret_cast<const uint4 *>(l);
+      }
     }
   }
 }
@@ -325,7 +338,7 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        const uint16_t *scales, const uint16_t *zeros, const int32_t *g_idx,
                        int64_t d_out, int64_t d_in, int group_size, int sym, const void *X,
                        int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
-                       const float *col_inv, float *Y) {
+                       const float *col_inv, float *Y, int bits) {
   if (group_size == 0) group_size = -1;  // per-tensor scales are stored per row
   const ReconLayout L = recon_layout(d_out, d_in, n_tok);
   uint8_t *base = static_cast<uint8_t *>(ws);
@@ -345,24 +358,24 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
     count_launch();
     return check_launch("recon_reduce_kernel");
   }
-  unsigned g = static_cast<unsigned>((d_out * (d_in / 8) + 255) / 256);
+  unsigned g = static_cast<unsigned>((d_out * (d_in / (bits == 4 ? 8 : 32)) + 255) / 256);
   const unsigned cap = static_cast<unsigned>(num_sms()) * 16;
   if (g > cap) g = cap;
   switch (dt) {
     case GQ_F32:
       dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
                                                     scales, zeros, g_idx, col_inv, d_out, d_in,
-                                                    group_size, sym, hi, lo, nullptr);
+                                                    group_size, sym, hi, lo, nullptr, bits);
       break;
     case GQ_F16:
       dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
                                                      scales, zeros, g_idx, col_inv, d_out,
-                                                     d_in, group_size, sym, hi, lo, nullptr);
+                                                     d_in, group_size, sym, hi, lo, nullptr, bits);
       break;
     case GQ_BF16:
       dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
           static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, col_inv, d_out,
-          d_in, group_size, sym, hi, lo, nullptr);
+          d_in, group_size, sym, hi, lo, nullptr, bits);
       break;
   }
   count_launch();
@@ -417,7 +430,7 @@ gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpack
                                const uint16_t *scales, const uint16_t *zeros,
                                const int32_t *g_idx, int64_t d_out, int64_t d_in, int group_size,
                                int sym, const float *H0, double *sse_dev, void *ws,
-                               cudaStream_t st) {
+                               cudaStream_t st, int bits) {
   if (group_size == 0) group_size = -1;  // per-tensor scales are stored per row
   const TraceLayout L = trace_layout(d_out, d_in);
   uint8_t *base = static_cast<uint8_t *>(ws);
@@ -425,24 +438,24 @@ gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpack
   double *partials = reinterpret_cast<double *>(base + L.off_partials);
   float *dw = reinterpret_cast<float *>(base + L.off_dw);
   if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
-  unsigned g = static_cast<unsigned>((d_out * (d_in / 8) + 255) / 256);
+  unsigned g = static_cast<unsigned>((d_out * (d_in / (bits == 4 ? 8 : 32)) + 255) / 256);
   const unsigned cap = static_cast<unsigned>(num_sms()) * 16;
   if (g > cap) g = cap;
   switch (dt) {
     case GQ_F32:
       dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
                                                     scales, zeros, g_idx, nullptr, d_out, d_in,
-                                                    group_size, sym, nullptr, nullptr, dw);
+                                                    group_size, sym, nullptr, nullptr, dw, bits);
       break;
     case GQ_F16:
       dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
                                                      scales, zeros, g_idx, nullptr, d_out, d_in,
-                                                     group_size, sym, nullptr, nullptr, dw);
+                                                     group_size, sym, nullptr, nullptr, dw, bits);
       break;
     case GQ_BF16:
       dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
           static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, nullptr, d_out,
-          d_in, group_size, sym, nullptr, nullptr, dw);
+          d_in, group_size, sym, nullptr, nullptr, dw, bits);
       break;
   }
   count_launch();

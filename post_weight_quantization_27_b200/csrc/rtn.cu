@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(256) tensor_stat_kernel(const T *__restrict__ 
 
 // part: n_part (a, b) pairs, or W itself (n_part == 0: a small tensor is
 // reduced here directly).
-template <typename T, bool SYM>
+template <typename T, bool SYM, int BITS = 4>
 __global__ void __launch_bounds__(256) tensor_params_kernel(const float *__restrict__ part,
                                                             int n_part, const T *__restrict__ W,
                                                             int64_t words, int64_t d_out,
@@ -379,7 +379,11 @@ __global__ void __launch_bounds__(256) tensor_params_kernel(const float *__restr
   block_combine<SYM>(st, sa, sb);
   if (threadIdx.x == 0) {
     bool small;
-    const GridParams g = st.grid(small);
+    GridParams g;
+    if constexpr (BITS == 4)
+      g = st.grid(small);
+    else
+      g = SYM ? grid_sym_b<BITS>(st.a) : grid_affine_b<BITS>(st.a, st.b);
     ps = g.s_bits;
     pz = SYM ? 0 : g.z_bits;
   }
@@ -405,6 +409,139 @@ __global__ void __launch_bounds__(256) tensor_pack_kernel(const T *__restrict__ 
     Vec8<T>::load(W + w * 8, v);
     q[w] = pack_word<SYM>(v, g, rs);
   }
+}
+
+// ---------------------------------------------------------------- other widths
+// Codes of BITS != 4 bits: a row is one little-endian bit stream along d_in
+// (column k at bits BITS k ..), so 32 consecutive columns make BITS whole
+// words.  One warp per segment (row, group), lanes over 32-column chunks:
+// a first pass for the statistic, a second (from L1 / L2) for the codes.
+// With params_given the scale (and zero) of each row are read instead
+// (per-tensor: one parameter set, stored per row).
+template <int BITS, int K = 0>
+__device__ __forceinline__ void pack_run(const float (&v)[32], const GridParams &g, float rs,
+                                         bool sym, uint32_t (&words)[BITS]) {
+  if constexpr (K < 32) {
+    uint32_t stored;
+    grid_code_b<BITS>(v[K], g, rs, sym, stored);
+    put_code<BITS, K>(words, stored);
+    pack_run<BITS, K + 1>(v, g, rs, sym, words);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load32(const T *p, float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float t[8];
+    Vec8<T>::load(p + 8 * i, t);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[8 * i + e] = t[e];
+  }
+}
+
+template <typename T, int BITS, bool SYM>
+__global__ void __launch_bounds__(256) rtn_bits_kernel(const T *__restrict__ W, int64_t d_out,
+                                                       int64_t d_in, int64_t seg_len,
+                                                       uint32_t *__restrict__ q,
+                                                       uint16_t *__restrict__ scales,
+                                                       uint16_t *__restrict__ zeros,
+                                                       int params_given) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t n_groups = d_in / seg_len, total = d_out * n_groups, chunks = seg_len / 32;
+  const int64_t row_words = d_in / 32 * BITS;
+  for (int64_t seg = warp; seg < total; seg += n_warps) {
+    const int64_t row = seg / n_groups, gi = seg - row * n_groups;
+    const T *src = W + row * d_in + gi * seg_len;
+    GridParams g{};
+    if (!params_given) {
+      SegStat<SYM> st;
+      for (int64_t c = lane; c < chunks; c += 32) {
+        float v[32];
+        load32(src + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) st.add(v[e]);
+      }
+      st.reduce(32);
+      g = SYM ? grid_sym_b<BITS>(st.a) : grid_affine_b<BITS>(st.a, st.b);
+      if (lane == 0) {
+        scales[seg] = g.s_bits;
+        if (zeros) zeros[seg] = SYM ? 0 : g.z_bits;
+      }
+    } else {
+      g.s = __half2float(__ushort_as_half(scales[seg]));
+      g.z = SYM ? 0.0f : __half2float(__ushort_as_half(zeros[seg]));
+    }
+    const float rs = __frcp_rn(g.s);
+    uint32_t *dst = q + row * row_words + gi * (seg_len / 32) * BITS;
+    for (int64_t c = lane; c < chunks; c += 32) {
+      float v[32];
+      load32(src + c * 32, v);
+      uint32_t words[BITS];
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) words[i] = 0u;
+      pack_run<BITS>(v, g, rs, SYM, words);
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) dst[c * BITS + i] = words[i];
+    }
+  }
+}
+
+template <typename T, int BITS>
+gq_status launch_bits(const void *W, int64_t d_out, int64_t d_in, int group_size, int sym,
+                      uint32_t *q, uint16_t *sc, uint16_t *z, cudaStream_t st) {
+  const T *w = static_cast<const T *>(W);
+  int params_given = 0;
+  int64_t seg_len = group_size <= 0 ? d_in : group_size;
+  if (group_size == 0) {  // per tensor: one parameter set (from block partials), then the codes
+    const int64_t words = d_out * d_in / 8;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
+    int64_t nb = (words + 255) / 256;
+    if (nb > cap) nb = cap;
+    if (nb > d_out * d_in * BITS / 32 / 2) nb = d_out * d_in * BITS / 32 / 2;
+    float *part = reinterpret_cast<float *>(q);  // the packed output as scratch
+    if (words <= 8192 || nb < 2) {
+      if (sym) tensor_params_kernel<T, true, BITS><<<1, 256, 0, st>>>(nullptr, 0, w, words, d_out, sc, z);
+      else tensor_params_kernel<T, false, BITS><<<1, 256, 0, st>>>(nullptr, 0, w, words, d_out, sc, z);
+      count_launch();
+    } else {
+      if (sym) {
+        tensor_stat_kernel<T, true><<<static_cast<unsigned>(nb), 256, 0, st>>>(w, words, part);
+        tensor_params_kernel<T, true, BITS><<<1, 256, 0, st>>>(part, static_cast<int>(nb), w, words, d_out, sc, z);
+      } else {
+        tensor_stat_kernel<T, false><<<static_cast<unsigned>(nb), 256, 0, st>>>(w, words, part);
+        tensor_params_kernel<T, false, BITS><<<1, 256, 0, st>>>(part, static_cast<int>(nb), w, words, d_out, sc, z);
+      }
+      count_launch(2);
+    }
+    params_given = 1;
+  }
+  const int64_t total = d_out * (d_in / seg_len);
+  int64_t blocks = (total + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (sym)
+    rtn_bits_kernel<T, BITS, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        w, d_out, d_in, seg_len, q, sc, z, params_given);
+  else
+    rtn_bits_kernel<T, BITS, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        w, d_out, d_in, seg_len, q, sc, z, params_given);
+  count_launch();
+  return check_launch("rtn_quantize_pack");
+}
+
+template <typename T>
+gq_status launch_typed_bits(const void *W, int64_t d_out, int64_t d_in, int group_size,
+                            int sym, int bits, uint32_t *q, uint16_t *sc, uint16_t *z,
+                            cudaStream_t st) {
+  switch (bits) {
+    case 2: return launch_bits<T, 2>(W, d_out, d_in, group_size, sym, q, sc, z, st);
+    case 3: return launch_bits<T, 3>(W, d_out, d_in, group_size, sym, q, sc, z, st);
+    case 8: return launch_bits<T, 8>(W, d_out, d_in, group_size, sym, q, sc, z, st);
+  }
+  return fail(GQ_ERR_ARG, "bits must be 2, 3, 4 or 8");
 }
 
 template <typename T, bool SYM>
@@ -501,9 +638,19 @@ gq_status launch_typed(const void *W, int64_t d_out, int64_t d_in, int group_siz
 
 // Per-tensor grid parameters of an fp32 matrix (the GPTQ working copy),
 // written once per row; scratch holds the block partials.
+template <int BITS>
+void tensor_params_f32_bits(const float *part, int n_part, const float *W, int64_t words,
+                            int64_t d_out, int sym, uint16_t *scales, uint16_t *zeros,
+                            cudaStream_t st) {
+  if (sym)
+    tensor_params_kernel<float, true, BITS><<<1, 256, 0, st>>>(part, n_part, W, words, d_out, scales, zeros);
+  else
+    tensor_params_kernel<float, false, BITS><<<1, 256, 0, st>>>(part, n_part, W, words, d_out, scales, zeros);
+}
+
 gq_status launch_tensor_params_f32(const float *W, int64_t d_out, int64_t d_in, int sym,
                                    uint16_t *scales, uint16_t *zeros, float *scratch,
-                                   int64_t scratch_floats, cudaStream_t st) {
+                                   int64_t scratch_floats, cudaStream_t st, int bits) {
   const int64_t words = d_out * d_in / 8;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 4;
   int64_t nb = (words + 255) / 256;
@@ -518,41 +665,50 @@ gq_status launch_tensor_params_f32(const float *W, int64_t d_out, int64_t d_in, 
     count_launch();
   }
   const int n_part = small ? 0 : static_cast<int>(nb);
-  if (sym)
-    tensor_params_kernel<float, true><<<1, 256, 0, st>>>(scratch, n_part, W, words, d_out, scales, zeros);
-  else
-    tensor_params_kernel<float, false><<<1, 256, 0, st>>>(scratch, n_part, W, words, d_out, scales, zeros);
+  switch (bits) {
+    case 2: tensor_params_f32_bits<2>(scratch, n_part, W, words, d_out, sym, scales, zeros, st); break;
+    case 3: tensor_params_f32_bits<3>(scratch, n_part, W, words, d_out, sym, scales, zeros, st); break;
+    case 8: tensor_params_f32_bits<8>(scratch, n_part, W, words, d_out, sym, scales, zeros, st); break;
+    default: tensor_params_f32_bits<4>(scratch, n_part, W, words, d_out, sym, scales, zeros, st);
+  }
   count_launch();
   return check_launch("per-tensor parameters");
 }
 
 gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, int group_size,
                      int sym, uint32_t *qpacked, uint16_t *scales, uint16_t *zeros,
-                     cudaStream_t st) {
+                     cudaStream_t st, int bits) {
   int wb = 0;
   gq_status s = GQ_OK;
   const int slot = timer_begin(GQ_KERNEL_RTN, st);
+  const bool b4 = bits == 4;
   switch (dt) {
     case GQ_F32:
       wb = 4;
-      s = launch_typed<float>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st);
+      s = b4 ? launch_typed<float>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st)
+             : launch_typed_bits<float>(W, d_out, d_in, group_size, sym, bits, qpacked, scales,
+                                        zeros, st);
       break;
     case GQ_F16:
       wb = 2;
-      s = launch_typed<__half>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st);
+      s = b4 ? launch_typed<__half>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros, st)
+             : launch_typed_bits<__half>(W, d_out, d_in, group_size, sym, bits, qpacked, scales,
+                                         zeros, st);
       break;
     case GQ_BF16:
       wb = 2;
-      s = launch_typed<__nv_bfloat16>(W, d_out, d_in, group_size, sym, qpacked, scales, zeros,
-                                      st);
+      s = b4 ? launch_typed<__nv_bfloat16>(W, d_out, d_in, group_size, sym, qpacked, scales,
+                                           zeros, st)
+             : launch_typed_bits<__nv_bfloat16>(W, d_out, d_in, group_size, sym, bits, qpacked,
+                                                scales, zeros, st);
       break;
     default:
       s = fail(GQ_ERR_DTYPE, "unknown dtype");
   }
-  // W read; codes (half a byte per weight), fp16 scales (and zeros) written
+  // W read; codes (bits / 8 bytes per weight), fp16 scales (and zeros) written
   const double n_groups = group_size <= 0 ? 1.0 : static_cast<double>(d_in / group_size);
   timer_end(slot, st,
-            static_cast<double>(d_out) * d_in * (wb + 0.5) +
+            static_cast<double>(d_out) * d_in * (wb + bits / 8.0) +
                 2.0 * d_out * n_groups * (sym ? 1 : 2));
   return s;
 }

@@ -72,21 +72,21 @@ def lib() -> ctypes.CDLL:
     L.gq_recon_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64]
     L.gq_recon_error.restype = _c_int
     L.gq_recon_error.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
-                                 _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp, _c_vp,
-                                 _c_sz, _c_vp]
+                                 _c_int, _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_vp,
+                                 _c_vp, _c_sz, _c_vp]
     L.gq_recon_error_hessian_workspace_size.restype = _c_sz
     L.gq_recon_error_hessian_workspace_size.argtypes = [_c_i64, _c_i64]
     L.gq_recon_error_hessian.restype = _c_int
     L.gq_recon_error_hessian.argtypes = [_c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64,
-                                         _c_i64, _c_int, _c_int, _c_vp, _c_i64, _c_vp, _c_vp,
-                                         _c_vp, _c_vp, _c_sz, _c_vp]
+                                         _c_i64, _c_int, _c_int, _c_int, _c_vp, _c_i64, _c_vp,
+                                         _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_w4a16_workspace_size.restype = _c_sz
     L.gq_w4a16_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64]
     L.gq_w4a16_matmul.restype = _c_int
     L.gq_w4a16_matmul.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_int, _c_int,
-                                  _c_vp, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
+                                  _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_awq_workspace_size.restype = _c_sz
-    L.gq_awq_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64, _c_int, _c_int]
+    L.gq_awq_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64, _c_int, _c_int, _c_int]
     L.gq_awq_rtn_search.restype = _c_int
     L.gq_awq_rtn_search.argtypes = [_c_vp, _c_int, _c_i64, _c_i64, _c_vp, _c_vp, _c_i64, _c_int,
                                     _c_int, _c_int, _c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
@@ -271,12 +271,15 @@ def _n_groups(d_in: int, group_size: int) -> int:
     return 1 if group_size <= 0 else d_in // group_size
 
 
-def _outputs(d_out, d_in, group_size, sym, dev, with_g_idx):
+def _outputs(d_out, d_in, group_size, sym, dev, with_g_idx, bits=4):
+    """Output tensors of a quantised layer; the dict also records its code
+    width (``bits``), which the consumers of the packed format read."""
     ng = _n_groups(d_in, group_size)
-    return dict(qpacked=torch.empty((d_out, d_in // 8), dtype=torch.int32, device=dev),
+    return dict(qpacked=torch.empty((d_out, bits * d_in // 32), dtype=torch.int32, device=dev),
                 scales=torch.empty((d_out, ng), dtype=torch.float16, device=dev),
                 zeros=None if sym else torch.empty((d_out, ng), dtype=torch.float16, device=dev),
-                g_idx=torch.empty(d_in, dtype=torch.int32, device=dev) if with_g_idx else None)
+                g_idx=torch.empty(d_in, dtype=torch.int32, device=dev) if with_g_idx else None,
+                bits=bits)
 
 
 def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, bits: int = 4, group_size: int = -1,
@@ -294,7 +297,8 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, bits: int = 4, group_s
         _dev(perm, "perm", torch.int32, (d_in,))
     if dead is not None:
         _dev(dead, "dead", torch.uint8, (d_in,))
-    o = _outputs(d_out, d_in, group_size, sym, W.device, perm is not None) if out is None else out
+    o = _outputs(d_out, d_in, group_size, sym, W.device, perm is not None, bits) \
+        if out is None else out
     ws = workspace(gptq_workspace_size(d_out, d_in, block_size), W.device) if ws is None else ws
     st = lib().gq_gptq_quantize_layer(_p(W), _DTYPES[W.dtype], d_out, d_in, _p(U), bits,
                                       group_size, block_size, int(bool(sym)), _p(perm), _p(dead),
@@ -308,12 +312,12 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, bits: int = 4, group_s
 
 def rtn_quantize_pack(W: torch.Tensor, bits: int = 4, group_size: int = -1, sym: bool = True,
                       out: dict | None = None, stream=None) -> dict:
-    """Round-to-nearest with int4 packing.  Same output layout as GPTQ."""
+    """Round-to-nearest with packing.  Same output layout as GPTQ."""
     _dev(W, "W")
     if W.dtype not in _DTYPES:
         raise ValueError(f"unsupported W dtype {W.dtype}")
     d_out, d_in = W.shape
-    o = _outputs(d_out, d_in, group_size, sym, W.device, False) if out is None else out
+    o = _outputs(d_out, d_in, group_size, sym, W.device, False, bits) if out is None else out
     st = lib().gq_rtn_quantize_pack(_p(W), _DTYPES[W.dtype], d_out, d_in, bits, group_size,
                                     int(bool(sym)), _p(o["qpacked"]), _p(o["scales"]),
                                     _p(o["zeros"]), _stream(stream))
@@ -341,8 +345,9 @@ def recon_error(W: torch.Tensor, q: dict, X: torch.Tensor, group_size: int = -1,
     ws = workspace(recon_workspace_size(d_out, d_in, n_tok), W.device) if ws is None else ws
     sse_h, mse_h = ctypes.c_double(0.0), ctypes.c_double(0.0)
     st = lib().gq_recon_error(_p(W), _DTYPES[W.dtype], _p(q["qpacked"]), _p(q["scales"]),
-                              _p(q.get("zeros")), _p(q.get("g_idx")), d_out, d_in, group_size,
-                              int(bool(sym)), _p(X), n_tok, _p(sse),
+                              _p(q.get("zeros")), _p(q.get("g_idx")), d_out, d_in,
+                              int(q.get("bits", 4)), group_size, int(bool(sym)), _p(X), n_tok,
+                              _p(sse),
                               ctypes.byref(sse_h) if sync else None,
                               ctypes.byref(mse_h) if sync else None,
                               _p(ws), ws.numel(), _stream(stream))
@@ -369,7 +374,8 @@ def recon_error_hessian(W: torch.Tensor, q: dict, H0: torch.Tensor, n_tok: int,
     sse_h, mse_h = ctypes.c_double(0.0), ctypes.c_double(0.0)
     st = lib().gq_recon_error_hessian(_p(W), _DTYPES[W.dtype], _p(q["qpacked"]),
                                       _p(q["scales"]), _p(q.get("zeros")), _p(q.get("g_idx")),
-                                      d_out, d_in, group_size, int(bool(sym)), _p(H0), n_tok,
+                                      d_out, d_in, int(q.get("bits", 4)), group_size,
+                                      int(bool(sym)), _p(H0), n_tok,
                                       _p(sse), ctypes.byref(sse_h) if sync else None,
                                       ctypes.byref(mse_h) if sync else None,
                                       _p(ws), ws.numel(), _stream(stream))
@@ -394,8 +400,9 @@ def w4a16_matmul(q: dict, d_in: int, X: torch.Tensor, group_size: int = -1, sym:
     Y = torch.empty((d_out, n_tok), dtype=torch.float32, device=X.device) if Y is None else Y
     ws = workspace(w4a16_workspace_size(d_out, d_in, n_tok), X.device) if ws is None else ws
     st = lib().gq_w4a16_matmul(_p(q["qpacked"]), _p(q["scales"]), _p(q.get("zeros")),
-                               _p(q.get("g_idx")), d_out, d_in, group_size, int(bool(sym)), _p(X),
-                               n_tok, _p(Y), _p(ws), ws.numel(), _stream(stream))
+                               _p(q.get("g_idx")), d_out, d_in, int(q.get("bits", 4)),
+                               group_size, int(bool(sym)), _p(X), n_tok, _p(Y), _p(ws),
+                               ws.numel(), _stream(stream))
     _check(st, "gq_w4a16_matmul")
     return Y
 
@@ -403,8 +410,9 @@ def w4a16_matmul(q: dict, d_in: int, X: torch.Tensor, group_size: int = -1, sym:
 # ------------------------------------------------------------------ activation-aware scaling
 
 def awq_workspace_size(d_out: int, d_in: int, n_tok: int, group_size: int = -1,
-                       sym: bool = True) -> int:
-    return int(lib().gq_awq_workspace_size(d_out, d_in, n_tok, group_size, int(bool(sym))))
+                       sym: bool = True, bits: int = 4) -> int:
+    return int(lib().gq_awq_workspace_size(d_out, d_in, n_tok, bits, group_size,
+                                           int(bool(sym))))
 
 
 def awq_rtn_search(W: torch.Tensor, H: torch.Tensor, X: torch.Tensor, bits: int = 4,
@@ -419,11 +427,11 @@ def awq_rtn_search(W: torch.Tensor, H: torch.Tensor, X: torch.Tensor, bits: int 
     _dev(X, "X", torch.bfloat16)
     d_out, d_in = W.shape
     n_tok = X.shape[0]
-    o = _outputs(d_out, d_in, group_size, sym, W.device, False)
+    o = _outputs(d_out, d_in, group_size, sym, W.device, False, bits)
     col = torch.empty(d_in, dtype=torch.float32, device=W.device)
     mse = np.zeros(n_grid, dtype=np.float64)
     best = ctypes.c_int32(-1)
-    ws = workspace(awq_workspace_size(d_out, d_in, n_tok, group_size, sym), W.device) \
+    ws = workspace(awq_workspace_size(d_out, d_in, n_tok, group_size, sym, bits), W.device) \
         if ws is None else ws
     st = lib().gq_awq_rtn_search(_p(W), _DTYPES[W.dtype], d_out, d_in, _p(H), _p(X), n_tok, bits,
                                  group_size, int(bool(sym)), n_grid, _p(o["qpacked"]),

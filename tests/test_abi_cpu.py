@@ -52,8 +52,12 @@ FAKE = ctypes.c_void_p(4096)   # never dereferenced: every call below fails vali
     (dict(dt=0, d_out=8, d_in=12, bits=4, g=-1, sym=1), 2),
     # group does not divide d_in
     (dict(dt=0, d_out=8, d_in=64, bits=4, g=48, sym=1), 2),
-    # bits != 4
-    (dict(dt=0, d_out=8, d_in=64, bits=3, g=-1, sym=1), 1),
+    # an unsupported code width
+    (dict(dt=0, d_out=8, d_in=64, bits=5, g=-1, sym=1), 1),
+    # 3-bit codes need d_in a multiple of 32
+    (dict(dt=0, d_out=8, d_in=72, bits=3, g=-1, sym=1), 2),
+    # 8-bit codes need the group a multiple of 32
+    (dict(dt=0, d_out=8, d_in=64, bits=8, g=16, sym=1), 2),
     # affine without zeros
     (dict(dt=0, d_out=8, d_in=64, bits=4, g=-1, sym=0), 1),
 ])
@@ -85,8 +89,14 @@ def test_other_argument_errors():
                                     FAKE, None, None, ctypes.c_void_p(4096 + 8), 1 << 40,
                                     None) == 4
     # recon: null sse_dev
-    assert L.gq_recon_error(FAKE, 0, FAKE, FAKE, None, None, 8, 64, -1, 1, FAKE, 16, None,
+    assert L.gq_recon_error(FAKE, 0, FAKE, FAKE, None, None, 8, 64, 4, -1, 1, FAKE, 16, None,
                             None, None, FAKE, 1 << 30, None) == 1
+    # GPTQ at another width than 4 bits needs block 128
+    assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 128, FAKE, 8, 64, 64, 1, None, None,
+                                    FAKE, FAKE, None, None, FAKE, 1 << 40, None) == 1
+    # trace route: null H0
+    assert L.gq_recon_error_hessian(FAKE, 0, FAKE, FAKE, None, None, 8, 64, 4, -1, 1, None, 16,
+                                    FAKE, None, None, FAKE, 1 << 30, None) == 1
 
 
 def test_kernel_timer_without_session():
@@ -112,7 +122,7 @@ def test_header_is_c_and_links_from_c(tmp_path):
         '#include "gq.h"\n#include <stdio.h>\n'
         "int main(void) {\n"
         '  printf("%s %zu %zu\\n", gq_status_string(GQ_ERR_NOT_PD),\n'
-        "         gq_hessian_workspace_size(2048, 768), gq_awq_workspace_size(8, 64, 16, -1, 1));\n"
+        "         gq_hessian_workspace_size(2048, 768), gq_awq_workspace_size(8, 64, 16, 4, -1, 1));\n"
         "  return gq_rtn_quantize_pack(0, GQ_F32, 8, 64, 4, -1, 1, 0, 0, 0, 0) == GQ_ERR_ARG ? 0 : 1;\n"
         "}\n")
     libdir = os.path.dirname(gq.LIB_PATH)

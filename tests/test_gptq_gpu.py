@@ -20,8 +20,8 @@ pytestmark = pytest.mark.gpu
 DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
 
-def _codes(out, d_in, sym):
-    return O.unpack_nibbles(u32(out["qpacked"]), d_in, sym)
+def _codes(out, d_in, sym, bits=4):
+    return O.unpack_nibbles(u32(out["qpacked"]), d_in, sym, bits)
 
 
 def code_agreement(got, ref):
@@ -29,10 +29,10 @@ def code_agreement(got, ref):
     return float(np.mean(diff == 0)), int(diff.max(initial=0))
 
 
-def check_gptq(out, oracle_run, d_in, sym, min_agree=0.999):
+def check_gptq(out, oracle_run, d_in, sym, min_agree=0.999, bits=4):
     """oracle_run(follow) -> GptqResult.  Asserts the parity bar (module
     docstring) and returns (raw agreement, replayed agreement, ties)."""
-    got = _codes(out, d_in, sym)
+    got = _codes(out, d_in, sym, bits)
     raw = oracle_run(None)
     raw_agree, _ = code_agreement(got, raw.codes)
     assert raw_agree >= min_agree, raw_agree
