@@ -488,6 +488,7 @@ KERNEL_BOUND = {
     "block_inverse": ("alu", "fp32 FMA", 1),
     "gptq_block": ("hbm", "HBM copy", 1),
     "rtn": ("hbm", "HBM copy", 1),
+    "qlinear": ("tensor", "bf16", 2),
 }
 
 

@@ -321,27 +321,47 @@ gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t
                                  size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
- * W4A16 product: a consumer of the packed format.
+ * Products with a quantised layer: consumers of the packed format.
  * "GPTQ: Post-Training INT4", "Group Quantization" and "Running GPTQ with
- * AutoGPTQ": the 4-bit codes with 16-bit scales (and zeros) are what a
- * quantised model is served from; this call multiplies them with 16-bit
- * activations: Y = W^ X^T with W^ = s (c - z) per group.
+ * AutoGPTQ": the packed codes with 16-bit scales (and zeros) are what a
+ * quantised model is served from.  Both calls multiply them with bf16
+ * activations, Y = W^ X^T with W^ = s (c - z) per group, in one tensor-core
+ * kernel that reads the packed codes and forms W^ in shared memory as it
+ * goes (no dequantised copy of W in device memory).  W^ is exact as a bf16
+ * hi + lo pair (an fp16 scale times a small integer), so the only error is
+ * the fp32 accumulation over d_in terms.
  *
  *   qpacked, scales, zeros, g_idx, d_out, d_in, bits, group_size, sym
  *              the quantised layer as produced by the calls above
  *   X          [n_tok][d_in] bf16 (device, 16-byte aligned)
- *   Y          [d_out][n_tok] fp32 (device, out, 16-byte aligned;
- *              n_tok a multiple of 4): the layer's outputs, feature-major
- *   ws         >= gq_w4a16_workspace_size(d_out, d_in, n_tok) bytes
- * W^ is formed in fp32 (exact: an fp16 scale times a small integer) and fed
- * to the tensor cores as a bf16 hi + lo pair, which holds it exactly; the
- * products accumulate in fp32.
+ *   ws         >= gq_w4a16_workspace_size(d_out, d_in, n_tok) bytes (the
+ *              device status word only)
+ *
+ * gq_w4a16_matmul: Y [d_out][n_tok] fp32 (device, out, 16-byte aligned;
+ * n_tok a multiple of 4), feature-major.
+ *
+ * gq_qlinear_bf16: the layer applied to X for the next layer's input,
+ * token-major: Z[t][j] = act((X W^T)[t][j]) + R[t][j], rounded once to bf16.
+ *   W_dense, w_dtype  used instead of the packed codes when qpacked is NULL
+ *              (the layer before quantisation: [d_out][d_in], 16-byte
+ *              aligned), else ignored
+ *   act        GQ_ACT_NONE, GQ_ACT_RELU or GQ_ACT_GELU (the tanh form,
+ *              0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))))
+ *   R          [n_tok][d_out] bf16 residual (device) or NULL
+ *   Z          [n_tok][d_out] bf16 (device, out)
  * ---------------------------------------------------------------------- */
+enum { GQ_ACT_NONE = 0, GQ_ACT_RELU = 1, GQ_ACT_GELU = 2 };
 size_t gq_w4a16_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok);
 gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
                           const uint16_t *zeros, const int32_t *g_idx, int64_t d_out,
                           int64_t d_in, int bits, int group_size, int sym, const void *X_bf16,
                           int64_t n_tok, float *Y, void *ws, size_t ws_bytes, void *stream);
+gq_status gq_qlinear_bf16(const uint32_t *qpacked, const uint16_t *scales,
+                          const uint16_t *zeros, const int32_t *g_idx, const void *W_dense,
+                          gq_dtype w_dtype, int64_t d_out, int64_t d_in, int bits,
+                          int group_size, int sym, const void *X_bf16, int64_t n_tok, int act,
+                          const void *R_bf16, void *Z_bf16, void *ws, size_t ws_bytes,
+                          void *stream);
 
 /* ------------------------------------------------------------------------
  * Activation-aware per-channel scaling before RTN.
@@ -435,8 +455,9 @@ gq_status gq_selftest_bounded_wait(int arrive, uint64_t limit_ns, void *ws, size
  *       destroys the events and ends the session.
  * The algorithmic work is counted in flops (2 per multiply-add) for
  * HESSIAN_MMA (symmetric half of X^T X), POTRF_TRSM, BLOCK_INVERSE,
- * GEMM_TF32X3 (the fp32 product; lower-triangle calls count the triangle)
- * and RECON_MMA (one product (W - W^) X^T), and in bytes that must cross
+ * GEMM_TF32X3 (the fp32 product; lower-triangle calls count the triangle),
+ * RECON_MMA (one product (W - W^) X^T) and QLINEAR (one product W^ X^T:
+ * 2 n_tok d_out d_in), and in bytes that must cross
  * HBM for GPTQ_BLOCK (the block's working weights read, Err written, the U
  * block, codes and scales) and RTN (W read, codes, scales and zeros
  * written).  One session at a time per process; the calls are thread safe.
@@ -449,7 +470,8 @@ typedef enum {
   GQ_KERNEL_GPTQ_BLOCK = 4,
   GQ_KERNEL_RTN = 5,
   GQ_KERNEL_RECON_MMA = 6,
-  GQ_KERNEL_COUNT = 7
+  GQ_KERNEL_QLINEAR = 7,
+  GQ_KERNEL_COUNT = 8
 } gq_kernel;
 
 gq_status gq_kernel_timer_start(uint32_t mask, int32_t capacity);

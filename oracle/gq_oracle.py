@@ -80,6 +80,7 @@ __all__ = [
     "recon_sse_trace", "bits_per_weight", "obs_quantize", "bruteforce_row",
     "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
     "gptq_layer", "awq_channel_scales", "awq_apply", "awq_rtn_search", "w4a16_matmul",
+    "round_to_bf16", "gelu_tanh", "apply_layer", "gptq_sequential",
 ]
 
 
@@ -555,6 +556,66 @@ def w4a16_matmul(qpacked, scales, zeros, d_in, group_size, sym, X, g_idx=None, b
     scales are what the quantised model is run from)."""
     What = dequantize_packed(qpacked, scales, zeros, d_in, group_size, sym, g_idx, bits)
     return What @ np.asarray(X, dtype=np.float64).T
+
+
+def round_to_bf16(x):
+    """Round fp64 values to the nearest bf16 value (8 significant bits, ties
+    to even), in one rounding step (no intermediate float32)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                     # x = m 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def gelu_tanh(x):
+    """GELU in its tanh form, 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715
+    x^3))), in fp64 (GPT-2's MLP activation)."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+
+def apply_layer(X, W_hat, act="none", residual=None):
+    """The layer applied to its input, as the next layer sees it: Z = act(X
+    W^T) (+ residual), fp64, rounded once to bf16.  X [n_tok, d_in], W_hat
+    [d_out, d_in]."""
+    Y = np.asarray(X, dtype=np.float64) @ np.asarray(W_hat, dtype=np.float64).T
+    if act == "relu":
+        Y = np.maximum(Y, 0.0)
+    elif act == "gelu":
+        Y = gelu_tanh(Y)
+    if residual is not None:
+        Y = Y + np.asarray(residual, dtype=np.float64)
+    return round_to_bf16(Y)
+
+
+def gptq_sequential(X0, layers, bits=4, group_size=-1, block_size=128, sym=True,
+                    damp_percent=0.01, quantized_inputs=True, follow=None):
+    """Layers quantised one after another, each calibrated on the input it
+    actually receives ("GPT-2 Quantization Reconstruction Error", "Key
+    findings": the per-layer errors were measured with the whole model
+    running, so each layer's input carries the error of the quantised layers
+    before it).  ``layers``: list of dicts with W [d_out, d_in], act ("none",
+    "relu", "gelu") and residual_from (None, or the index j <= l of an
+    earlier input X_j added to layer l's output, e.g. a block's input at the
+    end of an MLP block).  For each layer: H from its input X_l, GPTQ, the
+    layer error ||(W - W^) X_l^T||^2, then X_{l+1} = apply_layer(X_l, W^ (or
+    W when not ``quantized_inputs``), act, X_j).  ``follow``: per-layer
+    list of dicts (as for gptq_quantize) or None.  Returns (results, sse, xs)
+    with xs the inputs X_0 .. X_n."""
+    X = np.asarray(X0, dtype=np.float64)
+    results, sse, xs = [], [], [X]
+    for li, L in enumerate(layers):
+        W = np.asarray(L["W"], dtype=np.float64)
+        res, H0, U, perm, dead = gptq_layer(W, X, bits=bits, group_size=group_size,
+                                            block_size=block_size, sym=sym,
+                                            damp_percent=damp_percent,
+                                            follow=None if follow is None else follow[li])
+        results.append(res)
+        sse.append(recon_sse(W, res.W_hat, X))
+        j = L.get("residual_from")
+        X = apply_layer(X, res.W_hat if quantized_inputs else W, L.get("act", "none"),
+                        None if j is None else xs[j])
+        xs.append(X)
+    return results, sse, xs
 
 
 # --------------------------------------------------------------------------

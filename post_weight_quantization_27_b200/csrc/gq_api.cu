@@ -374,29 +374,61 @@ gq_status gq_recon_error_hessian(const void *W, gq_dtype w_dtype, const uint32_t
 
 size_t gq_w4a16_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok) {
   if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || n_tok < 0) return 0;
-  return recon_ws_bytes(d_out, d_in, n_tok);
+  return kWsHeader;
 }
+
+namespace {
+gq_status check_product(const uint32_t *qpacked, const uint16_t *scales, const uint16_t *zeros,
+                        int64_t d_out, int64_t d_in, int bits, int group_size, int sym,
+                        const void *X_bf16, int64_t n_tok, void *ws, size_t ws_bytes) {
+  if (qpacked && !scales) return fail(GQ_ERR_ARG, "null scales");
+  if (n_tok > 0 && !X_bf16) return fail(GQ_ERR_ARG, "null X");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (qpacked && sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
+  GQ_TRY(check_layer(d_out, d_in));
+  GQ_TRY(check_group(group_size, d_in));
+  if (qpacked) GQ_TRY(check_bits(bits, d_in, group_size));
+  if (n_tok < 0 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
+  if (d_out > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad d_out");
+  if (n_tok > 0 && !aligned(X_bf16, 16)) return fail(GQ_ERR_ARG, "X must be 16-byte aligned");
+  return check_ws(ws, ws_bytes, kWsHeader);
+}
+}  // namespace
 
 gq_status gq_w4a16_matmul(const uint32_t *qpacked, const uint16_t *scales,
                           const uint16_t *zeros, const int32_t *g_idx, int64_t d_out,
                           int64_t d_in, int bits, int group_size, int sym, const void *X_bf16,
                           int64_t n_tok, float *Y, void *ws, size_t ws_bytes, void *stream) {
   t_last_error.clear();
-  if (!qpacked || !scales || !Y || (n_tok > 0 && !X_bf16)) return fail(GQ_ERR_ARG, "null pointer");
-  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
-  if (sym == 0 && !zeros) return fail(GQ_ERR_ARG, "affine quantization needs zeros");
-  GQ_TRY(check_layer(d_out, d_in));
-  GQ_TRY(check_group(group_size, d_in));
-  GQ_TRY(check_bits(bits, d_in, group_size));
-  if (n_tok < 0 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
-  if (d_out > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad d_out");
-  if (n_tok > 0 && !aligned(X_bf16, 16)) return fail(GQ_ERR_ARG, "X must be 16-byte aligned");
+  if (!qpacked || !Y) return fail(GQ_ERR_ARG, "null pointer");
+  GQ_TRY(check_product(qpacked, scales, zeros, d_out, d_in, bits, group_size, sym, X_bf16, n_tok,
+                       ws, ws_bytes));
   if (!aligned(Y, 16) || n_tok % 4 != 0)
     return fail(GQ_ERR_ARG, "Y must be 16-byte aligned and n_tok a multiple of 4");
-  GQ_TRY(check_ws(ws, ws_bytes, recon_ws_bytes(d_out, d_in, n_tok)));
-  return launch_recon(nullptr, GQ_F32, qpacked, scales, zeros, g_idx, d_out, d_in, group_size,
-                      sym, X_bf16, n_tok, nullptr, ws, static_cast<cudaStream_t>(stream),
-                      nullptr, Y, bits);
+  return launch_qlinear(qpacked, scales, zeros, g_idx, nullptr, GQ_F32, d_out, d_in, bits,
+                        group_size, sym, X_bf16, n_tok, Y, nullptr, nullptr, GQ_ACT_NONE,
+                        static_cast<int *>(ws), static_cast<cudaStream_t>(stream));
+}
+
+gq_status gq_qlinear_bf16(const uint32_t *qpacked, const uint16_t *scales,
+                          const uint16_t *zeros, const int32_t *g_idx, const void *W_dense,
+                          gq_dtype w_dtype, int64_t d_out, int64_t d_in, int bits,
+                          int group_size, int sym, const void *X_bf16, int64_t n_tok, int act,
+                          const void *R_bf16, void *Z_bf16, void *ws, size_t ws_bytes,
+                          void *stream) {
+  t_last_error.clear();
+  if (!Z_bf16 || (!qpacked && !W_dense)) return fail(GQ_ERR_ARG, "null pointer");
+  if (!qpacked) {
+    GQ_TRY(check_dtype(w_dtype));
+    if (!aligned(W_dense, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
+  }
+  if (act != GQ_ACT_NONE && act != GQ_ACT_RELU && act != GQ_ACT_GELU)
+    return fail(GQ_ERR_ARG, "act must be GQ_ACT_NONE, GQ_ACT_RELU or GQ_ACT_GELU");
+  GQ_TRY(check_product(qpacked, scales, zeros, d_out, d_in, bits, group_size, sym, X_bf16, n_tok,
+                       ws, ws_bytes));
+  return launch_qlinear(qpacked, scales, zeros, g_idx, W_dense, w_dtype, d_out, d_in, bits,
+                        group_size, sym, X_bf16, n_tok, nullptr, Z_bf16, R_bf16, act,
+                        static_cast<int *>(ws), static_cast<cudaStream_t>(stream));
 }
 
 size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int bits,

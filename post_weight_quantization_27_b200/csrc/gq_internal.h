@@ -105,6 +105,15 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
                        int64_t n_tok, double *sse_dev, void *ws, cudaStream_t st,
                        const float *col_inv = nullptr, float *Y = nullptr, int bits = 4);
 
+// Y = W^ X^T with the codes dequantised inside the GEMM (qlinear.cu): Y
+// feature-major fp32 and / or Z = act(Y^T) + R token-major bf16; dense
+// weights when qpacked is NULL.  status: the call's device status word.
+gq_status launch_qlinear(const uint32_t *qpacked, const uint16_t *scales, const uint16_t *zeros,
+                         const int32_t *g_idx, const void *W_dense, gq_dtype w_dtype,
+                         int64_t d_out, int64_t d_in, int bits, int group_size, int sym,
+                         const void *X, int64_t n_tok, float *Y, void *Z, const void *R,
+                         int act, int *status, cudaStream_t st);
+
 // Activation-aware scaling before RTN (awq.cu).
 size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int sym,
                     int bits = 4);

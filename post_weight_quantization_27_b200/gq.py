@@ -85,6 +85,10 @@ def lib() -> ctypes.CDLL:
     L.gq_w4a16_matmul.restype = _c_int
     L.gq_w4a16_matmul.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_int, _c_int,
                                   _c_int, _c_vp, _c_i64, _c_vp, _c_vp, _c_sz, _c_vp]
+    L.gq_qlinear_bf16.restype = _c_int
+    L.gq_qlinear_bf16.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_i64, _c_i64,
+                                  _c_int, _c_int, _c_int, _c_vp, _c_i64, _c_int, _c_vp, _c_vp,
+                                  _c_vp, _c_sz, _c_vp]
     L.gq_awq_workspace_size.restype = _c_sz
     L.gq_awq_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64, _c_int, _c_int, _c_int]
     L.gq_awq_rtn_search.restype = _c_int
@@ -113,7 +117,7 @@ EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_w
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
            "gq_recon_workspace_size", "gq_recon_error", "gq_recon_error_hessian_workspace_size",
            "gq_recon_error_hessian", "gq_w4a16_workspace_size",
-           "gq_w4a16_matmul", "gq_awq_workspace_size",
+           "gq_w4a16_matmul", "gq_qlinear_bf16", "gq_awq_workspace_size",
            "gq_awq_rtn_search", "gq_workspace_status", "gq_selftest_bounded_wait",
            "gq_kernel_timer_start",
            "gq_kernel_timer_stop", "gq_kernel_timer_read", "gq_kernel_timer_release")
@@ -383,7 +387,10 @@ def recon_error_hessian(W: torch.Tensor, q: dict, H0: torch.Tensor, n_tok: int,
     return (sse_h.value, mse_h.value) if sync else sse
 
 
-# ------------------------------------------------------------------ W4A16 product
+# ------------------------------------------------------------------ products with a quantised layer
+
+ACT = {"none": 0, "relu": 1, "gelu": 2}
+
 
 def w4a16_workspace_size(d_out: int, d_in: int, n_tok: int) -> int:
     return int(lib().gq_w4a16_workspace_size(d_out, d_in, n_tok))
@@ -405,6 +412,28 @@ def w4a16_matmul(q: dict, d_in: int, X: torch.Tensor, group_size: int = -1, sym:
                                ws.numel(), _stream(stream))
     _check(st, "gq_w4a16_matmul")
     return Y
+
+
+def qlinear_bf16(X: torch.Tensor, d_out: int, q: dict | None = None, W: torch.Tensor | None = None,
+                 group_size: int = -1, sym: bool = True, act: str = "none",
+                 R: torch.Tensor | None = None, Z: torch.Tensor | None = None,
+                 ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Z = act(X W^T) (+ R), bf16 [n_tok][d_out]: the layer applied to its
+    input, from the packed layer ``q`` or (q None) from dense weights W."""
+    _dev(X, "X", torch.bfloat16)
+    n_tok, d_in = X.shape
+    Z = torch.empty((n_tok, d_out), dtype=torch.bfloat16, device=X.device) if Z is None else Z
+    if R is not None:
+        _dev(R, "R", torch.bfloat16, (n_tok, d_out))
+    ws = workspace(256, X.device) if ws is None else ws
+    qq = q or {}
+    st = lib().gq_qlinear_bf16(_p(qq.get("qpacked")), _p(qq.get("scales")), _p(qq.get("zeros")),
+                               _p(qq.get("g_idx")), _p(W), _DTYPES.get(W.dtype, 0) if W is not None else 0,
+                               d_out, d_in, int(qq.get("bits", 4)), group_size, int(bool(sym)),
+                               _p(X), n_tok, ACT[act], _p(R), _p(Z), _p(ws), ws.numel(),
+                               _stream(stream))
+    _check(st, "gq_qlinear_bf16")
+    return Z
 
 
 # ------------------------------------------------------------------ activation-aware scaling
@@ -446,9 +475,10 @@ def awq_rtn_search(W: torch.Tensor, H: torch.Tensor, X: torch.Tensor, bits: int 
 
 # gq_kernel values (include/gq.h) and the unit of each kernel's work figure
 KERNELS = ("hessian_mma", "potrf_trsm", "block_inverse", "gemm_tf32x3", "gptq_block", "rtn",
-           "recon_mma")
+           "recon_mma", "qlinear")
 KERNEL_UNITS = {"hessian_mma": "flop", "potrf_trsm": "flop", "block_inverse": "flop",
-                "gemm_tf32x3": "flop", "gptq_block": "byte", "rtn": "byte", "recon_mma": "flop"}
+                "gemm_tf32x3": "flop", "gptq_block": "byte", "rtn": "byte", "recon_mma": "flop",
+                "qlinear": "flop"}
 
 
 def kernel_timer_start(kernels, capacity: int) -> None:

@@ -770,3 +770,57 @@ def test_eight_bit_error_scales_with_the_step():
         Wh = O.dequantize_packed(r["qpacked"], r["scales"], r["zeros"], 4096, -1, True, bits=bits)
         err[bits] = np.mean((Wh - W) ** 2)
     assert err[8] / err[4] == pytest.approx((7 / 127) ** 2, rel=0.1)
+
+
+# ---------------------------------------------------------------- sequential pipeline
+
+def test_round_to_bf16_against_library_and_ties():
+    """One rounding to 8 significant bits, ties to even: checked at exact
+    midpoints and against torch's float32 -> bfloat16 conversion (a single
+    rounding for values that float32 holds exactly)."""
+    import torch
+    assert O.round_to_bf16(1.0 + 2.0 ** -8) == 1.0                  # tie -> even (1.0)
+    assert O.round_to_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6   # tie -> even
+    assert O.round_to_bf16(1.0 + 2.0 ** -8 + 2.0 ** -30) == 1.0 + 2.0 ** -7
+    assert O.round_to_bf16(-3.0) == -3.0 and O.round_to_bf16(0.0) == 0.0
+    v = np.random.default_rng(50).standard_normal(20000).astype(np.float32) * 10.0
+    ref = torch.from_numpy(v).to(torch.bfloat16).float().numpy().astype(np.float64)
+    assert np.array_equal(O.round_to_bf16(v.astype(np.float64)), ref)
+
+
+def test_gelu_tanh_closed_forms():
+    """gelu(0) = 0; gelu(x) - gelu(-x) = x exactly for the tanh form; the tanh
+    form of torch agrees to float32 precision."""
+    import torch
+    x = np.linspace(-6, 6, 1001)
+    assert O.gelu_tanh(0.0) == 0.0
+    assert np.allclose(O.gelu_tanh(x) - O.gelu_tanh(-x), x, rtol=0, atol=1e-12)
+    t = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    assert np.allclose(O.gelu_tanh(x), t, rtol=1e-12, atol=1e-12)
+
+
+def test_sequential_pipeline_structure():
+    """One layer: the pipeline is gptq_layer plus the layer error.  Two
+    layers: the second is calibrated on the first's quantised output, which
+    differs from its full-precision output, and the pipeline's errors are
+    its layers' errors on the inputs they received."""
+    rng = np.random.default_rng(51)
+    d, n = 64, 400
+    X0 = O.round_to_bf16(rng.standard_normal((n, d)))
+    W1 = rng.standard_normal((96, d)) * 0.1
+    W2 = rng.standard_normal((d, 96)) * 0.1
+    layers = [dict(W=W1, act="gelu"), dict(W=W2, act="none", residual_from=0)]
+    res, sse, xs = O.gptq_sequential(X0, layers[:1], group_size=32)
+    ref, *_ = O.gptq_layer(W1, X0, group_size=32)
+    assert np.array_equal(res[0].codes, ref.codes)
+    assert sse[0] == O.recon_sse(W1, ref.W_hat, X0)
+    res, sse, xs = O.gptq_sequential(X0, layers, group_size=32)
+    X1 = O.apply_layer(X0, res[0].W_hat, "gelu")
+    assert np.array_equal(xs[1], X1)
+    assert np.array_equal(xs[2], O.apply_layer(X1, res[1].W_hat, "none", X0))
+    ref2, *_ = O.gptq_layer(W2, X1, group_size=32)
+    assert np.array_equal(res[1].codes, ref2.codes)
+    assert sse[1] == O.recon_sse(W2, res[1].W_hat, X1)
+    _, _, xs_fp = O.gptq_sequential(X0, layers, group_size=32, quantized_inputs=False)
+    assert np.array_equal(xs_fp[1], O.apply_layer(X0, W1, "gelu"))
+    assert not np.array_equal(xs_fp[1], xs[1])
