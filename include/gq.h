@@ -364,6 +364,50 @@ gq_status gq_qlinear_bf16(const uint32_t *qpacked, const uint16_t *scales,
                           void *stream);
 
 /* ------------------------------------------------------------------------
+ * Sequential quantisation of a chain of layers, each calibrated on the input
+ * it actually receives: the output of the already quantised layers before
+ * it ("GPT-2 Quantization Reconstruction Error", "Key findings": the
+ * per-layer errors there were measured with the whole model running, so
+ * upstream quantisation error reaches every later layer).
+ *
+ * For l = 0 .. n_layers - 1, on `stream`:
+ *   H0 = 2 X_l^T X_l; dead columns, damping, U (no act-order); GPTQ of W_l
+ *   into the layer's outputs; sse_dev[l] = ||(W_l - W^_l) X_l^T||_F^2 (by
+ *   the Hessian route); X_{l+1}[t][j] = act_l((X_l W^_l^T)[t][j]) +
+ *   X_r[t][j] if the layer names an earlier input r, rounded to bf16.
+ *
+ *   X0         [n_tok][layers[0].d_in] bf16 (device), the first input
+ *   layers     host array of n_layers descriptors; layers[l].d_in must equal
+ *              layers[l-1].d_out; a residual input X_r (0 <= r <= l) must
+ *              have d_out columns
+ *   bits, group_size, block_size, sym, damp_percent
+ *              as for gq_gptq_quantize_layer / gq_damp_cholesky_inverse
+ *   sse_dev    [n_layers] double (device, out)
+ *   X_out      [n_tok][layers[n-1].d_out] bf16 (device, out) or NULL: the
+ *              chain's output
+ *   ws         >= gq_gptq_sequential_workspace_size(...) bytes: every input
+ *              X_0 .. X_n (bf16), three d x d fp32 matrices for the widest
+ *              layer, and the largest scratch of the steps
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  const void *W;          /* [d_out][d_in] (device, 16-byte aligned)          */
+  gq_dtype w_dtype;
+  int64_t d_out, d_in;
+  int act;                /* GQ_ACT_* applied to the layer's output           */
+  int residual_from;      /* -1, or r <= l: X_r is added to the output        */
+  uint32_t *qpacked;      /* GPTQ outputs (device), as gq_gptq_quantize_layer */
+  uint16_t *scales;
+  uint16_t *zeros;        /* NULL when sym                                    */
+} gq_seq_layer;
+
+size_t gq_gptq_sequential_workspace_size(const gq_seq_layer *layers, int n_layers,
+                                         int64_t n_tok, int block_size);
+gq_status gq_gptq_sequential(const void *X0_bf16, int64_t n_tok, const gq_seq_layer *layers,
+                             int n_layers, int bits, int group_size, int block_size, int sym,
+                             float damp_percent, double *sse_dev, void *X_out_bf16, void *ws,
+                             size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
  * Activation-aware per-channel scaling before RTN.
  * "Model Quantization Mechanics", section 2.2: a per-channel factor s
  * multiplies the weights of input channels whose activations are large and

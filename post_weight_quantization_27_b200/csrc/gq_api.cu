@@ -431,6 +431,59 @@ gq_status gq_qlinear_bf16(const uint32_t *qpacked, const uint16_t *scales,
                         static_cast<int *>(ws), static_cast<cudaStream_t>(stream));
 }
 
+size_t gq_gptq_sequential_workspace_size(const gq_seq_layer *layers, int n_layers,
+                                         int64_t n_tok, int block_size) {
+  if (!layers || n_layers < 1 || n_tok < 0) return 0;
+  if (block_size != 32 && block_size != 64 && block_size != 128) return 0;
+  for (int l = 0; l < n_layers; ++l)
+    if (layers[l].d_in < 8 || layers[l].d_in % 8 != 0 || layers[l].d_out < 1) return 0;
+  return seq_ws_bytes(layers, n_layers, n_tok, block_size);
+}
+
+gq_status gq_gptq_sequential(const void *X0_bf16, int64_t n_tok, const gq_seq_layer *layers,
+                             int n_layers, int bits, int group_size, int block_size, int sym,
+                             float damp_percent, double *sse_dev, void *X_out_bf16, void *ws,
+                             size_t ws_bytes, void *stream) {
+  t_last_error.clear();
+  if (!layers || n_layers < 1 || !sse_dev || (n_tok > 0 && !X0_bf16))
+    return fail(GQ_ERR_ARG, "null pointer or no layers");
+  if (n_tok < 1 || n_tok > (int64_t(1) << 31) - 256) return fail(GQ_ERR_SHAPE, "bad n_tok");
+  if (sym != 0 && sym != 1) return fail(GQ_ERR_ARG, "sym must be 0 or 1");
+  if (block_size != 32 && block_size != 64 && block_size != 128)
+    return fail(GQ_ERR_ARG, "block_size must be 32, 64 or 128");
+  if (!(damp_percent >= 0.0f) || !(damp_percent < 1e30f))
+    return fail(GQ_ERR_ARG, "damp_percent must be finite and >= 0");
+  if (!aligned(X0_bf16, 16)) return fail(GQ_ERR_ARG, "X0 must be 16-byte aligned");
+  for (int l = 0; l < n_layers; ++l) {
+    const gq_seq_layer &y = layers[l];
+    GQ_TRY(check_dtype(y.w_dtype));
+    if (!y.W || !y.qpacked || !y.scales || (sym == 0 && !y.zeros))
+      return fail(GQ_ERR_ARG, "layer " + std::to_string(l) + ": null pointer");
+    GQ_TRY(check_layer(y.d_out, y.d_in));
+    GQ_TRY(check_group(group_size, y.d_in));
+    GQ_TRY(check_bits(bits, y.d_in, group_size));
+    if (y.d_in > 65536) return fail(GQ_ERR_SHAPE, "d_in too large");
+    if (group_size > 0 && (group_size < 32 || block_size % group_size != 0))
+      return fail(GQ_ERR_ARG, "group_size must be -1, 0, 32, 64 or 128 and divide block_size");
+    if (bits != 4 && block_size != 128)
+      return fail(GQ_ERR_ARG, "codes of other widths than 4 bits need block_size 128");
+    if (l > 0 && y.d_in != layers[l - 1].d_out)
+      return fail(GQ_ERR_SHAPE, "layer " + std::to_string(l) + ": d_in != previous d_out");
+    if (y.act != GQ_ACT_NONE && y.act != GQ_ACT_RELU && y.act != GQ_ACT_GELU)
+      return fail(GQ_ERR_ARG, "bad act");
+    if (!aligned(y.W, 16)) return fail(GQ_ERR_ARG, "W must be 16-byte aligned");
+    if (y.residual_from >= 0) {
+      if (y.residual_from > l) return fail(GQ_ERR_ARG, "residual must be an earlier input");
+      const int64_t dr = layers[y.residual_from].d_in;
+      if (dr != y.d_out) return fail(GQ_ERR_SHAPE, "residual width != d_out");
+    }
+  }
+  GQ_TRY(check_ws(ws, ws_bytes, seq_ws_bytes(layers, n_layers, n_tok, block_size)));
+  return launch_sequential(X0_bf16, n_tok, layers, n_layers, bits, group_size, block_size, sym,
+                           damp_percent, sse_dev, X_out_bf16, ws,
+                           static_cast<cudaStream_t>(stream));
+}
+
 size_t gq_awq_workspace_size(int64_t d_out, int64_t d_in, int64_t n_tok, int bits,
                              int group_size, int sym) {
   if (d_out < 1 || d_in < 8 || d_in % 8 != 0 || n_tok < 1) return 0;

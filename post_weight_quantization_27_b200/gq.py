@@ -27,6 +27,14 @@ class GQError(RuntimeError):
         self.name = name
 
 
+class SeqLayer(ctypes.Structure):
+    """gq_seq_layer of include/gq.h."""
+    _fields_ = [("W", ctypes.c_void_p), ("w_dtype", ctypes.c_int32), ("d_out", ctypes.c_int64),
+                ("d_in", ctypes.c_int64), ("act", ctypes.c_int), ("residual_from", ctypes.c_int),
+                ("qpacked", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p)]
+
+
 _lib = None
 
 
@@ -89,6 +97,11 @@ def lib() -> ctypes.CDLL:
     L.gq_qlinear_bf16.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_i64, _c_i64,
                                   _c_int, _c_int, _c_int, _c_vp, _c_i64, _c_int, _c_vp, _c_vp,
                                   _c_vp, _c_sz, _c_vp]
+    L.gq_gptq_sequential_workspace_size.restype = _c_sz
+    L.gq_gptq_sequential_workspace_size.argtypes = [_c_vp, _c_int, _c_i64, _c_int]
+    L.gq_gptq_sequential.restype = _c_int
+    L.gq_gptq_sequential.argtypes = [_c_vp, _c_i64, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_f32, _c_vp, _c_vp, _c_vp, _c_sz, _c_vp]
     L.gq_awq_workspace_size.restype = _c_sz
     L.gq_awq_workspace_size.argtypes = [_c_i64, _c_i64, _c_i64, _c_int, _c_int, _c_int]
     L.gq_awq_rtn_search.restype = _c_int
@@ -117,7 +130,8 @@ EXPORTS = ("gq_status_string", "gq_last_error", "gq_launch_count", "gq_hessian_w
            "gq_gptq_workspace_size", "gq_gptq_quantize_layer", "gq_rtn_quantize_pack",
            "gq_recon_workspace_size", "gq_recon_error", "gq_recon_error_hessian_workspace_size",
            "gq_recon_error_hessian", "gq_w4a16_workspace_size",
-           "gq_w4a16_matmul", "gq_qlinear_bf16", "gq_awq_workspace_size",
+           "gq_w4a16_matmul", "gq_qlinear_bf16", "gq_gptq_sequential_workspace_size",
+           "gq_gptq_sequential", "gq_awq_workspace_size",
            "gq_awq_rtn_search", "gq_workspace_status", "gq_selftest_bounded_wait",
            "gq_kernel_timer_start",
            "gq_kernel_timer_stop", "gq_kernel_timer_read", "gq_kernel_timer_release")
@@ -434,6 +448,45 @@ def qlinear_bf16(X: torch.Tensor, d_out: int, q: dict | None = None, W: torch.Te
                                _stream(stream))
     _check(st, "gq_qlinear_bf16")
     return Z
+
+
+# ------------------------------------------------------------------ sequential quantisation
+
+def gptq_sequential(X0: torch.Tensor, layers: list, bits: int = 4, group_size: int = -1,
+                    block_size: int = 128, sym: bool = True, damp_percent: float = 0.01,
+                    stream=None):
+    """A chain of layers quantised one after another, each on the input it
+    receives from the quantised layers before it.  ``layers``: list of dicts
+    with W (device [d_out, d_in]), act ("none", "relu", "gelu") and
+    residual_from (None or the index of an earlier input added to the
+    output).  Returns (list of quantised-layer dicts, sse numpy [n_layers],
+    the chain's output [n_tok, d_out] bf16)."""
+    import numpy as np
+    _dev(X0, "X0", torch.bfloat16)
+    n_tok = X0.shape[0]
+    dev = X0.device
+    arr = (SeqLayer * len(layers))()
+    outs = []
+    for i, L in enumerate(layers):
+        W = _dev(L["W"], "W")
+        d_out, d_in = W.shape
+        o = _outputs(d_out, d_in, group_size, sym, dev, False, bits)
+        outs.append(o)
+        r = L.get("residual_from")
+        arr[i] = SeqLayer(W.data_ptr(), _DTYPES[W.dtype], d_out, d_in, ACT[L.get("act", "none")],
+                          -1 if r is None else int(r), o["qpacked"].data_ptr(),
+                          o["scales"].data_ptr(), _p(o["zeros"]))
+    lib_ = lib()
+    need = int(lib_.gq_gptq_sequential_workspace_size(ctypes.addressof(arr), len(layers), n_tok,
+                                                      block_size))
+    ws = workspace(need, dev)
+    sse = torch.empty(len(layers), dtype=torch.float64, device=dev)
+    X_out = torch.empty((n_tok, layers[-1]["W"].shape[0]), dtype=torch.bfloat16, device=dev)
+    st = lib_.gq_gptq_sequential(_p(X0), n_tok, ctypes.addressof(arr), len(layers), bits,
+                                 group_size, block_size, int(bool(sym)), float(damp_percent),
+                                 _p(sse), _p(X_out), _p(ws), ws.numel(), _stream(stream))
+    _check(st, "gq_gptq_sequential")
+    return outs, sse.cpu().numpy().astype(np.float64), X_out
 
 
 # ------------------------------------------------------------------ activation-aware scaling
