@@ -3,14 +3,17 @@ C-ABI library -- a fixed, small case for profilers (ncu) and for timing one
 stage by hand.
 
     python -m post_weight_quantization_27_b200.cases --workload 2 --layer 3
-           [--tokens N] [--repeat R] [--stages hessian,solve,gptq,rtn,recon,awq,w4a16]
+           [--tokens N] [--repeat R]
+           [--stages hessian,solve,gptq,rtn,recon,trace,awq,w4a16,qlinear]
 
 The stages always run in path order (H -> damp/U -> GPTQ -> RTN -> recon),
 each as many times as --repeat says; a stage that is not listed still runs
 once if a later listed stage needs its output.  Prints one line per stage
-with its CUDA-event time.  "awq" is the activation-aware scaling search
+with its CUDA-event time.  "trace" is the GPTQ layer's error from the
+Hessian (tr(dW H dW^T) / 2); "awq" is the activation-aware scaling search
 before RTN (20 values of alpha), which needs only H; "w4a16" multiplies the
-RTN layer with the first (at most 8192) tokens.
+RTN layer with the first (at most 8192) tokens; "qlinear" applies it to them
+(token-major bf16 output, GELU).
 """
 from __future__ import annotations
 
@@ -21,7 +24,7 @@ import torch
 from . import gq
 from . import inputs as I
 
-ORDER = ("hessian", "solve", "gptq", "rtn", "recon", "awq", "w4a16")
+ORDER = ("hessian", "solve", "gptq", "rtn", "recon", "trace", "awq", "w4a16", "qlinear")
 
 
 def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) -> dict:
@@ -32,12 +35,12 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
     X = I.make_x_device(spec, "cuda")
     last = max(ORDER.index(s) for s in stages)
     need = set(stages) | set(ORDER[:last])
-    if "recon" in stages:
+    if "recon" in stages or "trace" in stages:
         need |= {"gptq"}
     if stages == ["awq"]:  # needs only H
         need = {"hessian", "awq"}
-    if stages == ["w4a16"]:  # needs only the RTN output
-        need = {"rtn", "w4a16"}
+    if set(stages) <= {"w4a16", "qlinear"}:  # need only the RTN output
+        need = {"rtn"} | set(stages)
     times = {}
 
     def timed(name, fn):
@@ -67,11 +70,18 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
         r = timed("rtn", lambda: gq.rtn_quantize_pack(W, 4, spec.group_size, spec.sym))
     if "recon" in need:
         timed("recon", lambda: gq.recon_error(W, q, X, spec.group_size, spec.sym))
+    if "trace" in need:
+        timed("trace", lambda: gq.recon_error_hessian(W, q, H, X.shape[0], spec.group_size,
+                                                      spec.sym))
     if "awq" in need:
         timed("awq", lambda: gq.awq_rtn_search(W, H, X, 4, spec.group_size, spec.sym, 20))
     if "w4a16" in need:  # the RTN layer times the first (at most 8192) tokens
         Xs = X[:min(X.shape[0], 8192) // 4 * 4]
         timed("w4a16", lambda: gq.w4a16_matmul(r, spec.d_in, Xs, spec.group_size, spec.sym))
+    if "qlinear" in need:
+        Xs = X[:min(X.shape[0], 8192)]
+        timed("qlinear", lambda: gq.qlinear_bf16(Xs, spec.d_out, q=r, group_size=spec.group_size,
+                                                 sym=spec.sym, act="gelu"))
     return {"spec": spec, "ms": times}
 
 
