@@ -9,8 +9,9 @@ stage by hand.
 The stages always run in path order (H -> damp/U -> GPTQ -> RTN -> recon),
 each as many times as --repeat says; a stage that is not listed still runs
 once if a later listed stage needs its output.  Prints one line per stage
-with its CUDA-event time.  "trace" is the GPTQ layer's error from the
-Hessian (tr(dW H dW^T) / 2); "awq" is the activation-aware scaling search
+with its CUDA-event time.  "trace" is the error from the Hessian (tr(dW H
+dW^T) / 2) of the GPTQ layer (of the RTN layer when it is the only stage
+listed); "awq" is the activation-aware scaling search
 before RTN (20 values of alpha), which needs only H; "w4a16" multiplies the
 RTN layer with the first (at most 8192) tokens; "qlinear" applies it to them
 (token-major bf16 output, GELU).
@@ -35,10 +36,12 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
     X = I.make_x_device(spec, "cuda")
     last = max(ORDER.index(s) for s in stages)
     need = set(stages) | set(ORDER[:last])
-    if "recon" in stages or "trace" in stages:
+    if "recon" in stages:
         need |= {"gptq"}
     if stages == ["awq"]:  # needs only H
         need = {"hessian", "awq"}
+    if stages == ["trace"]:  # needs H and a quantised layer (the RTN one)
+        need = {"hessian", "rtn", "trace"}
     if set(stages) <= {"w4a16", "qlinear"}:  # need only the RTN output
         need = {"rtn"} | set(stages)
     times = {}
@@ -71,8 +74,8 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
     if "recon" in need:
         timed("recon", lambda: gq.recon_error(W, q, X, spec.group_size, spec.sym))
     if "trace" in need:
-        timed("trace", lambda: gq.recon_error_hessian(W, q, H, X.shape[0], spec.group_size,
-                                                      spec.sym))
+        timed("trace", lambda: gq.recon_error_hessian(W, q if q is not None else r, H,
+                                                      X.shape[0], spec.group_size, spec.sym))
     if "awq" in need:
         timed("awq", lambda: gq.awq_rtn_search(W, H, X, 4, spec.group_size, spec.sym, 20))
     if "w4a16" in need:  # the RTN layer times the first (at most 8192) tokens

@@ -22,6 +22,7 @@
 // trailing updates and the inverse's block steps are fp32 GEMMs on the
 // tensor cores (3 x TF32 split, gemm_tc.cu).
 #include <cfloat>
+#include <cmath>
 #include <climits>
 #include <map>
 #include <mutex>
@@ -540,6 +541,15 @@ __global__ void finish_info_kernel(int *status, int64_t d, int32_t *info_dev) {
 
 }  // namespace
 
+// Super-panel width: NB times the power of two nearest (on a log scale)
+// sqrt(d / NB).
+int64_t chol_super_cols(int64_t d) {
+  const double target = std::sqrt(static_cast<double>(NB) * static_cast<double>(d));
+  int64_t S = NB;
+  while (static_cast<double>(2 * S) <= target * 1.4142135623730951) S *= 2;
+  return S;
+}
+
 size_t chol_ws_bytes(int64_t d) {
   const int64_t n_panels = (d + NB - 1) / NB;
   return kWsHeader + round_up(static_cast<size_t>(d) * sizeof(float), 256) +
@@ -621,45 +631,77 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
     aux = aux_stream(st);
     if (aux) inv_st = aux->s;
   }
-  for (int64_t p = 0; p < n_panels; ++p) {
-    const int64_t k0 = p * NB;
-    const int nb = static_cast<int>(d - k0 < NB ? d - k0 : NB);
-    const int64_t k1 = k0 + nb;
-    const int rest = static_cast<int>(d - k1);
-    const unsigned tiles = static_cast<unsigned>(1 + (rest + NB - 1) / NB);
-    float *lp = w.linv + p * NB * NB;
-    int slot = timer_begin(GQ_KERNEL_POTRF_TRSM, st);
-    potrf_trsm_kernel<<<tiles, 256, PANEL_SMEM, st>>>(A, d, k0, nb, lp, w.status);
-    count_launch();
-    // Cholesky of the block nb^3 / 3, the panel solve rest nb^2
-    timer_end(slot, st, static_cast<double>(nb) * nb * (nb / 3.0 + rest));
-    if (aux) {
-      if (cudaEventRecord(aux->ev, st) != cudaSuccess ||
-          cudaStreamWaitEvent(aux->s, aux->ev, 0) != cudaSuccess)
-        return check_launch("stream fork");
-    }
-    if (rest > 0) {
-      // trailing: A[k1:, k1:] -= P P^T (lower part)
-      const gq_status s = launch_gemm_tf32x3(rest, rest, NB, -1.0f, A + k1 * d + k0, d,
-                                             A + k1 * d + k0, d, true, 1.0f, A + k1 * d + k1, d,
-                                             true, w.status, st);
+  // Two levels: panels of NB columns are grouped in super-panels of S
+  // columns.  After a panel, only the rest of its super-panel is updated
+  // (K = NB: a lower-triangular block and the rectangle below it), and
+  // after a super-panel the whole trailing matrix gets the super-panel's
+  // update in one SYRK with K = S; the inverse chain does the same with its
+  // block rows.  The same terms as the one-level scheme, summed in another
+  // order; the trailing matrix is read and written about S / 2 NB + d / 2 S
+  // times instead of d / 2 NB times.
+  const int64_t S = chol_super_cols(d);
+  for (int64_t s0 = 0; s0 < d; s0 += S) {
+    const int64_t s1 = s0 + S < d ? s0 + S : d;
+    for (int64_t k0 = s0; k0 < s1; k0 += NB) {
+      const int64_t p = k0 / NB;
+      const int nb = static_cast<int>(d - k0 < NB ? d - k0 : NB);
+      const int64_t k1 = k0 + nb;
+      const int rest = static_cast<int>(d - k1);
+      const unsigned tiles = static_cast<unsigned>(1 + (rest + NB - 1) / NB);
+      float *lp = w.linv + p * NB * NB;
+      int slot = timer_begin(GQ_KERNEL_POTRF_TRSM, st);
+      potrf_trsm_kernel<<<tiles, 256, PANEL_SMEM, st>>>(A, d, k0, nb, lp, w.status);
+      count_launch();
+      // Cholesky of the block nb^3 / 3, the panel solve rest nb^2
+      timer_end(slot, st, static_cast<double>(nb) * nb * (nb / 3.0 + rest));
+      if (aux) {
+        if (cudaEventRecord(aux->ev, st) != cudaSuccess ||
+            cudaStreamWaitEvent(aux->s, aux->ev, 0) != cudaSuccess)
+          return check_launch("stream fork");
+      }
+      const int in_sp = static_cast<int>(s1 - k1);  // columns left in the super-panel
+      if (in_sp > 0) {
+        // A[k1:s1, k1:s1] -= P P^T (lower part), P = A[k1:s1, k0:k1]
+        gq_status s = launch_gemm_tf32x3(in_sp, in_sp, nb, -1.0f, A + k1 * d + k0, d,
+                                         A + k1 * d + k0, d, true, 1.0f, A + k1 * d + k1, d,
+                                         true, w.status, st);
+        if (s != GQ_OK) return s;
+        if (d > s1) {
+          // A[s1:, k1:s1] -= A[s1:, k0:k1] A[k1:s1, k0:k1]^T
+          s = launch_gemm_tf32x3(static_cast<int>(d - s1), in_sp, nb, -1.0f, A + s1 * d + k0, d,
+                                 A + k1 * d + k0, d, true, 1.0f, A + s1 * d + k1, d, false,
+                                 w.status, st);
+          if (s != GQ_OK) return s;
+        }
+      }
+      // ---- inverse step p (on inv_st): X[k0:k1, 0:k1] := L_pp^-1 X[k0:k1, 0:k1]
+      slot = timer_begin(GQ_KERNEL_BLOCK_INVERSE, inv_st);
+      block_inverse_kernel<<<1, 256, INV_SMEM, inv_st>>>(lp);
+      count_launch();
+      timer_end(slot, inv_st, static_cast<double>(nb) * nb * nb / 3.0);
+      const int cols = static_cast<int>(k1);
+      // (in place: each output tile owns its columns)
+      gq_status s = launch_gemm_tf32x3(nb, cols, nb, 1.0f, lp, NB, X + k0 * d, d, false, 0.0f,
+                                       X + k0 * d, d, false, w.status, inv_st);
       if (s != GQ_OK) return s;
+      if (in_sp > 0) {
+        // X[k1:s1, 0:k1] -= L[k1:s1, k0:k1] X[k0:k1, 0:k1]
+        s = launch_gemm_tf32x3(in_sp, cols, nb, -1.0f, A + k1 * d + k0, d, X + k0 * d, d, false,
+                               1.0f, X + k1 * d, d, false, w.status, inv_st);
+        if (s != GQ_OK) return s;
+      }
     }
-    // ---- inverse step p (on inv_st)
-    slot = timer_begin(GQ_KERNEL_BLOCK_INVERSE, inv_st);
-    block_inverse_kernel<<<1, 256, INV_SMEM, inv_st>>>(lp);
-    count_launch();
-    timer_end(slot, inv_st, static_cast<double>(nb) * nb * nb / 3.0);
-    const int cols = static_cast<int>(k1);
-    // X[k0:k1, 0:cols] := L_pp^-1 X[k0:k1, 0:cols] (in place: each output
-    // tile owns its columns)
-    gq_status s = launch_gemm_tf32x3(nb, cols, nb, 1.0f, lp, NB, X + k0 * d, d, false, 0.0f,
-                                     X + k0 * d, d, false, w.status, inv_st);
-    if (s != GQ_OK) return s;
-    if (rest > 0) {
-      // X[k1:, 0:cols] -= L[k1:, k0:k1] X[k0:k1, 0:cols]
-      s = launch_gemm_tf32x3(rest, cols, nb, -1.0f, A + k1 * d + k0, d, X + k0 * d, d, false,
-                             1.0f, X + k1 * d, d, false, w.status, inv_st);
+    if (d > s1) {
+      const int rest = static_cast<int>(d - s1), sw = static_cast<int>(s1 - s0);
+      // A[s1:, s1:] -= L[s1:, s0:s1] L[s1:, s0:s1]^T (lower part)
+      gq_status s = launch_gemm_tf32x3(rest, rest, sw, -1.0f, A + s1 * d + s0, d,
+                                       A + s1 * d + s0, d, true, 1.0f, A + s1 * d + s1, d, true,
+                                       w.status, st);
+      if (s != GQ_OK) return s;
+      // X[s1:, 0:s1] -= L[s1:, s0:s1] X[s0:s1, 0:s1] (on inv_st, after the
+      // super-panel's last inverse step)
+      s = launch_gemm_tf32x3(rest, static_cast<int>(s1), sw, -1.0f, A + s1 * d + s0, d,
+                             X + s0 * d, d, false, 1.0f, X + s1 * d, d, false, w.status, inv_st);
       if (s != GQ_OK) return s;
     }
   }
