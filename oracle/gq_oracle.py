@@ -80,7 +80,7 @@ __all__ = [
     "recon_sse_trace", "bits_per_weight", "obs_quantize", "bruteforce_row",
     "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
     "gptq_layer", "awq_channel_scales", "awq_apply", "awq_rtn_search", "w4a16_matmul",
-    "round_to_bf16", "gelu_tanh", "apply_layer", "gptq_sequential",
+    "round_to_bf16", "gelu_tanh", "apply_layer", "gptq_sequential", "TIE_TOL", "TIE_REL",
 ]
 
 
@@ -353,22 +353,28 @@ def _fp16_tie_rel(s32):
     return np.abs(s - mid) / np.where(s > 0, s, 1.0)
 
 
-# Width of the rounding-tie window of the replay mode, in quantisation steps.
-# The other implementation computes each weight at its decision point in
-# fp32 after up to d_in accumulated updates; with unit roundoff u = 2^-24 and
-# error growth ~ sqrt(d_in) over sums whose terms are a few steps in size, its
-# value differs from the fp64 one by ~ sqrt(28672) * 6e-8 * (a few) ~ 1e-5
-# steps at the widest layer (measured: <= 2e-6 steps at d_in = 3072).  A
-# decision closer than this to a boundary k + 1/2 may go either way.  A scale
-# is a tie when its fp32 value lies within this relative distance of an fp16
-# rounding boundary (an error of eps steps in the group's extreme weight,
-# which spans 7 or 15 steps, moves the scale by at most eps relative), the
-# affine zero-point when -min'/s lies within this many steps of k + 1/2.
-TIE_TOL = 1e-5
+# Width of the rounding-tie window of the replay mode.  The other
+# implementation computes each weight at its decision point in fp32: the
+# in-block updates are fp32 FMAs, the lazy updates fp32-accuracy products on
+# tensor cores (three TF32 products per term, relative error <= ~2^-20 per
+# term) accumulated in fp32 (~sqrt(K) 2^-24 of the terms' magnitude over K
+# terms).  So the weight it decides on differs from the fp64 one by about
+# TIE_REL * E, with E = sum over the updates applied to that weight of
+# |delta_i U_ij| (tracked alongside, in fp64) and TIE_REL = 2^-18 (the
+# product error 2^-20 plus the typical accumulation error 2^-18.5, rounded
+# up).  A decision is a tie when w/s lies within max(TIE_TOL, TIE_REL * E/s)
+# steps of k + 1/2; TIE_TOL = 1e-6 steps covers the fp32 representation of
+# the weight and the division.  A scale is a tie when its fp32 value lies
+# within the same relative distance (the window on the group's extreme,
+# divided by the extreme) of an fp16 rounding boundary; an affine zero-point
+# when -min'/s lies within the window of k + 1/2.
+TIE_TOL = 1e-6
+TIE_REL = 2.0 ** -18
 
 
 def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
-                  perm=None, dead=None, follow=None, tie_tol=TIE_TOL) -> GptqResult:
+                  perm=None, dead=None, follow=None, tie_tol=TIE_TOL,
+                  tie_rel=TIE_REL) -> GptqResult:
     """GPTQ on one layer given U (upper, H^-1 = U^T U, in the column order
     the layer is processed in).
 
@@ -382,14 +388,16 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
 
     ``follow`` (optional, dict with "codes" [d_out, d_in] in original column
     order and "scales"/"zeros" [d_out, n_groups]) is the output of another
-    implementation.  Where the oracle's own decision is a rounding tie --
-    the value w/s lies within ``tie_tol`` steps of k + 1/2, or the fp32
-    scale within a relative ``tie_tol`` of an fp16 rounding boundary (see
-    TIE_TOL) -- both roundings are correct, and the oracle takes the other
-    implementation's choice so that the rest of the row can be checked
-    along it.  Nowhere else does ``follow`` change anything; ``n_followed``
-    counts the adopted decisions and ``max_follow_dist`` is the largest
-    distance from a boundary among them (steps, or relative for a scale)."""
+    implementation.  Where the oracle's own decision is a rounding tie at
+    the precision of that implementation -- w/s within max(tie_tol, tie_rel
+    E/s) steps of k + 1/2, E the accumulated magnitude of the updates applied
+    to w, or the fp32 scale within the same relative distance of an fp16
+    rounding boundary (see TIE_REL) -- both roundings are correct, and the
+    oracle takes the other implementation's choice so that the rest of the
+    row can be checked along it.  Nowhere else does ``follow`` change
+    anything; ``n_followed`` counts the adopted decisions and
+    ``max_follow_dist`` is the largest distance from a boundary among them
+    (steps, or relative for a scale)."""
     W = np.array(W, dtype=np.float64, copy=True)
     d_out, d_in = W.shape
     if dead is not None:
@@ -421,21 +429,32 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
         f_zeros = (np.asarray(follow["zeros"], dtype=np.float16)
                    if not sym else np.zeros_like(f_scales))
 
-    def group(vals, gi):
+    def group(vals, gi, evals=None):
         nonlocal n_followed, max_dist
         s, z = params(vals, bits)
         if follow is not None:
             v = np.asarray(vals, dtype=F32)
+            ev = (np.zeros(len(s)) if evals is None
+                  else tie_rel * np.max(np.asarray(evals), axis=-1))   # error of the extremes
             if sym:
+                ext = np.max(np.abs(v), axis=-1).astype(np.float64)
                 s32 = np.max(np.abs(v), axis=-1) / F32(2 ** (bits - 1) - 1)
-                zdist = np.full(len(s), np.inf)
+                win = np.maximum(tie_tol, ev / np.where(ext > 0, ext, 1.0))
+                dist = _fp16_tie_rel(s32)
             else:
                 mn = np.minimum(np.min(v, axis=-1), F32(0))
                 mx = np.maximum(np.max(v, axis=-1), F32(0))
+                ext = (mx - mn).astype(np.float64)
                 s32 = (mx - mn) / F32(2 ** bits - 1)
-                zdist = _tie_dist(-mn.astype(np.float64) / s.astype(np.float64))
-            dist = np.minimum(_fp16_tie_rel(s32), zdist)
-            take = (dist < tie_tol) & ((f_scales[:, gi] != s) | (f_zeros[:, gi] != z))
+                zd = _tie_dist(-mn.astype(np.float64) / s.astype(np.float64))
+                win_s = np.maximum(tie_tol, ev / np.where(ext > 0, ext, 1.0))
+                win_z = np.maximum(tie_tol, ev / s.astype(np.float64))
+                sd = _fp16_tie_rel(s32)
+                # compare each distance with its own window: report the one
+                # that is a tie (the smaller ratio)
+                dist = np.where(sd / win_s <= zd / win_z, sd, zd)
+                win = np.where(sd / win_s <= zd / win_z, win_s, win_z)
+            take = (dist < win) & ((f_scales[:, gi] != s) | (f_zeros[:, gi] != z))
             s = np.where(take, f_scales[:, gi], s)
             z = np.where(take, f_zeros[:, gi], z)
             n_followed += int(take.sum())
@@ -443,6 +462,8 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                 max_dist = max(max_dist, float(dist[take].max()))
         return s, z
 
+    # E: accumulated |update| per weight (only to size the tie windows)
+    E = np.zeros_like(W) if follow is not None else None
     if per_tensor:
         s, z = params(W.astype(F32).reshape(1, -1), bits)
         scales[:, 0], zeros[:, 0] = s[0], z[0]
@@ -452,20 +473,24 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     for b0 in range(0, d_in, block_size):
         b1 = min(b0 + block_size, d_in)
         Wb = W[:, b0:b1].copy()
+        Eb = E[:, b0:b1].copy() if E is not None else None
         Err = np.zeros_like(Wb)
         for j in range(b1 - b0):
             col = b0 + j
             if group_size != -1 and col % g == 0:
-                s, z = group(Wb[:, j:j + g].astype(F32), col // g)
+                s, z = group(Wb[:, j:j + g].astype(F32), col // g,
+                             None if Eb is None else Eb[:, j:j + g])
                 scales[:, col // g], zeros[:, col // g] = s, z
             gi = 0 if group_size == -1 else col // g
             s, z = scales[:, gi], zeros[:, gi]
             w = Wb[:, j]
             c = quantize_codes(w, s, z, sym, bits)
             if follow is not None:
-                r = w.astype(F32).astype(np.float64) / s.astype(np.float64)
+                s64 = s.astype(np.float64)
+                r = w.astype(F32).astype(np.float64) / s64
                 dist = _tie_dist(r)
-                take = ((dist < tie_tol) & (f_codes[:, col] != c)
+                win = np.maximum(tie_tol, tie_rel * Eb[:, j] / s64)
+                take = ((dist < win) & (f_codes[:, col] != c)
                         & (np.abs(f_codes[:, col] - c) == 1))
                 c = np.where(take, f_codes[:, col], c)
                 n_followed += int(take.sum())
@@ -477,8 +502,12 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
             delta = (w - q) / U[col, col]
             Err[:, j] = delta
             Wb[:, j + 1:] -= np.outer(delta, U[col, col + 1:b1])
+            if Eb is not None:
+                Eb[:, j + 1:] += np.outer(np.abs(delta), np.abs(U[col, col + 1:b1]))
         W[:, b0:b1] = Wb
         W[:, b1:] -= Err @ U[b0:b1, b1:]
+        if E is not None:
+            E[:, b1:] += np.abs(Err) @ np.abs(U[b0:b1, b1:])
 
     g_perm = np.arange(d_in) // g
     if perm is not None:
@@ -498,7 +527,8 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
 
 
 def gptq_layer(W, X, bits=4, group_size=-1, block_size=128, sym=True,
-               damp_percent=0.01, act_order=False, follow=None, tie_tol=TIE_TOL):
+               damp_percent=0.01, act_order=False, follow=None, tie_tol=TIE_TOL,
+               tie_rel=TIE_REL):
     """The whole per-layer path: H = 2 X^T X, dead columns and damping,
     optional act-order, U, then GPTQ.  Returns (GptqResult, H_undamped,
     U, perm, dead)."""
@@ -509,7 +539,7 @@ def gptq_layer(W, X, bits=4, group_size=-1, block_size=128, sym=True,
     U = upper_factor_of_inverse(Hp)
     res = gptq_quantize(W, U, bits=bits, group_size=group_size,
                         block_size=block_size, sym=sym, perm=perm, dead=dead,
-                        follow=follow, tie_tol=tie_tol)
+                        follow=follow, tie_tol=tie_tol, tie_rel=tie_rel)
     return res, H0, U, perm, dead
 
 

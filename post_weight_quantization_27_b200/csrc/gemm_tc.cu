@@ -53,6 +53,8 @@ struct TcArgs {
   int b_kmajor, lower;
   int *status;
   double *dot;  // dot mode: [n_tiles] sum over the tile of (alpha A B) * C; C not written
+                // (with lower: the strictly lower elements counted twice, the diagonal
+                // once, the rest not at all -- the full sum for symmetric A B and C)
 };
 
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool b_mn) {
@@ -298,16 +300,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float v[32];
           tmem_ld32(taddr + q * 32, v);
           const uint8_t *row = cs + q * (C_BYTES / 4) + r * 128;
-          float part = 0.0f;
+          float part = 0.0f, pdiag = 0.0f;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
+            float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
+            if (diag) {  // lower: keep n < m (counted twice below), the diagonal once
+              const int n = nt * TN + 32 * q + 4 * c;
+              if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
+              if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
+              if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
+              if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
+              if (n >= m) cv.x = 0.0f;
+              if (n + 1 >= m) cv.y = 0.0f;
+              if (n + 2 >= m) cv.z = 0.0f;
+              if (n + 3 >= m) cv.w = 0.0f;
+            }
             part = fmaf(a.alpha * v[4 * c], cv.x, part);
             part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
             part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
             part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
           }
-          rs += static_cast<double>(part);
+          rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) + static_cast<double>(pdiag);
         }
         tc_fence_before();
         __syncwarp();
@@ -389,8 +402,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // a diagonal tile is written back unchanged.
 // Dot mode (dot_partials non-NULL): nothing is written to C; instead
 // dot_partials[t] = sum over output tile t of (alpha A B) .* C (fp32 within
-// a row of the tile, fp64 across rows), for t < gemm_tf32x3_tiles(M, N).
-int gemm_tf32x3_tiles(int M, int N) { return ((M + TM - 1) / TM) * ((N + TN - 1) / TN); }
+// a row of the tile, fp64 across rows), for t < gemm_tf32x3_tiles(M, N,
+// lower).  With lower (M == N, A B and C symmetric) the tiles of the lower
+// triangle give the sum over the whole matrix: strictly lower elements
+// count twice, diagonal ones once.
+int gemm_tf32x3_tiles(int M, int N, bool lower) {
+  const int mt = (M + TM - 1) / TM, nt = (N + TN - 1) / TN;
+  return lower ? mt * (mt + 1) / 2 : mt * nt;
+}
 
 gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
                              const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
@@ -424,7 +443,7 @@ gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, i
   a.lower = lower ? 1 : 0;
   a.n_tiles = lower ? a.n_mt * (a.n_mt + 1) / 2 : a.n_mt * a.n_nt;
   a.status = status;
-  a.dot = lower ? nullptr : dot_partials;
+  a.dot = dot_partials;
   cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(SMEM_BYTES));
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();

@@ -78,12 +78,13 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
 
 // C = beta C + alpha A B in fp32 on the tensor cores (3 x TF32 split); with
 // dot_partials, per output tile the sum of (alpha A B) .* C instead (C is
-// read, not written; gemm_tf32x3_tiles(M, N) partials).
+// read, not written; gemm_tf32x3_tiles(M, N, lower) partials; with lower
+// the lower-triangle tiles give the full sum of a symmetric product).
 gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, int64_t lda,
                              const float *B, int64_t ldb, bool b_kmajor, float beta, float *C,
                              int64_t ldc, bool lower, int *status, cudaStream_t st,
                              double *dot_partials = nullptr);
-int gemm_tf32x3_tiles(int M, int N);
+int gemm_tf32x3_tiles(int M, int N, bool lower = false);
 
 size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size);
 gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,

@@ -404,20 +404,75 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
 
 // ---------------------------------------------------------------------------
 // The same SSE by the trace route: ||dW X^T||_F^2 = tr(dW X^T X dW^T) =
-// tr(dW H0 dW^T) / 2 with the undamped H0 = 2 X^T X.  dW in fp32, then one
-// fp32 GEMM P = dW H0 on the tensor cores (3 x TF32) whose epilogue sums
-// P .* dW over each output tile instead of storing P; fp64 partials added
-// in a fixed order.  2 d_out d_in^2 flops instead of 2 n_tok d_out d_in.
+// tr(dW H0 dW^T) / 2 = <H0, G>_F / 2 with G = dW^T dW and the undamped
+// H0 = 2 X^T X.  dW^T is formed in fp32, then G's lower triangle on the
+// tensor cores (a SYRK in fp32 accuracy, 3 x TF32) whose epilogue sums G .*
+// H0 over each tile instead of storing G (off-diagonal elements twice);
+// fp64 tile partials added in a fixed order.  d_out d_in^2 flops instead
+// of 2 n_tok d_out d_in.
 namespace {
+
+// dW^T [d_in][ldt] (ldt = d_out rounded up to 4, zero-padded): a block
+// takes 32 rows x 64 columns of dW, forms them in shared memory and writes
+// them transposed, 32 consecutive floats per column.
+template <typename T>
+__global__ void __launch_bounds__(256) dequant_diff_t_kernel(
+    const T *__restrict__ W, const uint32_t *__restrict__ q, const uint16_t *__restrict__ scales,
+    const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx, int64_t d_out,
+    int64_t d_in, int group_size, int sym, int bits, float *__restrict__ dwt, int64_t ldt) {
+  __shared__ float tile[64][33];
+  const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
+  const int64_t row_words = d_in * bits / 32;
+  const int offset = sym ? (1 << (bits - 1)) : 0;
+  const int64_t tiles_r = (d_out + 31) / 32, tiles_c = (d_in + 63) / 64;
+  for (int64_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
+    const int64_t r0 = (t % tiles_r) * 32, c0 = (t / tiles_r) * 64;
+    // read: thread -> (row r0 + i, 8 columns)
+    {
+      const int i = threadIdx.x >> 3, j0 = (threadIdx.x & 7) * 8;
+      const int64_t r = r0 + i;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int64_t c = c0 + j0 + k;
+        float dw = 0.0f;
+        if (r < d_out && c < d_in) {
+          int64_t gi = g_idx ? g_idx[c] : (group_size <= 0 ? 0 : c / group_size);
+          gi = gi < 0 ? 0 : (gi >= n_groups ? n_groups - 1 : gi);
+          const float sc = __half2float(__ushort_as_half(scales[r * n_groups + gi]));
+          const float z = sym ? 0.0f : __half2float(__ushort_as_half(zeros[r * n_groups + gi]));
+          const uint32_t stored = get_code(q + r * row_words, bits, static_cast<int>(c));
+          const float what = sc * (static_cast<float>(static_cast<int>(stored) - offset) - z);
+          dw = ld_w(W + r * d_in + c) - what;
+        }
+        tile[j0 + k][i] = dw;
+      }
+    }
+    __syncthreads();
+    // write: warp -> 8 columns, lane -> row
+    {
+      const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int cc = wp * 8 + k;
+        const int64_t c = c0 + cc, r = r0 + lane;
+        if (c < d_in && r < ldt) dwt[c * ldt + r] = r < d_out ? tile[cc][lane] : 0.0f;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 struct TraceLayout {
-  size_t off_partials, off_dw, total;
+  int64_t ldt;
+  size_t off_partials, off_dwt, total;
 };
 TraceLayout trace_layout(int64_t d_out, int64_t d_in) {
   TraceLayout L{};
+  L.ldt = (d_out + 3) / 4 * 4;
   L.off_partials = kWsHeader;
-  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_out), static_cast<int>(d_in));
-  L.off_dw = L.off_partials + round_up(static_cast<size_t>(tiles) * sizeof(double), 256);
-  L.total = L.off_dw + round_up(static_cast<size_t>(d_out) * d_in * sizeof(float), 256);
+  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_in), static_cast<int>(d_in), true);
+  L.off_dwt = L.off_partials + round_up(static_cast<size_t>(tiles) * sizeof(double), 256);
+  L.total = L.off_dwt + round_up(static_cast<size_t>(d_in) * L.ldt * sizeof(float), 256);
   return L;
 }
 }  // namespace
@@ -436,38 +491,39 @@ gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpack
   uint8_t *base = static_cast<uint8_t *>(ws);
   int *status = reinterpret_cast<int *>(base);
   double *partials = reinterpret_cast<double *>(base + L.off_partials);
-  float *dw = reinterpret_cast<float *>(base + L.off_dw);
+  float *dwt = reinterpret_cast<float *>(base + L.off_dwt);
   if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
-  unsigned g = static_cast<unsigned>((d_out * (d_in / (bits == 4 ? 8 : 32)) + 255) / 256);
-  const unsigned cap = static_cast<unsigned>(num_sms()) * 16;
+  int64_t g = ((L.ldt + 31) / 32) * ((d_in + 63) / 64);
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
   if (g > cap) g = cap;
+  const unsigned grid = static_cast<unsigned>(g);
   switch (dt) {
     case GQ_F32:
-      dequant_diff_kernel<float><<<g, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
-                                                    scales, zeros, g_idx, nullptr, d_out, d_in,
-                                                    group_size, sym, nullptr, nullptr, dw, bits);
+      dequant_diff_t_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
+                                                         scales, zeros, g_idx, d_out, d_in,
+                                                         group_size, sym, bits, dwt, L.ldt);
       break;
     case GQ_F16:
-      dequant_diff_kernel<__half><<<g, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
-                                                     scales, zeros, g_idx, nullptr, d_out, d_in,
-                                                     group_size, sym, nullptr, nullptr, dw, bits);
+      dequant_diff_t_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
+                                                          scales, zeros, g_idx, d_out, d_in,
+                                                          group_size, sym, bits, dwt, L.ldt);
       break;
     case GQ_BF16:
-      dequant_diff_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, nullptr, d_out,
-          d_in, group_size, sym, nullptr, nullptr, dw, bits);
+      dequant_diff_t_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, d_out, d_in,
+          group_size, sym, bits, dwt, L.ldt);
       break;
   }
   count_launch();
-  gq_status s = check_launch("dequant_diff_kernel");
+  gq_status s = check_launch("dequant_diff_t_kernel");
   if (s != GQ_OK) return s;
-  // P = dW H0 (H0 symmetric, so its rows serve as the K-major B operand);
-  // per tile sum of P .* dW
-  s = launch_gemm_tf32x3(static_cast<int>(d_out), static_cast<int>(d_in), static_cast<int>(d_in),
-                         1.0f, dw, d_in, H0, d_in, true, 0.0f, dw, d_in, false, status, st,
-                         partials);
+  // G = dW^T dW (lower triangle, K = d_out; rows of dW^T are K-major for
+  // both operands), each tile summed against H0's
+  s = launch_gemm_tf32x3(static_cast<int>(d_in), static_cast<int>(d_in), static_cast<int>(L.ldt),
+                         1.0f, dwt, L.ldt, dwt, L.ldt, true, 0.0f, const_cast<float *>(H0), d_in,
+                         true, status, st, partials);
   if (s != GQ_OK) return s;
-  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_out), static_cast<int>(d_in));
+  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_in), static_cast<int>(d_in), true);
   recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, tiles, status, sse_dev, 0.5);
   count_launch();
   return check_launch("recon_reduce_kernel");

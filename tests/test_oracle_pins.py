@@ -824,3 +824,23 @@ def test_sequential_pipeline_structure():
     _, _, xs_fp = O.gptq_sequential(X0, layers, group_size=32, quantized_inputs=False)
     assert np.array_equal(xs_fp[1], O.apply_layer(X0, W1, "gelu"))
     assert not np.array_equal(xs_fp[1], xs[1])
+
+
+def test_tie_window_grows_with_the_updates_a_weight_received():
+    """The replay window of a decision is max(TIE_TOL, TIE_REL * E / s) with
+    E the accumulated |delta U| applied to the weight: a near-tie inside
+    that window is adopted, one just outside it is not."""
+    s = 2.0 ** -7                              # fp16-exact scale: absmax 7 s
+    U = np.array([[1.0, 50.0, 0.0], [0.0, 1.0, 0.0], [0.0, 0.0, 1.0]])
+    w0 = 3.02 * s                              # code 3, delta 0.02 s: column 1 gets 1 step of update
+    win = max(O.TIE_TOL, O.TIE_REL * 1.0)
+    assert win > O.TIE_TOL
+    for off, adopted in ((0.5 * win, True), (2.0 * win, False)):
+        W = np.array([[w0, (3.5 + off) * s, 7 * s]])   # column 1 decides at (2.5 + off) steps
+        r = O.gptq_quantize(W, U, group_size=-1)
+        assert float(r.scales[0, 0]) == s and r.codes[0, 1] == 3
+        other = r.codes.copy()
+        other[0, 1] = 2
+        rf = O.gptq_quantize(W, U, group_size=-1, follow=dict(codes=other, scales=r.scales))
+        assert (rf.codes[0, 1] == 2) == adopted, (off, win)
+        assert rf.n_followed == int(adopted)
