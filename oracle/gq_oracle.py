@@ -334,6 +334,7 @@ class GptqResult:
     W_hat: np.ndarray      # [d_out, d_in] fp64 dequantised, original column order
     n_followed: int = 0    # tie decisions adopted from ``follow``
     max_follow_dist: float = 0.0   # largest boundary distance among them
+    expected_ties: float = 0.0     # expected number of decisions inside their tie windows
 
 
 def _tie_dist(x):
@@ -421,6 +422,7 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     zeros = np.zeros((d_out, n_groups), dtype=np.float16)
     n_followed = 0
     max_dist = 0.0
+    expected = 0.0   # sum over decisions of the chance that a decision lands in its window
     if follow is not None:
         f_codes = np.asarray(follow["codes"], dtype=np.int64)
         if perm is not None:
@@ -430,7 +432,7 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                    if not sym else np.zeros_like(f_scales))
 
     def group(vals, gi, evals=None):
-        nonlocal n_followed, max_dist
+        nonlocal n_followed, max_dist, expected
         s, z = params(vals, bits)
         if follow is not None:
             v = np.asarray(vals, dtype=F32)
@@ -454,6 +456,8 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                 # that is a tie (the smaller ratio)
                 dist = np.where(sd / win_s <= zd / win_z, sd, zd)
                 win = np.where(sd / win_s <= zd / win_z, win_s, win_z)
+            # fp16 rounding boundaries are an ulp (2^-11 .. 2^-10 relative) apart
+            expected += float(np.sum(np.minimum(1.0, 2.0 * win / 2.0 ** -11)))
             take = (dist < win) & ((f_scales[:, gi] != s) | (f_zeros[:, gi] != z))
             s = np.where(take, f_scales[:, gi], s)
             z = np.where(take, f_zeros[:, gi], z)
@@ -490,6 +494,7 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                 r = w.astype(F32).astype(np.float64) / s64
                 dist = _tie_dist(r)
                 win = np.maximum(tie_tol, tie_rel * Eb[:, j] / s64)
+                expected += float(np.sum(np.minimum(1.0, 2.0 * win)))
                 take = ((dist < win) & (f_codes[:, col] != c)
                         & (np.abs(f_codes[:, col] - c) == 1))
                 c = np.where(take, f_codes[:, col], c)
@@ -521,7 +526,7 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
     assert codes.min() >= lo
     return GptqResult(codes=codes, scales=scales, zeros=zeros,
                       g_idx=g_idx.astype(np.int32), n_followed=n_followed,
-                      max_follow_dist=max_dist,
+                      max_follow_dist=max_dist, expected_ties=expected,
                       qpacked=pack_nibbles(codes, sym, bits) if (bits * d_in) % 32 == 0 else None,
                       W_hat=Q)
 

@@ -511,9 +511,13 @@ __global__ void __launch_bounds__(256) block_inverse_kernel(float *__restrict__ 
 
 // X := I on the lower triangle and on the whole NB x NB diagonal blocks
 // (the right-hand side of L X = I); the rest of the upper part is never read.
-__global__ void __launch_bounds__(256) eye_lower_kernel(float *__restrict__ X, int64_t d) {
+// X := I on the lower triangle and on every super-panel's diagonal block
+// (the upper part of those blocks is read by the inverse's K = S updates;
+// the rest of the upper triangle is never read).
+__global__ void __launch_bounds__(256) eye_lower_kernel(float *__restrict__ X, int64_t d,
+                                                        int64_t S) {
   for (int64_t r = blockIdx.y; r < d; r += gridDim.y) {
-    int64_t end = (r / NB + 1) * NB;
+    int64_t end = (r / S + 1) * S;
     if (end > d) end = d;
     for (int64_t c = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; c < end;
          c += static_cast<int64_t>(gridDim.x) * 256)
@@ -620,7 +624,7 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
   cudaFuncSetAttribute(block_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(INV_SMEM));
   const int64_t n_panels = (d + NB - 1) / NB;
-  eye_lower_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d);
+  eye_lower_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d, chol_super_cols(d));
   count_launch();
   // The inverse X = L^-1 (blocked forward substitution on the identity) runs
   // as a second chain: its step p needs the panel p of L and step p-1 only,

@@ -70,9 +70,10 @@ __device__ __forceinline__ void ql_tile(int t, int n_mt, int n_nt, int &mt, int 
 
 __device__ __forceinline__ float activate(float v, int act) {
   if (act == 1) return fmaxf(v, 0.0f);
-  if (act == 2) {  // GELU, tanh form
+  if (act == 2) {  // GELU, tanh form: 0.5 v (1 + tanh u) = v / (1 + e^(-2u)), which keeps
+                   // its relative accuracy for large negative v (no 1 + tanh cancellation)
     const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
-    return 0.5f * v * (1.0f + tanhf(u));
+    return v / (1.0f + expf(-2.0f * u));
   }
   return v;
 }
