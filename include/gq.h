@@ -383,8 +383,10 @@ gq_status gq_qlinear_bf16(const uint32_t *qpacked, const uint16_t *scales,
  *   bits, group_size, block_size, sym, damp_percent
  *              as for gq_gptq_quantize_layer / gq_damp_cholesky_inverse
  *   sse_dev    [n_layers] double (device, out)
- *   X_out      [n_tok][layers[n-1].d_out] bf16 (device, out) or NULL: the
- *              chain's output
+ *   X_all_out  bf16 (device, out) or NULL: receives every input X_0 .. X_n
+ *              (X_n is the chain's output), one after another, X_l taking
+ *              n_tok * d_l elements with d_l = layers[l].d_in (d_n =
+ *              layers[n-1].d_out)
  *   ws         >= gq_gptq_sequential_workspace_size(...) bytes: every input
  *              X_0 .. X_n (bf16), three d x d fp32 matrices for the widest
  *              layer, and the largest scratch of the steps
@@ -404,8 +406,8 @@ size_t gq_gptq_sequential_workspace_size(const gq_seq_layer *layers, int n_layer
                                          int64_t n_tok, int block_size);
 gq_status gq_gptq_sequential(const void *X0_bf16, int64_t n_tok, const gq_seq_layer *layers,
                              int n_layers, int bits, int group_size, int block_size, int sym,
-                             float damp_percent, double *sse_dev, void *X_out_bf16, void *ws,
-                             size_t ws_bytes, void *stream);
+                             float damp_percent, double *sse_dev, void *X_all_out_bf16,
+                             void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Activation-aware per-channel scaling before RTN.

@@ -358,19 +358,20 @@ def _fp16_tie_rel(s32):
 # implementation computes each weight at its decision point in fp32: the
 # in-block updates are fp32 FMAs, the lazy updates fp32-accuracy products on
 # tensor cores (three TF32 products per term, relative error <= ~2^-20 per
-# term) accumulated in fp32 (~sqrt(K) 2^-24 of the terms' magnitude over K
-# terms).  So the weight it decides on differs from the fp64 one by about
-# TIE_REL * E, with E = sum over the updates applied to that weight of
-# |delta_i U_ij| (tracked alongside, in fp64) and TIE_REL = 2^-18 (the
-# product error 2^-20 plus the typical accumulation error 2^-18.5, rounded
-# up).  A decision is a tie when w/s lies within max(TIE_TOL, TIE_REL * E/s)
-# steps of k + 1/2; TIE_TOL = 1e-6 steps covers the fp32 representation of
-# the weight and the division.  A scale is a tie when its fp32 value lies
+# term) accumulated in fp32.  So the weight it decides on differs from the
+# fp64 one by about TIE_REL * E, with E = sum over the updates applied to
+# that weight of |delta_i U_ij| (tracked alongside, in fp64) and TIE_REL =
+# 2^-20, the bound of the split's product error; the measured divergences of
+# the column loop at d_in up to 28672 all lie inside this window, at about a
+# tenth of the count it predicts (the fp32 accumulation errors mostly
+# cancel).  A decision is a tie when w/s lies within max(TIE_TOL, TIE_REL *
+# E/s) steps of k + 1/2; TIE_TOL = 1e-6 steps covers the fp32 representation
+# of the weight and the division.  A scale is a tie when its fp32 value lies
 # within the same relative distance (the window on the group's extreme,
 # divided by the extreme) of an fp16 rounding boundary; an affine zero-point
 # when -min'/s lies within the window of k + 1/2.
 TIE_TOL = 1e-6
-TIE_REL = 2.0 ** -18
+TIE_REL = 2.0 ** -20
 
 
 def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
@@ -608,22 +609,45 @@ def gelu_tanh(x):
     return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
 
 
-def apply_layer(X, W_hat, act="none", residual=None):
+def apply_layer(X, W_hat, act="none", residual=None, follow=None, tie_rel=TIE_REL):
     """The layer applied to its input, as the next layer sees it: Z = act(X
     W^T) (+ residual), fp64, rounded once to bf16.  X [n_tok, d_in], W_hat
-    [d_out, d_in]."""
-    Y = np.asarray(X, dtype=np.float64) @ np.asarray(W_hat, dtype=np.float64).T
+    [d_out, d_in].
+
+    ``follow`` (optional, [n_tok, d_out], another implementation's bf16
+    values): where the fp64 value lies within that implementation's error
+    of a bf16 rounding boundary -- tie_rel * (|X| |W|^T + |residual| +
+    |Z|), the error bound of an fp32 sum of those terms -- both roundings
+    are correct and the other implementation's value is taken when it is
+    the other neighbour.  Returns Z, or (Z, adopted) with ``follow``."""
+    Xa = np.asarray(X, dtype=np.float64)
+    Wa = np.asarray(W_hat, dtype=np.float64)
+    Y = Xa @ Wa.T
     if act == "relu":
         Y = np.maximum(Y, 0.0)
     elif act == "gelu":
         Y = gelu_tanh(Y)
     if residual is not None:
         Y = Y + np.asarray(residual, dtype=np.float64)
-    return round_to_bf16(Y)
+    Z = round_to_bf16(Y)
+    if follow is None:
+        return Z
+    f = np.asarray(follow, dtype=np.float64)
+    mag = np.abs(Xa) @ np.abs(Wa).T + np.abs(Y)
+    if residual is not None:
+        mag = mag + np.abs(np.asarray(residual, dtype=np.float64))
+    m, e = np.frexp(Y)
+    k = np.floor(np.abs(m) * 256.0)                   # the bf16 neighbours of Y:
+    a = np.sign(Y) * np.ldexp(k, e - 8)               # k and k + 1 units of 2^(e-8)
+    b = np.sign(Y) * np.ldexp(k + 1.0, e - 8)
+    mid = np.sign(Y) * np.ldexp(k + 0.5, e - 8)
+    near = np.abs(Y - mid) < tie_rel * mag
+    take = near & (f != Z) & ((f == a) | (f == b))
+    return np.where(take, f, Z), int(take.sum())
 
 
 def gptq_sequential(X0, layers, bits=4, group_size=-1, block_size=128, sym=True,
-                    damp_percent=0.01, quantized_inputs=True, follow=None):
+                    damp_percent=0.01, quantized_inputs=True, follow=None, follow_x=None):
     """Layers quantised one after another, each calibrated on the input it
     actually receives ("GPT-2 Quantization Reconstruction Error", "Key
     findings": the per-layer errors were measured with the whole model
@@ -634,8 +658,10 @@ def gptq_sequential(X0, layers, bits=4, group_size=-1, block_size=128, sym=True,
     end of an MLP block).  For each layer: H from its input X_l, GPTQ, the
     layer error ||(W - W^) X_l^T||^2, then X_{l+1} = apply_layer(X_l, W^ (or
     W when not ``quantized_inputs``), act, X_j).  ``follow``: per-layer
-    list of dicts (as for gptq_quantize) or None.  Returns (results, sse, xs)
-    with xs the inputs X_0 .. X_n."""
+    list of dicts (as for gptq_quantize) or None; ``follow_x``: another
+    implementation's X_1 .. X_n (its bf16 roundings are taken at ties, as in
+    apply_layer).  Returns (results, sse, xs) with xs the inputs X_0 ..
+    X_n."""
     X = np.asarray(X0, dtype=np.float64)
     results, sse, xs = [], [], [X]
     for li, L in enumerate(layers):
@@ -648,7 +674,10 @@ def gptq_sequential(X0, layers, bits=4, group_size=-1, block_size=128, sym=True,
         sse.append(recon_sse(W, res.W_hat, X))
         j = L.get("residual_from")
         X = apply_layer(X, res.W_hat if quantized_inputs else W, L.get("act", "none"),
-                        None if j is None else xs[j])
+                        None if j is None else xs[j],
+                        follow=None if follow_x is None else follow_x[li])
+        if follow_x is not None:
+            X = X[0]
         xs.append(X)
     return results, sse, xs
 

@@ -36,13 +36,14 @@
 namespace gq {
 namespace {
 
-constexpr int TM = 128, TN = 128, TK = 32, STAGES = 2;
+constexpr int TM = 128, TN = 128, TK = 32, STAGES = 3;
 constexpr int TILE_BYTES = TM * TK * 4;         // 16 KB, A or B tile
 constexpr int STAGE_BYTES = 4 * TILE_BYTES;     // A_h, A_l, B_h, B_l
-constexpr int C_BYTES = TM * TN * 4;            // C staging: 4 boxes [128 rows][32 fp32]
+constexpr int C_BYTES = TM * TN * 4;            // a C tile: 4 boxes [128 rows][32 fp32]
+constexpr int C_STAGE_BYTES = C_BYTES / 2;      // staged half a tile (64 columns) at a time
 constexpr int NUM_THREADS = 320;
 constexpr uint32_t TMEM_COLS = 256;
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + C_BYTES + 1024 + 256;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + C_STAGE_BYTES + 1024 + 256;
 
 struct TcArgs {
   int M, N, K;
@@ -105,15 +106,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *cs = smem + STAGES * STAGE_BYTES;  // C staging, 1024-byte aligned
-  uint64_t *bars = reinterpret_cast<uint64_t *>(cs + C_BYTES);
+  uint8_t *cs = smem + STAGES * STAGE_BYTES;  // C staging (half a tile), 1024-byte aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(cs + C_STAGE_BYTES);
   uint64_t *full = bars;                  // TMA landed
   uint64_t *split = bars + STAGES;        // h / l split done
   uint64_t *empty = bars + 2 * STAGES;    // MMAs done with the stage
   uint64_t *acc_full = bars + 3 * STAGES;
   uint64_t *acc_empty = acc_full + 2;
   uint64_t *drain = acc_empty + 2;
-  uint64_t *c_full = drain + 1;           // C tile landed in the staging buffer
+  uint64_t *c_full = drain + 1;           // a C half tile landed in the staging buffer
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 1);
   double *red = reinterpret_cast<double *>(bars + 16);  // dot mode: one per epilogue warp
 
@@ -261,123 +262,131 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) set_status(a.status, kDevTimeout);
     }
   } else {
-    // ---------------- epilogue: warps 6..9 (thread = accumulator row)
+    // ---------------- epilogue: warps 6..9 (thread = accumulator row).  The
+    // C tile passes through the staging buffer in two halves of 64 columns:
+    // half h is fetched by TMA (while the tile multiplies, for h = 0),
+    // combined with the accumulator in place and stored by TMA, then the
+    // buffer takes the next half.  After a failed wait the warps skip the
+    // work but keep meeting the named barriers, so none is left waiting.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;               // row within the tile
     const bool leader = threadIdx.x == 192;          // issues the C copies
     const bool dot = a.dot != nullptr;
     const bool need_c = a.beta != 0.0f || a.lower != 0 || dot;
-    uint32_t ch = 0;
+    uint32_t ch = 0, n_c = 0;                        // tiles done, C halves waited for
     bool ok = true;
-    auto load_c = [&](int t) {
+    auto load_half = [&](int t, int h) {
       int mt, nt;
       tile_of(a, t, mt, nt);
-      mbar_arrive_expect_tx(c_full, C_BYTES);
+      mbar_arrive_expect_tx(c_full, C_STAGE_BYTES);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tma_load_2d(cs + q * (C_BYTES / 4), &tmC, c_full, nt * TN + 32 * q, mt * TM);
+      for (int q = 0; q < 2; ++q)
+        tma_load_2d(cs + q * (C_BYTES / 4), &tmC, c_full, nt * TN + 64 * h + 32 * q, mt * TM);
     };
-    if (leader && need_c && static_cast<int>(blockIdx.x) < a.n_tiles) load_c(blockIdx.x);
+    if (leader && need_c && static_cast<int>(blockIdx.x) < a.n_tiles) load_half(blockIdx.x, 0);
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++ch) {
       int mt, nt;
       tile_of(a, t, mt, nt);
       const uint32_t buf = ch & 1, use = ch >> 1;
-      bool got = true;
-      if (need_c) got = mbar_wait(c_full, ch & 1);
-      got = mbar_wait(&acc_full[buf], use & 1) && got;
-      ok = __all_sync(0xffffffffu, got);
-      if (!ok) break;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1));
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * TN;
       const int m = mt * TM + r;
       const bool diag = a.lower && mt == nt;
-      if (dot) {
-        // sum over the tile of (alpha acc) * C: each thread its row (fp32
-        // over 32 columns, fp64 across), then the four warps in order
-        double rs = 0.0;
+      double rs = 0.0;  // dot mode: this row's sum
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          float v[32];
-          tmem_ld32(taddr + q * 32, v);
-          const uint8_t *row = cs + q * (C_BYTES / 4) + r * 128;
-          float part = 0.0f, pdiag = 0.0f;
+      for (int h = 0; h < 2; ++h) {
+        if (need_c && ok) ok = __all_sync(0xffffffffu, mbar_wait(c_full, n_c & 1));
+        ++n_c;
+        if (ok) {
+#pragma unroll 1
+          for (int qq = 0; qq < 2; ++qq) {
+            const int q = 2 * h + qq;
+            float v[32];
+            tmem_ld32(taddr + q * 32, v);
+            uint8_t *row = cs + qq * (C_BYTES / 4) + r * 128;
+            if (dot) {
+              // (alpha acc) * C over the row (fp32 over 32 columns, fp64 across)
+              float part = 0.0f, pdiag = 0.0f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
-            if (diag) {  // lower: keep n < m (counted twice below), the diagonal once
-              const int n = nt * TN + 32 * q + 4 * c;
-              if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
-              if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
-              if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
-              if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
-              if (n >= m) cv.x = 0.0f;
-              if (n + 1 >= m) cv.y = 0.0f;
-              if (n + 2 >= m) cv.z = 0.0f;
-              if (n + 3 >= m) cv.w = 0.0f;
+              for (int c = 0; c < 8; ++c) {
+                float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
+                if (diag) {  // lower: keep n < m (counted twice below), the diagonal once
+                  const int n = nt * TN + 32 * q + 4 * c;
+                  if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
+                  if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
+                  if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
+                  if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
+                  if (n >= m) cv.x = 0.0f;
+                  if (n + 1 >= m) cv.y = 0.0f;
+                  if (n + 2 >= m) cv.z = 0.0f;
+                  if (n + 3 >= m) cv.w = 0.0f;
+                }
+                part = fmaf(a.alpha * v[4 * c], cv.x, part);
+                part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
+                part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
+                part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
+              }
+              rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) +
+                    static_cast<double>(pdiag);
+              continue;
             }
-            part = fmaf(a.alpha * v[4 * c], cv.x, part);
-            part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
-            part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
-            part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+              float4 *p = reinterpret_cast<float4 *>(row + ((c ^ (r & 7)) << 4));
+              const float4 old = need_c ? *p : make_float4(0.f, 0.f, 0.f, 0.f);
+              float4 o;
+              o.x = fmaf(a.beta, old.x, a.alpha * v[4 * c]);
+              o.y = fmaf(a.beta, old.y, a.alpha * v[4 * c + 1]);
+              o.z = fmaf(a.beta, old.z, a.alpha * v[4 * c + 2]);
+              o.w = fmaf(a.beta, old.w, a.alpha * v[4 * c + 3]);
+              if (diag) {  // keep the strict upper part of a diagonal tile
+                const int n = nt * TN + 32 * q + 4 * c;
+                if (n > m) o.x = old.x;
+                if (n + 1 > m) o.y = old.y;
+                if (n + 2 > m) o.z = old.z;
+                if (n + 3 > m) o.w = old.w;
+              }
+              *p = o;
+            }
           }
-          rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) + static_cast<double>(pdiag);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (h == 1) {
+          // the accumulator buffer is free once its columns are in registers
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        if (!dot) fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader && ok) {
+          if (!dot) {
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq)
+              tma_store_2d(&tmC, cs + qq * (C_BYTES / 4), nt * TN + 64 * h + 32 * qq, mt * TM);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // staging buffer reusable
+          }
+          if (need_c) {
+            if (h == 0) {
+              load_half(t, 1);
+            } else {
+              const int tn = t + static_cast<int>(gridDim.x);
+              if (tn < a.n_tiles) load_half(tn, 0);
+            }
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+      if (dot) {
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
         if (lane == 0) red[quarter] = rs;
         named_bar_sync(1, 128);
-        if (leader) {
-          a.dot[t] = ((red[0] + red[1]) + red[2]) + red[3];
-          const int tn = t + static_cast<int>(gridDim.x);
-          if (tn < a.n_tiles) load_c(tn);
-        }
+        if (leader && ok) a.dot[t] = ((red[0] + red[1]) + red[2]) + red[3];
         named_bar_sync(1, 128);
-        continue;
       }
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        tmem_ld32(taddr + q * 32, v);
-        uint8_t *row = cs + q * (C_BYTES / 4) + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
-          float4 *p = reinterpret_cast<float4 *>(row + ((c ^ (r & 7)) << 4));
-          const float4 old = need_c ? *p : make_float4(0.f, 0.f, 0.f, 0.f);
-          float4 o;
-          o.x = fmaf(a.beta, old.x, a.alpha * v[4 * c]);
-          o.y = fmaf(a.beta, old.y, a.alpha * v[4 * c + 1]);
-          o.z = fmaf(a.beta, old.z, a.alpha * v[4 * c + 2]);
-          o.w = fmaf(a.beta, old.w, a.alpha * v[4 * c + 3]);
-          if (diag) {  // keep the strict upper part of a diagonal tile
-            const int n = nt * TN + 32 * q + 4 * c;
-            if (n > m) o.x = old.x;
-            if (n + 1 > m) o.y = old.y;
-            if (n + 2 > m) o.z = old.z;
-            if (n + 3 > m) o.w = old.w;
-          }
-          *p = o;
-        }
-      }
-      // the accumulator buffer is free once its columns are in registers
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          tma_store_2d(&tmC, cs + q * (C_BYTES / 4), nt * TN + 32 * q, mt * TM);
-        bulk_commit_group();
-        bulk_wait_group_read0();  // staging buffer reusable
-        const int tn = t + static_cast<int>(gridDim.x);
-        if (need_c && tn < a.n_tiles) load_c(tn);
-      }
-      named_bar_sync(1, 128);
     }
     if (leader) bulk_wait_group0();
     if (!ok && lane == 0) set_status(a.status, kDevTimeout);

@@ -442,8 +442,8 @@ size_t gq_gptq_sequential_workspace_size(const gq_seq_layer *layers, int n_layer
 
 gq_status gq_gptq_sequential(const void *X0_bf16, int64_t n_tok, const gq_seq_layer *layers,
                              int n_layers, int bits, int group_size, int block_size, int sym,
-                             float damp_percent, double *sse_dev, void *X_out_bf16, void *ws,
-                             size_t ws_bytes, void *stream) {
+                             float damp_percent, double *sse_dev, void *X_all_out_bf16,
+                             void *ws, size_t ws_bytes, void *stream) {
   t_last_error.clear();
   if (!layers || n_layers < 1 || !sse_dev || (n_tok > 0 && !X0_bf16))
     return fail(GQ_ERR_ARG, "null pointer or no layers");
@@ -480,7 +480,7 @@ gq_status gq_gptq_sequential(const void *X0_bf16, int64_t n_tok, const gq_seq_la
   }
   GQ_TRY(check_ws(ws, ws_bytes, seq_ws_bytes(layers, n_layers, n_tok, block_size)));
   return launch_sequential(X0_bf16, n_tok, layers, n_layers, bits, group_size, block_size, sym,
-                           damp_percent, sse_dev, X_out_bf16, ws,
+                           damp_percent, sse_dev, X_all_out_bf16, ws,
                            static_cast<cudaStream_t>(stream));
 }
 

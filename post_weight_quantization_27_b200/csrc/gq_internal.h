@@ -119,7 +119,7 @@ gq_status launch_qlinear(const uint32_t *qpacked, const uint16_t *scales, const 
 size_t seq_ws_bytes(const gq_seq_layer *layers, int n_layers, int64_t n_tok, int block_size);
 gq_status launch_sequential(const void *X0, int64_t n_tok, const gq_seq_layer *layers, int n,
                             int bits, int group_size, int block_size, int sym, float damp,
-                            double *sse_dev, void *X_out, void *ws, cudaStream_t st);
+                            double *sse_dev, void *X_all, void *ws, cudaStream_t st);
 
 // Activation-aware scaling before RTN (awq.cu).
 size_t awq_ws_bytes(int64_t d_out, int64_t d_in, int64_t n_tok, int group_size, int sym,

@@ -59,7 +59,7 @@ size_t seq_ws_bytes(const gq_seq_layer *layers, int n_layers, int64_t n_tok, int
 
 gq_status launch_sequential(const void *X0, int64_t n_tok, const gq_seq_layer *layers, int n,
                             int bits, int group_size, int block_size, int sym, float damp,
-                            double *sse_dev, void *X_out, void *ws, cudaStream_t st) {
+                            double *sse_dev, void *X_all, void *ws, cudaStream_t st) {
   const SeqLayout L = seq_layout(layers, n, n_tok, block_size);
   uint8_t *base = static_cast<uint8_t *>(ws);
   int *status = reinterpret_cast<int *>(base);
@@ -97,9 +97,17 @@ gq_status launch_sequential(const void *X0, int64_t n_tok, const gq_seq_layer *l
                        y.act, reinterpret_cast<int *>(scr), st);
     if (s != GQ_OK) return s;
   }
-  if (X_out && cudaMemcpyAsync(X_out, xbuf(n), static_cast<size_t>(n_tok) * layers[n - 1].d_out * 2,
-                               cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return check_launch("copy X_out");
+  if (X_all) {  // every input X_0 .. X_n, one after another (as the workspace holds them)
+    size_t off = 0;
+    for (int l = 0; l <= n; ++l) {
+      const int64_t dl = l < n ? layers[l].d_in : layers[n - 1].d_out;
+      const size_t bytes = static_cast<size_t>(n_tok) * dl * 2;
+      if (cudaMemcpyAsync(static_cast<uint8_t *>(X_all) + off, xbuf(l), bytes,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return check_launch("copy X_all");
+      off += bytes;
+    }
+  }
   return check_launch("gptq_sequential");
 }
 

@@ -460,7 +460,8 @@ def gptq_sequential(X0: torch.Tensor, layers: list, bits: int = 4, group_size: i
     with W (device [d_out, d_in]), act ("none", "relu", "gelu") and
     residual_from (None or the index of an earlier input added to the
     output).  Returns (list of quantised-layer dicts, sse numpy [n_layers],
-    the chain's output [n_tok, d_out] bf16)."""
+    list of the inputs X_0 .. X_n as bf16 device tensors, X_n the chain's
+    output)."""
     import numpy as np
     _dev(X0, "X0", torch.bfloat16)
     n_tok = X0.shape[0]
@@ -481,12 +482,17 @@ def gptq_sequential(X0: torch.Tensor, layers: list, bits: int = 4, group_size: i
                                                       block_size))
     ws = workspace(need, dev)
     sse = torch.empty(len(layers), dtype=torch.float64, device=dev)
-    X_out = torch.empty((n_tok, layers[-1]["W"].shape[0]), dtype=torch.bfloat16, device=dev)
+    widths = [L["W"].shape[1] for L in layers] + [layers[-1]["W"].shape[0]]
+    X_all = torch.empty(n_tok * sum(widths), dtype=torch.bfloat16, device=dev)
     st = lib_.gq_gptq_sequential(_p(X0), n_tok, ctypes.addressof(arr), len(layers), bits,
                                  group_size, block_size, int(bool(sym)), float(damp_percent),
-                                 _p(sse), _p(X_out), _p(ws), ws.numel(), _stream(stream))
+                                 _p(sse), _p(X_all), _p(ws), ws.numel(), _stream(stream))
     _check(st, "gq_gptq_sequential")
-    return outs, sse.cpu().numpy().astype(np.float64), X_out
+    xs, off = [], 0
+    for d in widths:
+        xs.append(X_all[off:off + n_tok * d].view(n_tok, d))
+        off += n_tok * d
+    return outs, sse.cpu().numpy().astype(np.float64), xs
 
 
 # ------------------------------------------------------------------ activation-aware scaling

@@ -17,7 +17,7 @@ import torch
 
 import oracle as O
 from post_weight_quantization_27_b200 import gq, inputs as I
-from tests.gpu_util import f16, u32
+from tests.gpu_util import f16, rel_fro, u32
 
 pytestmark = pytest.mark.gpu
 DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
@@ -58,13 +58,31 @@ def _layer(d_out, d_in, n_tok, seed, dtype="f32", outlier="cols:0.02:8"):
     return I.make_weights(spec), I.make_x(spec)
 
 
-def _run_gpu(W, X, group_size, sym, act_order=False, block_size=128, damp=0.01):
+def e2e_tie_rel(U_gpu, X, damp=0.01, perm=None):
+    """Scale of the tie windows for an end-to-end comparison.  There the GPU
+    runs GPTQ with its own fp32 U, whose relative error against the
+    oracle's fp64 U perturbs every update term as the column loop's own
+    rounding does: the window scale is the larger of TIE_REL and that
+    measured error (relative Frobenius)."""
+    Hd, _ = O.damp_hessian(O.hessian(X), damp)
+    if perm is not None:
+        Hd = Hd[np.ix_(perm, perm)]
+    Uo = O.upper_factor_of_inverse(Hd)
+    return max(O.TIE_REL, rel_fro(U_gpu.cpu().numpy(), Uo))
+
+
+def _run_gpu(W, X, group_size, sym, act_order=False, block_size=128, damp=0.01, bits=4):
+    """The whole GPU path; returns (quantised layer, perm, end-to-end tie
+    window scale)."""
     Wd, Xd = W.cuda(), X.cuda()
     H = gq.hessian(Xd)
     U, perm, dead, info = gq.damp_cholesky_inverse(H, damp, act_order=act_order)
-    out = gq.gptq_quantize_layer(Wd, U, 4, group_size, block_size, sym, perm=perm, dead=dead)
+    out = gq.gptq_quantize_layer(Wd, U, bits, group_size, block_size, sym, perm=perm, dead=dead)
     torch.cuda.synchronize()
-    return out, perm
+    p = None if perm is None else perm.cpu().numpy()
+    if p is not None:   # the order the oracle takes (reading 15)
+        p, _ = O.act_order_perm(O.damp_hessian(O.hessian(X.float().numpy()), damp)[0], follow=p)
+    return out, perm, e2e_tie_rel(U, X.float().numpy(), damp, p)
 
 
 @pytest.mark.parametrize("d_out,d_in,n_tok,group_size,sym,dt", [
@@ -80,19 +98,20 @@ def _run_gpu(W, X, group_size, sym, act_order=False, block_size=128, damp=0.01):
 ])
 def test_gptq_end_to_end(d_out, d_in, n_tok, group_size, sym, dt):
     W, X = _layer(d_out, d_in, n_tok, d_out + d_in, dt)
-    out, _ = _run_gpu(W, X, group_size, sym)
+    out, _, tr = _run_gpu(W, X, group_size, sym)
     Wn, Xn = W.float().numpy(), X.float().numpy()
     check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=group_size, sym=sym,
-                                           follow=f)[0], d_in, sym)
+                                           follow=f, tie_rel=tr)[0], d_in, sym)
 
 
 @pytest.mark.parametrize("block_size,group_size", [(64, -1), (64, 64), (32, 32), (128, 32)])
 def test_gptq_block_sizes(block_size, group_size):
     W, X = _layer(80, 320, 900, block_size + group_size)
-    out, _ = _run_gpu(W, X, group_size, True, block_size=block_size)
+    out, _, tr = _run_gpu(W, X, group_size, True, block_size=block_size)
     Wn, Xn = W.numpy(), X.float().numpy()
     check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=group_size,
-                                           block_size=block_size, follow=f)[0], 320, True)
+                                           block_size=block_size, follow=f, tie_rel=tr)[0],
+               320, True)
 
 
 def test_gptq_with_oracle_u_is_near_exact():
@@ -123,24 +142,27 @@ def test_gptq_with_oracle_u_is_near_exact():
 
 def test_gptq_act_order_affine():
     W, X = _layer(64, 384, 1200, 11, "bf16", "cols:0.02:10")
-    out, perm = _run_gpu(W, X, 128, False, act_order=True)
+    out, perm, tr = _run_gpu(W, X, 128, False, act_order=True)
     Wn, Xn = W.float().numpy(), X.float().numpy()
-    ref, H0, U, pref, dead = O.gptq_layer(Wn, Xn, group_size=128, sym=False, act_order=True)
-    if not np.array_equal(perm.cpu().numpy(), pref):
-        pytest.skip("act-order keys tie at fp32 precision")
+    Hd, dead = O.damp_hessian(O.hessian(Xn), 0.01)
+    pref, _ = O.act_order_perm(Hd, follow=perm.cpu().numpy())     # reading 15
+    assert np.array_equal(perm.cpu().numpy(), pref)
+    Uo = O.upper_factor_of_inverse(Hd[np.ix_(pref, pref)])
+    ref = O.gptq_quantize(Wn, Uo, group_size=128, sym=False, perm=pref, dead=dead)
     assert np.array_equal(out["g_idx"].cpu().numpy(), ref.g_idx)
-    check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=128, sym=False, act_order=True,
-                                           follow=f)[0], 384, False)
+    check_gptq(out, lambda f: O.gptq_quantize(Wn, Uo, group_size=128, sym=False, perm=pref,
+                                              dead=dead, follow=f, tie_rel=tr), 384, False)
 
 
 def test_gptq_dead_columns():
     W, X = _layer(32, 256, 600, 12)
     X[:, [3, 77]] = 0
-    out, _ = _run_gpu(W, X, -1, True)
+    out, _, tr = _run_gpu(W, X, -1, True)
     codes = _codes(out, 256, True)
     assert np.all(codes[:, [3, 77]] == 0)
     Wn, Xn = W.numpy(), X.float().numpy()
-    check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=-1, follow=f)[0], 256, True)
+    check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=-1, follow=f, tie_rel=tr)[0],
+               256, True)
 
 
 def test_gptq_diagonal_hessian_is_rtn():
@@ -150,7 +172,7 @@ def test_gptq_diagonal_hessian_is_rtn():
     X[torch.arange(d_in), torch.arange(d_in)] = torch.linspace(0.5, 3.0, d_in).to(torch.bfloat16)
     W, _ = _layer(48, d_in, 10, 13)
     for gs, sym in ((-1, True), (128, False), (32, True), (0, True), (0, False)):
-        out, _ = _run_gpu(W, X, gs, sym)
+        out, _, _ = _run_gpu(W, X, gs, sym)
         rtn = gq.rtn_quantize_pack(W.cuda(), 4, gs, sym)
         torch.cuda.synchronize()
         assert np.array_equal(u32(out["qpacked"]), u32(rtn["qpacked"]))
@@ -161,10 +183,10 @@ def test_gptq_diagonal_hessian_is_rtn():
 def test_gptq_workload_layers(workload, idx):
     spec = I.workload_layers(workload)[idx]
     W, X = I.make_weights(spec), I.make_x(spec)
-    out, _ = _run_gpu(W, X, spec.group_size, spec.sym)
+    out, _, tr = _run_gpu(W, X, spec.group_size, spec.sym)
     Wn, Xn = W.float().numpy(), X.float().numpy()
     check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, group_size=spec.group_size, sym=spec.sym,
-                                           follow=f)[0], spec.d_in, spec.sym)
+                                           follow=f, tie_rel=tr)[0], spec.d_in, spec.sym)
 
 
 def test_gptq_division_matches_ieee_at_midpoints():
@@ -187,7 +209,7 @@ def test_gptq_division_matches_ieee_at_midpoints():
     X = torch.zeros((d_in, d_in), dtype=torch.bfloat16)
     X[torch.arange(d_in), torch.arange(d_in)] = torch.linspace(0.5, 2.0, d_in).to(torch.bfloat16)
     for gs, sym in ((-1, True), (128, True), (64, False)):
-        out, _ = _run_gpu(W, X, gs, sym)
+        out, _, _ = _run_gpu(W, X, gs, sym)
         rtn = gq.rtn_quantize_pack(W.cuda(), 4, gs, sym)
         torch.cuda.synchronize()
         assert np.array_equal(u32(out["qpacked"]), u32(rtn["qpacked"])), (gs, sym)

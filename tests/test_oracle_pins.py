@@ -831,16 +831,36 @@ def test_tie_window_grows_with_the_updates_a_weight_received():
     E the accumulated |delta U| applied to the weight: a near-tie inside
     that window is adopted, one just outside it is not."""
     s = 2.0 ** -7                              # fp16-exact scale: absmax 7 s
-    U = np.array([[1.0, 50.0, 0.0], [0.0, 1.0, 0.0], [0.0, 0.0, 1.0]])
-    w0 = 3.02 * s                              # code 3, delta 0.02 s: column 1 gets 1 step of update
-    win = max(O.TIE_TOL, O.TIE_REL * 1.0)
+    # columns 0 and 1 (delta 0.2 s each) update column 2 by -5 s and +5 s:
+    # no net change, E = 10 steps
+    U = np.eye(4)
+    U[0, 2], U[1, 2] = 25.0, -25.0
+    win = max(O.TIE_TOL, O.TIE_REL * 10.0)
     assert win > O.TIE_TOL
     for off, adopted in ((0.5 * win, True), (2.0 * win, False)):
-        W = np.array([[w0, (3.5 + off) * s, 7 * s]])   # column 1 decides at (2.5 + off) steps
+        W = np.array([[3.2 * s, 1.2 * s, (2.5 + off) * s, 7 * s]])
         r = O.gptq_quantize(W, U, group_size=-1)
-        assert float(r.scales[0, 0]) == s and r.codes[0, 1] == 3
+        assert float(r.scales[0, 0]) == s and r.codes[0, 2] == 3
         other = r.codes.copy()
-        other[0, 1] = 2
+        other[0, 2] = 2
         rf = O.gptq_quantize(W, U, group_size=-1, follow=dict(codes=other, scales=r.scales))
-        assert (rf.codes[0, 1] == 2) == adopted, (off, win)
+        assert (rf.codes[0, 2] == 2) == adopted, (off, win)
         assert rf.n_followed == int(adopted)
+
+
+def test_apply_layer_follow_only_at_rounding_ties():
+    """The replay of bf16 roundings takes the other value only where the
+    fp64 result sits within the fp32 error of a bf16 rounding boundary
+    (window 2^-20 * (|X||W| + |Z|) ~ 2^-19 here)."""
+    X = np.array([[1.0, 1.0]])
+    # Z = 1 + 2^-8 + off: just above the bf16 midpoint between 1 and 1 + 2^-7
+    for off, adopted in ((2.0 ** -40, True), (2.0 ** -16, False)):
+        W = np.array([[0.5 + 2.0 ** -8 + off, 0.5]])
+        Z = O.apply_layer(X, W)
+        assert Z[0, 0] == 1.0 + 2.0 ** -7
+        Zf, n = O.apply_layer(X, W, follow=np.array([[1.0]]))
+        assert (n == 1) == adopted and (Zf[0, 0] == 1.0) == adopted
+    # a value two steps away is never taken
+    W = np.array([[0.5 + 2.0 ** -8 + 2.0 ** -40, 0.5]])
+    Zf, n = O.apply_layer(X, W, follow=np.array([[1.0 + 2.0 ** -6]]))
+    assert n == 0 and Zf[0, 0] == 1.0 + 2.0 ** -7

@@ -12,7 +12,7 @@ import torch
 import oracle as O
 from post_weight_quantization_27_b200 import gq, inputs as I
 from tests.gpu_util import f16, u32
-from tests.test_gptq_gpu import check_gptq
+from tests.test_gptq_gpu import check_gptq, e2e_tie_rel
 
 pytestmark = pytest.mark.gpu
 DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
@@ -62,8 +62,9 @@ def test_gptq_widths(bits, group_size, sym):
     out = gq.gptq_quantize_layer(Wd, U, bits, group_size, 128, sym, dead=dead)
     torch.cuda.synchronize()
     Wn, Xn = W.float().numpy(), X.float().numpy()
+    tr = e2e_tie_rel(U, Xn)
     check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, bits=bits, group_size=group_size, sym=sym,
-                                           follow=f)[0], 384, sym, bits=bits)
+                                           follow=f, tie_rel=tr)[0], 384, sym, bits=bits)
 
 
 @pytest.mark.parametrize("bits", [3, 8])
@@ -74,12 +75,14 @@ def test_gptq_widths_act_order(bits):
     out = gq.gptq_quantize_layer(Wd, U, bits, 128, 128, False, perm=perm, dead=dead)
     torch.cuda.synchronize()
     Wn, Xn = W.float().numpy(), X.float().numpy()
-    ref, H0, Uo, pref, dead_o = O.gptq_layer(Wn, Xn, bits=bits, group_size=128, sym=False,
-                                            act_order=True)
-    pref, _ = O.act_order_perm(O.damp_hessian(H0, 0.01)[0], follow=perm.cpu().numpy())
+    Hd, dead_o = O.damp_hessian(O.hessian(Xn), 0.01)
+    pref, _ = O.act_order_perm(Hd, follow=perm.cpu().numpy())
     assert np.array_equal(perm.cpu().numpy(), pref)
-    check_gptq(out, lambda f: O.gptq_layer(Wn, Xn, bits=bits, group_size=128, sym=False,
-                                           act_order=True, follow=f)[0], 256, False, bits=bits)
+    Uo = O.upper_factor_of_inverse(Hd[np.ix_(pref, pref)])
+    tr = e2e_tie_rel(U, Xn, perm=pref)
+    check_gptq(out, lambda f: O.gptq_quantize(Wn, Uo, bits=bits, group_size=128, sym=False,
+                                              perm=pref, dead=dead_o, follow=f, tie_rel=tr),
+               256, False, bits=bits)
 
 
 @pytest.mark.parametrize("bits", [2, 3, 8])
