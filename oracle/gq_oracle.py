@@ -615,11 +615,15 @@ def apply_layer(X, W_hat, act="none", residual=None, follow=None, tie_rel=TIE_RE
     [d_out, d_in].
 
     ``follow`` (optional, [n_tok, d_out], another implementation's bf16
-    values): where the fp64 value lies within that implementation's error
-    of a bf16 rounding boundary -- tie_rel * (|X| |W|^T + |residual| +
-    |Z|), the error bound of an fp32 sum of those terms -- both roundings
-    are correct and the other implementation's value is taken when it is
-    the other neighbour.  Returns Z, or (Z, adopted) with ``follow``."""
+    values): that implementation computes the value before rounding with an
+    error of at most w = tie_rel * (|X| |W|^T + |residual| + |Z|), the
+    error bound of an fp32 sum of those terms, so any bf16 value that is
+    the rounding of some t in [Z - w, Z + w] is a correct result.  Rounding
+    is monotone, so those are exactly the bf16 values between
+    round(Z - w) and round(Z + w); the other implementation's value is
+    taken where it is one of them (the other neighbour at a rounding tie;
+    where Z cancels to far below |X| |W|^T, w can span several bf16 steps).
+    Returns Z, or (Z, adopted) with ``follow``."""
     Xa = np.asarray(X, dtype=np.float64)
     Wa = np.asarray(W_hat, dtype=np.float64)
     Y = Xa @ Wa.T
@@ -636,13 +640,9 @@ def apply_layer(X, W_hat, act="none", residual=None, follow=None, tie_rel=TIE_RE
     mag = np.abs(Xa) @ np.abs(Wa).T + np.abs(Y)
     if residual is not None:
         mag = mag + np.abs(np.asarray(residual, dtype=np.float64))
-    m, e = np.frexp(Y)
-    k = np.floor(np.abs(m) * 256.0)                   # the bf16 neighbours of Y:
-    a = np.sign(Y) * np.ldexp(k, e - 8)               # k and k + 1 units of 2^(e-8)
-    b = np.sign(Y) * np.ldexp(k + 1.0, e - 8)
-    mid = np.sign(Y) * np.ldexp(k + 0.5, e - 8)
-    near = np.abs(Y - mid) < tie_rel * mag
-    take = near & (f != Z) & ((f == a) | (f == b))
+    w = tie_rel * mag
+    lo, hi = round_to_bf16(Y - w), round_to_bf16(Y + w)
+    take = (f != Z) & (f >= lo) & (f <= hi)
     return np.where(take, f, Z), int(take.sum())
 
 

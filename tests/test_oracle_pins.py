@@ -849,8 +849,8 @@ def test_tie_window_grows_with_the_updates_a_weight_received():
 
 
 def test_apply_layer_follow_only_at_rounding_ties():
-    """The replay of bf16 roundings takes the other value only where the
-    fp64 result sits within the fp32 error of a bf16 rounding boundary
+    """The replay of bf16 roundings takes the other value only where it is
+    the rounding of a value within the fp32 error of the fp64 result
     (window 2^-20 * (|X||W| + |Z|) ~ 2^-19 here)."""
     X = np.array([[1.0, 1.0]])
     # Z = 1 + 2^-8 + off: just above the bf16 midpoint between 1 and 1 + 2^-7
@@ -864,3 +864,11 @@ def test_apply_layer_follow_only_at_rounding_ties():
     W = np.array([[0.5 + 2.0 ** -8 + 2.0 ** -40, 0.5]])
     Zf, n = O.apply_layer(X, W, follow=np.array([[1.0 + 2.0 ** -6]]))
     assert n == 0 and Zf[0, 0] == 1.0 + 2.0 ** -7
+    # cancellation: Z = 2^-30 far below |X||W| = 1, so the window 2^-20 (1 +
+    # Z) spans many bf16 steps of Z: any value that rounds some t within it
+    # is taken (2^-21, -2^-22), one beyond it is not (2^-19)
+    W = np.array([[0.5, -0.5 + 2.0 ** -30]])
+    assert O.apply_layer(X, W)[0, 0] == 2.0 ** -30
+    for f, adopted in ((2.0 ** -21, True), (-(2.0 ** -22), True), (2.0 ** -19, False)):
+        Zf, n = O.apply_layer(X, W, follow=np.array([[f]]))
+        assert (n == 1) == adopted and (Zf[0, 0] == f) == adopted
