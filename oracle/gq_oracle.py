@@ -647,7 +647,8 @@ def apply_layer(X, W_hat, act="none", residual=None, follow=None, tie_rel=TIE_RE
 
 
 def gptq_sequential(X0, layers, bits=4, group_size=-1, block_size=128, sym=True,
-                    damp_percent=0.01, quantized_inputs=True, follow=None, follow_x=None):
+                    damp_percent=0.01, quantized_inputs=True, follow=None, follow_x=None,
+                    tie_rel=TIE_REL, x_tie_rel=TIE_REL):
     """Layers quantised one after another, each calibrated on the input it
     actually receives ("GPT-2 Quantization Reconstruction Error", "Key
     findings": the per-layer errors were measured with the whole model
@@ -660,22 +661,26 @@ def gptq_sequential(X0, layers, bits=4, group_size=-1, block_size=128, sym=True,
     W when not ``quantized_inputs``), act, X_j).  ``follow``: per-layer
     list of dicts (as for gptq_quantize) or None; ``follow_x``: another
     implementation's X_1 .. X_n (its bf16 roundings are taken at ties, as in
-    apply_layer).  Returns (results, sse, xs) with xs the inputs X_0 ..
-    X_n."""
+    apply_layer); ``tie_rel``: the GPTQ tie window scale (see TIE_REL), one
+    for all layers or a list with one per layer; ``x_tie_rel``: the window
+    scale of the activations' replay (apply_layer's tie_rel).  Returns
+    (results, sse, xs) with xs the inputs X_0 .. X_n."""
     X = np.asarray(X0, dtype=np.float64)
     results, sse, xs = [], [], [X]
     for li, L in enumerate(layers):
         W = np.asarray(L["W"], dtype=np.float64)
+        tr = tie_rel[li] if isinstance(tie_rel, (list, tuple)) else tie_rel
         res, H0, U, perm, dead = gptq_layer(W, X, bits=bits, group_size=group_size,
                                             block_size=block_size, sym=sym,
                                             damp_percent=damp_percent,
-                                            follow=None if follow is None else follow[li])
+                                            follow=None if follow is None else follow[li],
+                                            tie_rel=tr)
         results.append(res)
         sse.append(recon_sse(W, res.W_hat, X))
         j = L.get("residual_from")
         X = apply_layer(X, res.W_hat if quantized_inputs else W, L.get("act", "none"),
                         None if j is None else xs[j],
-                        follow=None if follow_x is None else follow_x[li])
+                        follow=None if follow_x is None else follow_x[li], tie_rel=x_tie_rel)
         if follow_x is not None:
             X = X[0]
         xs.append(X)

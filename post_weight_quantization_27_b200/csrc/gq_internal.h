@@ -63,6 +63,7 @@ gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, in
 
 struct HessPlan {
   int n_bi, n_bj, n_tiles, n_split, nkb_total, kb_per_split;
+  int pairs;  // 256 x 256 tiles on CTA pairs (else 128 x 256 on single CTAs)
   size_t ws_bytes;
 };
 HessPlan hessian_plan(int64_t n_tok, int64_t d_in);
@@ -85,6 +86,14 @@ gq_status launch_gemm_tf32x3(int M, int N, int K, float alpha, const float *A, i
                              int64_t ldc, bool lower, int *status, cudaStream_t st,
                              double *dot_partials = nullptr);
 int gemm_tf32x3_tiles(int M, int N, bool lower = false);
+// sum over the lower triangle of (A A^T) .* C with A = A_h + A_l in bf16
+// parts [M][lda] (K contiguous, lda a multiple of 8), C symmetric fp32:
+// syrk_dot_bf16x3_partials(M) fp64 partials (strictly lower elements
+// twice, the diagonal once); ~2^-16 relative per product term.
+int syrk_dot_bf16x3_partials(int M);
+gq_status launch_syrk_dot_bf16x3(int M, int K, const uint16_t *A_h, const uint16_t *A_l,
+                                 int64_t lda, const float *C, int64_t ldc, double *dot_partials,
+                                 int *status, cudaStream_t st);
 
 size_t gptq_ws_bytes(int64_t d_out, int64_t d_in, int block_size);
 gq_status launch_gptq(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, const float *U,

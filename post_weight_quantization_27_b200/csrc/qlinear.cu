@@ -89,48 +89,88 @@ __device__ __forceinline__ float ld_dense<__nv_bfloat16>(const __nv_bfloat16 *p)
   return __bfloat162float(*p);
 }
 
-// The 64 weights of row m, columns k0 .. k0 + 63, in fp32 (zero past d_in).
-template <int BITS, typename T>
-__device__ __forceinline__ void row_weights(const QlArgs &a, int64_t m, int64_t k0,
-                                            float (&w)[64]) {
-  if constexpr (BITS == 0) {
-    const T *src = static_cast<const T *>(a.Wd) + m * a.d_in;
+// Dense mode: the 64 weights of row m, columns k0 .. k0 + 63, in fp32
+// (zero past d_in).
+template <typename T>
+__device__ __forceinline__ void dense_weights(const QlArgs &a, int64_t m, int64_t k0,
+                                              float (&w)[64]) {
+  const T *src = static_cast<const T *>(a.Wd) + m * a.d_in;
 #pragma unroll
-    for (int k = 0; k < 64; ++k) w[k] = k0 + k < a.d_in ? ld_dense<T>(src + k0 + k) : 0.0f;
-  } else {
-    constexpr int NW = 2 * BITS;  // words of 64 codes
-    const int64_t row_words = a.d_in * BITS / 32;
-    const uint32_t *src = a.q + m * row_words + (k0 * BITS) / 32;
-    const int64_t left = row_words - (k0 * BITS) / 32;
-    uint32_t wd[NW];
+  for (int k = 0; k < 64; ++k) w[k] = k0 + k < a.d_in ? ld_dense<T>(src + k0 + k) : 0.0f;
+}
+
+// The packed codes of row m for columns k0 .. k0 + 63 (2 BITS words) and,
+// when one group covers the whole K step, its scale and zero: loaded one
+// K step ahead of their use, so the loads' latency hides behind the
+// previous step's work.
+template <int BITS>
+struct CodeSlot {
+  uint32_t wd[2 * BITS];
+  float s, z;
+};
+
+template <int BITS>
+__device__ __forceinline__ void load_slot(const QlArgs &a, int64_t m, int64_t k0, bool uniform,
+                                          CodeSlot<BITS> &c) {
+  constexpr int NW = 2 * BITS;
+  c.s = 0.0f;
+  c.z = 0.0f;
+  if (m >= a.d_out) {
 #pragma unroll
-    for (int i = 0; i < NW; ++i) wd[i] = i < left ? __ldg(src + i) : 0u;
-    const bool uniform = a.g_idx == nullptr && (a.group_size <= 0 || a.group_size % 64 == 0);
-    float s = 0.0f, z = 0.0f;
-    if (uniform) {
-      const int64_t gi = a.group_size <= 0 ? 0 : k0 / a.group_size;
-      s = __half2float(__ushort_as_half(a.scales[m * a.n_groups + gi]));
-      z = a.sym ? 0.0f : __half2float(__ushort_as_half(a.zeros[m * a.n_groups + gi]));
-    }
-    const int offset = a.sym ? (1 << (BITS - 1)) : 0;
-#pragma unroll
-    for (int k = 0; k < 64; ++k) {
-      const int bit = BITS * k, wi = bit >> 5, off = bit & 31;
-      uint32_t v = wd[wi] >> off;
-      if (off + BITS > 32) v |= wd[wi + 1] << (32 - off);
-      v &= (1u << BITS) - 1u;
-      float sk = s, zk = z;
-      if (!uniform) {
-        const int64_t c = k0 + k < a.d_in ? k0 + k : a.d_in - 1;
-        int64_t gi = a.g_idx ? a.g_idx[c] : (a.group_size <= 0 ? 0 : c / a.group_size);
-        gi = gi < 0 ? 0 : (gi >= a.n_groups ? a.n_groups - 1 : gi);
-        sk = __half2float(__ushort_as_half(a.scales[m * a.n_groups + gi]));
-        zk = a.sym ? 0.0f : __half2float(__ushort_as_half(a.zeros[m * a.n_groups + gi]));
-      }
-      const float code = static_cast<float>(static_cast<int>(v) - offset);
-      w[k] = k0 + k < a.d_in ? sk * (code - zk) : 0.0f;
-    }
+    for (int i = 0; i < NW; ++i) c.wd[i] = 0u;
+    return;
   }
+  const int64_t row_words = a.d_in * BITS / 32;
+  const uint32_t *src = a.q + m * row_words + (k0 * BITS) / 32;
+  const int64_t left = row_words - (k0 * BITS) / 32;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) c.wd[i] = i < left ? __ldg(src + i) : 0u;
+  if (uniform) {
+    const int64_t gi = a.group_size <= 0 ? 0 : k0 / a.group_size;
+    c.s = __half2float(__ushort_as_half(a.scales[m * a.n_groups + gi]));
+    c.z = a.sym ? 0.0f : __half2float(__ushort_as_half(a.zeros[m * a.n_groups + gi]));
+  }
+}
+
+// W^ of the 8 columns k0 + 8 cb .. k0 + 8 cb + 7 of row m from its codes.
+template <int BITS>
+__device__ __forceinline__ void slot_chunk(const QlArgs &a, int64_t m, int64_t k0, bool uniform,
+                                           const CodeSlot<BITS> &c, int cb, float (&w)[8]) {
+  const int offset = a.sym ? (1 << (BITS - 1)) : 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int k = 8 * cb + e;
+    const int bit = BITS * k, wi = bit >> 5, off = bit & 31;
+    uint32_t v = c.wd[wi] >> off;
+    if (off + BITS > 32) v |= c.wd[wi + 1] << (32 - off);
+    v &= (1u << BITS) - 1u;
+    float sk = c.s, zk = c.z;
+    if (!uniform && m < a.d_out) {
+      const int64_t col = k0 + k < a.d_in ? k0 + k : a.d_in - 1;
+      int64_t gi = a.g_idx ? a.g_idx[col] : (a.group_size <= 0 ? 0 : col / a.group_size);
+      gi = gi < 0 ? 0 : (gi >= a.n_groups ? a.n_groups - 1 : gi);
+      sk = __half2float(__ushort_as_half(a.scales[m * a.n_groups + gi]));
+      zk = a.sym ? 0.0f : __half2float(__ushort_as_half(a.zeros[m * a.n_groups + gi]));
+    }
+    const float code = static_cast<float>(static_cast<int>(v) - offset);
+    w[e] = (k0 + k < a.d_in && m < a.d_out) ? sk * (code - zk) : 0.0f;
+  }
+}
+
+// 8 fp32 weights as bf16 hi + lo into chunk cb of row r of the stage's A
+// tiles (128-byte swizzle: 16-byte chunk cb of row r sits at cb ^ (r % 8)).
+__device__ __forceinline__ void store_chunk(uint8_t *hi_row, uint8_t *lo_row, int r, int cb,
+                                            const float (&w)[8]) {
+  __align__(16) __nv_bfloat16 h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const __nv_bfloat16 hb = __float2bfloat16_rn(w[e]);
+    h[e] = hb;
+    l[e] = __float2bfloat16_rn(w[e] - __bfloat162float(hb));
+  }
+  const int pc = (cb ^ (r & 7)) << 4;
+  *reinterpret_cast<uint4 *>(hi_row + pc) = *reinterpret_cast<const uint4 *>(h);
+  *reinterpret_cast<uint4 *>(lo_row + pc) = *reinterpret_cast<const uint4 *>(l);
 }
 
 template <int BITS, typename T>
@@ -200,41 +240,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = threadIdx.x - 64;  // row of the tile, 0..127
     bool ok = true;
     uint32_t it = 0;
-    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-      int mt, nt;
-      ql_tile(t, a.n_mt, a.n_nt, mt, nt);
-      const int64_t m = static_cast<int64_t>(mt) * BM + r;
-      for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+    if constexpr (BITS == 0) {
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        int mt, nt;
+        ql_tile(t, a.n_mt, a.n_nt, mt, nt);
+        const int64_t m = static_cast<int64_t>(mt) * BM + r;
+        for (int kb = 0; kb < a.nkb; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = it / STAGES;
+          ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], (ph & 1) ^ 1));
+          if (!ok) break;
+          float w[64];
+          if (m < a.d_out) {
+            dense_weights<T>(a, m, static_cast<int64_t>(kb) * BK, w);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 64; ++k) w[k] = 0.0f;
+          }
+          uint8_t *hi_row = smem + s * STAGE_BYTES + r * 128;
+#pragma unroll
+          for (int cb = 0; cb < 8; ++cb) {
+            float w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w8[e] = w[8 * cb + e];
+            store_chunk(hi_row, hi_row + A_BYTES, r, cb, w8);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[s]);
+        }
+      }
+    } else {
+      const bool uniform = a.g_idx == nullptr && (a.group_size <= 0 || a.group_size % 64 == 0);
+      // (t, kb) in processing order; the codes of the next step are loaded
+      // before waiting for this step's stage
+      int t = blockIdx.x, kb = 0;
+      CodeSlot<BITS> nxt;
+      auto row_of = [&](int tt) {
+        int mt, nt;
+        ql_tile(tt, a.n_mt, a.n_nt, mt, nt);
+        return static_cast<int64_t>(mt) * BM + r;
+      };
+      if (t < n_tiles) load_slot<BITS>(a, row_of(t), 0, uniform, nxt);
+      while (t < n_tiles && ok) {
+        const CodeSlot<BITS> cur = nxt;
+        const int64_t m = row_of(t);
+        const int64_t k0 = static_cast<int64_t>(kb) * BK;
+        int t2 = t, kb2 = kb + 1;
+        if (kb2 == a.nkb) {
+          t2 = t + static_cast<int>(gridDim.x);
+          kb2 = 0;
+        }
+        if (t2 < n_tiles) load_slot<BITS>(a, row_of(t2), static_cast<int64_t>(kb2) * BK, uniform, nxt);
         const uint32_t s = it % STAGES, ph = it / STAGES;
         ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], (ph & 1) ^ 1));
         if (!ok) break;
-        float w[64];
-        if (m < a.d_out) {
-          row_weights<BITS, T>(a, m, static_cast<int64_t>(kb) * BK, w);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 64; ++k) w[k] = 0.0f;
-        }
         uint8_t *hi_row = smem + s * STAGE_BYTES + r * 128;
-        uint8_t *lo_row = hi_row + A_BYTES;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          __align__(16) __nv_bfloat16 h[8], l[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float v = w[8 * c + e];
-            const __nv_bfloat16 hb = __float2bfloat16_rn(v);
-            h[e] = hb;
-            l[e] = __float2bfloat16_rn(v - __bfloat162float(hb));
-          }
-          // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
-          const int pc = (c ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4 *>(hi_row + pc) = *reinterpret_cast<const uint4 *>(h);
-          *reinterpret_cast<uint4 *>(lo_row + pc) = *reinterpret_cast<const uint4 *>(l);
+        for (int cb = 0; cb < 8; ++cb) {
+          float w8[8];
+          slot_chunk<BITS>(a, m, k0, uniform, cur, cb, w8);
+          store_chunk(hi_row, hi_row + A_BYTES, r, cb, w8);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[s]);
+        ++it;
+        t = t2;
+        kb = kb2;
       }
     }
     if (!ok && lane == 0) set_status(a.status, kDevTimeout);

@@ -405,21 +405,24 @@ gq_status launch_recon(const void *W, gq_dtype dt, const uint32_t *qpacked,
 // ---------------------------------------------------------------------------
 // The same SSE by the trace route: ||dW X^T||_F^2 = tr(dW X^T X dW^T) =
 // tr(dW H0 dW^T) / 2 = <H0, G>_F / 2 with G = dW^T dW and the undamped
-// H0 = 2 X^T X.  dW^T is formed in fp32, then G's lower triangle on the
-// tensor cores (a SYRK in fp32 accuracy, 3 x TF32) whose epilogue sums G .*
-// H0 over each tile instead of storing G (off-diagonal elements twice);
-// fp64 tile partials added in a fixed order.  d_out d_in^2 flops instead
-// of 2 n_tok d_out d_in.
+// H0 = 2 X^T X.  dW^T is formed as a bf16 pair hi + lo (16 significant
+// bits), then G's lower triangle on the tensor cores (a SYRK of three bf16
+// products, ~2^-16 relative per term) whose epilogue sums G .* H0 over each
+// tile instead of storing G (off-diagonal elements twice); fp64 tile
+// partials added in a fixed order.  d_out d_in^2 flops instead of 2 n_tok
+// d_out d_in.
 namespace {
 
-// dW^T [d_in][ldt] (ldt = d_out rounded up to 4, zero-padded): a block
-// takes 32 rows x 64 columns of dW, forms them in shared memory and writes
-// them transposed, 32 consecutive floats per column.
+// dW^T as bf16 hi + lo, [d_in][ldt] each (ldt = d_out rounded up to 8,
+// zero-padded): a block takes 32 rows x 64 columns of dW, forms them in
+// shared memory and writes them transposed, 32 consecutive values per
+// column.
 template <typename T>
 __global__ void __launch_bounds__(256) dequant_diff_t_kernel(
     const T *__restrict__ W, const uint32_t *__restrict__ q, const uint16_t *__restrict__ scales,
     const uint16_t *__restrict__ zeros, const int32_t *__restrict__ g_idx, int64_t d_out,
-    int64_t d_in, int group_size, int sym, int bits, float *__restrict__ dwt, int64_t ldt) {
+    int64_t d_in, int group_size, int sym, int bits, __nv_bfloat16 *__restrict__ dth,
+    __nv_bfloat16 *__restrict__ dtl, int64_t ldt) {
   __shared__ float tile[64][33];
   const int64_t n_groups = group_size <= 0 ? 1 : d_in / group_size;
   const int64_t row_words = d_in * bits / 32;
@@ -455,7 +458,12 @@ __global__ void __launch_bounds__(256) dequant_diff_t_kernel(
       for (int k = 0; k < 8; ++k) {
         const int cc = wp * 8 + k;
         const int64_t c = c0 + cc, r = r0 + lane;
-        if (c < d_in && r < ldt) dwt[c * ldt + r] = r < d_out ? tile[cc][lane] : 0.0f;
+        if (c < d_in && r < ldt) {
+          const float v = r < d_out ? tile[cc][lane] : 0.0f;
+          const __nv_bfloat16 h = __float2bfloat16_rn(v);
+          dth[c * ldt + r] = h;
+          dtl[c * ldt + r] = __float2bfloat16_rn(v - __bfloat162float(h));
+        }
       }
     }
     __syncthreads();
@@ -464,15 +472,17 @@ __global__ void __launch_bounds__(256) dequant_diff_t_kernel(
 
 struct TraceLayout {
   int64_t ldt;
-  size_t off_partials, off_dwt, total;
+  size_t off_partials, off_dth, off_dtl, total;
 };
 TraceLayout trace_layout(int64_t d_out, int64_t d_in) {
   TraceLayout L{};
-  L.ldt = (d_out + 3) / 4 * 4;
+  L.ldt = (d_out + 7) / 8 * 8;
   L.off_partials = kWsHeader;
-  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_in), static_cast<int>(d_in), true);
-  L.off_dwt = L.off_partials + round_up(static_cast<size_t>(tiles) * sizeof(double), 256);
-  L.total = L.off_dwt + round_up(static_cast<size_t>(d_in) * L.ldt * sizeof(float), 256);
+  const int parts = syrk_dot_bf16x3_partials(static_cast<int>(d_in));
+  const size_t part = round_up(static_cast<size_t>(d_in) * L.ldt * 2, 256);
+  L.off_dth = L.off_partials + round_up(static_cast<size_t>(parts) * sizeof(double), 256);
+  L.off_dtl = L.off_dth + part;
+  L.total = L.off_dtl + part;
   return L;
 }
 }  // namespace
@@ -491,7 +501,8 @@ gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpack
   uint8_t *base = static_cast<uint8_t *>(ws);
   int *status = reinterpret_cast<int *>(base);
   double *partials = reinterpret_cast<double *>(base + L.off_partials);
-  float *dwt = reinterpret_cast<float *>(base + L.off_dwt);
+  auto *dth = reinterpret_cast<__nv_bfloat16 *>(base + L.off_dth);
+  auto *dtl = reinterpret_cast<__nv_bfloat16 *>(base + L.off_dtl);
   if (cudaMemsetAsync(status, 0, kWsHeader, st) != cudaSuccess) return check_launch("memset");
   int64_t g = ((L.ldt + 31) / 32) * ((d_in + 63) / 64);
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
@@ -501,30 +512,31 @@ gq_status launch_recon_hessian(const void *W, gq_dtype dt, const uint32_t *qpack
     case GQ_F32:
       dequant_diff_t_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(W), qpacked,
                                                          scales, zeros, g_idx, d_out, d_in,
-                                                         group_size, sym, bits, dwt, L.ldt);
+                                                         group_size, sym, bits, dth, dtl, L.ldt);
       break;
     case GQ_F16:
       dequant_diff_t_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half *>(W), qpacked,
                                                           scales, zeros, g_idx, d_out, d_in,
-                                                          group_size, sym, bits, dwt, L.ldt);
+                                                          group_size, sym, bits, dth, dtl, L.ldt);
       break;
     case GQ_BF16:
       dequant_diff_t_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
           static_cast<const __nv_bfloat16 *>(W), qpacked, scales, zeros, g_idx, d_out, d_in,
-          group_size, sym, bits, dwt, L.ldt);
+          group_size, sym, bits, dth, dtl, L.ldt);
       break;
   }
   count_launch();
   gq_status s = check_launch("dequant_diff_t_kernel");
   if (s != GQ_OK) return s;
-  // G = dW^T dW (lower triangle, K = d_out; rows of dW^T are K-major for
-  // both operands), each tile summed against H0's
-  s = launch_gemm_tf32x3(static_cast<int>(d_in), static_cast<int>(d_in), static_cast<int>(L.ldt),
-                         1.0f, dwt, L.ldt, dwt, L.ldt, true, 0.0f, const_cast<float *>(H0), d_in,
-                         true, status, st, partials);
+  // G = dW^T dW (lower triangle, K = d_out; rows of dW^T are K-major),
+  // each tile summed against H0's
+  s = launch_syrk_dot_bf16x3(static_cast<int>(d_in), static_cast<int>(d_out),
+                             reinterpret_cast<const uint16_t *>(dth),
+                             reinterpret_cast<const uint16_t *>(dtl), L.ldt, H0, d_in, partials,
+                             status, st);
   if (s != GQ_OK) return s;
-  const int tiles = gemm_tf32x3_tiles(static_cast<int>(d_in), static_cast<int>(d_in), true);
-  recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, tiles, status, sse_dev, 0.5);
+  const int parts = syrk_dot_bf16x3_partials(static_cast<int>(d_in));
+  recon_reduce_kernel<<<1, 1024, 0, st>>>(partials, parts, status, sse_dev, 0.5);
   count_launch();
   return check_launch("recon_reduce_kernel");
 }

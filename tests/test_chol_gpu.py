@@ -19,7 +19,9 @@ def _H(n_tok, d, seed, dead=()):
     return O.hessian(X).astype(np.float32)
 
 
-@pytest.mark.parametrize("n_tok,d", [(64, 8), (300, 136), (2048, 768), (1500, 1032), (4000, 3072)])
+# (the last case's trailing updates are large enough to run on CTA pairs)
+@pytest.mark.parametrize("n_tok,d", [(64, 8), (300, 136), (2048, 768), (1500, 1032), (4000, 3072),
+                                     (8192, 6144)])
 def test_upper_factor_matches_oracle(n_tok, d):
     H32 = _H(n_tok, d, d)
     U, perm, dead, info = gq.damp_cholesky_inverse(torch.from_numpy(H32).cuda(), 0.01)

@@ -19,8 +19,11 @@ def _x(n_tok, d_in, seed):
     return I.make_x(spec)
 
 
+# d_in >= 1024 runs on CTA pairs (256 x 256 tiles): 1032 and 1304 leave
+# ragged pair tiles, 20000 x 1304 splits the tokens over few tiles
 @pytest.mark.parametrize("n_tok,d_in", [(64, 8), (100, 136), (2048, 768), (1000, 264),
-                                        (4097, 520), (2560, 3072), (300, 1032), (70000, 256)])
+                                        (4097, 520), (2560, 3072), (300, 1032), (70000, 256),
+                                        (20000, 1304)])
 def test_hessian_matches_oracle(n_tok, d_in):
     X = _x(n_tok, d_in, n_tok + d_in)
     H = gq.hessian(X.cuda()).cpu().numpy()

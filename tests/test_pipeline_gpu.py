@@ -14,7 +14,7 @@ import torch
 
 import oracle as O
 from post_weight_quantization_27_b200 import gq, inputs as I
-from tests.gpu_util import f16, u32
+from tests.gpu_util import f16, rel_fro, u32
 from tests.test_gptq_gpu import check_gptq
 
 pytestmark = pytest.mark.gpu
@@ -93,6 +93,14 @@ def _chain(seed, d=256, n=2048):
     return X0, layers
 
 
+def _u_err(x: torch.Tensor) -> float:
+    """Relative Frobenius error of the GPU's U (from its H of the bf16 input
+    x) against the oracle's U of the same input."""
+    U, _, _, _ = gq.damp_cholesky_inverse(gq.hessian(x.contiguous()), 0.01)
+    Hd, _ = O.damp_hessian(O.hessian(x.float().cpu().numpy()), 0.01)
+    return rel_fro(U.cpu().numpy(), O.upper_factor_of_inverse(Hd))
+
+
 @pytest.mark.parametrize("bits,group_size,sym", [(4, 128, True), (4, -1, False), (8, 64, True)])
 def test_sequential_pipeline_matches_oracle(bits, group_size, sym):
     """The whole chain against the oracle's: each layer's codes to the GPTQ
@@ -114,8 +122,18 @@ def test_sequential_pipeline_matches_oracle(bits, group_size, sym):
                            scales=f16(o["scales"]),
                            zeros=None if sym else f16(o["zeros"])))
     fx = [x.float().cpu().numpy() for x in xs_gpu[1:]]
+    # each layer's GPTQ decisions are taken with the GPU's fp32 U of its own
+    # input: its measured error widens the tie windows (as end to end in
+    # test_configs_gpu)
+    tie_rel = [max(O.TIE_REL, _u_err(x)) for x in xs_gpu[:-1]]
+    # the GPU multiplies with W^ held as a bf16 pair (16 significant bits):
+    # exact for symmetric codes of <= 5 bits (an fp16 scale times a small
+    # integer), within 2^-16 relative per weight otherwise (8-bit codes, an
+    # fp16 zero-point), which widens the activations' window by 2^-16 |X||W^|
+    x_tie = O.TIE_REL + (0.0 if sym and bits <= 5 else 2.0 ** -16)
     res, sse_ref, xs = O.gptq_sequential(X0n, layers, bits=bits, group_size=group_size, sym=sym,
-                                         follow=follow, follow_x=fx)
+                                         follow=follow, follow_x=fx, tie_rel=tie_rel,
+                                         x_tie_rel=x_tie)
     for li, (o, L) in enumerate(zip(outs, layers)):
         d_in = L["W"].shape[1]
         got = follow[li]["codes"]
