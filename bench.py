@@ -388,10 +388,10 @@ def stage_work(spec, recon_route="hessian"):
         "hessian_flops": spec.n_tok * spec.d_in * (spec.d_in + 1),
         # read W, write codes + fp16 scales (+ zeros)
         "rtn_bytes": spec.d_out * spec.d_in * (wb + 0.5) + 2 * spec.d_out * n_groups + zero_bytes,
-        # two reconstruction errors: 2 N d_out d_in each (direct), or
-        # 2 d_out d_in^2 each from the Hessian
+        # two reconstruction errors: 2 N d_out d_in each (direct), or the
+        # lower triangle of dW^T dW, d_out d_in (d_in + 1) each, from the Hessian
         "recon_flops": (2 * 2 * spec.n_tok * spec.d_out * spec.d_in if recon_route == "direct"
-                        else 2 * 2 * spec.d_out * spec.d_in ** 2),
+                        else 2 * spec.d_out * spec.d_in * (spec.d_in + 1)),
         "weights": spec.d_out * spec.d_in,
     }
 
@@ -477,7 +477,7 @@ def gpu_arm(args, world, rank, local):
         # per-kernel rates from the serialised eager pass (work / event time)
         "xtx_tflops": rate(shares, "hessian_mma", 1e12),
         "rtn_gbs": rate(shares, "rtn", 1e9),
-        "recon_tflops": rate(shares, "recon_mma", 1e12),
+        "recon_tflops": rate(shares, "recon_mma" if args.recon == "direct" else "syrk_bf16", 1e12),
         "tf32x3_gemm_tflops": rate(shares, "gemm_tf32x3", 1e12),
         "gptq_block_gbs": rate(shares, "gptq_block", 1e9),
         "roofline": roof,
@@ -514,6 +514,7 @@ KERNEL_BOUND = {
     "gptq_block": ("hbm", "HBM copy", 1),
     "rtn": ("hbm", "HBM copy", 1),
     "qlinear": ("tensor", "bf16", 2),
+    "syrk_bf16": ("tensor", "bf16", 3),
 }
 
 

@@ -502,8 +502,10 @@ gq_status gq_selftest_bounded_wait(int arrive, uint64_t limit_ns, void *ws, size
  * The algorithmic work is counted in flops (2 per multiply-add) for
  * HESSIAN_MMA (symmetric half of X^T X), POTRF_TRSM, BLOCK_INVERSE,
  * GEMM_TF32X3 (the fp32 product; lower-triangle calls count the triangle),
- * RECON_MMA (one product (W - W^) X^T) and QLINEAR (one product W^ X^T:
- * 2 n_tok d_out d_in), and in bytes that must cross
+ * RECON_MMA (one product (W - W^) X^T), QLINEAR (one product W^ X^T:
+ * 2 n_tok d_out d_in) and SYRK_BF16 (the lower triangle of dW^T dW in the
+ * error from the Hessian, three bf16 products: d_in (d_in + 1) d_out),
+ * and in bytes that must cross
  * HBM for GPTQ_BLOCK (the block's working weights read, Err written, the U
  * block, codes and scales) and RTN (W read, codes, scales and zeros
  * written).  One session at a time per process; the calls are thread safe.
@@ -517,7 +519,8 @@ typedef enum {
   GQ_KERNEL_RTN = 5,
   GQ_KERNEL_RECON_MMA = 6,
   GQ_KERNEL_QLINEAR = 7,
-  GQ_KERNEL_COUNT = 8
+  GQ_KERNEL_SYRK_BF16 = 8,
+  GQ_KERNEL_COUNT = 9
 } gq_kernel;
 
 gq_status gq_kernel_timer_start(uint32_t mask, int32_t capacity);

@@ -81,6 +81,7 @@ __all__ = [
     "round_to_grid", "round_error_carried_forward", "gptq_fixed_grid",
     "gptq_layer", "awq_channel_scales", "awq_apply", "awq_rtn_search", "w4a16_matmul",
     "round_to_bf16", "gelu_tanh", "apply_layer", "gptq_sequential", "TIE_TOL", "TIE_REL",
+    "QUOT_REL",
 ]
 
 
@@ -364,14 +365,18 @@ def _fp16_tie_rel(s32):
 # 2^-20, the bound of the split's product error; the measured divergences of
 # the column loop at d_in up to 28672 all lie inside this window, at about a
 # tenth of the count it predicts (the fp32 accumulation errors mostly
-# cancel).  A decision is a tie when w/s lies within max(TIE_TOL, TIE_REL *
-# E/s) steps of k + 1/2; TIE_TOL = 1e-6 steps covers the fp32 representation
-# of the weight and the division.  A scale is a tie when its fp32 value lies
+# cancel).  A decision is a tie when w/s lies within max(TIE_TOL,
+# QUOT_REL |w/s|, TIE_REL * E/s) steps of k + 1/2: the fp32 weight (one
+# rounding, 2^-24 relative) and the correctly rounded quotient (2^-24) put
+# w/s within 2^-23 |w/s| steps of the fp64 quotient, covered twice over by
+# QUOT_REL = 2^-22 (1.5e-5 steps at |w/s| = 127, the 8-bit range; 2e-6 at
+# 4 bits); TIE_TOL = 1e-6 steps is the floor near zero.  A scale is a tie when its fp32 value lies
 # within the same relative distance (the window on the group's extreme,
 # divided by the extreme) of an fp16 rounding boundary; an affine zero-point
 # when -min'/s lies within the window of k + 1/2.
 TIE_TOL = 1e-6
 TIE_REL = 2.0 ** -20
+QUOT_REL = 2.0 ** -22
 
 
 def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
@@ -449,9 +454,11 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                 mx = np.maximum(np.max(v, axis=-1), F32(0))
                 ext = (mx - mn).astype(np.float64)
                 s32 = (mx - mn) / F32(2 ** bits - 1)
-                zd = _tie_dist(-mn.astype(np.float64) / s.astype(np.float64))
+                zr = -mn.astype(np.float64) / s.astype(np.float64)
+                zd = _tie_dist(zr)
                 win_s = np.maximum(tie_tol, ev / np.where(ext > 0, ext, 1.0))
-                win_z = np.maximum(tie_tol, ev / s.astype(np.float64))
+                win_z = np.maximum(np.maximum(tie_tol, QUOT_REL * np.abs(zr)),
+                                   ev / s.astype(np.float64))
                 sd = _fp16_tie_rel(s32)
                 # compare each distance with its own window: report the one
                 # that is a tie (the smaller ratio)
@@ -494,7 +501,8 @@ def gptq_quantize(W, U, bits=4, group_size=-1, block_size=128, sym=True,
                 s64 = s.astype(np.float64)
                 r = w.astype(F32).astype(np.float64) / s64
                 dist = _tie_dist(r)
-                win = np.maximum(tie_tol, tie_rel * Eb[:, j] / s64)
+                win = np.maximum(np.maximum(tie_tol, QUOT_REL * np.abs(r)),
+                                 tie_rel * Eb[:, j] / s64)
                 expected += float(np.sum(np.minimum(1.0, 2.0 * win)))
                 take = ((dist < win) & (f_codes[:, col] != c)
                         & (np.abs(f_codes[:, col] - c) == 1))

@@ -893,7 +893,7 @@ gq_status launch_syrk_dot_bf16x3(int M, int K, const uint16_t *A_h, const uint16
   cudaFuncSetAttribute(gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(SMEM_BYTES));
   const int n_pairs = a.n_tiles < sms / 2 ? a.n_tiles : sms / 2;
-  const int slot = timer_begin(GQ_KERNEL_GEMM_TF32X3, st);
+  const int slot = timer_begin(GQ_KERNEL_SYRK_BF16, st);
   gemm_pair_kernel<true><<<2 * n_pairs, NUM_THREADS, SMEM_BYTES, st>>>(tH, tL, tC, a);
   count_launch();
   timer_end(slot, st, static_cast<double>(M) * (M + 1) * K);

@@ -63,8 +63,8 @@ gq_status launch_rtn(const void *W, gq_dtype dt, int64_t d_out, int64_t d_in, in
 
 struct HessPlan {
   int n_bi, n_bj, n_tiles, n_split, nkb_total, kb_per_split;
-  int pairs;  // 256 x 256 tiles on CTA pairs (else 128 x 256 on single CTAs)
-  size_t ws_bytes;
+  int align_groups, align_waves;  // token-alignment counters (0: none)
+  size_t off_align, ws_bytes;
 };
 HessPlan hessian_plan(int64_t n_tok, int64_t d_in);
 gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, void *ws,

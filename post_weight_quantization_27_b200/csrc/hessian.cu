@@ -12,12 +12,15 @@
 //     B = X^T are both "MN-major" operands of tcgen05.mma (columns of X
 //     are contiguous), so no transpose is ever materialised.
 //   * warp 1 (one elected thread) issues tcgen05.mma kind::f16 bf16 x bf16
-//     -> fp32 into one of two 256-column TMEM accumulators.  Every 1024
+//     -> fp32 into one of two 256-column TMEM accumulators.  Every 512
 //     tokens the accumulator is handed to the epilogue and the other one
 //     is used, so the tensor pipe never waits for the drain.
-//   * warps 2..9 add each 1024-token partial into fp32 registers (one TMEM
+//   * warps 2..9 add each 512-token partial into fp32 registers (one TMEM
 //     lane = one tile row per thread).  Short accumulation chains inside
 //     the tensor core keep the fp32 error small at 262144 tokens.
+//   * the producers of a wave of tiles stay within a few token steps of
+//     each other (see ALIGN_G), so the L2 keeps serving the X slabs they
+//     share.
 //   * tiles are split over token ranges when there are too few tiles for
 //     the SMs, or when a split makes the last wave of tiles less ragged;
 //     each (split, tile) writes its raw partial tile to the workspace and
@@ -35,18 +38,13 @@ namespace gq {
 namespace {
 
 #ifndef GQ_HESS_CHUNK_KB
-#define GQ_HESS_CHUNK_KB 2
+#define GQ_HESS_CHUNK_KB 8
 #endif
 // K-blocks (of 64 tokens) accumulated inside TMEM before the partial is
 // drained into fp32 registers.  The tensor core's fp32 accumulation error
-// grows with the length of this chain; 2 (128 tokens) keeps H within a few
-// fp32 ulps of the exact sum while the drain still overlaps the MMAs.
-#ifndef GQ_HESS_PAIR_MIN_D
-#define GQ_HESS_PAIR_MIN_D (1 << 30)
-#endif
-// Smallest d_in computed on CTA pairs (256 x 256 tiles); below it, single
-// CTAs with 128 x 256 tiles.
-constexpr int64_t PAIR_MIN_D = GQ_HESS_PAIR_MIN_D;
+// grows with the length of this chain (measured against 128-token chains:
+// 7.9e-7 relative at 512 tokens, 1.8e-6 at 1024), the drain's cost shrinks
+// with it: 8 (512 tokens) ran the 8192-wide layer 25% faster than 2.
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, CHUNK_KB = GQ_HESS_CHUNK_KB;
 constexpr int A_BYTES = BM * BK * 2;  // two 64x64 boxes
 constexpr int B_BYTES = BN * BK * 2;  // four 64x64 boxes
@@ -60,7 +58,42 @@ struct HessArgs {
   int n_bi, n_bj, n_tiles, n_split, kb_per_split, nkb_total;
   float *P;
   int *status;
+  int *align;        // token-alignment counters [waves][align_groups], zeroed; or NULL
+  int align_groups;
 };
+
+// Token alignment of the tiles in flight.  All tiles of a wave of the
+// persistent grid read the same token rows of X at about the same time, so
+// the L2 serves the X slabs they share -- as long as the CTAs stay close in
+// the token dimension.  Over many waves they drift apart (a CTA that misses
+// in L2 slows down and misses more), and at d = 28672 the tiles re-read X
+// from DRAM ~120 times.  So the producers of a wave count the groups of
+// ALIGN_G k-blocks they have issued, and a producer does not run more than
+// ALIGN_LEAD groups ahead of the slowest CTA of its wave.  The wait is
+// short and soft: after ALIGN_WAIT_NS without progress (a CTA of the wave
+// is not resident, e.g. while another kernel holds SMs) the producer stops
+// waiting for the rest of the launch; it still counts its groups, so the
+// others are never held up by it.  Only the timing depends on this.
+#ifndef GQ_HESS_ALIGN
+#define GQ_HESS_ALIGN 1
+#endif
+constexpr int ALIGN_G = 8, ALIGN_LEAD = 4;
+constexpr uint64_t ALIGN_WAIT_NS = 20000;
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool wait_count(const int *p, int target) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(100);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if (globaltimer_ns() - t0 > ALIGN_WAIT_NS) return false;
+  }
+}
 
 // Tiles of row-block b are the column blocks b/2 .. n_bj-1 (a 128-row block
 // starting at 128b meets the diagonal in column block floor(128b/256)).
@@ -145,6 +178,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- TMA producer
     if (lane == 0) {
       bool ok = true;
+      bool align = a.align != nullptr;  // (only with one token range per tile)
       uint32_t it = 0;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         const int split = item / a.n_tiles, t = item % a.n_tiles;
@@ -152,7 +186,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         raster_tile(t, a.n_bi, a.n_bj, bi, bj);
         const int kb0 = split * a.kb_per_split;
         const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
+        const int wave = (item - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+        const int in_wave = min(static_cast<int>(gridDim.x), n_items - wave * static_cast<int>(gridDim.x));
+        int *cnt = a.align ? a.align + static_cast<size_t>(wave) * a.align_groups : nullptr;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int g = (kb - kb0) / ALIGN_G;
+          if (align && (kb - kb0) % ALIGN_G == 0 && g >= ALIGN_LEAD)
+            align = wait_count(cnt + g - ALIGN_LEAD, in_wave);
           const uint32_t s = it % STAGES, r = it / STAGES;
           if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
@@ -163,6 +203,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d(sa + BOX_BYTES, &tmX, &full[s], bi * BM + 64, tok);
 #pragma unroll
           for (int q = 0; q < 4; ++q) tma_load_2d(sb + q * BOX_BYTES, &tmX, &full[s], bj * BN + 64 * q, tok);
+          if (cnt && ((kb - kb0) % ALIGN_G == ALIGN_G - 1 || kb == kb1 - 1)) atomicAdd(cnt + g, 1);
         }
       }
       // every load issued must have landed before the CTA may exit
@@ -264,247 +305,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// ---------------------------------------------------------------- CTA pairs
-// The same sum on 256 x 256 upper tiles (bi <= bj), each computed by a pair
-// of CTAs on two SMs (a cluster of two; tcgen05 cta_group::2): CTA r stages
-// X columns 256 bi + 128 r .. (its half of A) and 256 bj + 128 r .. (its
-// half of B); CTA 0 issues MMAs of M = 256, N = 256 that read both CTAs'
-// halves, and each CTA's TMEM receives its 128 rows x 256 columns.  Per SM
-// and flop that is two thirds of the one-CTA kernel's operand traffic (the
-// B slab is shared by the pair), which bounds the one-CTA kernel's tensor
-// pipe.  The partial tiles are 256 x 256, in row-major order over the
-// upper tiles.
-//   full[s]       per CTA: its own TMA loads landed
-//   empty[s]      per CTA: the MMAs reading stage s completed (multicast commit)
-//   acc_full[b]   per CTA: a chunk's MMAs completed (multicast commit)
-//   acc_empty[b]  CTA 0: both CTAs' epilogues drained accumulator b (16 warps)
-// The MMA issuer waits for its own CTA's full[s] and for the peer's, which
-// the peer's producer forwards to CTA 0's peer_full[s] once its loads landed.
-constexpr int PB = 256;                  // pair tile edge
-constexpr int P_STAGE_BYTES = 2 * A_BYTES;  // A half + B half, 128 columns each
-constexpr int P_STAGES = 6;
-constexpr size_t P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 256;
-
-__host__ __device__ __forceinline__ int64_t pair_row_start(int64_t b, int64_t n_b) {
-  return b * n_b - b * (b - 1) / 2;
-}
-
-// Processing position r -> upper tile (bi, bj), groups of RASTER_G row
-// blocks, column block by column block inside a group.
-__device__ __forceinline__ void pair_raster_tile(int r, int n_b, int &bi, int &bj) {
-  for (int b0 = 0; b0 < n_b; b0 += RASTER_G) {
-    const int b1 = min(b0 + RASTER_G, n_b);
-    // column j >= b0 holds the group's rows b <= j: min(b1, j + 1) - b0 of them
-    int count = 0;
-    for (int j = b0; j < n_b; ++j) count += min(b1, j + 1) - b0;
-    if (r >= count) {
-      r -= count;
-      continue;
-    }
-    for (int j = b0; j < n_b; ++j) {
-      const int c = min(b1, j + 1) - b0;
-      if (r < c) {
-        bi = b0 + r;
-        bj = j;
-        return;
-      }
-      r -= c;
-    }
-  }
-  bi = 0;
-  bj = 0;
-}
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
-    hessian_pair_kernel(const __grid_constant__ CUtensorMap tmX, HessArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + P_STAGES * P_STAGE_BYTES);
-  uint64_t *full = bars;
-  uint64_t *peer_full = bars + P_STAGES;
-  uint64_t *empty = bars + 2 * P_STAGES;
-  uint64_t *acc_full = bars + 3 * P_STAGES;
-  uint64_t *acc_empty = acc_full + 2;
-  uint64_t *drain = acc_empty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int pair = static_cast<int>(blockIdx.x >> 1), n_pairs = static_cast<int>(gridDim.x >> 1);
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < P_STAGES; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&peer_full[st], 1);
-      mbar_init(&empty[st], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 16);
-    }
-    mbar_init(drain, 1);
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  if (threadIdx.x == 0) tma_prefetch_desc(&tmX);
-  tc_fence_before();
-  cluster_sync();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const int n_items = a.n_tiles * a.n_split;
-  const int half0 = static_cast<int>(rank) * (PB / 2);
-
-  if (warp == 0) {
-    // ---------------- TMA producer (each CTA its own halves)
-    if (lane == 0) {
-      bool ok = true;
-      uint32_t it = 0;
-      for (int item = pair; item < n_items && ok; item += n_pairs) {
-        const int split = item / a.n_tiles, t = item % a.n_tiles;
-        int bi, bj;
-        pair_raster_tile(t, a.n_bi, bi, bj);
-        const int kb0 = split * a.kb_per_split;
-        const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const uint32_t s = it % P_STAGES, r = it / P_STAGES;
-          if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[s], P_STAGE_BYTES);
-          uint8_t *sa = smem + s * P_STAGE_BYTES;
-          uint8_t *sb = sa + A_BYTES;
-          const int tok = kb * BK;
-          tma_load_2d(sa, &tmX, &full[s], bi * PB + half0, tok);
-          tma_load_2d(sa + BOX_BYTES, &tmX, &full[s], bi * PB + half0 + 64, tok);
-          tma_load_2d(sb, &tmX, &full[s], bj * PB + half0, tok);
-          tma_load_2d(sb + BOX_BYTES, &tmX, &full[s], bj * PB + half0 + 64, tok);
-        }
-      }
-      const uint32_t n_wait = it < P_STAGES ? it : P_STAGES;
-      for (uint32_t k = 0; k < n_wait; ++k) {
-        const uint32_t j = it - 1 - k;
-        if (!mbar_wait(&full[j % P_STAGES], (j / P_STAGES) & 1)) ok = false;
-      }
-      if (!ok) set_status(a.status, kDevTimeout);
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (CTA 0 of the pair)
-    if (lane == 0 && rank == 0) {
-      bool ok = true;
-      uint32_t it = 0, ch = 0;
-      constexpr uint32_t idesc = idesc_bf16_f32(PB, PB, true, true);
-      for (int item = pair; item < n_items && ok; item += n_pairs) {
-        const int split = item / a.n_tiles;
-        const int kb0 = split * a.kb_per_split;
-        const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
-        for (int c0 = kb0; c0 < kb1 && ok; c0 += CHUNK_KB, ++ch) {
-          const int c1 = min(c0 + CHUNK_KB, kb1);
-          const uint32_t buf = ch & 1, use = ch >> 1;
-          if (!mbar_wait_cluster(&acc_empty[buf], (use & 1) ^ 1)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + buf * PB;
-          for (int kb = c0; kb < c1; ++kb, ++it) {
-            const uint32_t s = it % P_STAGES, r = it / P_STAGES;
-            if (!mbar_wait(&full[s], r & 1) || !mbar_wait_cluster(&peer_full[s], r & 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(smem + s * P_STAGE_BYTES);
-            const uint32_t sb = sa + A_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(sa + kk * 2048, BOX_BYTES, 1024);
-              const uint64_t bd = smem_desc_sw128(sb + kk * 2048, BOX_BYTES, 1024);
-              mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > c0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit_pair(&empty[s], 3);
-          }
-          if (!ok) break;
-          mma_commit_pair(&acc_full[buf], 3);
-        }
-      }
-      mma_commit_pair(drain, 1);
-      if (!mbar_wait(drain, 0)) ok = false;
-      if (!ok) set_status(a.status, kDevTimeout);
-    } else if (lane == 0) {
-      // CTA 1: forward the landing of each stage to CTA 0's MMA issuer
-      bool ok = true;
-      uint32_t it = 0;
-      for (int item = pair; item < n_items && ok; item += n_pairs) {
-        const int split = item / a.n_tiles;
-        const int kb0 = split * a.kb_per_split;
-        const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const uint32_t s = it % P_STAGES, r = it / P_STAGES;
-          if (!mbar_wait(&full[s], r & 1)) { ok = false; break; }
-          mbar_arrive_cluster(&peer_full[s], 0);
-        }
-      }
-      if (!ok) set_status(a.status, kDevTimeout);
-    }
-  } else {
-    // ---------------- epilogue: warps 2..9 of each CTA
-    const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int row = quarter * 32 + lane;
-    uint32_t ch = 0;
-    bool ok = true;
-    for (int item = pair; item < n_items && ok; item += n_pairs) {
-      const int split = item / a.n_tiles;
-      const int kb0 = split * a.kb_per_split;
-      const int kb1 = min(kb0 + a.kb_per_split, a.nkb_total);
-      float m[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) m[i] = 0.0f;
-      for (int c0 = kb0; c0 < kb1; c0 += CHUNK_KB, ++ch) {
-        const uint32_t buf = ch & 1, use = ch >> 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], use & 1));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * PB + half * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) m[c * 32 + i] += v[i];
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(&acc_empty[buf], 0);
-      }
-      if (!ok) break;
-      int bi, bj;
-      pair_raster_tile(item % a.n_tiles, a.n_bi, bi, bj);
-      const size_t slot = static_cast<size_t>(split) * a.n_tiles +
-                          static_cast<size_t>(pair_row_start(bi, a.n_bi) + (bj - bi));
-      float *dst = a.P + (slot * PB + half0 + row) * PB + half * 128;
-#pragma unroll
-      for (int c = 0; c < 128; c += 4)
-        *reinterpret_cast<float4 *>(dst + c) = make_float4(m[c], m[c + 1], m[c + 2], m[c + 3]);
-    }
-    if (!ok && lane == 0) set_status(a.status, kDevTimeout);
-  }
-
-  tc_fence_before();
-  __syncwarp();
-  cluster_sync();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, TMEM_COLS);
-  }
-}
-
 // H[i][j] (i <= j) := H[i][j] + 2 * sum_s P_s(i, j) (without the H term
 // when !accumulate); H[j][i] := H[i][j].
 __global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__ H, int d,
                                                              const float *__restrict__ P,
                                                              int n_tiles, int n_bj, int n_split,
-                                                             const int *status, int accumulate,
-                                                             int pairs) {
+                                                             const int *status, int accumulate) {
   const int bi = blockIdx.y, bj = blockIdx.x;
   if (bi > bj) return;
   __shared__ float tile[32][33];
@@ -514,18 +320,11 @@ __global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__
     const int i = bi * 32 + r, j = bj * 32 + tx;
     float val = 0.0f;
     if (i < d && j < d && i <= j) {
+      const int tb = i / BM, tj = j / BN;
+      const int t = static_cast<int>(tile_row_start(tb, n_bj)) + (tj - (tb >> 1));
       float sum = 0.0f;
-      if (pairs) {
-        const int tb = i / PB, tj = j / PB;
-        const int t = static_cast<int>(pair_row_start(tb, n_bj)) + (tj - tb);
-        for (int s = 0; s < n_split; ++s)
-          sum += P[(static_cast<size_t>(s * n_tiles + t) * PB + (i - tb * PB)) * PB + (j - tj * PB)];
-      } else {
-        const int tb = i / BM, tj = j / BN;
-        const int t = static_cast<int>(tile_row_start(tb, n_bj)) + (tj - (tb >> 1));
-        for (int s = 0; s < n_split; ++s)
-          sum += P[(static_cast<size_t>(s * n_tiles + t) * BM + (i - tb * BM)) * BN + (j - tj * BN)];
-      }
+      for (int s = 0; s < n_split; ++s)
+        sum += P[(static_cast<size_t>(s * n_tiles + t) * BM + (i - tb * BM)) * BN + (j - tj * BN)];
       val = accumulate ? H[static_cast<size_t>(i) * d + j] + 2.0f * sum : 2.0f * sum;
       if (bad) val = __int_as_float(0x7fc00000);
       H[static_cast<size_t>(i) * d + j] = val;
@@ -543,18 +342,12 @@ __global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__
 
 HessPlan hessian_plan(int64_t n_tok, int64_t d_in) {
   HessPlan p{};
-  p.pairs = d_in >= PAIR_MIN_D ? 1 : 0;
-  if (p.pairs) {
-    p.n_bi = p.n_bj = static_cast<int>((d_in + PB - 1) / PB);
-    p.n_tiles = static_cast<int>(pair_row_start(p.n_bi, p.n_bi));
-  } else {
-    p.n_bi = static_cast<int>((d_in + BM - 1) / BM);
-    p.n_bj = static_cast<int>((d_in + BN - 1) / BN);
-    p.n_tiles = static_cast<int>(tile_row_start(p.n_bi, p.n_bj));
-  }
+  p.n_bi = static_cast<int>((d_in + BM - 1) / BM);
+  p.n_bj = static_cast<int>((d_in + BN - 1) / BN);
+  p.n_tiles = static_cast<int>(tile_row_start(p.n_bi, p.n_bj));
   p.nkb_total = static_cast<int>((n_tok + BK - 1) / BK);
   int split = 1;
-  const int sms = p.pairs ? num_sms() / 2 : num_sms();  // concurrent work items
+  const int sms = num_sms();
   const int target = 2 * sms;
   if (p.nkb_total > 0 && p.n_tiles < target) {
     const int want = (target + p.n_tiles - 1) / p.n_tiles;
@@ -582,8 +375,14 @@ HessPlan hessian_plan(int64_t n_tok, int64_t d_in) {
     p.kb_per_split = (p.nkb_total + split - 1) / split;
     p.n_split = (p.nkb_total + p.kb_per_split - 1) / p.kb_per_split;
   }
-  const size_t tile_elems = p.pairs ? static_cast<size_t>(PB) * PB : static_cast<size_t>(BM) * BN;
-  p.ws_bytes = kWsHeader + static_cast<size_t>(p.n_split) * p.n_tiles * tile_elems * sizeof(float);
+  p.off_align = kWsHeader + static_cast<size_t>(p.n_split) * p.n_tiles * BM * BN * sizeof(float);
+  if (GQ_HESS_ALIGN && p.n_split == 1 && p.n_tiles > sms) {
+    const int grid = p.n_tiles < sms ? p.n_tiles : sms;
+    p.align_waves = (p.n_tiles + grid - 1) / grid;
+    p.align_groups = (p.nkb_total + ALIGN_G - 1) / ALIGN_G;
+  }
+  p.ws_bytes = p.off_align + round_up(static_cast<size_t>(p.align_waves) * p.align_groups *
+                                          sizeof(int), 256);
   return p;
 }
 
@@ -598,20 +397,22 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
     gq_status s = make_tmap_2d(&tm, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d_in, n_tok, d_in,
                                64, BK);
     if (s != GQ_OK) return s;
-    HessArgs a{p.n_bi, p.n_bj, p.n_tiles, p.n_split, p.kb_per_split, p.nkb_total, P, status};
+    int *align = nullptr;
+    if (p.align_groups > 0) {
+      align = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + p.off_align);
+      if (cudaMemsetAsync(align, 0,
+                          static_cast<size_t>(p.align_waves) * p.align_groups * sizeof(int),
+                          st) != cudaSuccess)
+        return check_launch("memset");
+    }
+    HessArgs a{p.n_bi, p.n_bj, p.n_tiles, p.n_split, p.kb_per_split, p.nkb_total, P, status,
+               align, p.align_groups};
     const int sms = num_sms();
     const int slot = timer_begin(GQ_KERNEL_HESSIAN_MMA, st);
-    if (p.pairs) {
-      cudaFuncSetAttribute(hessian_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(P_SMEM_BYTES));
-      const int n_pairs = n_items < sms / 2 ? n_items : sms / 2;
-      hessian_pair_kernel<<<2 * n_pairs, NUM_THREADS, P_SMEM_BYTES, st>>>(tm, a);
-    } else {
-      cudaFuncSetAttribute(hessian_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(SMEM_BYTES));
-      const int grid = n_items < sms ? n_items : sms;
-      hessian_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, a);
-    }
+    cudaFuncSetAttribute(hessian_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(SMEM_BYTES));
+    const int grid = n_items < sms ? n_items : sms;
+    hessian_mma_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, a);
     count_launch();
     // symmetric half of X^T X: n_tok d_in (d_in + 1) flops
     timer_end(slot, st, static_cast<double>(n_tok) * d_in * (d_in + 1));
@@ -621,7 +422,7 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
   const int nb = static_cast<int>((d_in + 31) / 32);
   hessian_finish_kernel<<<dim3(nb, nb), 256, 0, st>>>(H, static_cast<int>(d_in), P, p.n_tiles,
                                                       p.n_bj, p.n_split, status,
-                                                      accumulate ? 1 : 0, p.pairs);
+                                                      accumulate ? 1 : 0);
   count_launch();
   return check_launch("hessian_finish_kernel");
 }

@@ -534,10 +534,10 @@ def awq_rtn_search(W: torch.Tensor, H: torch.Tensor, X: torch.Tensor, bits: int 
 
 # gq_kernel values (include/gq.h) and the unit of each kernel's work figure
 KERNELS = ("hessian_mma", "potrf_trsm", "block_inverse", "gemm_tf32x3", "gptq_block", "rtn",
-           "recon_mma", "qlinear")
+           "recon_mma", "qlinear", "syrk_bf16")
 KERNEL_UNITS = {"hessian_mma": "flop", "potrf_trsm": "flop", "block_inverse": "flop",
                 "gemm_tf32x3": "flop", "gptq_block": "byte", "rtn": "byte", "recon_mma": "flop",
-                "qlinear": "flop"}
+                "qlinear": "flop", "syrk_bf16": "flop"}
 
 
 def kernel_timer_start(kernels, capacity: int) -> None:

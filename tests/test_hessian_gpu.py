@@ -19,8 +19,8 @@ def _x(n_tok, d_in, seed):
     return I.make_x(spec)
 
 
-# d_in >= 1024 runs on CTA pairs (256 x 256 tiles): 1032 and 1304 leave
-# ragged pair tiles, 20000 x 1304 splits the tokens over few tiles
+# ragged tiles in both directions (136, 264, 520, 1032, 1304); 20000 x 1304
+# splits the tokens over few tiles; 70000 x 256 runs several waves
 @pytest.mark.parametrize("n_tok,d_in", [(64, 8), (100, 136), (2048, 768), (1000, 264),
                                         (4097, 520), (2560, 3072), (300, 1032), (70000, 256),
                                         (20000, 1304)])

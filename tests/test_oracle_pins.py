@@ -848,6 +848,28 @@ def test_tie_window_grows_with_the_updates_a_weight_received():
         assert rf.n_followed == int(adopted)
 
 
+def test_tie_window_scales_with_the_quotient():
+    """Near the end of the 8-bit range the fp32 weight and quotient are
+    within 2^-23 |w/s| steps of the exact quotient, far more than TIE_TOL:
+    the window's floor is QUOT_REL |w/s|.  w/s = 100.5 + off with off one
+    fp32 ulp of the quotient (inside 2^-22 * 100.5) is a tie, eight ulps is
+    not."""
+    s = 2.0 ** -7                              # absmax 127 s: fp16-exact scale s
+    U = np.eye(4)
+    win = O.QUOT_REL * 100.5
+    assert win > O.TIE_TOL
+    for off, adopted in ((2.0 ** -17, True), (8 * 2.0 ** -17, False)):
+        W = np.array([[127 * s, (100.5 + off) * s, 3 * s, -5 * s]])
+        r = O.gptq_quantize(W, U, group_size=-1, bits=8)
+        assert float(r.scales[0, 0]) == s and r.codes[0, 1] == 101
+        other = r.codes.copy()
+        other[0, 1] = 100
+        rf = O.gptq_quantize(W, U, group_size=-1, bits=8,
+                             follow=dict(codes=other, scales=r.scales))
+        assert (rf.codes[0, 1] == 100) == adopted, (off, win)
+        assert rf.n_followed == int(adopted)
+
+
 def test_apply_layer_follow_only_at_rounding_ties():
     """The replay of bf16 roundings takes the other value only where it is
     the rounding of a value within the fp32 error of the fp64 result

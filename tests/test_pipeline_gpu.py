@@ -138,6 +138,11 @@ def test_sequential_pipeline_matches_oracle(bits, group_size, sym):
         d_in = L["W"].shape[1]
         got = follow[li]["codes"]
         agree = np.mean(got == res[li].codes)
+        diff = np.argwhere(got != res[li].codes)
+        print(f"[pipeline {bits}-bit layer {li}] codes agree {agree:.6f} ({len(diff)} differ, "
+              f"rows {sorted(set(diff[:, 0].tolist()))[:8]}), ties followed "
+              f"{res[li].n_followed}, expected {res[li].expected_ties:.1f}, tie_rel "
+              f"{tie_rel[li]:.2e}, X equal {np.mean(fx[li] == xs[li + 1]):.6f}")
         assert agree >= 0.999 and np.max(np.abs(got - res[li].codes)) <= 1, (li, agree)
         assert abs(sse[li] - sse_ref[li]) <= 1e-3 * sse_ref[li], (li, sse[li], sse_ref[li])
         assert np.array_equal(fx[li], xs[li + 1]), (li, np.mean(fx[li] == xs[li + 1]))
