@@ -8,13 +8,13 @@ stage by hand.
 
 The stages always run in path order (H -> damp/U -> GPTQ -> RTN -> recon),
 each as many times as --repeat says; a stage that is not listed still runs
-once if a later listed stage needs its output.  Prints one line per stage
-with its CUDA-event time.  "trace" is the error from the Hessian (tr(dW H
-dW^T) / 2) of the GPTQ layer (of the RTN layer when it is the only stage
-listed); "awq" is the activation-aware scaling search
-before RTN (20 values of alpha), which needs only H; "w4a16" multiplies the
-RTN layer with the first (at most 8192) tokens; "qlinear" applies it to them
-(token-major bf16 output, GELU).
+once if a listed stage needs its output.  Prints one line per stage with its
+CUDA-event time.  "recon" is the direct error ||(W - W^) X^T||^2 of the GPTQ
+and RTN layers; "trace" is the error from the Hessian (tr(dW H dW^T) / 2) of
+the GPTQ layer (of the RTN layer when GPTQ is not listed); "awq" is the
+activation-aware scaling search before RTN (20 values of alpha), which needs
+only H; "w4a16" multiplies the RTN layer with the first (at most 8192)
+tokens; "qlinear" applies it to them (token-major bf16 output, GELU).
 """
 from __future__ import annotations
 
@@ -34,16 +34,14 @@ def run(workload: int, layer: int, tokens: int | None, stages, repeat: int = 1) 
         spec = spec.with_tokens(tokens)
     W = I.make_weights(spec).cuda()
     X = I.make_x_device(spec, "cuda")
-    last = max(ORDER.index(s) for s in stages)
-    need = set(stages) | set(ORDER[:last])
-    if "recon" in stages:
-        need |= {"gptq"}
-    if stages == ["awq"]:  # needs only H
-        need = {"hessian", "awq"}
-    if stages == ["trace"]:  # needs H and a quantised layer (the RTN one)
-        need = {"hessian", "rtn", "trace"}
-    if set(stages) <= {"w4a16", "qlinear"}:  # need only the RTN output
-        need = {"rtn"} | set(stages)
+    # what each stage needs run before it
+    deps = {"hessian": set(), "solve": {"hessian"}, "gptq": {"hessian", "solve"}, "rtn": set(),
+            "recon": {"hessian", "solve", "gptq", "rtn"}, "awq": {"hessian"},
+            "trace": {"hessian"} | ({"solve", "gptq"} if "gptq" in stages else {"rtn"}),
+            "w4a16": {"rtn"}, "qlinear": {"rtn"}}
+    need = set(stages)
+    for st in stages:
+        need |= deps[st]
     times = {}
 
     def timed(name, fn):
