@@ -40,7 +40,8 @@ constexpr int TM = 128, TN = 128, TK = 32, STAGES = 3;
 constexpr int TILE_BYTES = TM * TK * 4;         // 16 KB, A or B tile
 constexpr int STAGE_BYTES = 4 * TILE_BYTES;     // A_h, A_l, B_h, B_l
 constexpr int C_BYTES = TM * TN * 4;            // a C tile: 4 boxes [128 rows][32 fp32]
-constexpr int C_STAGE_BYTES = C_BYTES / 2;      // staged half a tile (64 columns) at a time
+constexpr int C_STAGE_BYTES = C_BYTES / 2;      // two staging buffers of 32 columns each
+constexpr int C_BUF_BYTES = C_BYTES / 4;        // one buffer: [128 rows][32 fp32], one TMA box
 constexpr int NUM_THREADS = 320;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + C_STAGE_BYTES + 1024 + 256;
@@ -124,9 +125,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t *acc_full = bars + 3 * STAGES;
   uint64_t *acc_empty = acc_full + 2;
   uint64_t *drain = acc_empty + 2;
-  uint64_t *c_full = drain + 1;           // a C half tile landed in the staging buffer
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 1);
-  double *red = reinterpret_cast<double *>(bars + 16);  // dot mode: one per epilogue warp
+  uint64_t *c_full = drain + 1;           // [2]: a C chunk landed in staging buffer b
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 2);
+  double *red = reinterpret_cast<double *>(bars + 17);  // dot mode: one per epilogue warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&acc_empty[b], 4);
     }
     mbar_init(drain, 1);
-    mbar_init(c_full, 1);
+    mbar_init(&c_full[0], 1);
+    mbar_init(&c_full[1], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -273,27 +275,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ---------------- epilogue: warps 6..9 (thread = accumulator row).  The
-    // C tile passes through the staging buffer in two halves of 64 columns:
-    // half h is fetched by TMA (while the tile multiplies, for h = 0),
-    // combined with the accumulator in place and stored by TMA, then the
-    // buffer takes the next half.  After a failed wait the warps skip the
-    // work but keep meeting the named barriers, so none is left waiting.
+    // C tile passes through two staging buffers in chunks of 32 columns:
+    // while chunk k is combined with the accumulator in buffer k % 2 and
+    // stored by TMA, chunk k + 1 (of this tile or of the next) is already
+    // being fetched into the other buffer.  After a failed wait the warps
+    // skip the work but keep meeting the named barrier, so none is left
+    // waiting.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;               // row within the tile
     const bool leader = threadIdx.x == 192;          // issues the C copies
     const bool dot = a.dot != nullptr;
     const bool need_c = a.beta != 0.0f || a.lower != 0 || dot;
-    uint32_t ch = 0, n_c = 0;                        // tiles done, C halves waited for
+    constexpr int NCH = TN / 32;                     // chunks per tile
+    uint32_t ch = 0, cc = 0;                         // tiles done, chunks done
     bool ok = true;
-    auto load_half = [&](int t, int h) {
+    auto load_chunk = [&](int t, int h, uint32_t b) {
       int mt, nt;
       tile_of(a, t, mt, nt);
-      mbar_arrive_expect_tx(c_full, C_STAGE_BYTES);
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-        tma_load_2d(cs + q * (C_BYTES / 4), &tmC, c_full, nt * TN + 64 * h + 32 * q, mt * TM);
+      mbar_arrive_expect_tx(&c_full[b], C_BUF_BYTES);
+      tma_load_2d(cs + b * C_BUF_BYTES, &tmC, &c_full[b], nt * TN + 32 * h, mt * TM);
     };
-    if (leader && need_c && static_cast<int>(blockIdx.x) < a.n_tiles) load_half(blockIdx.x, 0);
+    if (leader && need_c && static_cast<int>(blockIdx.x) < a.n_tiles) load_chunk(blockIdx.x, 0, 0);
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++ch) {
       int mt, nt;
       tile_of(a, t, mt, nt);
@@ -305,42 +307,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool diag = a.lower && mt == nt;
       double rs = 0.0;  // dot mode: this row's sum
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        if (need_c && ok) ok = __all_sync(0xffffffffu, mbar_wait(c_full, n_c & 1));
-        ++n_c;
+      for (int h = 0; h < NCH; ++h, ++cc) {
+        const uint32_t b = cc & 1;
+        if (need_c && ok) ok = __all_sync(0xffffffffu, mbar_wait(&c_full[b], (cc >> 1) & 1));
+        if (leader && ok && need_c) {
+          // the other buffer's last store has been read out: fetch the next chunk into it
+          if (!dot) bulk_wait_group_read0();
+          if (h + 1 < NCH) {
+            load_chunk(t, h + 1, b ^ 1u);
+          } else {
+            const int tn = t + static_cast<int>(gridDim.x);
+            if (tn < a.n_tiles) load_chunk(tn, 0, b ^ 1u);
+          }
+        }
         if (ok) {
-#pragma unroll 1
-          for (int qq = 0; qq < 2; ++qq) {
-            const int q = 2 * h + qq;
-            float v[32];
-            tmem_ld32(taddr + q * 32, v);
-            uint8_t *row = cs + qq * (C_BYTES / 4) + r * 128;
-            if (dot) {
-              // (alpha acc) * C over the row (fp32 over 32 columns, fp64 across)
-              float part = 0.0f, pdiag = 0.0f;
+          float v[32];
+          tmem_ld32(taddr + h * 32, v);
+          uint8_t *row = cs + b * C_BUF_BYTES + r * 128;
+          if (dot) {
+            // (alpha acc) * C over the row (fp32 over 32 columns, fp64 across)
+            float part = 0.0f, pdiag = 0.0f;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
-                if (diag) {  // lower: keep n < m (counted twice below), the diagonal once
-                  const int n = nt * TN + 32 * q + 4 * c;
-                  if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
-                  if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
-                  if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
-                  if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
-                  if (n >= m) cv.x = 0.0f;
-                  if (n + 1 >= m) cv.y = 0.0f;
-                  if (n + 2 >= m) cv.z = 0.0f;
-                  if (n + 3 >= m) cv.w = 0.0f;
-                }
-                part = fmaf(a.alpha * v[4 * c], cv.x, part);
-                part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
-                part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
-                part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
+            for (int c = 0; c < 8; ++c) {
+              float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
+              if (diag) {  // lower: keep n < m (counted twice below), the diagonal once
+                const int n = nt * TN + 32 * h + 4 * c;
+                if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
+                if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
+                if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
+                if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
+                if (n >= m) cv.x = 0.0f;
+                if (n + 1 >= m) cv.y = 0.0f;
+                if (n + 2 >= m) cv.z = 0.0f;
+                if (n + 3 >= m) cv.w = 0.0f;
               }
-              rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) +
-                    static_cast<double>(pdiag);
-              continue;
+              part = fmaf(a.alpha * v[4 * c], cv.x, part);
+              part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
+              part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
+              part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
             }
+            rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) + static_cast<double>(pdiag);
+          } else {
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
@@ -352,7 +359,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               o.z = fmaf(a.beta, old.z, a.alpha * v[4 * c + 2]);
               o.w = fmaf(a.beta, old.w, a.alpha * v[4 * c + 3]);
               if (diag) {  // keep the strict upper part of a diagonal tile
-                const int n = nt * TN + 32 * q + 4 * c;
+                const int n = nt * TN + 32 * h + 4 * c;
                 if (n > m) o.x = old.x;
                 if (n + 1 > m) o.y = old.y;
                 if (n + 2 > m) o.z = old.z;
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        if (h == 1) {
+        if (h == NCH - 1) {
           // the accumulator buffer is free once its columns are in registers
           tc_fence_before();
           __syncwarp();
@@ -370,24 +377,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!dot) fence_proxy_async_smem();
         named_bar_sync(1, 128);
-        if (leader && ok) {
-          if (!dot) {
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq)
-              tma_store_2d(&tmC, cs + qq * (C_BYTES / 4), nt * TN + 64 * h + 32 * qq, mt * TM);
-            bulk_commit_group();
-            bulk_wait_group_read0();  // staging buffer reusable
-          }
-          if (need_c) {
-            if (h == 0) {
-              load_half(t, 1);
-            } else {
-              const int tn = t + static_cast<int>(gridDim.x);
-              if (tn < a.n_tiles) load_half(tn, 0);
-            }
-          }
+        if (leader && ok && !dot) {
+          tma_store_2d(&tmC, cs + b * C_BUF_BYTES, nt * TN + 32 * h, mt * TM);
+          bulk_commit_group();
+          // without C loads nothing else orders the buffer's reuse two chunks on
+          if (!need_c) bulk_wait_group_read0();
         }
-        named_bar_sync(1, 128);
       }
       if (dot) {
 #pragma unroll
@@ -456,9 +451,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   uint64_t *acc_full = bars + 3 * STAGES;
   uint64_t *acc_empty = acc_full + 2;
   uint64_t *drain = acc_empty + 2;
-  uint64_t *c_full = drain + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 1);
-  double *red = reinterpret_cast<double *>(bars + 16);
+  uint64_t *c_full = drain + 1;           // [2]: a C chunk landed in staging buffer b
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c_full + 2);
+  double *red = reinterpret_cast<double *>(bars + 17);  // dot mode: one per epilogue warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -474,7 +469,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&acc_empty[b], 8);
     }
     mbar_init(drain, 1);
-    mbar_init(c_full, 1);
+    mbar_init(&c_full[0], 1);
+    mbar_init(&c_full[1], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -627,24 +623,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (!ok) set_status(a.status, kDevTimeout);
     }
   } else {
-    // ---------------- epilogue: warps 6..9 of each CTA, its 128 rows
+    // ---------------- epilogue: warps 6..9 of each CTA, its 128 rows; the C
+    // tile in chunks of 32 columns through two staging buffers, as in the
+    // one-CTA kernel
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const bool leader = threadIdx.x == 192;
     const bool dot = a.dot != nullptr;
     const bool need_c = a.beta != 0.0f || a.lower != 0 || dot;
-    uint32_t ch = 0, n_c = 0;
+    constexpr int NCH = PN / 32;
+    uint32_t ch = 0, cc = 0;
     bool ok = true;
-    auto load_chunk = [&](int t, int h) {
+    auto load_chunk = [&](int t, int h, uint32_t b) {
       int mt, nt;
       tile_of(a, t, mt, nt);
-      mbar_arrive_expect_tx(c_full, C_STAGE_BYTES);
-#pragma unroll
-      for (int q = 0; q < 2; ++q)
-        tma_load_2d(cs + q * (C_BYTES / 4), &tmC, c_full, nt * PN + 64 * h + 32 * q,
-                    mt * PM + row0);
+      mbar_arrive_expect_tx(&c_full[b], C_BUF_BYTES);
+      tma_load_2d(cs + b * C_BUF_BYTES, &tmC, &c_full[b], nt * PN + 32 * h, mt * PM + row0);
     };
-    if (leader && need_c && pair < a.n_tiles) load_chunk(pair, 0);
+    if (leader && need_c && pair < a.n_tiles) load_chunk(pair, 0, 0);
     for (int t = pair; t < a.n_tiles; t += n_pairs, ++ch) {
       int mt, nt;
       tile_of(a, t, mt, nt);
@@ -656,41 +652,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const bool diag = a.lower && mt == nt;
       double rs = 0.0;
 #pragma unroll 1
-      for (int h = 0; h < PN / 64; ++h) {
-        if (need_c && ok) ok = __all_sync(0xffffffffu, mbar_wait(c_full, n_c & 1));
-        ++n_c;
+      for (int h = 0; h < NCH; ++h, ++cc) {
+        const uint32_t b = cc & 1;
+        if (need_c && ok) ok = __all_sync(0xffffffffu, mbar_wait(&c_full[b], (cc >> 1) & 1));
+        if (leader && ok && need_c) {
+          if (!dot) bulk_wait_group_read0();
+          if (h + 1 < NCH) {
+            load_chunk(t, h + 1, b ^ 1u);
+          } else {
+            const int tn = t + n_pairs;
+            if (tn < a.n_tiles) load_chunk(tn, 0, b ^ 1u);
+          }
+        }
         if (ok) {
-#pragma unroll 1
-          for (int qq = 0; qq < 2; ++qq) {
-            const int q = 2 * h + qq;
-            float v[32];
-            tmem_ld32(taddr + q * 32, v);
-            uint8_t *row = cs + qq * (C_BYTES / 4) + r * 128;
-            if (dot) {
-              float part = 0.0f, pdiag = 0.0f;
+          float v[32];
+          tmem_ld32(taddr + h * 32, v);
+          uint8_t *row = cs + b * C_BUF_BYTES + r * 128;
+          if (dot) {
+            float part = 0.0f, pdiag = 0.0f;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
-                if (diag) {
-                  const int n = nt * PN + 32 * q + 4 * c;
-                  if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
-                  if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
-                  if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
-                  if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
-                  if (n >= m) cv.x = 0.0f;
-                  if (n + 1 >= m) cv.y = 0.0f;
-                  if (n + 2 >= m) cv.z = 0.0f;
-                  if (n + 3 >= m) cv.w = 0.0f;
-                }
-                part = fmaf(a.alpha * v[4 * c], cv.x, part);
-                part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
-                part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
-                part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
+            for (int c = 0; c < 8; ++c) {
+              float4 cv = *reinterpret_cast<const float4 *>(row + ((c ^ (r & 7)) << 4));
+              if (diag) {
+                const int n = nt * PN + 32 * h + 4 * c;
+                if (n == m) pdiag = fmaf(a.alpha * v[4 * c], cv.x, pdiag);
+                if (n + 1 == m) pdiag = fmaf(a.alpha * v[4 * c + 1], cv.y, pdiag);
+                if (n + 2 == m) pdiag = fmaf(a.alpha * v[4 * c + 2], cv.z, pdiag);
+                if (n + 3 == m) pdiag = fmaf(a.alpha * v[4 * c + 3], cv.w, pdiag);
+                if (n >= m) cv.x = 0.0f;
+                if (n + 1 >= m) cv.y = 0.0f;
+                if (n + 2 >= m) cv.z = 0.0f;
+                if (n + 3 >= m) cv.w = 0.0f;
               }
-              rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) +
-                    static_cast<double>(pdiag);
-              continue;
+              part = fmaf(a.alpha * v[4 * c], cv.x, part);
+              part = fmaf(a.alpha * v[4 * c + 1], cv.y, part);
+              part = fmaf(a.alpha * v[4 * c + 2], cv.z, part);
+              part = fmaf(a.alpha * v[4 * c + 3], cv.w, part);
             }
+            rs += (a.lower ? 2.0 : 1.0) * static_cast<double>(part) + static_cast<double>(pdiag);
+          } else {
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               float4 *p = reinterpret_cast<float4 *>(row + ((c ^ (r & 7)) << 4));
@@ -701,7 +701,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               o.z = fmaf(a.beta, old.z, a.alpha * v[4 * c + 2]);
               o.w = fmaf(a.beta, old.w, a.alpha * v[4 * c + 3]);
               if (diag) {
-                const int n = nt * PN + 32 * q + 4 * c;
+                const int n = nt * PN + 32 * h + 4 * c;
                 if (n > m) o.x = old.x;
                 if (n + 1 > m) o.y = old.y;
                 if (n + 2 > m) o.z = old.z;
@@ -711,7 +711,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        if (h == PN / 64 - 1) {
+        if (h == NCH - 1) {
           // both CTAs' epilogues free the accumulator on CTA 0's barrier
           tc_fence_before();
           __syncwarp();
@@ -719,25 +719,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         if (!dot) fence_proxy_async_smem();
         named_bar_sync(1, 128);
-        if (leader && ok) {
-          if (!dot) {
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq)
-              tma_store_2d(&tmC, cs + qq * (C_BYTES / 4), nt * PN + 64 * h + 32 * qq,
-                           mt * PM + row0);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-          }
-          if (need_c) {
-            if (h + 1 < PN / 64) {
-              load_chunk(t, h + 1);
-            } else {
-              const int tn = t + n_pairs;
-              if (tn < a.n_tiles) load_chunk(tn, 0);
-            }
-          }
+        if (leader && ok && !dot) {
+          tma_store_2d(&tmC, cs + b * C_BUF_BYTES, nt * PN + 32 * h, mt * PM + row0);
+          bulk_commit_group();
+          if (!need_c) bulk_wait_group_read0();
         }
-        named_bar_sync(1, 128);
       }
       if (dot) {
 #pragma unroll

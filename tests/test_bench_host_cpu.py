@@ -72,10 +72,10 @@ def test_every_timed_kernel_has_a_ceiling():
 
 
 def test_traffic_table_parses():
-    t = bench.profiled_traffic("potrf_trsm", 2)
+    t = bench.profiled_traffic("hessian_mma", 5)
     assert t is not None and t > 0
-    assert bench.profiled_traffic("potrf_trsm", 99) is None
-    assert bench.profiled_traffic("no_such_kernel", 2) is None
+    assert bench.profiled_traffic("hessian_mma", 99) is None
+    assert bench.profiled_traffic("no_such_kernel", 5) is None
 
 
 def test_rate():
