@@ -290,6 +290,14 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
     import torch
     from post_weight_quantization_27_b200 import gq
     main, sides = streams if streams is not None else make_streams(n_streams)
+    sched = schedule(runs, n_streams)
+    if host is not None:
+        # the inputs come in on their own stream, in the order the layers
+        # run, so that a layer's copy overlaps the compute of the layers
+        # before it; the results go back on another
+        h2d_st, d2h_st = torch.cuda.Stream(), torch.cuda.Stream()
+        order = [i for pos in range(max(len(x) for x in sched))
+                 for x in sched if pos < len(x) for i in [x[pos]]]
     g = torch.cuda.CUDAGraph()
     events = []
     n0 = gq.launch_count()
@@ -300,14 +308,23 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
         fork.record(main)
         for sd in sides:
             sd.wait_event(fork)
-        for si, idxs in enumerate(schedule(runs, n_streams)):
+        ready = {}
+        if host is not None:
+            h2d_st.wait_event(fork)
+            d2h_st.wait_event(fork)
+            with torch.cuda.stream(h2d_st):
+                for i in order:
+                    runs[i].W.copy_(host[i]["W"], non_blocking=True)
+                    runs[i].X.copy_(host[i]["X"], non_blocking=True)
+                    ready[i] = torch.cuda.Event()
+                    ready[i].record(h2d_st)
+        for si, idxs in enumerate(sched):
             sd = sides[si]
             with torch.cuda.stream(sd):
                 for i in idxs:
                     r = runs[i]
                     if host is not None:
-                        r.W.copy_(host[i]["W"], non_blocking=True)
-                        r.X.copy_(host[i]["X"], non_blocking=True)
+                        sd.wait_event(ready[i])
                     for st in LayerRun.STAGES:
                         if timed:
                             e0 = torch.cuda.Event(enable_timing=True, external=True)
@@ -318,12 +335,16 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
                             e1.record(sd)
                             events.append((i, st, e0, e1))
                     if host is not None:
+                        done = torch.cuda.Event()
+                        done.record(sd)
+                        d2h_st.wait_event(done)
                         h = host[i]
-                        h["q"].copy_(r.q_gptq["qpacked"], non_blocking=True)
-                        h["s"].copy_(r.q_gptq["scales"], non_blocking=True)
-                        h["qr"].copy_(r.q_rtn["qpacked"], non_blocking=True)
-                        h["sse"].copy_(r.sse, non_blocking=True)
-        for sd in sides:
+                        with torch.cuda.stream(d2h_st):
+                            h["q"].copy_(r.q_gptq["qpacked"], non_blocking=True)
+                            h["s"].copy_(r.q_gptq["scales"], non_blocking=True)
+                            h["qr"].copy_(r.q_rtn["qpacked"], non_blocking=True)
+                            h["sse"].copy_(r.sse, non_blocking=True)
+        for sd in sides + ([h2d_st, d2h_st] if host is not None else []):
             j = torch.cuda.Event()
             j.record(sd)
             main.wait_event(j)
@@ -575,8 +596,9 @@ def roofline(kernel, recs, peaks, workload, ms_per_step):
 def e2e_run(runs, args, dev, world, n_streams, streams=None):
     """Same metric through the C-ABI with host buffers: every step copies
     each layer's W and X from pinned host memory and reads back the packed
-    codes, scales and both SSEs (copies and compute in one captured graph,
-    on the same streams)."""
+    codes, scales and both SSEs (copies and compute in one captured graph;
+    the copies on their own streams, each layer's compute waiting for its
+    inputs only)."""
     import torch
     host = []
     for r in runs:

@@ -140,13 +140,49 @@ constexpr int TT = 2 * NB + 4;  // row stride of the transposed sub-panel (float
 // row, the row in registers); rd gets the reciprocals of its diagonal.
 // Column J: the pivot is broadcast by a shuffle, the column of L goes
 // through colbuf (32 floats, read back as broadcast float4s) to every
-// row's update.  The column loop is not unrolled (the body selects the
-// registers of column J by predicated moves), which keeps the code small:
-// a fully unrolled factor is large enough that its instruction fetches
-// dominate on an SM that has not run it recently.  Entries right of a
-// lane's diagonal are updated too; they are never read.  A pivot that is
-// not positive and finite is replaced by 1; returns the first such column
-// (32 if none).
+// row's update.  The column loop runs over J = 8 J8 + E with E unrolled
+// (chol32_step<E>), so a column's register is picked among 4 candidates
+// and the update needs no per-element test; the 8-step body keeps the code
+// small (a fully unrolled factor is large enough that its instruction
+// fetches dominate on an SM that has not run it recently).  The pivot step
+// is the panel's serial chain -- the other warps wait for it -- so its
+// latency is what counts.  Entries right of a lane's diagonal are updated
+// too; they are never read; entries left of column J see l_k = 0.  A pivot
+// that is not positive and finite is replaced by 1; returns the first such
+// column (32 if none).
+template <int E>
+__device__ __forceinline__ void chol32_step(float (&w)[32], int J8, float *colbuf, int lane,
+                                            float &my_rd, int &bad) {
+  const int J = 8 * J8 + E;
+  const float a0 = (J8 & 1) ? w[8 + E] : w[E];
+  const float a1 = (J8 & 1) ? w[24 + E] : w[16 + E];
+  const float wj = (J8 & 2) ? a1 : a0;  // w[J]
+  float piv = __shfl_sync(0xffffffffu, wj, J);
+  const bool ill = !(piv > 0.0f) || !(piv < FLT_MAX);
+  bad = (ill && bad == 32) ? J : bad;
+  piv = ill ? 1.0f : piv;
+  // 1 / sqrt(piv): hardware estimate plus one Newton step r (3 - piv r^2) / 2
+  float rj = rsqrtf(piv);
+  rj = rj * fmaf(-0.5f * piv, rj * rj, 1.5f);
+  const float lij = lane > J ? wj * rj : (lane == J ? piv * rj : 0.0f);
+  my_rd = lane == J ? rj : my_rd;
+  colbuf[lane] = lij;
+  __syncwarp();
+#pragma unroll
+  for (int k4 = 0; k4 < 8; ++k4) {
+    const float4 l4 = reinterpret_cast<const float4 *>(colbuf)[k4];
+    const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k = 4 * k4 + q;
+      const float u = fmaf(-lij, lk[q], w[k]);
+      if (k % 8 == E) w[k] = (k / 8 == J8) ? lij : u;
+      else w[k] = u;
+    }
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ int chol32_piece(float *S, float *rd, float *colbuf, int c0,
                                             int lane) {
   float w[32];
@@ -155,32 +191,15 @@ __device__ __forceinline__ int chol32_piece(float *S, float *rd, float *colbuf, 
   float my_rd = 1.0f;
   int bad = 32;
 #pragma unroll 1
-  for (int J = 0; J < 32; ++J) {
-    float wj = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) wj = (k == J) ? w[k] : wj;
-    float piv = __shfl_sync(0xffffffffu, wj, J);
-    const bool ill = !(piv > 0.0f) || !(piv < FLT_MAX);
-    bad = (ill && bad == 32) ? J : bad;
-    piv = ill ? 1.0f : piv;
-    // 1 / sqrt(piv): hardware estimate plus one Newton step r (3 - piv r^2) / 2
-    float rj = rsqrtf(piv);
-    rj = rj * fmaf(-0.5f * piv, rj * rj, 1.5f);
-    const float lij = lane > J ? wj * rj : (lane == J ? piv * rj : 0.0f);
-    my_rd = lane == J ? rj : my_rd;
-    colbuf[lane] = lij;
-    __syncwarp();
-#pragma unroll
-    for (int k4 = 0; k4 < 8; ++k4) {
-      const float4 l4 = reinterpret_cast<const float4 *>(colbuf)[k4];
-      const float lk[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = 4 * k4 + e;
-        w[k] = (k == J) ? lij : fmaf(-lij, lk[e], w[k]);
-      }
-    }
-    __syncwarp();
+  for (int J8 = 0; J8 < 4; ++J8) {
+    chol32_step<0>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<1>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<2>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<3>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<4>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<5>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<6>(w, J8, colbuf, lane, my_rd, bad);
+    chol32_step<7>(w, J8, colbuf, lane, my_rd, bad);
   }
 #pragma unroll
   for (int k = 0; k < 32; ++k)
