@@ -566,7 +566,14 @@ __global__ void finish_info_kernel(int *status, int64_t d, int32_t *info_dev) {
 
 // Super-panel width: NB times the power of two nearest (on a log scale)
 // sqrt(d / NB).
+#ifndef GQ_CHOL_TWO_LEVEL_MIN_D
+#define GQ_CHOL_TWO_LEVEL_MIN_D 0
+#endif
+// Super-panel width S: about sqrt(NB d) (a power-of-two multiple of NB);
+// below GQ_CHOL_TWO_LEVEL_MIN_D one level (S = d), whose fewer launches
+// matter more than the trailing matrix's traffic when it sits in L2.
 int64_t chol_super_cols(int64_t d) {
+  if (d < GQ_CHOL_TWO_LEVEL_MIN_D) return d;
   const double target = std::sqrt(static_cast<double>(NB) * static_cast<double>(d));
   int64_t S = NB;
   while (static_cast<double>(2 * S) <= target * 1.4142135623730951) S *= 2;
