@@ -567,11 +567,12 @@ __global__ void finish_info_kernel(int *status, int64_t d, int32_t *info_dev) {
 // Super-panel width: NB times the power of two nearest (on a log scale)
 // sqrt(d / NB).
 #ifndef GQ_CHOL_TWO_LEVEL_MIN_D
-#define GQ_CHOL_TWO_LEVEL_MIN_D 0
+#define GQ_CHOL_TWO_LEVEL_MIN_D 4097
 #endif
 // Super-panel width S: about sqrt(NB d) (a power-of-two multiple of NB);
-// below GQ_CHOL_TWO_LEVEL_MIN_D one level (S = d), whose fewer launches
-// matter more than the trailing matrix's traffic when it sits in L2.
+// below GQ_CHOL_TWO_LEVEL_MIN_D one level (S = d): there the fewer launches
+// matter more than the trailing matrix's traffic, which mostly stays in L2
+// (the 49-layer GPT-2-small step, widths 768 and 3072: 24.9 -> 23.9 ms).
 int64_t chol_super_cols(int64_t d) {
   if (d < GQ_CHOL_TWO_LEVEL_MIN_D) return d;
   const double target = std::sqrt(static_cast<double>(NB) * static_cast<double>(d));
