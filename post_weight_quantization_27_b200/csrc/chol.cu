@@ -120,14 +120,25 @@ __global__ void __launch_bounds__(256) gather_reversed_kernel(const float *__res
                                                               int64_t d,
                                                               const int32_t *__restrict__ perm,
                                                               float *__restrict__ A) {
-  for (int64_t a = blockIdx.y; a < d; a += gridDim.y) {
+  // one warp per row; without a permutation a row of A is a row of H read
+  // backwards, one aligned float4 per lane (d is a multiple of 4); the
+  // float4 that holds the diagonal may also write up to three elements
+  // right of it, whose values are the symmetric matrix's own (the strict
+  // upper part is never read)
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t a = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       a < d; a += nw) {
     const int64_t sa = d - 1 - a;
-    const int64_t ra = perm ? perm[sa] : sa;
-    for (int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; b <= a;
-         b += static_cast<int64_t>(gridDim.x) * 256) {
-      const int64_t sb = d - 1 - b;
-      const int64_t cb = perm ? perm[sb] : sb;
-      A[a * d + b] = H[ra * d + cb];
+    if (perm) {
+      const int64_t ra = perm[sa];
+      for (int64_t b = lane; b <= a; b += 32) A[a * d + b] = H[ra * d + perm[d - 1 - b]];
+    } else {
+      const float *hr = H + sa * d;
+      for (int64_t b = 4 * lane; b <= a; b += 128) {
+        const float4 v = *reinterpret_cast<const float4 *>(hr + (d - 4 - b));
+        *reinterpret_cast<float4 *>(A + a * d + b) = make_float4(v.w, v.z, v.y, v.x);
+      }
     }
   }
 }
@@ -535,23 +546,42 @@ __global__ void __launch_bounds__(256) block_inverse_kernel(float *__restrict__ 
 // the rest of the upper triangle is never read).
 __global__ void __launch_bounds__(256) eye_lower_kernel(float *__restrict__ X, int64_t d,
                                                         int64_t S) {
-  for (int64_t r = blockIdx.y; r < d; r += gridDim.y) {
+  // one warp per row, float4 stores (d and S are multiples of 4)
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < d; r += nw) {
     int64_t end = (r / S + 1) * S;
     if (end > d) end = d;
-    for (int64_t c = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; c < end;
-         c += static_cast<int64_t>(gridDim.x) * 256)
-      X[r * d + c] = r == c ? 1.0f : 0.0f;
+    for (int64_t c = 4 * lane; c < end; c += 128) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r == c) v.x = 1.0f;
+      if (r == c + 1) v.y = 1.0f;
+      if (r == c + 2) v.z = 1.0f;
+      if (r == c + 3) v.w = 1.0f;
+      *reinterpret_cast<float4 *>(X + r * d + c) = v;
+    }
   }
 }
 
-// U[a][b] = X[d-1-a][d-1-b] for a <= b, 0 below the diagonal; also turns
-// the recorded pivot failure into the info value.
+// U[a][b] = X[d-1-a][d-1-b] for a <= b, 0 below the diagonal: one warp per
+// row, a row of X read backwards as aligned float4s.
 __global__ void __launch_bounds__(256) reverse_upper_kernel(const float *__restrict__ X,
                                                             int64_t d, float *__restrict__ U) {
-  for (int64_t a = blockIdx.y; a < d; a += gridDim.y)
-    for (int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; b < d;
-         b += static_cast<int64_t>(gridDim.x) * 256)
-      U[a * d + b] = b >= a ? X[(d - 1 - a) * d + (d - 1 - b)] : 0.0f;
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t a = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       a < d; a += nw) {
+    const float *xr = X + (d - 1 - a) * d;
+    for (int64_t b = 4 * lane; b < d; b += 128) {
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (b + 3 >= a) {
+        const float4 v = *reinterpret_cast<const float4 *>(xr + (d - 4 - b));
+        o = make_float4(b >= a ? v.w : 0.f, b + 1 >= a ? v.z : 0.f, b + 2 >= a ? v.y : 0.f, v.x);
+      }
+      *reinterpret_cast<float4 *>(U + a * d + b) = o;
+    }
+  }
 }
 
 // The factorisation runs on the reversed matrix: reversed pivot k is column
@@ -635,12 +665,12 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
     rank_kernel<<<static_cast<unsigned>((d + 255) / 256), 256, 0, st>>>(w.key, d, perm_out);
     count_launch();
   }
-  const unsigned gx = static_cast<unsigned>((d + 255) / 256);
-  const unsigned gy = static_cast<unsigned>(d < 65535 ? d : 65535);
+  // row kernels: one warp per row, 8 rows per block
+  const int64_t row_blocks = (d + 7) / 8, cap = static_cast<int64_t>(num_sms()) * 16;
+  const unsigned gr = static_cast<unsigned>(row_blocks < cap ? row_blocks : cap);
   float *A = U;  // the factorisation lives in the U buffer
   float *X = H;  // L^-1 is built in the H buffer
-  gather_reversed_kernel<<<dim3(gx, gy), 256, 0, st>>>(
-      H, d, act_order ? perm_out : nullptr, A);
+  gather_reversed_kernel<<<gr, 256, 0, st>>>(H, d, act_order ? perm_out : nullptr, A);
   count_launch();
   {
     const gq_status s = check_launch("damp/gather");
@@ -651,7 +681,7 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
   cudaFuncSetAttribute(block_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(INV_SMEM));
   const int64_t n_panels = (d + NB - 1) / NB;
-  eye_lower_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d, chol_super_cols(d));
+  eye_lower_kernel<<<gr, 256, 0, st>>>(X, d, chol_super_cols(d));
   count_launch();
   // The inverse X = L^-1 (blocked forward substitution on the identity) runs
   // as a second chain: its step p needs the panel p of L and step p-1 only,
@@ -741,7 +771,7 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
         cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess)
       return check_launch("stream join");
   }
-  reverse_upper_kernel<<<dim3(gx, gy), 256, 0, st>>>(X, d, U);
+  reverse_upper_kernel<<<gr, 256, 0, st>>>(X, d, U);
   count_launch();
   finish_info_kernel<<<1, 1, 0, st>>>(w.status, d, info_dev);
   count_launch();

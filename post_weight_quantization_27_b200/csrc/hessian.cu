@@ -307,34 +307,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // H[i][j] (i <= j) := H[i][j] + 2 * sum_s P_s(i, j) (without the H term
 // when !accumulate); H[j][i] := H[i][j].
+// Tiles of 64 x 64 on or above the diagonal, enumerated column by column
+// (t -> (bi, bj), bi <= bj) so that no block is spent on the lower half;
+// each thread moves 4 consecutive columns of a row (float4; d is a
+// multiple of 8 and a tile's 64 columns never straddle two 256-column
+// partial tiles).
 __global__ void __launch_bounds__(256) hessian_finish_kernel(float *__restrict__ H, int d,
                                                              const float *__restrict__ P,
                                                              int n_tiles, int n_bj, int n_split,
                                                              const int *status, int accumulate) {
-  const int bi = blockIdx.y, bj = blockIdx.x;
-  if (bi > bj) return;
-  __shared__ float tile[32][33];
+  constexpr int FT = 64;
+  __shared__ float tile[FT][FT + 1];
   const bool bad = status != nullptr && *status != 0;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int r = ty; r < 32; r += 8) {
-    const int i = bi * 32 + r, j = bj * 32 + tx;
-    float val = 0.0f;
-    if (i < d && j < d && i <= j) {
-      const int tb = i / BM, tj = j / BN;
-      const int t = static_cast<int>(tile_row_start(tb, n_bj)) + (tj - (tb >> 1));
-      float sum = 0.0f;
-      for (int s = 0; s < n_split; ++s)
-        sum += P[(static_cast<size_t>(s * n_tiles + t) * BM + (i - tb * BM)) * BN + (j - tj * BN)];
-      val = accumulate ? H[static_cast<size_t>(i) * d + j] + 2.0f * sum : 2.0f * sum;
-      if (bad) val = __int_as_float(0x7fc00000);
-      H[static_cast<size_t>(i) * d + j] = val;
+  const int cx = (threadIdx.x & 15) * 4, ry = threadIdx.x >> 4;  // 4 columns, 16 rows per pass
+  const int nb = (d + FT - 1) / FT;
+  const int64_t n_up = static_cast<int64_t>(nb) * (nb + 1) / 2;
+  for (int64_t t = blockIdx.x; t < n_up; t += gridDim.x) {
+    int bj = static_cast<int>((sqrt(8.0 * static_cast<double>(t) + 1.0) - 1.0) * 0.5);
+    while (static_cast<int64_t>(bj) * (bj + 1) / 2 > t) --bj;
+    while (static_cast<int64_t>(bj + 1) * (bj + 2) / 2 <= t) ++bj;
+    const int bi = static_cast<int>(t - static_cast<int64_t>(bj) * (bj + 1) / 2);
+    const int j = bj * FT + cx;
+    for (int r = ry; r < FT; r += 16) {
+      const int i = bi * FT + r;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < d && j < d && i <= j + 3) {
+        const int tb = i / BM, tj = j / BN;
+        const int tt = static_cast<int>(tile_row_start(tb, n_bj)) + (tj - (tb >> 1));
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < n_split; ++s) {
+          const float4 p = *reinterpret_cast<const float4 *>(
+              P + (static_cast<size_t>(s * n_tiles + tt) * BM + (i - tb * BM)) * BN + (j - tj * BN));
+          sum.x += p.x; sum.y += p.y; sum.z += p.z; sum.w += p.w;
+        }
+        float *h = H + static_cast<size_t>(i) * d + j;
+        const float4 old = accumulate ? *reinterpret_cast<const float4 *>(h)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        v = make_float4(old.x + 2.0f * sum.x, old.y + 2.0f * sum.y, old.z + 2.0f * sum.z,
+                        old.w + 2.0f * sum.w);
+        if (!accumulate) v = make_float4(2.0f * sum.x, 2.0f * sum.y, 2.0f * sum.z, 2.0f * sum.w);
+        if (bad) v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                 __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+        // only the elements with i <= j belong to this triangle
+        if (i <= j) {
+          *reinterpret_cast<float4 *>(h) = v;
+        } else {
+          if (i <= j + 1) h[1] = v.y;
+          if (i <= j + 2) h[2] = v.z;
+          h[3] = v.w;
+        }
+      }
+      tile[r][cx] = v.x;
+      tile[r][cx + 1] = v.y;
+      tile[r][cx + 2] = v.z;
+      tile[r][cx + 3] = v.w;
     }
-    tile[r][tx] = val;
-  }
-  __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int j = bj * 32 + r, i = bi * 32 + tx;
-    if (i < d && j < d && i < j) H[static_cast<size_t>(j) * d + i] = tile[tx][r];
+    __syncthreads();
+    // the mirror: H[j'][i'] = H[i'][j'] for i' < j', rows j' of the tile's columns
+    for (int r = ry; r < FT; r += 16) {
+      const int jr = bj * FT + r, ic = bi * FT + cx;
+      if (jr >= d || ic >= d) continue;
+      float *h = H + static_cast<size_t>(jr) * d + ic;
+      if (ic + 3 < jr) {
+        *reinterpret_cast<float4 *>(h) =
+            make_float4(tile[cx][r], tile[cx + 1][r], tile[cx + 2][r], tile[cx + 3][r]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (ic + q < jr) h[q] = tile[cx + q][r];
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -419,10 +462,10 @@ gq_status launch_hessian(const void *X, int64_t n_tok, int64_t d_in, float *H, v
     s = check_launch("hessian_mma_kernel");
     if (s != GQ_OK) return s;
   }
-  const int nb = static_cast<int>((d_in + 31) / 32);
-  hessian_finish_kernel<<<dim3(nb, nb), 256, 0, st>>>(H, static_cast<int>(d_in), P, p.n_tiles,
-                                                      p.n_bj, p.n_split, status,
-                                                      accumulate ? 1 : 0);
+  const int64_t nb = (d_in + 63) / 64, n_up = nb * (nb + 1) / 2;
+  const int64_t fcap = static_cast<int64_t>(num_sms()) * 16;
+  hessian_finish_kernel<<<static_cast<unsigned>(n_up < fcap ? n_up : fcap), 256, 0, st>>>(
+      H, static_cast<int>(d_in), P, p.n_tiles, p.n_bj, p.n_split, status, accumulate ? 1 : 0);
   count_launch();
   return check_launch("hessian_finish_kernel");
 }
