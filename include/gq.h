@@ -139,11 +139,11 @@ gq_status gq_hessian_compute(const void *X_bf16, int64_t n_tok, int64_t d_in, fl
  *   4. U := the upper-triangular matrix with positive diagonal such that
  *      H^-1 = U^T U (written to U; the strictly lower part is zero).
  *
- *   H          [d_in][d_in] fp32, exactly symmetric (device, in; used as
- *              scratch: contents unspecified on return)
+ *   H          [d_in][d_in] fp32, exactly symmetric (device, in, 16-byte
+ *              aligned; used as scratch: contents unspecified on return)
  *   perm_out   [d_in] int32 (device, out) -- required iff act_order != 0
  *   dead_out   [d_in] uint8 (device, out) or NULL
- *   U          [d_in][d_in] fp32 (device, out)
+ *   U          [d_in][d_in] fp32 (device, out, 16-byte aligned)
  *   info_dev   int32 (device, out) or NULL: -1 on success, else a column
  *              (in processing order) at which the factorisation met a
  *              non-positive or non-finite pivot.

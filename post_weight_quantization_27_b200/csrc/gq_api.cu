@@ -216,6 +216,8 @@ gq_status gq_damp_cholesky_inverse(float *H, int64_t d_in, float damp_percent, i
                                    size_t ws_bytes, void *stream) {
   t_last_error.clear();
   if (!H || !U) return fail(GQ_ERR_ARG, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(U)) % 16 != 0)
+    return fail(GQ_ERR_ARG, "H and U must be 16-byte aligned");
   if (act_order != 0 && !perm_out) return fail(GQ_ERR_ARG, "act_order needs perm_out");
   if (!(damp_percent >= 0.0f) || !(damp_percent < 1e30f))
     return fail(GQ_ERR_ARG, "damp_percent must be finite and >= 0");

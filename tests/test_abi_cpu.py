@@ -81,6 +81,14 @@ def test_other_argument_errors():
     # negative damping
     assert L.gq_damp_cholesky_inverse(FAKE, 64, -1.0, 0, None, None, FAKE, None, None,
                                       FAKE, 1 << 30, None) == 1
+    # H or U not 16-byte aligned (the row kernels read them as float4)
+    odd = ctypes.c_void_p(4096 + 4)
+    assert L.gq_damp_cholesky_inverse(odd, 64, 0.01, 0, None, None, FAKE, None, None,
+                                      FAKE, 1 << 30, None) == 1
+    assert L.gq_damp_cholesky_inverse(FAKE, 64, 0.01, 0, None, None, odd, None, None,
+                                      FAKE, 1 << 30, None) == 1
+    assert L.gq_damp_cholesky_inverse_noalloc(odd, 64, 0.01, 0, None, None, FAKE, None,
+                                              None, None) == 1
     # group_size must divide block_size
     assert L.gq_gptq_quantize_layer(FAKE, 0, 8, 192, FAKE, 4, 48, 96, 1, None, None,
                                     FAKE, FAKE, None, None, FAKE, 1 << 40, None) == 1
