@@ -283,8 +283,8 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
     """One whole step (every layer, every stage) captured as a CUDA graph:
     the layers run on ``n_streams`` streams forked from and joined back to
     one capture stream.  ``timed`` adds timing event nodes around each
-    stage call; ``kernel`` adds the library's per-launch event pairs around
-    every launch of that kernel (read with gq.kernel_timer_read after the
+    stage call; ``kernel`` (a name or a list of names) adds the library's per-launch
+    event pairs around every launch of that kernel (read with gq.kernel_timer_read after the
     replays); ``host`` adds the pinned host <-> device copies of the
     end-to-end run.  Returns (graph, stream, stage events, launches/step)."""
     import torch
@@ -302,7 +302,8 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
     events = []
     n0 = gq.launch_count()
     if kernel is not None:
-        gq.kernel_timer_start([kernel], capacity)
+        gq.kernel_timer_start(list(kernel) if isinstance(kernel, (list, tuple)) else [kernel],
+                              capacity)
     with torch.cuda.graph(g, stream=main):
         fork = torch.cuda.Event()
         fork.record(main)
@@ -371,10 +372,11 @@ def replay(graph, stream, n, timed=False):
     return t0.elapsed_time(t1) / max(n, 1) if timed else None
 
 
-def kernel_shares(runs):
-    """One eager pass of the whole step on one stream with every kernel's
-    launches timed: per kernel (total ms, launches), serialised like an ncu
-    launch list; picks the dominant kernel."""
+def kernel_shares(runs, n_streams, streams):
+    """Per kernel (total ms, launches, work) over one step, timed inside a
+    captured graph of the step (the library's per-launch event pairs on
+    every launch; device time, no host gaps between launches); picks the
+    dominant kernel."""
     import torch
     from post_weight_quantization_27_b200 import gq
     n0 = gq.launch_count()
@@ -383,15 +385,15 @@ def kernel_shares(runs):
             getattr(r, st)()
     torch.cuda.synchronize()
     cap = int(1.2 * (gq.launch_count() - n0)) + 64
-    gq.kernel_timer_start(gq.KERNELS, cap)
+    graph, gstream, _, _ = capture_step(runs, n_streams, kernel=list(gq.KERNELS), capacity=cap,
+                                        streams=streams)
     try:
-        for r in runs:
-            for st in LayerRun.STAGES:
-                getattr(r, st)()
+        replay(graph, gstream, 2)
         torch.cuda.synchronize()
         recs = gq.kernel_timer_read()
     finally:
         gq.kernel_timer_release()
+        del graph
     tot = {}
     for k, ms, w in recs:
         t, n, wk = tot.get(k, (0.0, 0, 0.0))
@@ -432,7 +434,7 @@ def gpu_arm(args, world, rank, local):
     # captured step with the dominant kernel's launches timed
     streams = make_streams(n_streams)
     warm_streams(runs, streams[1])
-    shares = kernel_shares(runs)
+    shares = kernel_shares(runs, n_streams, streams)
     dom_kernel = max(shares, key=lambda k: shares[k][0])
     graph, gstream, events, launches_per_step = capture_step(
         runs, n_streams, timed=True, kernel=dom_kernel, capacity=shares[dom_kernel][1] + 64,
@@ -492,10 +494,10 @@ def gpu_arm(args, world, rank, local):
                        sum(r.W.numel() * r.W.element_size() + r.X.numel() * 2 for r in runs) / 1e6)},
         "mweights_per_s": round(world * tot["weights"] / (ms / 1e3) / 1e6, 2),
         "stage_ms_sum_of_calls": {k: round(v, 4) for k, v in stage_ms.items()},
-        "kernel_share_eager": {k: {"ms": round(t, 3), "launches": n,
-                                   "share": round(t / sum(v[0] for v in shares.values()), 4)}
-                               for k, (t, n, _) in sorted(shares.items(), key=lambda x: -x[1][0])},
-        # per-kernel rates from the serialised eager pass (work / event time)
+        "kernel_share": {k: {"ms": round(t, 3), "launches": n,
+                             "share": round(t / sum(v[0] for v in shares.values()), 4)}
+                         for k, (t, n, _) in sorted(shares.items(), key=lambda x: -x[1][0])},
+        # per-kernel rates from the timed graph pass (work / event time)
         "xtx_tflops": rate(shares, "hessian_mma", 1e12),
         "rtn_gbs": rate(shares, "rtn", 1e9),
         "recon_tflops": rate(shares, "recon_mma" if args.recon == "direct" else "syrk_bf16", 1e12),
