@@ -144,6 +144,10 @@ def measured_peaks() -> dict:
 
 # ----------------------------------------------------------------------------- GPU arm
 
+# token chunks of a layer's X in the end-to-end run (copied in one after another;
+# the Hessian accumulates over each as it lands)
+E2E_CHUNKS = 8
+
 class LayerRun:
     """Device buffers of one layer and the calls of one step on it."""
 
@@ -158,7 +162,9 @@ class LayerRun:
         self.H0 = torch.empty((d_in, d_in), dtype=torch.float32, **f)   # undamped, kept
         self.H = torch.empty((d_in, d_in), dtype=torch.float32, **f)    # the solve's scratch
         self.U = torch.empty((d_in, d_in), dtype=torch.float32, **f)
-        self.ws_h = gq.workspace(gq.hessian_workspace_size(n, d_in), dev)
+        self.n_chunks = E2E_CHUNKS if n % E2E_CHUNKS == 0 and n >= 8192 * E2E_CHUNKS else 1
+        self.ws_h = gq.workspace(max(gq.hessian_workspace_size(n, d_in),
+                                     gq.hessian_workspace_size(n // self.n_chunks, d_in)), dev)
         self.ws_c = gq.workspace(gq.damp_cholesky_workspace_size(d_in), dev)
         self.ws_g = gq.workspace(gq.gptq_workspace_size(d_out, d_in, spec.block_size), dev)
         self.ws_r = gq.workspace(gq.recon_workspace_size(d_out, d_in, n) if recon_route == "direct"
@@ -176,6 +182,18 @@ class LayerRun:
         gq._check(L.gq_hessian_compute(gq._p(self.X), self.spec.n_tok, self.spec.d_in,
                                        gq._p(self.H0), gq._p(self.ws_h), self.ws_h.numel(), s),
                   "hessian")
+
+    def hessian_part(self, c):
+        """H0 over token chunk c of n_chunks: := for the first, += after
+        (the end-to-end run accumulates H while the later chunks of X are
+        still being copied in)."""
+        from post_weight_quantization_27_b200 import gq
+        L, s = gq.lib(), gq._stream(None)
+        n = self.spec.n_tok // self.n_chunks
+        x = gq._p(self.X) + c * n * self.spec.d_in * 2
+        fn = L.gq_hessian_compute if c == 0 else L.gq_hessian_accumulate
+        gq._check(fn(x, n, self.spec.d_in, gq._p(self.H0), gq._p(self.ws_h), self.ws_h.numel(),
+                     s), "hessian")
 
     def solve(self):
         from post_weight_quantization_27_b200 import gq
@@ -315,18 +333,28 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
             d2h_st.wait_event(fork)
             with torch.cuda.stream(h2d_st):
                 for i in order:
-                    runs[i].W.copy_(host[i]["W"], non_blocking=True)
-                    runs[i].X.copy_(host[i]["X"], non_blocking=True)
-                    ready[i] = torch.cuda.Event()
-                    ready[i].record(h2d_st)
+                    r, nc = runs[i], runs[i].n_chunks
+                    r.W.copy_(host[i]["W"], non_blocking=True)
+                    ready[i] = []
+                    rows = r.spec.n_tok // nc
+                    for c in range(nc):
+                        r.X[c * rows:(c + 1) * rows].copy_(host[i]["X"][c * rows:(c + 1) * rows],
+                                                           non_blocking=True)
+                        ready[i].append(torch.cuda.Event())
+                        ready[i][-1].record(h2d_st)
         for si, idxs in enumerate(sched):
             sd = sides[si]
             with torch.cuda.stream(sd):
                 for i in idxs:
                     r = runs[i]
+                    stages = LayerRun.STAGES
                     if host is not None:
-                        sd.wait_event(ready[i])
-                    for st in LayerRun.STAGES:
+                        # H over the chunks of X as they land, then the rest
+                        for c, ev in enumerate(ready[i]):
+                            sd.wait_event(ev)
+                            r.hessian_part(c)
+                        stages = stages[1:]
+                    for st in stages:
                         if timed:
                             e0 = torch.cuda.Event(enable_timing=True, external=True)
                             e1 = torch.cuda.Event(enable_timing=True, external=True)
