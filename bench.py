@@ -400,11 +400,13 @@ def replay(graph, stream, n, timed=False):
     return t0.elapsed_time(t1) / max(n, 1) if timed else None
 
 
-def kernel_shares(runs, n_streams, streams):
+def kernel_shares(runs):
     """Per kernel (total ms, launches, work) over one step, timed inside a
-    captured graph of the step (the library's per-launch event pairs on
-    every launch; device time, no host gaps between launches); picks the
-    dominant kernel."""
+    captured graph of the step on one fresh stream (the library's per-launch
+    event pairs on every launch: device time with no host gaps, and no
+    helper stream, since none is created during a capture, so the kernels
+    run one after another as in an ncu launch list); picks the dominant
+    kernel."""
     import torch
     from post_weight_quantization_27_b200 import gq
     n0 = gq.launch_count()
@@ -413,8 +415,8 @@ def kernel_shares(runs, n_streams, streams):
             getattr(r, st)()
     torch.cuda.synchronize()
     cap = int(1.2 * (gq.launch_count() - n0)) + 64
-    graph, gstream, _, _ = capture_step(runs, n_streams, kernel=list(gq.KERNELS), capacity=cap,
-                                        streams=streams)
+    graph, gstream, _, _ = capture_step(runs, 1, kernel=list(gq.KERNELS), capacity=cap,
+                                        streams=make_streams(1))
     try:
         replay(graph, gstream, 2)
         torch.cuda.synchronize()
@@ -462,7 +464,7 @@ def gpu_arm(args, world, rank, local):
     # captured step with the dominant kernel's launches timed
     streams = make_streams(n_streams)
     warm_streams(runs, streams[1])
-    shares = kernel_shares(runs, n_streams, streams)
+    shares = kernel_shares(runs)
     dom_kernel = max(shares, key=lambda k: shares[k][0])
     graph, gstream, events, launches_per_step = capture_step(
         runs, n_streams, timed=True, kernel=dom_kernel, capacity=shares[dom_kernel][1] + 64,
@@ -525,7 +527,7 @@ def gpu_arm(args, world, rank, local):
         "kernel_share": {k: {"ms": round(t, 3), "launches": n,
                              "share": round(t / sum(v[0] for v in shares.values()), 4)}
                          for k, (t, n, _) in sorted(shares.items(), key=lambda x: -x[1][0])},
-        # per-kernel rates from the timed graph pass (work / event time)
+        # per-kernel rates from the serialised graph pass (work / event time)
         "xtx_tflops": rate(shares, "hessian_mma", 1e12),
         "rtn_gbs": rate(shares, "rtn", 1e9),
         "recon_tflops": rate(shares, "recon_mma" if args.recon == "direct" else "syrk_bf16", 1e12),
