@@ -273,7 +273,8 @@ constexpr size_t PANEL_SMEM = (2 * NB * SP + NB + 32 * TT + 32) * sizeof(float);
 
 __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, int64_t d,
                                                          int64_t k0, int nb,
-                                                         float *__restrict__ lpp, int *status) {
+                                                         float *__restrict__ lpp, int *status,
+                                                         int n_rb) {
   extern __shared__ float sm[];
   float *S = sm;            // [NB][SP]  the diagonal block, then its factor L (lower)
   float *P = S + NB * SP;   // [NB][SP]  this CTA's panel rows (CTA 0: unused)
@@ -445,6 +446,68 @@ __global__ void __launch_bounds__(256) potrf_trsm_kernel(float *__restrict__ A, 
       const int r = e >> 5, c = (e & 31) * 4;
       if (r < prows && c < nb)
         *reinterpret_cast<float4 *>(A + (row0 + r) * d + k0 + c) =
+            make_float4(P[r * SP + c], P[r * SP + c + 1], P[r * SP + c + 2], P[r * SP + c + 3]);
+    }
+  }
+
+  // Further row blocks (a grid smaller than the panel's n_rb row blocks):
+  // the diagonal block's factor stays in S and rd, and each further block
+  // of 128 rows is solved against it as the CTA's own rows were above --
+  // the same operations in the same order, without factoring the block
+  // again.  T's block part is refilled from S for each sub-panel.
+  for (int rb = static_cast<int>(blockIdx.x + gridDim.x); rb < n_rb;
+       rb += static_cast<int>(gridDim.x)) {
+    const int64_t r0 = k0 + static_cast<int64_t>(rb) * NB;
+    const int pr = static_cast<int>(d - r0 < NB ? d - r0 : NB);
+    __syncthreads();  // the previous rows are written out; P and T are free
+    for (int e = tid; e < NB * NB / 4; e += 256) {
+      const int r = e >> 5, c = (e & 31) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < pr && c < nb) v = *reinterpret_cast<const float4 *>(A + (r0 + r) * d + k0 + c);
+      P[r * SP + c] = v.x;
+      P[r * SP + c + 1] = v.y;
+      P[r * SP + c + 2] = v.z;
+      P[r * SP + c + 3] = v.w;
+    }
+    __syncthreads();
+    for (int c0 = 0; c0 < NB; c0 += 32) {
+      const int base = c0 + 32;
+      for (int i = tid; i < NB; i += 256) {
+        float *row = P + i * SP;
+        float a[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) a[k] = row[c0 + k];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float x = a[j] * rd[c0 + j];
+          a[j] = x;
+#pragma unroll
+          for (int k = j + 1; k < 32; ++k) a[k] = fmaf(-x, S[(c0 + k) * SP + c0 + j], a[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          row[c0 + k] = a[k];
+          T[k * TT + NB + i] = a[k];
+        }
+      }
+      if (base >= NB) break;
+      for (int e = tid; e < 32 * (NB - base); e += 256) {
+        const int k = e / (NB - base), q = base + e % (NB - base);
+        T[k * TT + q] = S[q * SP + c0 + k];
+      }
+      __syncthreads();
+      const int m8 = (NB - base) / 8;
+      for (int t = tid; t < (NB / 8) * m8; t += 256) {
+        const int tp = t / m8, tk = t % m8;
+        update_tile8(T, NB + 8 * tp, base + 8 * tk, P, SP, false, 8 * tp, base + 8 * tk);
+      }
+      __syncthreads();
+    }
+    __syncthreads();
+    for (int e = tid; e < NB * NB / 4; e += 256) {
+      const int r = e >> 5, c = (e & 31) * 4;
+      if (r < pr && c < nb)
+        *reinterpret_cast<float4 *>(A + (r0 + r) * d + k0 + c) =
             make_float4(P[r * SP + c], P[r * SP + c + 1], P[r * SP + c + 2], P[r * SP + c + 3]);
     }
   }
@@ -708,10 +771,11 @@ gq_status launch_damp_chol(float *H, int64_t d, float damp, int act_order, int32
       const int nb = static_cast<int>(d - k0 < NB ? d - k0 : NB);
       const int64_t k1 = k0 + nb;
       const int rest = static_cast<int>(d - k1);
-      const unsigned tiles = static_cast<unsigned>(1 + (rest + NB - 1) / NB);
+      const int tiles = static_cast<int>(1 + (rest + NB - 1) / NB);
+      const int pgrid = tiles < num_sms() ? tiles : num_sms();  // one wave; CTAs loop
       float *lp = w.linv + p * NB * NB;
       int slot = timer_begin(GQ_KERNEL_POTRF_TRSM, st);
-      potrf_trsm_kernel<<<tiles, 256, PANEL_SMEM, st>>>(A, d, k0, nb, lp, w.status);
+      potrf_trsm_kernel<<<pgrid, 256, PANEL_SMEM, st>>>(A, d, k0, nb, lp, w.status, tiles);
       count_launch();
       // Cholesky of the block nb^3 / 3, the panel solve rest nb^2
       timer_end(slot, st, static_cast<double>(nb) * nb * (nb / 3.0 + rest));
