@@ -297,14 +297,16 @@ def warm_streams(runs, sides):
 
 
 def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=0,
-                 streams=None):
+                 streams=None, serial=()):
     """One whole step (every layer, every stage) captured as a CUDA graph:
     the layers run on ``n_streams`` streams forked from and joined back to
     one capture stream.  ``timed`` adds timing event nodes around each
     stage call; ``kernel`` (a name or a list of names) adds the library's per-launch
     event pairs around every launch of that kernel (read with gq.kernel_timer_read after the
     replays); ``host`` adds the pinned host <-> device copies of the
-    end-to-end run.  Returns (graph, stream, stage events, launches/step)."""
+    end-to-end run; stages named in ``serial`` run one layer at a time
+    across the streams (each waits for the previous layer's, in issue
+    order).  Returns (graph, stream, stage events, launches/step)."""
     import torch
     from post_weight_quantization_27_b200 import gq
     main, sides = streams if streams is not None else make_streams(n_streams)
@@ -327,7 +329,7 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
         fork.record(main)
         for sd in sides:
             sd.wait_event(fork)
-        ready = {}
+        ready, last = {}, {}
         if host is not None:
             h2d_st.wait_event(fork)
             d2h_st.wait_event(fork)
@@ -350,16 +352,26 @@ def capture_step(runs, n_streams, timed=False, host=None, kernel=None, capacity=
                     stages = LayerRun.STAGES
                     if host is not None:
                         # H over the chunks of X as they land, then the rest
+                        if "hessian" in serial and "hessian" in last:
+                            sd.wait_event(last["hessian"])
                         for c, ev in enumerate(ready[i]):
                             sd.wait_event(ev)
                             r.hessian_part(c)
+                        if "hessian" in serial:
+                            last["hessian"] = torch.cuda.Event()
+                            last["hessian"].record(sd)
                         stages = stages[1:]
                     for st in stages:
+                        if st in serial and st in last:
+                            sd.wait_event(last[st])
                         if timed:
                             e0 = torch.cuda.Event(enable_timing=True, external=True)
                             e1 = torch.cuda.Event(enable_timing=True, external=True)
                             e0.record(sd)
                         getattr(r, st)()
+                        if st in serial:
+                            last[st] = torch.cuda.Event()
+                            last[st].record(sd)
                         if timed:
                             e1.record(sd)
                             events.append((i, st, e0, e1))
@@ -466,9 +478,10 @@ def gpu_arm(args, world, rank, local):
     warm_streams(runs, streams[1])
     shares = kernel_shares(runs)
     dom_kernel = max(shares, key=lambda k: shares[k][0])
+    serial = tuple(x for x in args.serial_stages.split(",") if x)
     graph, gstream, events, launches_per_step = capture_step(
         runs, n_streams, timed=True, kernel=dom_kernel, capacity=shares[dom_kernel][1] + 64,
-        streams=streams)
+        streams=streams, serial=serial)
 
     replay(graph, gstream, args.warmup)
     torch.cuda.synchronize()
@@ -519,7 +532,8 @@ def gpu_arm(args, world, rank, local):
         "config": {"workload": WORKLOAD_NAMES[args.workload], "layers": n_layers,
                    "recon_route": args.recon,
                    "weights_per_step": tot["weights"], "parallelism": f"layers x{world} (weak)",
-                   "streams": n_streams, "cuda_graph": True,
+                   "streams": n_streams, "serial_stages": args.serial_stages,
+                   "cuda_graph": True,
                    "l2": "inputs larger than L2 (%.0f MB of W and X per step)" % (
                        sum(r.W.numel() * r.W.element_size() + r.X.numel() * 2 for r in runs) / 1e6)},
         "mweights_per_s": round(world * tot["weights"] / (ms / 1e3) / 1e6, 2),
@@ -642,7 +656,9 @@ def e2e_run(runs, args, dev, world, n_streams, streams=None):
     h2d = sum(h["W"].numel() * h["W"].element_size() + h["X"].numel() * 2 for h in host)
     d2h = sum(h["q"].numel() * 4 + h["s"].numel() * 2 + h["qr"].numel() * 4 + 16 for h in host)
     graph, gstream, _, _ = capture_step(runs, n_streams, timed=False, host=host,
-                                        streams=streams)
+                                        streams=streams,
+                                        serial=tuple(x for x in args.serial_stages.split(",")
+                                                     if x))
     steps = max(1, min(args.steps, 5))
     replay(graph, gstream, 1)
     torch.cuda.synchronize()
@@ -859,6 +875,9 @@ def main():
     ap.add_argument("--recon", default="hessian", choices=["hessian", "direct"],
                     help="reconstruction error route: from the Hessian (tr(dW H0 dW^T) / 2) "
                          "or directly (||dW X^T||^2)")
+    ap.add_argument("--serial-stages", default="",
+                    help="stages (comma-separated, e.g. hessian) that run one layer at a time "
+                         "across the streams")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

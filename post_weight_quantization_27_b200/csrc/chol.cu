@@ -17,8 +17,10 @@
 // inverse) goes to a [NB][NB] slot of the workspace; X = L^-1 is built in
 // the H buffer (the caller's H is scratch); the last kernel writes
 // U = J X J back into the U buffer.
-// Blocked right-looking algorithms with 128-wide panels; one CTA factors a
-// diagonal block in shared memory (and inverts it), the panel solve, the
+// Blocked right-looking algorithms with 128-wide panels grouped in
+// super-panels (two levels, above a width); each CTA of the panel kernel
+// factors the diagonal block in shared memory and solves its panel rows
+// against it, one CTA inverts the block for the inverse's chain, and the
 // trailing updates and the inverse's block steps are fp32 GEMMs on the
 // tensor cores (3 x TF32 split, gemm_tc.cu).
 #include <cfloat>

@@ -21,11 +21,14 @@
 //              releasing the stage to the MMA warp
 //   warp 1     three MMAs per 8-wide K step into one of two TMEM
 //              accumulators (the epilogue of one tile overlaps the next)
-//   warps 6-9  epilogue: the C tile is fetched by TMA into a staging buffer
-//              while the tile's MMAs run; each thread (one accumulator row)
-//              forms beta C + alpha acc in the staging buffer, and TMA
-//              stores it (clipped at the matrix edge).  Global memory is
-//              only touched by whole-tile TMA copies.
+//   warps 6-9  epilogue: the C tile passes through two staging buffers in
+//              chunks of 32 columns -- the next chunk is fetched by TMA
+//              while each thread (one accumulator row) forms beta C + alpha
+//              acc of the current one, which TMA stores (clipped at the
+//              matrix edge).  Global memory is only touched by TMA copies.
+// Large products run on CTA pairs instead (gemm_pair_kernel, below: 256 x
+// 256 tiles, tcgen05 cta_group::2), as does the bf16 SYRK of the error
+// from the Hessian.
 // A is K-major (A(m, k) = A[m lda + k]); B is either K-major (B(k, n) =
 // B[n ldb + k]) or N-major (B(k, n) = B[k ldb + n]); an N-major TF32 operand
 // must be staged with the 32-byte-atom variant of the 128-byte swizzle.  With `lower` only
