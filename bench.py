@@ -647,8 +647,14 @@ def e2e_run(runs, args, dev, world, n_streams, streams=None):
     inputs only)."""
     import torch
     host = []
+
+    def pinned_copy(t):  # one pinned host copy (no pageable intermediate)
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
     for r in runs:
-        host.append(dict(W=r.W.cpu().pin_memory(), X=r.X.cpu().pin_memory(),
+        host.append(dict(W=pinned_copy(r.W), X=pinned_copy(r.X),
                          q=torch.empty(r.q_gptq["qpacked"].shape, dtype=torch.int32).pin_memory(),
                          s=torch.empty(r.q_gptq["scales"].shape, dtype=torch.float16).pin_memory(),
                          qr=torch.empty(r.q_rtn["qpacked"].shape, dtype=torch.int32).pin_memory(),
