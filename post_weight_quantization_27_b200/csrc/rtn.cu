@@ -12,6 +12,7 @@
 // 16-byte vector loads and every packed word is written by one coalesced
 // 4-byte store.  Rows longer than 32 * 8 words stream twice through L2
 // instead (second kernel).
+#include <cstring>
 #include <type_traits>
 
 #include "gq_device.cuh"
@@ -83,13 +84,14 @@ struct Raw8Half {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float2 f;
-      if constexpr (sizeof(H2) == 4 && std::is_same<H2, __half2>::value)
-        f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
-      else
-        f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
+      if constexpr (std::is_same<H2, __half2>::value) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      } else {  // a bf16 value is the upper half of the fp32 with the same value
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
     }
   }
 };
@@ -105,6 +107,57 @@ struct Raw8<__nv_bfloat16> : Raw8Half<__nv_bfloat162> {
     u = __ldg(reinterpret_cast<const uint4 *>(p));
   }
 };
+
+// Running min and max of 0 and the weights seen, in the weights' own type
+// (min and max are exact in every format, and a 16-bit pair takes one
+// instruction for two weights), read out as fp32 once per segment.  NaN is
+// passed over, as fminf / fmaxf do.
+template <typename T>
+struct MinMax;
+template <>
+struct MinMax<float> {
+  float mn = 0.0f, mx = 0.0f;
+  __device__ __forceinline__ void add(const Raw8<float> &r) {
+    float v[8];
+    r.get(v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      mn = fminf(mn, v[e]);
+      mx = fmaxf(mx, v[e]);
+    }
+  }
+  __device__ __forceinline__ void get(float &lo, float &hi) const {
+    lo = mn;
+    hi = mx;
+  }
+};
+template <typename H2>
+struct MinMaxHalf {
+  H2 mn, mx;
+  __device__ __forceinline__ MinMaxHalf() {
+    const uint32_t zero = 0u;
+    memcpy(&mn, &zero, 4);
+    memcpy(&mx, &zero, 4);
+  }
+  __device__ __forceinline__ void add(const Raw8Half<H2> &r) {
+    const uint32_t w[4] = {r.u.x, r.u.y, r.u.z, r.u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      H2 h;
+      memcpy(&h, &w[i], 4);
+      mn = __hmin2(mn, h);
+      mx = __hmax2(mx, h);
+    }
+  }
+  __device__ __forceinline__ void get(float &lo, float &hi) const {
+    lo = fminf(__low2float(mn), __high2float(mn));
+    hi = fmaxf(__low2float(mx), __high2float(mx));
+  }
+};
+template <>
+struct MinMax<__half> : MinMaxHalf<__half2> {};
+template <>
+struct MinMax<__nv_bfloat16> : MinMaxHalf<__nv_bfloat162> {};
 
 // Code word of 8 weights.  rs = RN(1 / s): the quotient w / s is formed as a
 // correctly rounded division from the reciprocal and rounded exactly with a
@@ -124,26 +177,74 @@ __device__ __forceinline__ uint32_t pack_word(const float (&v)[8], const GridPar
 }
 
 // The same codes for a group whose quotients are known to be small (see
-// RtnGrid::fast): q = w / s needs no clamp before the magic-constant
-// rounding, C + rint(q) is exact, and the code is read from the bits of
-// that sum as an integer (symmetric: the range -7..7 is already guaranteed;
-// affine: rint(q) + z clamped to 0..15 in integer arithmetic).
+// SegStat::grid: |w / s| < 23), so C + OFF + rint(q) is exact and the code is
+// read from the bits of that sum as an integer.
+//
+// Two weights at a time: the division from the reciprocal and the rounding
+// addition run on the paired fp32 pipe (f32x2 mul / fma / add, each half an
+// IEEE round-to-nearest operation, so the quotient and its rounding are those
+// of the scalar route; OFF is even, so ties still go to the even integer).
+// Symmetric: OFF = 8 and the sum's bits are Cb + c + 8 with c + 8 in 1..15.
+// Affine: OFF = 2^14 and the low half of the sum's bits is 2^14 + rint(q);
+// the low halves of two weights share a register and are clamped together
+// to [2^14 - z, 2^14 - z + 15], i.e. rint(q) + z clamped to 0..15 plus the
+// base 2^14 - z.  Either way each value is a base plus its 4-bit code, so the
+// word is sum_k value_k 16^k minus base * 0x11111111 in 32-bit modular
+// arithmetic (linear, and the codes themselves do not overlap).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t r, uint32_t &lo, uint32_t &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(r));
+}
+// RN(RN(w / s) + c) for a pair of weights: rs2 = (RN(1/s), RN(1/s)), ns2 = (-s, -s),
+// c2 = (c, c).  The steps of div_by_recip, in pairs.
+__device__ __forceinline__ uint64_t quotient_plus_f32x2(uint64_t w, uint64_t rs2, uint64_t ns2,
+                                                        uint64_t c2) {
+  uint64_t q0, e, q, t;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(w), "l"(rs2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e) : "l"(q0), "l"(ns2), "l"(w));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(e), "l"(rs2), "l"(q0));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(q), "l"(c2));
+  return t;
+}
+__device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 template <bool SYM>
-__device__ __forceinline__ uint32_t pack_word_small(const float (&v)[8], const GridParams &g,
-                                                    float rs, int zi) {
-  constexpr float C = 12582912.0f;  // 1.5 * 2^23; its low mantissa bits are 0
-  uint32_t word = 0;
+__device__ __forceinline__ uint32_t pack_word_small(const float (&v)[8], float s, float rs,
+                                                    int zi) {
+  constexpr float C = 12582912.0f;  // 1.5 * 2^23; its low 22 mantissa bits are 0
+  constexpr uint32_t Cb = 0x4B400000u;
+  constexpr float OFF = SYM ? 8.0f : 16384.0f;
+  const uint64_t rs2 = f32x2_pack(rs, rs), ns2 = f32x2_pack(-s, -s);
+  const uint64_t c2 = f32x2_pack(C + OFF, C + OFF);
+  uint32_t t[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t t = __float_as_uint(__fadd_rn(div_by_recip(v[k], g.s, rs), C));
-    uint32_t nib;
-    if (SYM) {
-      nib = (t + 8u) & 0xFu;
-    } else {
-      const int c = static_cast<int>(t - __float_as_uint(C)) + zi;
-      nib = static_cast<uint32_t>(min(max(c, 0), 15));
-    }
-    word |= nib << (4 * k);
+  for (int p = 0; p < 4; ++p)
+    f32x2_unpack(quotient_plus_f32x2(f32x2_pack(v[2 * p], v[2 * p + 1]), rs2, ns2, c2),
+                 t[2 * p], t[2 * p + 1]);
+  if (SYM) {
+    uint32_t word = 0u - Cb * 0x11111111u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) word = mad_u32(t[k], 1u << (4 * k), word);
+    return word;
+  }
+  const uint32_t b16 = 16384u - static_cast<uint32_t>(zi);
+  const uint32_t lo2 = b16 * 0x10001u, hi2 = (b16 + 15u) * 0x10001u;
+  uint32_t word = 0u - b16 * 0x11111111u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t pr;  // low half of t_j, then low half of t_{j+4} (nibble j + 4 = 16 bits up)
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(pr) : "r"(t[j]), "r"(t[j + 4]));
+    asm("max.u16x2 %0, %0, %1;" : "+r"(pr) : "r"(lo2));
+    asm("min.u16x2 %0, %0, %1;" : "+r"(pr) : "r"(hi2));
+    word = mad_u32(pr, 1u << (4 * j), word);
   }
   return word;
 }
@@ -161,6 +262,15 @@ struct SegStat {
       b = fmaxf(b, x);
     }
   }
+  // from the min and max of 0 and the weights (lo <= 0 <= hi)
+  __device__ __forceinline__ void set(float lo, float hi) {
+    if (SYM) {
+      a = fmaxf(-lo, hi);
+    } else {
+      a = lo;
+      b = hi;
+    }
+  }
   __device__ __forceinline__ void reduce(int width) {
     for (int off = width / 2; off > 0; off >>= 1) {
       if (SYM) {
@@ -174,8 +284,11 @@ struct SegStat {
   // Same values as grid_sym / grid_affine, with the divisions by 7 and 15
   // done from their correctly rounded reciprocals.  small: every finite
   // weight of the segment has |w / s| < 7.5 (symmetric: the fp16 scale is
-  // a normal number, or the group is all but zero) or < 2^22 (affine: the
-  // scale did not saturate), so pack_word_small gives the same codes.
+  // a normal number, or the group is all but zero) or < 23 (affine: the
+  // scale did not saturate; then |w| <= b - a <= 15 s32 (1 + 2^-22), a
+  // normal fp16 s is at least s32 (1 - 2^-11), a subnormal one at least
+  // s32 / 1.5, and a zero one is replaced by 1 for weights below
+  // 15 * 2^-24), so pack_word_small gives the same codes.
   __device__ __forceinline__ GridParams grid(bool &small) const {
     GridParams g;
     float s32 = SYM ? div_by_recip(a, 7.0f, 1.0f / 7.0f)
@@ -236,14 +349,13 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
     }
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
+      MinMax<T> mm;
+#pragma unroll
+      for (int k = 0; k < WPL; ++k) mm.add(raw[u][k]);
+      float lo, hi;
+      mm.get(lo, hi);
       SegStat<SYM> st;
-#pragma unroll
-      for (int k = 0; k < WPL; ++k) {
-        float v[8];
-        raw[u][k].get(v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) st.add(v[e]);
-      }
+      st.set(lo, hi);
       st.reduce(TEAM);
       if (seg[u] >= total) continue;
       bool small;
@@ -261,7 +373,7 @@ __global__ void __launch_bounds__(256) rtn_reg_kernel(const T *__restrict__ W, i
         if (w < seg_words) {
           float v[8];
           raw[u][k].get(v);
-          dst[w] = small ? pack_word_small<SYM>(v, g, rs, zi) : pack_word<SYM>(v, g, rs);
+          dst[w] = small ? pack_word_small<SYM>(v, g.s, rs, zi) : pack_word<SYM>(v, g, rs);
         }
       }
     }
