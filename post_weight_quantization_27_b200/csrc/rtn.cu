@@ -686,7 +686,11 @@ void launch_reg(const void *W, int64_t d_out, int64_t seg_words, int64_t n_group
   const int64_t total = d_out * n_groups;
   const int64_t per_block = (256 / 32) * (32 / TEAM) * UNROLL;
   int64_t blocks = (total + per_block - 1) / per_block;
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  // 16-bit weights: up to one segment group per warp on the largest layers,
+  // so that the block scheduler balances the tail (a grid-stride of 2-3
+  // rounds per warp left the last round part-empty: 8192 x 28672 fp16
+  // 104 -> 100 us); fp32 rows (lm_head) run better on a capped grid
+  const int64_t cap = static_cast<int64_t>(num_sms()) * (sizeof(T) == 2 ? 64 : 8);
   if (blocks > cap) blocks = cap;
   const T *w = static_cast<const T *>(W);
   if (sym)
