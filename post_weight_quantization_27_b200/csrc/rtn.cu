@@ -184,13 +184,15 @@ __device__ __forceinline__ uint32_t pack_word(const float (&v)[8], const GridPar
 // addition run on the paired fp32 pipe (f32x2 mul / fma / add, each half an
 // IEEE round-to-nearest operation, so the quotient and its rounding are those
 // of the scalar route; OFF is even, so ties still go to the even integer).
-// Symmetric: OFF = 8 and the sum's bits are Cb + c + 8 with c + 8 in 1..15.
-// Affine: OFF = 2^14 and the low half of the sum's bits is 2^14 + rint(q);
-// the low halves of two weights share a register and are clamped together
-// to [2^14 - z, 2^14 - z + 15], i.e. rint(q) + z clamped to 0..15 plus the
-// base 2^14 - z.  Either way each value is a base plus its 4-bit code, so the
-// word is sum_k value_k 16^k minus base * 0x11111111 in 32-bit modular
-// arithmetic (linear, and the codes themselves do not overlap).
+// The low halves of the sums' bits (Cb's are 0) of weights k and k + 4 share
+// a register.  Symmetric: OFF = 8 and the low half is the stored code
+// c + 8 in 1..15 (clamped to 15 as well, which only a NaN weight reaches, so
+// that it cannot spill into its neighbours).  Affine: OFF = 2^14, the low
+// half is 2^14 + rint(q) and is clamped to [2^14 - z, 2^14 - z + 15], i.e.
+// rint(q) + z clamped to 0..15 plus the base 2^14 - z.  Either way each
+// half is a base plus its 4-bit code, so the word is sum_j pair_j 16^j minus
+// base * 0x11111111 in 32-bit modular arithmetic (linear, and the codes
+// themselves do not overlap).
 __device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -220,7 +222,6 @@ template <bool SYM>
 __device__ __forceinline__ uint32_t pack_word_small(const float (&v)[8], float s, float rs,
                                                     int zi) {
   constexpr float C = 12582912.0f;  // 1.5 * 2^23; its low 22 mantissa bits are 0
-  constexpr uint32_t Cb = 0x4B400000u;
   constexpr float OFF = SYM ? 8.0f : 16384.0f;
   const uint64_t rs2 = f32x2_pack(rs, rs), ns2 = f32x2_pack(-s, -s);
   const uint64_t c2 = f32x2_pack(C + OFF, C + OFF);
@@ -229,20 +230,16 @@ __device__ __forceinline__ uint32_t pack_word_small(const float (&v)[8], float s
   for (int p = 0; p < 4; ++p)
     f32x2_unpack(quotient_plus_f32x2(f32x2_pack(v[2 * p], v[2 * p + 1]), rs2, ns2, c2),
                  t[2 * p], t[2 * p + 1]);
-  if (SYM) {
-    uint32_t word = 0u - Cb * 0x11111111u;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) word = mad_u32(t[k], 1u << (4 * k), word);
-    return word;
-  }
-  const uint32_t b16 = 16384u - static_cast<uint32_t>(zi);
+  // symmetric: base 0 (the low halves are the stored codes themselves); the
+  // upper clamp only acts on a NaN weight, whose code it keeps in its nibble
+  const uint32_t b16 = SYM ? 0u : 16384u - static_cast<uint32_t>(zi);
   const uint32_t lo2 = b16 * 0x10001u, hi2 = (b16 + 15u) * 0x10001u;
   uint32_t word = 0u - b16 * 0x11111111u;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     uint32_t pr;  // low half of t_j, then low half of t_{j+4} (nibble j + 4 = 16 bits up)
     asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(pr) : "r"(t[j]), "r"(t[j + 4]));
-    asm("max.u16x2 %0, %0, %1;" : "+r"(pr) : "r"(lo2));
+    if (!SYM) asm("max.u16x2 %0, %0, %1;" : "+r"(pr) : "r"(lo2));
     asm("min.u16x2 %0, %0, %1;" : "+r"(pr) : "r"(hi2));
     word = mad_u32(pr, 1u << (4 * j), word);
   }

@@ -140,3 +140,31 @@ def test_rtn_per_tensor(dt, shape):
     W.view(-1)[shape[0] * shape[1] // 2] = 0.3      # the extreme sits in the middle
     _check(W, 0, True)
     _check(W, 0, False)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("group_size,sym", [(-1, True), (-1, False), (128, True), (128, False)])
+def test_rtn_nan_weight_keeps_the_other_codes(dt, group_size, sym):
+    """A NaN weight has no defined code.  The group statistic passes over it
+    (as fminf / fmaxf do), and it must not disturb any other code of its word
+    or group: with the NaN positions set to 0 (inside every group's range
+    already, since the range includes 0) the oracle's scales, zeros and the
+    codes of every other position are the GPU's."""
+    d_out, d_in = 16, 512
+    g = torch.Generator().manual_seed(77 + group_size + int(sym))
+    W = (torch.randn((d_out, d_in), generator=g) * 0.02).to(DT[dt])
+    nan_at = [(r, (37 * r + 5) % d_in) for r in range(0, d_out, 2)]
+    Wn, W0 = W.clone(), W.float().numpy().copy()
+    for r, c in nan_at:
+        Wn[r, c] = float("nan")
+        W0[r, c] = 0.0
+    out = gq.rtn_quantize_pack(Wn.cuda(), 4, group_size, sym)
+    torch.cuda.synchronize()
+    ref = O.rtn_quantize(W0, group_size, sym)
+    assert np.array_equal(f16(out["scales"]).view(np.uint16), ref["scales"].view(np.uint16))
+    if not sym:
+        assert np.array_equal(f16(out["zeros"]).view(np.uint16), ref["zeros"].view(np.uint16))
+    mask = np.full(ref["qpacked"].shape, 0xFFFFFFFF, dtype=np.uint32)
+    for r, c in nan_at:
+        mask[r, c // 8] &= np.uint32(~(0xF << (4 * (c % 8))) & 0xFFFFFFFF)
+    assert np.array_equal(u32(out["qpacked"]) & mask, ref["qpacked"] & mask)
